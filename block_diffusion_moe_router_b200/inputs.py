@@ -1,0 +1,197 @@
+"""Seeded synthetic inputs for the top-k mixture-of-experts FFN layer.
+
+This module only draws random tensors and packs integer codes into bytes.  It
+holds none of the layer's arithmetic, so both the CUDA path and the CPU oracle
+can consume its output without sharing any computation.
+
+Workloads (shapes and distributions follow the DiffusionGemma 26B-A4B pages:
+128 experts with 8 active per token, a 256-token canvas, hidden 2816 and
+per-expert intermediate 704, symmetric int4 weights in groups of 128):
+
+  tiny     T=16,   d=256,  E=16,  k=2, f=64,  bf16 weights
+  canvas   T=256,  d=2816, E=128, k=8, f=704, bf16 weights
+  canvas4  T=256,  d=2816, E=128, k=8, f=704, int4 w4g128 weights + fp16 scales
+  encode   T=2048, d=2816, E=128, k=8, f=704, bf16 weights (prompt + canvas)
+  stack30  30 layers of `canvas`, distinct weights, Zipf(1.1)-skewed router bias,
+           residual carried between layers
+
+Distributions: x ~ N(0,1) rounded to bf16; router W ~ N(0, 1/d) (variance 1/d,
+so logits have unit scale) in fp32; gamma ~ N(0, 0.1^2) in fp32; expert weights
+~ N(0, 0.02^2) rounded to bf16; int4 codes uniform on [-8, 7] and scales
+U(0.001, 0.01) rounded to fp16.  Seeds: 1000*workload_id + 10*layer + tensor_id.
+
+Layouts (all row-major, contiguous):
+  x            [T, d]            bf16
+  router_w     [E, d]            fp32
+  router_gamma [d]               fp32 (applied as 1 + gamma)
+  router_bias  [E]               fp32 or None
+  w_gate_up    [E, 2f, d]        bf16 (rows [0,f) gate, [f,2f) up)
+               [E, 2f, d/2]      uint8 for int4 (element i in byte i/2, low
+                                 nibble for even i, 4-bit two's complement)
+  w_down       [E, d, f]         bf16, or [E, d, f/2] uint8 for int4
+  scales_gu    [E, 2f, ceil(d/128)] fp16 (int4 only)
+  scales_d     [E, d, ceil(f/128)]  fp16 (int4 only)
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+GROUP = 128  # int4 quantisation group along the input dimension
+
+WDTYPE_BF16 = 0
+WDTYPE_INT4 = 1
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    wid: int          # workload id used in the seed formula
+    T: int
+    d: int
+    E: int
+    k: int
+    f: int
+    wdtype: int = WDTYPE_BF16
+    layers: int = 1
+    zipf_s: float = 0.0   # > 0: router bias drawn so expert load is Zipf(s)-skewed
+    residual: bool = False
+    act_wid: Optional[int] = None  # take x / router tensors from another workload's seeds
+
+    @property
+    def n_groups_d(self) -> int:
+        return (self.d + GROUP - 1) // GROUP
+
+    @property
+    def n_groups_f(self) -> int:
+        return (self.f + GROUP - 1) // GROUP
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 0, T=16, d=256, E=16, k=2, f=64),
+    "canvas": Workload("canvas", 1, T=256, d=2816, E=128, k=8, f=704),
+    "canvas4": Workload("canvas4", 2, T=256, d=2816, E=128, k=8, f=704,
+                        wdtype=WDTYPE_INT4, act_wid=1),
+    "encode": Workload("encode", 3, T=2048, d=2816, E=128, k=8, f=704),
+    "stack30": Workload("stack30", 4, T=256, d=2816, E=128, k=8, f=704,
+                        layers=30, zipf_s=1.1, residual=True),
+}
+
+# tensor ids inside the seed formula
+_TID_X, _TID_RW, _TID_GAMMA, _TID_WGU, _TID_WD, _TID_SGU, _TID_SD, _TID_BIAS = range(8)
+
+
+def seed_for(wid: int, layer: int, tensor_id: int) -> int:
+    return 1000 * wid + 10 * layer + tensor_id
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _randn(shape, std, seed, device, dtype):
+    g = _gen(seed, device)
+    t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(dtype)
+
+
+def pack_int4(codes: torch.Tensor) -> torch.Tensor:
+    """Pack int8 codes in [-8, 7] along the last dim: element i -> byte i/2,
+    low nibble for even i (4-bit two's complement)."""
+    assert codes.shape[-1] % 2 == 0
+    c = codes.to(torch.int16) & 0xF
+    lo = c[..., 0::2]
+    hi = c[..., 1::2]
+    return (lo | (hi << 4)).to(torch.uint8)
+
+
+def unpack_int4(packed: torch.Tensor) -> torch.Tensor:
+    """Inverse of pack_int4 (pure bit manipulation): uint8 -> int8 codes."""
+    p = packed.to(torch.int16)
+    lo = p & 0xF
+    hi = (p >> 4) & 0xF
+    out = torch.stack([lo, hi], dim=-1).reshape(*packed.shape[:-1], packed.shape[-1] * 2)
+    out = torch.where(out >= 8, out - 16, out)
+    return out.to(torch.int8)
+
+
+def make_int4(shape, seed_codes, seed_scales, device):
+    """Random int4 codes uniform on [-8, 7] (packed) and U(0.001, 0.01) fp16
+    scales, one per group of 128 along the last (input) dimension."""
+    E, rows, cols = shape
+    g = _gen(seed_codes, device)
+    codes = torch.randint(-8, 8, (E, rows, cols), generator=g, device=device, dtype=torch.int8)
+    ng = (cols + GROUP - 1) // GROUP
+    gs = _gen(seed_scales, device)
+    scales = (torch.rand((E, rows, ng), generator=gs, device=device, dtype=torch.float32)
+              * 0.009 + 0.001).to(torch.float16)
+    return pack_int4(codes), scales
+
+
+def zipf_bias(E: int, s: float, seed: int, device) -> torch.Tensor:
+    """Router bias whose exp() follows a Zipf(s) law over a seeded random
+    ranking of the experts: b_e = -s * ln(rank_e), rank_e in 1..E."""
+    g = _gen(seed, "cpu")
+    rank = torch.randperm(E, generator=g).to(torch.float64) + 1.0
+    return (-s * torch.log(rank)).to(torch.float32).to(device)
+
+
+def make_layer(w: Workload, layer: int = 0, device="cpu", T: Optional[int] = None,
+               with_x: bool = True) -> dict:
+    """All tensors of one layer of workload `w` (see module docstring)."""
+    T = w.T if T is None else T
+    awid = w.wid if w.act_wid is None else w.act_wid
+    out = {}
+    if with_x:
+        out["x"] = _randn((T, w.d), 1.0, seed_for(awid, 0, _TID_X), device, torch.bfloat16)
+    out["router_w"] = _randn((w.E, w.d), 1.0 / math.sqrt(w.d),
+                             seed_for(awid, layer, _TID_RW), device, torch.float32)
+    out["router_gamma"] = _randn((w.d,), 0.1, seed_for(awid, layer, _TID_GAMMA), device,
+                                 torch.float32)
+    out["router_bias"] = (zipf_bias(w.E, w.zipf_s, seed_for(w.wid, layer, _TID_BIAS), device)
+                          if w.zipf_s > 0 else None)
+    if w.wdtype == WDTYPE_BF16:
+        out["w_gate_up"] = _randn((w.E, 2 * w.f, w.d), 0.02, seed_for(w.wid, layer, _TID_WGU),
+                                  device, torch.bfloat16)
+        out["w_down"] = _randn((w.E, w.d, w.f), 0.02, seed_for(w.wid, layer, _TID_WD),
+                               device, torch.bfloat16)
+        out["scales_gate_up"] = None
+        out["scales_down"] = None
+    else:
+        out["w_gate_up"], out["scales_gate_up"] = make_int4(
+            (w.E, 2 * w.f, w.d), seed_for(w.wid, layer, _TID_WGU),
+            seed_for(w.wid, layer, _TID_SGU), device)
+        out["w_down"], out["scales_down"] = make_int4(
+            (w.E, w.d, w.f), seed_for(w.wid, layer, _TID_WD),
+            seed_for(w.wid, layer, _TID_SD), device)
+    return out
+
+
+def make_small(T, d, E, k, f, seed, wdtype=WDTYPE_BF16, bias=False, residual=False,
+               device="cpu", w_std=0.02, gamma_std=0.1) -> dict:
+    """A small random layer of arbitrary shape for tests (same distributions)."""
+    base = 100000 + 1000 * seed
+    out = {
+        "x": _randn((T, d), 1.0, base + 1, device, torch.bfloat16),
+        "router_w": _randn((E, d), 1.0 / math.sqrt(d), base + 2, device, torch.float32),
+        "router_gamma": _randn((d,), gamma_std, base + 3, device, torch.float32),
+        "router_bias": _randn((E,), 1.0, base + 4, device, torch.float32) if bias else None,
+        "residual": _randn((T, d), 1.0, base + 5, device, torch.bfloat16) if residual else None,
+    }
+    if wdtype == WDTYPE_BF16:
+        out["w_gate_up"] = _randn((E, 2 * f, d), w_std, base + 6, device, torch.bfloat16)
+        out["w_down"] = _randn((E, d, f), w_std, base + 7, device, torch.bfloat16)
+        out["scales_gate_up"] = None
+        out["scales_down"] = None
+    else:
+        out["w_gate_up"], out["scales_gate_up"] = make_int4((E, 2 * f, d), base + 6, base + 8,
+                                                            device)
+        out["w_down"], out["scales_down"] = make_int4((E, d, f), base + 7, base + 9, device)
+    return out

@@ -1,0 +1,22 @@
+"""CPU oracle of the top-k mixture-of-experts FFN layer (fp64, plain C).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
+baseline are the only callers.  The product path never imports this package
+and shares no code with it.  See moe_oracle.c for the definition it follows.
+"""
+from .oracle import (  # noqa: F401
+    build,
+    lib,
+    gelu_tanh,
+    rmsnorm_plus_one,
+    select_topk,
+    route_weights,
+    route,
+    moe_forward,
+    expert_ffn,
+    weight_row,
+    decode_bf16,
+    decode_fp16,
+    set_threads,
+    get_threads,
+)

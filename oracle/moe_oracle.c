@@ -1,0 +1,301 @@
+/*
+ * moe_oracle.c -- plain, slow, fp64 CPU oracle of the top-k mixture-of-experts
+ * FFN layer of DiffusionGemma 26B-A4B.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg may load this library.  It shares no code, header, table
+ * or helper with the CUDA path, and the CUDA path never calls it.
+ *
+ * Sources (page title, section):
+ *  [QT]  Quant-Tuner pull request "Add DiffusionGemma (Gemma-4 MoE
+ *        block-diffusion) support": Summary (128 experts, 8 active);
+ *        "Answers to the motivating questions" (the router reads the raw
+ *        residual through its own internal norm; the fused 3-D
+ *        experts.gate_up_proj; Gemma's (1+gamma) RMSNorm convention).
+ *  [AR]  auto-round pull request "Add quantization support for DiffusionGemma":
+ *        Description (fused gate_up_proj / down_proj), transformers backend
+ *        test log (act_fn GELUTanh; gate_proj 2816->704, up_proj 2816->704,
+ *        down_proj 704->2816; quantization_config bits 4, group_size 128,
+ *        sym True, data_type int).
+ *  [RF]  Hugging Face card "kingjones777/DiffusionGemma-26B-A4B-it-ROCmFP4-GGUF":
+ *        header (128 experts / top-8).
+ *
+ * Where the pages are silent this file follows the readings adopted by the
+ * library (they are listed once, here):
+ *  - routing: p = softmax over all E logits; S = the k largest logits, the
+ *    lower expert index winning ties, ordered by (logit desc, index asc);
+ *    w_j = p[S_j] / sum_{j'} p[S_j'];  gap = z_(k) - z_(k+1);
+ *  - gated form: out = down(gelu_tanh(gate(x)) * up(x)), gate = rows [0,f)
+ *    of the fused gate_up weight, up = rows [f,2f);
+ *  - the experts read x as given (any expert-side pre-norm is the caller's);
+ *  - RMSNorm: u_i = x_i / sqrt(mean_i x_i^2 + eps) * (1 + gamma_i);
+ *  - router bias (optional) is added to the logits before the softmax;
+ *  - int4: element i of a row sits in byte i/2, low nibble for even i, 4-bit
+ *    two's complement; w = code * scale[i / 128] with fp16 scales, exact here;
+ *  - out = residual + sum_j w_j y_j, summed in j order (residual optional).
+ *
+ * Everything is computed in double precision from the exact bf16 / fp16 /
+ * int4 values the GPU receives; nothing is rounded in between.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_W_BF16 0
+#define ORACLE_W_INT4 1
+#define ORACLE_GROUP 128
+
+/* ---- scalar decoders (IEEE definitions) -------------------------------- */
+
+/* bfloat16: the upper 16 bits of an IEEE binary32. */
+static double bf16_to_double(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* IEEE binary16: 1 sign bit, 5 exponent bits (bias 15), 10 mantissa bits. */
+static double fp16_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int ex = (h >> 10) & 0x1f;
+  int man = h & 0x3ff;
+  double v;
+  if (ex == 0)
+    v = ldexp((double)man, -24); /* subnormal: man * 2^-14 * 2^-10 */
+  else if (ex == 31)
+    v = man ? NAN : INFINITY;
+  else
+    v = ldexp(1.0 + man / 1024.0, ex - 15);
+  return sign ? -v : v;
+}
+
+/* 4-bit two's complement code of element i of a packed row. */
+static int int4_code(const uint8_t* row, int i) {
+  int byte = row[i / 2];
+  int nib = (i % 2 == 0) ? (byte & 0xf) : ((byte >> 4) & 0xf);
+  return nib >= 8 ? nib - 16 : nib;
+}
+
+/* One expert-weight element W[e][r][i] of a [E, R, C] weight in either
+ * storage format.  int4: code * fp16 scale of group i/128 ([AR] w4g128). */
+static double weight_elem(int wdtype, const void* w, const uint16_t* scales, int R, int C, int e,
+                          int r, int i) {
+  size_t row = (size_t)e * R + r;
+  if (wdtype == ORACLE_W_BF16) {
+    const uint16_t* wb = (const uint16_t*)w;
+    return bf16_to_double(wb[row * C + i]);
+  }
+  const uint8_t* wp = (const uint8_t*)w + row * (size_t)(C / 2);
+  int ng = (C + ORACLE_GROUP - 1) / ORACLE_GROUP;
+  double s = fp16_to_double(scales[row * ng + i / ORACLE_GROUP]);
+  return (double)int4_code(wp, i) * s;
+}
+
+/* ---- the layer, step by step -------------------------------------------- */
+
+/* GELU, tanh form ([AR] act_fn GELUTanh):
+ * 0.5 a (1 + tanh( sqrt(2/pi) (a + 0.044715 a^3) )). */
+double oracle_gelu_tanh(double a) {
+  const double c = sqrt(2.0 / M_PI);
+  return 0.5 * a * (1.0 + tanh(c * (a + 0.044715 * a * a * a)));
+}
+
+/* The router's own norm on the raw residual, Gemma (1+gamma) form ([QT]). */
+void oracle_rmsnorm_plus_one(int d, const double* x, const float* gamma, double eps,
+                             double* u) {
+  double ss = 0.0;
+  for (int i = 0; i < d; i++) ss += x[i] * x[i];
+  double r = sqrt(ss / d + eps);
+  for (int i = 0; i < d; i++) u[i] = x[i] / r * (1.0 + (double)gamma[i]);
+}
+
+/* Router logits z_e = sum_i W_r[e][i] u_i (+ b_e) ([QT]; fp32 weights). */
+void oracle_router_logits(int E, int d, const double* u, const float* router_w,
+                          const float* bias, double* z) {
+  for (int e = 0; e < E; e++) {
+    double acc = 0.0;
+    for (int i = 0; i < d; i++) acc += (double)router_w[(size_t)e * d + i] * u[i];
+    z[e] = acc + (bias ? (double)bias[e] : 0.0);
+  }
+}
+
+/* Top-k of E ([QT] Summary, [RF]: 8 of 128): k rounds, each taking the
+ * largest remaining logit; a strict '>' while scanning e upward keeps the
+ * lower index on ties.  gap = z_(k) - z_(k+1) (+inf when k == E). */
+void oracle_select_topk(int E, int k, const double* z, int32_t* idx, double* gap) {
+  char* taken = (char*)calloc((size_t)E, 1);
+  for (int j = 0; j < k; j++) {
+    int best = -1;
+    for (int e = 0; e < E; e++)
+      if (!taken[e] && (best < 0 || z[e] > z[best])) best = e;
+    idx[j] = best;
+    taken[best] = 1;
+  }
+  if (gap) {
+    int next = -1;
+    for (int e = 0; e < E; e++)
+      if (!taken[e] && (next < 0 || z[e] > z[next])) next = e;
+    *gap = (next < 0) ? INFINITY : z[idx[k - 1]] - z[next];
+  }
+  free(taken);
+}
+
+/* Routing weights: softmax over all E logits, restricted to S and
+ * renormalised so that the k weights sum to one. */
+void oracle_route_weights(int E, int k, const double* z, const int32_t* idx, double* w) {
+  double m = z[0];
+  for (int e = 1; e < E; e++)
+    if (z[e] > m) m = z[e];
+  double den = 0.0;
+  for (int e = 0; e < E; e++) den += exp(z[e] - m);
+  double sel = 0.0;
+  for (int j = 0; j < k; j++) {
+    w[j] = exp(z[idx[j]] - m) / den; /* p[S_j] */
+    sel += w[j];
+  }
+  for (int j = 0; j < k; j++) w[j] /= sel;
+}
+
+/* One expert e on one token ([QT] fused 3-D gate_up; [AR] gate/up 2816->704,
+ * down 704->2816, GELUTanh):
+ *   g_r = sum_i Wgu[e][r][i] x_i,  v_r = sum_i Wgu[e][f+r][i] x_i   (r < f)
+ *   h_r = gelu_tanh(g_r) * v_r
+ *   y_m = sum_r Wd[e][m][r] h_r                                    (m < d) */
+void oracle_expert_ffn(int d, int f, int wdtype, const void* w_gu, const void* w_d,
+                       const uint16_t* s_gu, const uint16_t* s_d, int e, const double* x,
+                       double* y, double* h_out) {
+  double* h = (double*)malloc(sizeof(double) * (size_t)f);
+  for (int r = 0; r < f; r++) {
+    double g = 0.0, v = 0.0;
+    for (int i = 0; i < d; i++) {
+      g += weight_elem(wdtype, w_gu, s_gu, 2 * f, d, e, r, i) * x[i];
+      v += weight_elem(wdtype, w_gu, s_gu, 2 * f, d, e, f + r, i) * x[i];
+    }
+    h[r] = oracle_gelu_tanh(g) * v;
+  }
+  for (int m = 0; m < d; m++) {
+    double acc = 0.0;
+    for (int r = 0; r < f; r++) acc += weight_elem(wdtype, w_d, s_d, d, f, e, m, r) * h[r];
+    y[m] = acc;
+  }
+  if (h_out) memcpy(h_out, h, sizeof(double) * (size_t)f);
+  free(h);
+}
+
+/* Dequantised (or widened) row r of expert e of a [E, R, C] weight. */
+void oracle_weight_row(int wdtype, const void* w, const uint16_t* scales, int R, int C, int e,
+                       int r, double* out) {
+  for (int i = 0; i < C; i++) out[i] = weight_elem(wdtype, w, scales, R, C, e, r, i);
+}
+
+/* Routing of one token: norm -> logits -> top-k -> weights. */
+static void route_token(int E, int k, int d, const uint16_t* x_row, const float* router_w,
+                        const float* gamma, const float* bias, double eps,
+                        const int32_t* forced_idx, double* xs, double* u, double* z,
+                        int32_t* idx, double* w, double* gap) {
+  for (int i = 0; i < d; i++) xs[i] = bf16_to_double(x_row[i]);
+  oracle_rmsnorm_plus_one(d, xs, gamma, eps, u);
+  oracle_router_logits(E, d, u, router_w, bias, z);
+  double g = 0.0;
+  oracle_select_topk(E, k, z, idx, &g);
+  if (gap) *gap = g;
+  if (forced_idx)
+    for (int j = 0; j < k; j++) idx[j] = forced_idx[j];
+  oracle_route_weights(E, k, z, idx, w);
+}
+
+static int n_threads_wanted = 0;
+
+void oracle_set_threads(int n) { n_threads_wanted = n; }
+
+int oracle_get_threads(void) {
+#ifdef _OPENMP
+  return n_threads_wanted > 0 ? n_threads_wanted : omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* Routing only, for T tokens.  Outputs: idx [T,k], w [T,k], gap [T],
+ * z [T,E] (any output may be NULL except idx and w). */
+void oracle_route(int T, int E, int k, int d, const uint16_t* x, const float* router_w,
+                  const float* gamma, const float* bias, double eps, int32_t* idx, double* w,
+                  double* gap, double* z_out) {
+#pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_get_threads())
+  for (int t = 0; t < T; t++) {
+    double* xs = (double*)malloc(sizeof(double) * (size_t)d);
+    double* u = (double*)malloc(sizeof(double) * (size_t)d);
+    double* z = (double*)malloc(sizeof(double) * (size_t)E);
+    route_token(E, k, d, x + (size_t)t * d, router_w, gamma, bias, eps, NULL, xs, u, z,
+                idx + (size_t)t * k, w + (size_t)t * k, gap ? gap + t : NULL);
+    if (z_out) memcpy(z_out + (size_t)t * E, z, sizeof(double) * (size_t)E);
+    free(xs);
+    free(u);
+    free(z);
+  }
+}
+
+/* The whole layer for T tokens, one token at a time over its k selected
+ * experts.  forced_idx [T,k] (or NULL) replaces the selected set S (the j
+ * order is then the given order); residual [T,d] bf16 (or NULL) is added.
+ * Outputs: out [T,d] (double), idx [T,k], w [T,k], gap [T] (NULL allowed
+ * for w and gap). */
+void oracle_moe_forward(int T, int E, int k, int d, int f, int wdtype, const uint16_t* x,
+                        const float* router_w, const float* gamma, const float* bias,
+                        double eps, const void* w_gu, const void* w_d, const uint16_t* s_gu,
+                        const uint16_t* s_d, const uint16_t* residual,
+                        const int32_t* forced_idx, double* out, int32_t* idx_out,
+                        double* w_out, double* gap_out) {
+#pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_get_threads())
+  for (int t = 0; t < T; t++) {
+    double* xs = (double*)malloc(sizeof(double) * (size_t)d);
+    double* u = (double*)malloc(sizeof(double) * (size_t)d);
+    double* z = (double*)malloc(sizeof(double) * (size_t)E);
+    double* y = (double*)malloc(sizeof(double) * (size_t)d);
+    int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* w = (double*)malloc(sizeof(double) * (size_t)k);
+    double gap = 0.0;
+    route_token(E, k, d, x + (size_t)t * d, router_w, gamma, bias, eps,
+                forced_idx ? forced_idx + (size_t)t * k : NULL, xs, u, z, idx, w, &gap);
+    double* o = out + (size_t)t * d;
+    for (int m = 0; m < d; m++)
+      o[m] = residual ? bf16_to_double(residual[(size_t)t * d + m]) : 0.0;
+    for (int j = 0; j < k; j++) {
+      oracle_expert_ffn(d, f, wdtype, w_gu, w_d, s_gu, s_d, idx[j], xs, y, NULL);
+      for (int m = 0; m < d; m++) o[m] += w[j] * y[m];
+    }
+    if (idx_out) memcpy(idx_out + (size_t)t * k, idx, sizeof(int32_t) * (size_t)k);
+    if (w_out) memcpy(w_out + (size_t)t * k, w, sizeof(double) * (size_t)k);
+    if (gap_out) gap_out[t] = gap;
+    free(xs);
+    free(u);
+    free(z);
+    free(y);
+    free(idx);
+    free(w);
+  }
+}
+
+/* Vector helpers for the pins: GELU-tanh and the (1+gamma) norm on rows. */
+void oracle_gelu_tanh_vec(int n, const double* a, double* out) {
+  for (int i = 0; i < n; i++) out[i] = oracle_gelu_tanh(a[i]);
+}
+
+void oracle_rmsnorm_rows(int T, int d, const double* x, const float* gamma, double eps,
+                         double* u) {
+  for (int t = 0; t < T; t++)
+    oracle_rmsnorm_plus_one(d, x + (size_t)t * d, gamma, eps, u + (size_t)t * d);
+}
+
+void oracle_decode_bf16(int n, const uint16_t* in, double* out) {
+  for (int i = 0; i < n; i++) out[i] = bf16_to_double(in[i]);
+}
+
+void oracle_decode_fp16(int n, const uint16_t* in, double* out) {
+  for (int i = 0; i < n; i++) out[i] = fp16_to_double(in[i]);
+}
