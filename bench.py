@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Throughput of the top-8-of-128 MoE FFN layer on a 256-token canvas.
+
+One step = one moe_forward (router -> plan -> gather -> expert GEMMs ->
+combine) over one canvas of T=256 tokens, d=2816, 128 experts, top-8,
+f=704, bf16 weights (synthetic, seeded; inputs resident in HBM).  The metric
+is canvas tokens/s per MoE layer; the JSON line also carries the expert
+kernel's HBM roofline fraction, an end-to-end figure through
+moe_forward_host (host buffers, copies inside the timed region) and the CPU
+oracle timed on a bounded sample.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (one canvas per GPU, no collective on the
+data path), launched one process per GPU by torch.distributed.run.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "canvas tokens/s per MoE layer (T=256, bf16) and % of HBM/tensor roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "expert_kernel_canvas.txt")
+EXPERT_SOURCES = ["block_diffusion_moe_router_b200/csrc/expert.cu",
+                  "block_diffusion_moe_router_b200/csrc/common.cuh"]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=100)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="canvas")
+    p.add_argument("--sets", type=int, default=0, help="input sets rotated (0: enough to exceed L2)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            m = json.load(fh)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), float(
+            m.get("bf16_tflops_sustained", m["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in EXPERT_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the expert kernel from the committed ncu
+    summary, or None if the summary is missing or the kernel changed since."""
+    try:
+        kv = {}
+        for line in open(PROFILE_SUMMARY):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("source_sha256_16") != source_hash():
+            return None
+        return float(kv["dram_bytes_per_launch_full_canvas"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.reasons |= int(r)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self._h is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples),
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+
+
+def layer_costs(w, touched: float, T: int):
+    """Algorithmic bytes and FLOPs of one layer call: weights of the experts
+    that receive a token (streamed once), x in, router tensors, out."""
+    if w.wdtype == 0:
+        wbytes = 3 * w.f * w.d * 2
+    else:
+        wbytes = 3 * w.f * w.d // 2 + 2 * (2 * w.f * w.n_groups_d + w.d * w.n_groups_f)
+    expert_bytes = touched * wbytes
+    act = T * w.d * 2 * (3 if w.residual else 2)
+    router = w.E * w.d * 4 + w.d * 4 + (w.E * 4 if w.zipf_s > 0 else 0)
+    flops = T * w.k * 2 * (3 * w.f * w.d) + 2 * T * w.E * w.d
+    return expert_bytes, expert_bytes + act + router, flops, wbytes
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+
+def oracle_sample_rate(lay_cpu, k, n_tokens, eps=1e-6):
+    """Tokens/s of the oracle on the first n_tokens rows (all host threads)."""
+    import oracle
+    x = lay_cpu["x"][:n_tokens]
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, lay_cpu["router_w"], lay_cpu["router_gamma"],
+                       lay_cpu.get("router_bias"), lay_cpu["w_gate_up"], lay_cpu["w_down"], k,
+                       scales_gate_up=lay_cpu.get("scales_gate_up"),
+                       scales_down=lay_cpu.get("scales_down"), eps=eps)
+    return n_tokens / (time.perf_counter() - t0)
+
+
+def cpu_baseline(lay_cpu, w, budget_s=12.0):
+    import oracle
+    cores = oracle.get_threads()
+    probe = max(1, min(w.T, cores))
+    r = oracle_sample_rate(lay_cpu, w.k, probe)
+    n = int(max(probe, min(w.T, round(r * budget_s / cores) * cores)))
+    r = oracle_sample_rate(lay_cpu, w.k, n)
+    return {"value": r, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of the {w.T} canvas tokens, fp64 oracle, one layer"}
+
+
+# ---------------------------------------------------------------- arms
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+    import oracle
+    from block_diffusion_moe_router_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    lay = {k: (v.cpu() if isinstance(v, torch.Tensor) else v)
+           for k, v in inputs.make_layer(w, device=dev).items()}
+    cores = oracle.get_threads()
+    r1 = oracle_sample_rate(lay, w.k, min(w.T, cores))
+    steps = args.steps + args.warmup
+    per = max(1, min(w.T, int(120.0 * r1 / steps)))
+    pos = 0
+
+    def step():
+        nonlocal pos
+        rows = [(pos + i) % w.T for i in range(per)]
+        pos = (pos + per) % w.T
+        sub = dict(lay)
+        sub["x"] = lay["x"][rows]
+        oracle.moe_forward(sub["x"], sub["router_w"], sub["router_gamma"],
+                           sub.get("router_bias"), sub["w_gate_up"], sub["w_down"], w.k,
+                           scales_gate_up=sub.get("scales_gate_up"),
+                           scales_down=sub.get("scales_down"))
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = args.steps * per / dt
+    sample = f"{per} of the {w.T} canvas tokens per step (rotating), fp64 oracle, one layer"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: T={w.T} d={w.d} E={w.E} k={w.k} f={w.f} bf16 weights",
+                   "sample_tokens_per_step": per},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import block_diffusion_moe_router_b200 as moe
+    from block_diffusion_moe_router_b200 import inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = inputs.WORKLOADS[args.workload]
+    T = w.T
+    lay = inputs.make_layer(w, device="cuda", with_x=False)
+    # rotate the small per-call inputs so that, with the weights, the working
+    # set exceeds L2 on every step
+    small = T * w.d * 2 * 2 + w.E * w.d * 4 + w.d * 4
+    nsets = args.sets or max(2, math.ceil(1.1 * L2_BYTES / small))
+    xs = [inputs._randn((T, w.d), 1.0, 777000 + 1000 * rank + i, "cuda", torch.bfloat16)
+          for i in range(nsets)]
+    rws = [lay["router_w"]] + [lay["router_w"][torch.randperm(w.E, device="cuda")].contiguous()
+                               for _ in range(nsets - 1)]
+    gms = [lay["router_gamma"]] + [lay["router_gamma"].roll(i).contiguous()
+                                   for i in range(1, nsets)]
+    outs = [torch.empty((T, w.d), dtype=torch.bfloat16, device="cuda") for _ in range(nsets)]
+    plan = moe.moe_plan_create(w.E, w.k, w.d, w.f, w.wdtype)
+    moe.moe_plan_reserve(plan, T)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        j = i % nsets
+        moe.moe_forward(plan, T, xs[j], rws[j], gms[j], lay["router_bias"], lay["w_gate_up"],
+                        lay["w_down"], lay["scales_gate_up"], lay["scales_down"], None, outs[j],
+                        stream)
+
+    # touched experts per set (weights the layer must stream)
+    touched = []
+    for i in range(nsets):
+        step(i)
+        off = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+        moe.moe_plan_routing(plan, off, None, None, stream)
+        touched.append(int(((off[1:] - off[:-1]) > 0).sum().item()))
+    st = moe.moe_plan_sync_status(plan, stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(moe.moe_status_str(st))
+    mean_touched = sum(touched) / len(touched)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(K, profile):
+        moe.moe_plan_set_option(plan, moe.MOE_OPT_PROFILE, 1 if profile else 0)
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = e0.elapsed_time(e1)
+        moe.moe_plan_set_option(plan, moe.MOE_OPT_PROFILE, 0)
+        if world > 1:
+            t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    for kk in range(moe.MOE_K_COMBINE + 1):  # discard warm-up records
+        moe.moe_plan_profile(plan, kk)
+    with ClockSampler(local) as clk:
+        ms = timed(args.steps, profile=True)
+    kern = {}
+    for kk, name in enumerate(moe.KERNEL_NAMES):
+        tot, n = moe.moe_plan_profile(plan, kk)
+        kern[name] = (tot / n) if n else None
+    ms_plain = timed(args.steps, profile=False)
+    st = moe.moe_plan_sync_status(plan, stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(moe.moe_status_str(st))
+
+    # end to end through moe_forward_host: host x in, host out back, every step
+    x_host = [xs[i].cpu().pin_memory() for i in range(min(nsets, 4))]
+    out_host = torch.empty((T, w.d), dtype=torch.bfloat16).pin_memory()
+    K2 = args.steps
+    barrier()
+    t0 = time.perf_counter()
+    for i in range(K2):
+        moe.moe_forward_host(plan, T, x_host[i % len(x_host)], rws[0], gms[0], lay["router_bias"],
+                             lay["w_gate_up"], lay["w_down"], lay["scales_gate_up"],
+                             lay["scales_down"], None, out_host, stream)
+    e2e_s = time.perf_counter() - t0
+    if world > 1:
+        t = torch.tensor([e2e_s], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    st = moe.moe_plan_sync_status(plan, stream)
+    if st != moe.MOE_OK:
+        raise RuntimeError(moe.moe_status_str(st))
+
+    hbm, bf16, bf16_sus, basis = peaks()
+    expert_bytes, layer_bytes, flops, wbytes = layer_costs(w, mean_touched, T)
+    ms_step = ms / args.steps
+    k_ms = kern["expert"]
+    achieved = expert_bytes / (k_ms * 1e-3) / 1e9 if k_ms else None
+    traffic = recorded_traffic()
+    line = {
+        "metric": METRIC,
+        "value": world * T * args.steps / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{w.name}: one MoE layer over a T={T} token canvas, d={w.d}, E={w.E}, "
+                        f"top-{w.k}, f={w.f}, bf16 weights",
+            "global_batch": world * T, "seq_len": T,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"weights {wbytes * w.E / 1e9:.2f} GB > L2; x/router/out rotated over "
+                  f"{nsets} sets ({nsets * small / 2**20:.0f} MiB)",
+            "timed_region": "per-kernel CUDA events recorded inside the timed steps",
+            "ms_per_step_without_events": ms_plain / args.steps,
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "expert (grouped gate_up + down GEMMs)",
+            "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": (achieved / hbm) if achieved else None, "traffic": traffic,
+            "peak_basis": f"{basis} HBM copy bandwidth",
+            "alg_bytes_per_launch": expert_bytes,
+            "alg_bytes_rule": f"{mean_touched:.2f} touched experts x {wbytes} B of expert "
+                              f"weights",
+            "kernel_ms": k_ms,
+        },
+        "layer_roofline": {
+            "alg_bytes": layer_bytes, "flops": flops,
+            "t_hbm_ms": layer_bytes / (hbm * 1e9) * 1e3,
+            "t_tensor_ms": flops / (bf16 * 1e12) * 1e3,
+            "frac_of_roofline": (max(layer_bytes / (hbm * 1e9), flops / (bf16 * 1e12)) * 1e3)
+                                / ms_step,
+        },
+        "kernel_ms": kern,
+        "gpu_launches": 5 * args.steps,
+        "e2e": {"value": world * T * K2 / e2e_s, "unit": "tokens/s",
+                "h2d_bytes_per_step": T * w.d * 2, "d2h_bytes_per_step": T * w.d * 2},
+        "clocks": clk.summary(),
+    }
+    moe.moe_plan_destroy(plan)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        lay_cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in lay.items()}
+        lay_cpu["x"] = xs[0].cpu()
+        line["cpu_baseline"] = cpu_baseline(lay_cpu, w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,300 @@
+// common.cuh -- sm_100a building blocks shared by the MoE kernels:
+// mbarriers with bounded waits, TMA tile loads, tcgen05 (UMMA + TMEM)
+// wrappers, the device status word, and launch-parameter structs.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- layout constants
+constexpr int kBM = 128;           // UMMA M: weight rows per tile
+constexpr int kBK = 64;            // K elements per pipeline stage (bf16: 128 bytes/row)
+constexpr int kUmmaK = 16;         // K of one kind::f16 UMMA
+constexpr int kMaxN = 256;         // tokens per unit (UMMA N upper bound)
+constexpr int kBRows = 32;         // rows per B-operand TMA box
+constexpr int kGuHalf = 64;        // gate rows (and up rows) per gate_up tile
+constexpr int kTmemCols = 512;     // whole TMEM: 2 accumulators x 256 columns
+constexpr int kRouterTT = 8;       // tokens per router CTA
+constexpr int kRouterTE = 32;      // experts per router CTA
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 32;
+
+// Device status / scheduler words kept by the plan (one small int array).
+struct Ctl {
+  int status;        // 0 or an moe_status_t, first error wins
+  int where;         // code of the wait or check that failed
+  int work_next;     // next unit index handed out by the expert scheduler
+  int n_chunks;      // number of (expert, 256-token chunk) pairs this call
+  int max_chunk;     // largest chunk (tokens) this call
+  int pad[3];
+};
+
+__device__ __forceinline__ void record_error(Ctl* ctl, int code, int where) {
+  if (atomicCAS(&ctl->status, 0, code) == 0) atomicExch(&ctl->where, where);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete.  Gives up after
+// timeout_ns (records MOE_ERR_TIMEOUT with `where`) or when another role of
+// the CTA has already given up (*abort != 0).  Returns true on success.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          Ctl* ctl, uint64_t timeout_ns, int where) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(a, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      record_error(ctl, MOE_ERR_TIMEOUT, where);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- TMA
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// 2-D tiled TMA load (no multicast): box at element coordinates (x, y),
+// x innermost.  Completes `bytes` on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, int x, int y,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// ---------------------------------------------------------------- tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on `bar` when every UMMA issued so far by this thread is done.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 D.
+//   [4,6) D format = 1 (f32), [7,10) A = 1 (bf16), [10,13) B = 1 (bf16),
+//   [15] A major = 0 (K), [16] B major = 0 (K), [17,23) N >> 3, [24,29) M >> 4.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor for a K-major tile written by TMA with
+// 128-byte swizzling: rows of 128 bytes, 8-row swizzle atoms 1024 bytes
+// apart (SBO), leading offset unused for swizzled K-major (1), version 1,
+// layout type 2 (SWIZZLE_128B).  The atom base must be 1024-byte aligned;
+// stepping K inside the 128-byte row adds bytes to the start address.
+__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// 32 lanes x 32 bit, 32 consecutive columns: thread i of the warp gets TMEM
+// lane (warp's quarter base + i), columns [col, col+32).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------- launch params
+struct RouterArgs {
+  int T, E, k, d;
+  float eps;
+  const __nv_bfloat16* x;
+  const float* router_w;
+  const float* gamma;
+  const float* bias;
+  int32_t* idx;
+  float* w;
+  float* gap;
+  Ctl* ctl;
+};
+
+struct PlanArgs {
+  int T, E, k, d, f;
+  const int32_t* idx;    // [T*k]
+  int32_t* offsets;      // [E+1]
+  int32_t* perm;         // [T*k] slot -> token
+  int32_t* slot_of;      // [T*k] assignment -> slot
+  int32_t* chunk_e;      // [max_chunks] chunk -> expert
+  int32_t* chunk_c;      // [max_chunks] chunk -> chunk index within expert
+  int32_t* ready;        // [max_chunks] gate_up tiles finished per chunk
+  Ctl* ctl;
+};
+
+struct GatherArgs {
+  int rows, d;
+  const int32_t* perm;
+  const __nv_bfloat16* x;
+  __nv_bfloat16* x_perm;
+};
+
+struct ExpertArgs {
+  int T, E, k, d, f;
+  const int32_t* offsets;
+  const int32_t* chunk_e;
+  const int32_t* chunk_c;
+  int32_t* ready;
+  __nv_bfloat16* h;   // [T*k, f]
+  float* y;           // [T*k, d]
+  Ctl* ctl;
+  uint64_t timeout_ns;
+  int test_stall;
+};
+
+struct CombineArgs {
+  int T, k, d;
+  const int32_t* slot_of;
+  const float* w;
+  const float* y;
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* out;
+};
+
+}  // namespace moe
+
+// Host-side launchers (one per kernel file).
+cudaError_t moe_launch_router(const moe::RouterArgs& a, cudaStream_t s);
+cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s);
+cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s);
+cudaError_t moe_launch_expert(const moe::ExpertArgs& a, const CUtensorMap& tm_wgu,
+                              const CUtensorMap& tm_wd, const CUtensorMap& tm_xp,
+                              const CUtensorMap& tm_h, int num_sms, cudaStream_t s);
+cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s);

@@ -1,0 +1,436 @@
+// expert.cu -- grouped expert GEMMs of the MoE FFN on tcgen05 tensor cores.
+//
+// One persistent kernel runs every (expert, 256-token chunk) work unit of both
+// projections (auto-round pull request "Add quantization support for
+// DiffusionGemma", transformers backend test log: gate_proj / up_proj
+// 2816->704, down_proj 704->2816, act GELUTanh; Quant-Tuner pull request,
+// "Answers to the motivating questions": one fused 3-D gate_up projection):
+//
+//   gate_up unit (e, chunk, m): 64 gate rows [m*64, m*64+64) and the 64 up rows
+//     [f + m*64, ...) of W_gu[e] are stacked into one 128-row A tile, so a
+//     single M=128 UMMA per K step computes both for the chunk's tokens (N);
+//     the epilogue pairs TMEM lane r (gate) with lane 64+r (up) and writes
+//     h = gelu_tanh(gate) * up in bf16.
+//   down unit (e, chunk, m): rows [m*128, m*128+128) of W_d[e] against the
+//     chunk's h rows; the epilogue writes y (fp32) per slot.
+//
+// "Swap-AB": weight rows are the UMMA M dimension and the tokens routed to
+// the expert are N (16..256), so every weight byte is streamed from HBM once
+// per chunk, and at 256 tokens per canvas one chunk covers every expert.
+//
+// Roles (192 threads): warp 0 = TMA producer (also the scheduler: it claims
+// units from a global counter), warp 1 = UMMA issuer (owns the TMEM
+// allocation), warps 2..5 = epilogue (TMEM -> registers -> global).  Smem
+// holds a ring of A/B stages sized at run time from the largest chunk; TMEM
+// holds two 256-column fp32 accumulators so the epilogue of one unit overlaps
+// the MMAs of the next.  A down unit may start only when all gate_up units of
+// its chunk have published h (per-chunk counter, acquire/release).
+//
+// Every wait is bounded by %globaltimer; on expiry the kernel records
+// MOE_ERR_TIMEOUT, the roles leave their loops, in-flight TMA copies and
+// UMMAs are drained (again bounded) and TMEM is released.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kUnitRing = 4;
+constexpr int kMaxStages = 8;
+constexpr int kRingBytes = 200 * 1024;
+constexpr int kXchgStride = 33;  // floats per exchanged row (bank-conflict padding)
+constexpr int kXchgBytes = 64 * kXchgStride * 4;
+constexpr int kABytes = kBM * kBK * 2;  // 16 KB
+constexpr int kBarBytes = 8 * (2 * kMaxStages + 4 + 2 * kUnitRing + 1);
+constexpr int kSmemBytes = 1024 + kRingBytes + kXchgBytes + kBarBytes + 256;
+
+enum { kUnitGateUp = 0, kUnitDown = 1, kUnitStop = -1 };
+
+struct UnitInfo {
+  int type;
+  int e;      // expert
+  int m;      // row tile inside the expert's weight
+  int n;      // tokens in this chunk (1..256)
+  int slot0;  // first slot of the chunk
+  int q;      // chunk index (scheduler table)
+};
+
+enum {
+  kWhereUnitEmpty = 1,
+  kWhereStageEmpty,
+  kWhereReady,
+  kWhereUnitFullMma,
+  kWhereTmemEmpty,
+  kWhereStageFull,
+  kWhereUnitFullEpi,
+  kWhereTmemFull,
+  kWhereDrain
+};
+
+__device__ __forceinline__ float gelu_tanh(float g) {
+  // 0.5 g (1 + tanh( sqrt(2/pi) (g + 0.044715 g^3) ))
+  const float c = 0.7978845608028654f;
+  return 0.5f * g * (1.f + tanhf(c * fmaf(0.044715f * g, g * g, g)));
+}
+
+// Spin until *p >= need (acquire), bounded like mbar_wait.
+__device__ bool wait_count(const int* p, int need, volatile int* abort, Ctl* ctl,
+                           uint64_t timeout_ns, int where) {
+  if (ld_acquire_gpu(p) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i) {
+      __nanosleep(64);
+      if (ld_acquire_gpu(p) >= need) return true;
+    }
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      record_error(ctl, MOE_ERR_TIMEOUT, where);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag (used only while draining).
+__device__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, Ctl* ctl, uint64_t timeout_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      record_error(ctl, MOE_ERR_TIMEOUT, kWhereDrain);
+      return false;
+    }
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    expert_kernel(const __grid_constant__ CUtensorMap tm_wgu,
+                  const __grid_constant__ CUtensorMap tm_wd,
+                  const __grid_constant__ CUtensorMap tm_xp,
+                  const __grid_constant__ CUtensorMap tm_h, ExpertArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  float* xchg = reinterpret_cast<float*>(smem + kRingBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kXchgBytes);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* ufull = tempty + 2;
+  uint64_t* uempty = ufull + kUnitRing;
+  uint64_t* drain = uempty + kUnitRing;
+  UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(units + kUnitRing);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_bcast = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int GU = a.f / kGuHalf;
+  const int DN = a.d / kBM;
+  Ctl* ctl = a.ctl;
+
+  // B-operand rows per stage: the largest chunk, rounded up to the TMA box.
+  const int maxn = max(1, min(kMaxN, ctl->max_chunk));
+  const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
+  const int stage_bytes = kABytes + NB * kBK * 2;
+  const int S = min(kMaxStages, kRingBytes / stage_bytes);
+  const int n_chunks = ctl->n_chunks;
+  const int U = n_chunks * (GU + DN);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);  // one arrival per epilogue warp
+    }
+    for (int i = 0; i < kUnitRing; ++i) {
+      mbar_init(&ufull[i], 1);
+      mbar_init(&uempty[i], 2);  // UMMA issuer + epilogue leader
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_wgu);
+    tma_prefetch_desc(&tm_wd);
+    tma_prefetch_desc(&tm_xp);
+    tma_prefetch_desc(&tm_h);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_act = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int ur = 0;
+      uint32_t uphase = 0;
+      uint32_t issued = 0, issued_par = 0;  // stages with a copy issued, and its parity
+      while (true) {
+        if (*s_abort) break;
+        const int u = atomicAdd(&ctl->work_next, 1);
+        UnitInfo ui;
+        ui.type = kUnitStop;
+        ui.e = ui.m = ui.n = ui.slot0 = ui.q = 0;
+        if (u < U) {
+          int q, m;
+          if (u < n_chunks * GU) {
+            ui.type = kUnitGateUp;
+            q = u / GU;
+            m = u - q * GU;
+          } else {
+            const int v = u - n_chunks * GU;
+            ui.type = kUnitDown;
+            q = v / DN;
+            m = v - q * DN;
+          }
+          const int e = a.chunk_e[q];
+          const int c = a.chunk_c[q];
+          const int seg0 = a.offsets[e];
+          const int ne = a.offsets[e + 1] - seg0;
+          ui.e = e;
+          ui.m = m;
+          ui.q = q;
+          ui.slot0 = seg0 + c * kMaxN;
+          ui.n = min(kMaxN, ne - c * kMaxN);
+          if (ui.n < 1 || ui.n > NB) {  // corrupt plan: never index outside the ring
+            record_error(ctl, MOE_ERR_DEVICE_CHECK, 200);
+            *s_abort = 1;
+            break;
+          }
+        }
+        if (ui.type == kUnitDown) {
+          const int need = GU + (a.test_stall ? (1 << 30) : 0);
+          if (!wait_count(a.ready + ui.q, need, s_abort, ctl, a.timeout_ns, kWhereReady)) break;
+          fence_proxy_async_global();
+        }
+        if (!mbar_wait(&uempty[ur], uphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereUnitEmpty))
+          break;
+        units[ur] = ui;
+        mbar_arrive(&ufull[ur]);
+        if (++ur == kUnitRing) {
+          ur = 0;
+          uphase ^= 1;
+        }
+        if (ui.type == kUnitStop) break;
+
+        const int nkb = (ui.type == kUnitGateUp) ? a.d / kBK : a.f / kBK;
+        const int nbox = (ui.n + kBRows - 1) / kBRows;
+        const uint32_t tx = kABytes + nbox * kBRows * kBK * 2;
+        const CUtensorMap* tb = (ui.type == kUnitGateUp) ? &tm_xp : &tm_h;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
+                         kWhereStageEmpty)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = ring + stage * stage_bytes;
+          uint8_t* sb = sa + kABytes;
+          mbar_arrive_expect_tx(&full[stage], tx);
+          const int kx = kb * kBK;
+          if (ui.type == kUnitGateUp) {
+            const int r0 = ui.e * 2 * a.f + ui.m * kGuHalf;
+            tma_load_2d(sa, &tm_wgu, kx, r0, &full[stage], pol_w);
+            tma_load_2d(sa + kGuHalf * kBK * 2, &tm_wgu, kx, r0 + a.f, &full[stage], pol_w);
+          } else {
+            tma_load_2d(sa, &tm_wd, kx, ui.e * a.d + ui.m * kBM, &full[stage], pol_w);
+          }
+          for (int bx = 0; bx < nbox; ++bx)
+            tma_load_2d(sb + bx * kBRows * kBK * 2, tb, kx, ui.slot0 + bx * kBRows, &full[stage],
+                        pol_act);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      // Drain: every issued copy must land before the CTA may exit.
+      for (int s2 = 0; s2 < S; ++s2)
+        if ((issued >> s2) & 1u) mbar_wait_drain(&full[s2], (issued_par >> s2) & 1u, ctl,
+                                                 a.timeout_ns);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int ur = 0;
+      uint32_t uphase = 0;
+      int acc = 0;
+      uint32_t aphase = 0;
+      while (true) {
+        if (!mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullMma)) break;
+        const UnitInfo ui = units[ur];
+        if (ui.type == kUnitStop) break;
+        const int nkb = (ui.type == kUnitGateUp) ? a.d / kBK : a.f / kBK;
+        const int N = (ui.n + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(kBM, N);
+        if (!mbar_wait(&tempty[acc], aphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereTmemEmpty))
+          break;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + (uint32_t)(acc * kMaxN);
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, s_abort, ctl, a.timeout_ns, kWhereStageFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(ring + stage * stage_bytes);
+          const uint32_t sb = sa + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+            umma_bf16(dt, sdesc_k_sw128(sa + kk * kUmmaK * 2), sdesc_k_sw128(sb + kk * kUmmaK * 2),
+                      idesc, (kb | kk) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        mbar_arrive(&uempty[ur]);
+        if (++ur == kUnitRing) {
+          ur = 0;
+          uphase ^= 1;
+        }
+        acc ^= 1;
+        if (acc == 0) aphase ^= 1;
+      }
+      // Drain: all issued UMMAs complete before TMEM is released.
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, ctl, a.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;          // TMEM lane quarter this warp may access
+    const int row = q4 * 32 + lane;   // accumulator row (TMEM lane)
+    const int et = threadIdx.x - 64;  // 0..127
+    int ur = 0;
+    uint32_t uphase = 0;
+    int acc = 0;
+    uint32_t aphase = 0;
+    while (true) {
+      // The leader waits; the decision is broadcast so the 128 threads always
+      // take the same path through the named barriers below.
+      if (et == 0) {
+        bool ok = mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullEpi);
+        if (ok && units[ur].type != kUnitStop)
+          ok = mbar_wait(&tfull[acc], aphase, s_abort, ctl, a.timeout_ns, kWhereTmemFull);
+        *s_bcast = ok ? 1 : 0;
+      }
+      named_barrier(1, 128);
+      const bool ok = *s_bcast != 0;
+      const UnitInfo ui = units[ur];
+      named_barrier(1, 128);
+      if (!ok || ui.type == kUnitStop) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kMaxN);
+      const int nch = (ui.n + 31) / 32;
+      if (ui.type == kUnitGateUp) {
+        __nv_bfloat16* hcol = a.h + (size_t)ui.slot0 * a.f + ui.m * kGuHalf + row;
+        for (int cc = 0; cc < nch; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tbase + cc * 32, v);
+          tmem_wait_ld();
+          if (row >= kGuHalf) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              xchg[(row - kGuHalf) * kXchgStride + i] = __uint_as_float(v[i]);
+          }
+          named_barrier(1, 128);
+          if (row < kGuHalf) {
+            const int cmax = min(32, ui.n - cc * 32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i < cmax) {
+                const float g = __uint_as_float(v[i]);
+                const float up = xchg[row * kXchgStride + i];
+                hcol[(size_t)(cc * 32 + i) * a.f] = __float2bfloat16(gelu_tanh(g) * up);
+              }
+            }
+          }
+          named_barrier(1, 128);
+        }
+      } else {
+        float* ycol = a.y + (size_t)ui.slot0 * a.d + ui.m * kBM + row;
+        for (int cc = 0; cc < nch; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tbase + cc * 32, v);
+          tmem_wait_ld();
+          const int cmax = min(32, ui.n - cc * 32);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __uint_as_float(v[i]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (ui.type == kUnitGateUp) __threadfence();  // h visible before the chunk counter
+      named_barrier(1, 128);
+      if (et == 0) {
+        if (ui.type == kUnitGateUp) {
+          __threadfence();
+          fence_proxy_async_global();
+          atomicAdd(a.ready + ui.q, 1);
+        }
+        mbar_arrive(&uempty[ur]);
+      }
+      if (++ur == kUnitRing) {
+        ur = 0;
+        uphase ^= 1;
+      }
+      acc ^= 1;
+      if (acc == 0) aphase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+}  // namespace moe
+
+cudaError_t moe_launch_expert(const moe::ExpertArgs& a, const CUtensorMap& tm_wgu,
+                              const CUtensorMap& tm_wd, const CUtensorMap& tm_xp,
+                              const CUtensorMap& tm_h, int num_sms, cudaStream_t s) {
+  static_assert(moe::kSmemBytes <= 232448, "expert kernel smem above the sm_100 limit");
+  cudaError_t err = cudaFuncSetAttribute(moe::expert_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         moe::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  moe::expert_kernel<<<num_sms, moe::kThreads, moe::kSmemBytes, s>>>(tm_wgu, tm_wd, tm_xp, tm_h,
+                                                                      a);
+  return cudaGetLastError();
+}

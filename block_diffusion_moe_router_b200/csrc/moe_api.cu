@@ -1,0 +1,514 @@
+// moe_api.cu -- host side of the C ABI declared in include/moe.h: plan
+// objects, argument validation, the plan-owned workspace, TMA tensor maps and
+// the launch sequence router -> plan -> gather -> expert GEMMs -> combine.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "moe.h"
+
+namespace {
+
+using moe::Ctl;
+
+struct ProfRec {
+  int kernel;
+  cudaEvent_t start, stop;
+};
+
+}  // namespace
+
+struct moe_plan_s {
+  int E, k, d, f;
+  moe_wdtype_t wdtype;
+  int device;
+  int num_sms;
+  float eps;
+  int timeout_ms;
+  int profile;
+  int test_stall;
+  int cap_T;
+  int last_T;
+  void* ws;  // one device allocation holding everything below
+  Ctl* ctl;
+  int32_t *idx, *perm, *slot_of, *offsets, *chunk_e, *chunk_c, *ready;
+  float *w, *gap, *y;
+  __nv_bfloat16 *x_perm, *h, *x_dev, *res_dev, *out_dev;
+  std::vector<ProfRec> prof;
+  std::vector<cudaEvent_t> ev_pool;
+};
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix, 128-byte swizzle,
+// box = box_rows x 64 columns (128 bytes).
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+int max_chunks(int E, int T, int k) { return E + (T * k) / moe::kMaxN + 1; }
+
+moe_status_t check_device(moe_plan_t p) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  return dev == p->device ? MOE_OK : MOE_ERR_INVALID_ARG;
+}
+
+moe_status_t ensure_workspace(moe_plan_t p, int T) {
+  if (p->ws && T <= p->cap_T) return MOE_OK;
+  int cap = p->cap_T > 0 ? p->cap_T : 16;
+  while (cap < T) cap *= 2;
+  const size_t A = (size_t)cap * p->k;
+  const size_t MC = (size_t)max_chunks(p->E, cap, p->k);
+  size_t sz = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = sz;
+    sz += align256(bytes);
+    return o;
+  };
+  const size_t o_ctl = take(sizeof(Ctl));
+  const size_t o_idx = take(A * 4), o_w = take(A * 4), o_gap = take((size_t)cap * 4);
+  const size_t o_perm = take(A * 4), o_slot = take(A * 4), o_off = take((size_t)(p->E + 1) * 4);
+  const size_t o_ce = take(MC * 4), o_cc = take(MC * 4), o_rd = take(MC * 4);
+  const size_t o_xp = take(A * p->d * 2), o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
+  const size_t o_xd = take((size_t)cap * p->d * 2), o_rs = take((size_t)cap * p->d * 2);
+  const size_t o_od = take((size_t)cap * p->d * 2);
+  if (p->ws) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    cudaFree(p->ws);
+    p->ws = nullptr;
+  }
+  void* ws = nullptr;
+  if (cudaMalloc(&ws, sz) != cudaSuccess) {
+    cudaGetLastError();
+    p->cap_T = 0;
+    return MOE_ERR_ALLOC;
+  }
+  if (cudaMemset(ws, 0, sz) != cudaSuccess) return MOE_ERR_CUDA;
+  char* b = static_cast<char*>(ws);
+  p->ws = ws;
+  p->ctl = reinterpret_cast<Ctl*>(b + o_ctl);
+  p->idx = reinterpret_cast<int32_t*>(b + o_idx);
+  p->w = reinterpret_cast<float*>(b + o_w);
+  p->gap = reinterpret_cast<float*>(b + o_gap);
+  p->perm = reinterpret_cast<int32_t*>(b + o_perm);
+  p->slot_of = reinterpret_cast<int32_t*>(b + o_slot);
+  p->offsets = reinterpret_cast<int32_t*>(b + o_off);
+  p->chunk_e = reinterpret_cast<int32_t*>(b + o_ce);
+  p->chunk_c = reinterpret_cast<int32_t*>(b + o_cc);
+  p->ready = reinterpret_cast<int32_t*>(b + o_rd);
+  p->x_perm = reinterpret_cast<__nv_bfloat16*>(b + o_xp);
+  p->h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
+  p->y = reinterpret_cast<float*>(b + o_y);
+  p->x_dev = reinterpret_cast<__nv_bfloat16*>(b + o_xd);
+  p->res_dev = reinterpret_cast<__nv_bfloat16*>(b + o_rs);
+  p->out_dev = reinterpret_cast<__nv_bfloat16*>(b + o_od);
+  p->cap_T = cap;
+  return MOE_OK;
+}
+
+cudaEvent_t take_event(moe_plan_t p) {
+  if (!p->ev_pool.empty()) {
+    cudaEvent_t e = p->ev_pool.back();
+    p->ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Records an event pair around one launch when profiling is on.
+struct ProfScope {
+  moe_plan_t p;
+  int kernel;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr, b = nullptr;
+  ProfScope(moe_plan_t p_, int k_, cudaStream_t s_) : p(p_), kernel(k_), s(s_) {
+    if (p->profile && p->prof.size() < 65536) {
+      a = take_event(p);
+      b = take_event(p);
+      if (a && b) cudaEventRecord(a, s);
+    }
+  }
+  ~ProfScope() {
+    if (a && b) {
+      cudaEventRecord(b, s);
+      p->prof.push_back({kernel, a, b});
+    }
+  }
+};
+
+moe_status_t validate_route(moe_plan_t p, int T, const void* x, const float* rw,
+                            const float* gamma, const float* bias) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !rw || !gamma) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(rw) || !aligned16(gamma)) return MOE_ERR_INVALID_ARG;
+  if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return MOE_ERR_INVALID_ARG;
+  return check_device(p);
+}
+
+moe_status_t launch_router(moe_plan_t p, int T, const void* x, const float* rw,
+                           const float* gamma, const float* bias, int32_t* idx, float* w,
+                           float* gap, cudaStream_t s) {
+  moe::RouterArgs ra;
+  ra.T = T;
+  ra.E = p->E;
+  ra.k = p->k;
+  ra.d = p->d;
+  ra.eps = p->eps;
+  ra.x = static_cast<const __nv_bfloat16*>(x);
+  ra.router_w = rw;
+  ra.gamma = gamma;
+  ra.bias = bias;
+  ra.idx = idx;
+  ra.w = w;
+  ra.gap = gap;
+  ra.ctl = p->ctl;
+  ProfScope ps(p, MOE_K_ROUTER, s);
+  return moe_launch_router(ra, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_str(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: bad pointer, size, alignment or aliasing";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape or dtype outside the kernels' limits";
+    case MOE_ERR_ALLOC: return "MOE_ERR_ALLOC: workspace allocation failed";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or launch failed";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a device-side bounded wait ran out";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: a kernel saw an out-of-range index";
+  }
+  return "unknown moe_status_t";
+}
+
+moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, moe_plan_t* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (E < 1 || E > moe::kMaxE || k < 1 || k > E || k > moe::kMaxK) return MOE_ERR_UNSUPPORTED;
+  if (d < 128 || d > 4096 || d % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (f < 64 || f > 4096 || f % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (wdtype != MOE_W_BF16 && wdtype != MOE_W_INT4_G128) return MOE_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  moe_plan_s* p = new moe_plan_s();
+  p->E = E;
+  p->k = k;
+  p->d = d;
+  p->f = f;
+  p->wdtype = wdtype;
+  p->device = dev;
+  p->num_sms = sms;
+  p->eps = 1e-6f;
+  p->timeout_ms = 1000;
+  p->profile = 0;
+  p->test_stall = 0;
+  p->cap_T = 0;
+  p->last_T = 0;
+  p->ws = nullptr;
+  *out = p;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_set_option(moe_plan_t p, int key, double value) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  switch (key) {
+    case MOE_OPT_EPS:
+      if (!(value >= 0.0)) return MOE_ERR_INVALID_ARG;
+      p->eps = (float)value;
+      return MOE_OK;
+    case MOE_OPT_TIMEOUT_MS:
+      if (!(value >= 1.0 && value <= 600000.0)) return MOE_ERR_INVALID_ARG;
+      p->timeout_ms = (int)value;
+      return MOE_OK;
+    case MOE_OPT_PROFILE:
+      p->profile = value != 0.0;
+      return MOE_OK;
+    case MOE_OPT_TEST_STALL:
+      p->test_stall = value != 0.0;
+      return MOE_OK;
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+moe_status_t moe_plan_reserve(moe_plan_t p, int max_T) {
+  if (!p || max_T < 0) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device(p);
+  if (st != MOE_OK) return st;
+  return ensure_workspace(p, max_T > 0 ? max_T : 1);
+}
+
+moe_status_t moe_route(moe_plan_t p, int T, const void* x, const float* router_w,
+                       const float* router_gamma, const float* router_bias, int32_t* idx_out,
+                       float* w_out, float* gap_out, void* stream) {
+  moe_status_t st = validate_route(p, T, x, router_w, router_gamma, router_bias);
+  if (st != MOE_OK || T == 0) return st;
+  if (!idx_out || !w_out) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx_out) & 3u) || (reinterpret_cast<uintptr_t>(w_out) & 3u) ||
+      (gap_out && (reinterpret_cast<uintptr_t>(gap_out) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  st = ensure_workspace(p, 1);
+  if (st != MOE_OK) return st;
+  return launch_router(p, T, x, router_w, router_gamma, router_bias, idx_out, w_out, gap_out,
+                       static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router_w,
+                         const float* router_gamma, const float* router_bias,
+                         const void* w_gate_up, const void* w_down, const void* scales_gate_up,
+                         const void* scales_down, const void* residual, void* out, void* stream) {
+  moe_status_t st = validate_route(p, T, x, router_w, router_gamma, router_bias);
+  if (st != MOE_OK || T == 0) return st;
+  if (!w_gate_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
+  if (p->wdtype == MOE_W_BF16) {
+    if (scales_gate_up || scales_down) return MOE_ERR_INVALID_ARG;
+  } else {
+    if (!scales_gate_up || !scales_down) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(scales_gate_up) || !aligned16(scales_down)) return MOE_ERR_INVALID_ARG;
+    return MOE_ERR_UNSUPPORTED;  // int4 expert kernels not built yet
+  }
+  const size_t act = (size_t)T * p->d * 2;
+  if (overlap(out, act, x, act)) return MOE_ERR_INVALID_ARG;
+  if (residual && residual != out && overlap(out, act, residual, act)) return MOE_ERR_INVALID_ARG;
+  st = ensure_workspace(p, T);
+  if (st != MOE_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int A = T * p->k;
+  CUtensorMap tm_wgu, tm_wd, tm_xp, tm_h;
+  if (!make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) ||
+      !make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM) ||
+      !make_map_bf16(&tm_xp, p->x_perm, (uint64_t)A, p->d, moe::kBRows) ||
+      !make_map_bf16(&tm_h, p->h, (uint64_t)A, p->f, moe::kBRows))
+    return MOE_ERR_CUDA;
+
+  st = launch_router(p, T, x, router_w, router_gamma, router_bias, p->idx, p->w, p->gap, s);
+  if (st != MOE_OK) return st;
+
+  moe::PlanArgs pa;
+  pa.T = T;
+  pa.E = p->E;
+  pa.k = p->k;
+  pa.d = p->d;
+  pa.f = p->f;
+  pa.idx = p->idx;
+  pa.offsets = p->offsets;
+  pa.perm = p->perm;
+  pa.slot_of = p->slot_of;
+  pa.chunk_e = p->chunk_e;
+  pa.chunk_c = p->chunk_c;
+  pa.ready = p->ready;
+  pa.ctl = p->ctl;
+  {
+    ProfScope ps(p, MOE_K_PLAN, s);
+    if (moe_launch_plan(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  moe::GatherArgs ga;
+  ga.rows = A;
+  ga.d = p->d;
+  ga.perm = p->perm;
+  ga.x = static_cast<const __nv_bfloat16*>(x);
+  ga.x_perm = p->x_perm;
+  {
+    ProfScope ps(p, MOE_K_GATHER, s);
+    if (moe_launch_gather(ga, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  moe::ExpertArgs ea;
+  ea.T = T;
+  ea.E = p->E;
+  ea.k = p->k;
+  ea.d = p->d;
+  ea.f = p->f;
+  ea.offsets = p->offsets;
+  ea.chunk_e = p->chunk_e;
+  ea.chunk_c = p->chunk_c;
+  ea.ready = p->ready;
+  ea.h = p->h;
+  ea.y = p->y;
+  ea.ctl = p->ctl;
+  ea.timeout_ns = (uint64_t)p->timeout_ms * 1000000ull;
+  ea.test_stall = p->test_stall;
+  {
+    ProfScope ps(p, MOE_K_EXPERT, s);
+    if (moe_launch_expert(ea, tm_wgu, tm_wd, tm_xp, tm_h, p->num_sms, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+
+  moe::CombineArgs ca;
+  ca.T = T;
+  ca.k = p->k;
+  ca.d = p->d;
+  ca.slot_of = p->slot_of;
+  ca.w = p->w;
+  ca.y = p->y;
+  ca.residual = static_cast<const __nv_bfloat16*>(residual);
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  {
+    ProfScope ps(p, MOE_K_COMBINE, s);
+    if (moe_launch_combine(ca, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  p->last_T = T;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward_host(moe_plan_t p, int T, const void* x_host, const float* router_w,
+                              const float* router_gamma, const float* router_bias,
+                              const void* w_gate_up, const void* w_down,
+                              const void* scales_gate_up, const void* scales_down,
+                              const void* residual_host, void* out_host, void* stream) {
+  if (!p || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device(p);
+  if (st != MOE_OK) return st;
+  st = ensure_workspace(p, T);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t act = (size_t)T * p->d * 2;
+  if (cudaMemcpyAsync(p->x_dev, x_host, act, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (residual_host &&
+      cudaMemcpyAsync(p->res_dev, residual_host, act, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = moe_forward(p, T, p->x_dev, router_w, router_gamma, router_bias, w_gate_up, w_down,
+                   scales_gate_up, scales_down, residual_host ? p->res_dev : nullptr, p->out_dev,
+                   stream);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(out_host, p->out_dev, act, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_routing(moe_plan_t p, int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                              void* stream) {
+  if (!p || !p->ws) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t A = (size_t)p->last_T * p->k;
+  if (offsets && cudaMemcpyAsync(offsets, p->offsets, (p->E + 1) * 4, cudaMemcpyDeviceToDevice,
+                                 s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (perm && A && cudaMemcpyAsync(perm, p->perm, A * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (slot_of && A &&
+      cudaMemcpyAsync(slot_of, p->slot_of, A * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_sync_status(moe_plan_t p, void* stream) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!p->ws) return MOE_OK;
+  Ctl c;
+  if (cudaMemcpy(&c, p->ctl, sizeof(Ctl), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (c.status != 0) {
+    const int zero[2] = {0, 0};
+    if (cudaMemcpy(p->ctl, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  return static_cast<moe_status_t>(c.status);
+}
+
+moe_status_t moe_plan_profile(moe_plan_t p, int kernel, double* total_ms, int* launches) {
+  if (!p || !total_ms || !launches || kernel < 0 || kernel >= MOE_K_COUNT)
+    return MOE_ERR_INVALID_ARG;
+  double tot = 0.0;
+  int n = 0;
+  std::vector<ProfRec> keep;
+  for (const ProfRec& r : p->prof) {
+    if (r.kernel != kernel) {
+      keep.push_back(r);
+      continue;
+    }
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) return MOE_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) return MOE_ERR_CUDA;
+    tot += ms;
+    ++n;
+    p->ev_pool.push_back(r.start);
+    p->ev_pool.push_back(r.stop);
+  }
+  p->prof.swap(keep);
+  *total_ms = tot;
+  *launches = n;
+  return MOE_OK;
+}
+
+void moe_plan_destroy(moe_plan_t p) {
+  if (!p) return;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  if (prev != p->device) cudaSetDevice(p->device);
+  if (p->ws) {
+    cudaDeviceSynchronize();
+    cudaFree(p->ws);
+  }
+  for (const ProfRec& r : p->prof) {
+    cudaEventDestroy(r.start);
+    cudaEventDestroy(r.stop);
+  }
+  for (cudaEvent_t e : p->ev_pool) cudaEventDestroy(e);
+  if (prev >= 0 && prev != p->device) cudaSetDevice(prev);
+  delete p;
+}
+
+}  // extern "C"

@@ -1,0 +1,165 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) top-k mixture-of-experts FFN layer.
+ *
+ * The layer is the MoE FFN of DiffusionGemma 26B-A4B applied to a whole
+ * denoising canvas at once:
+ *   - 128 experts, 8 active per token (Quant-Tuner pull request "Add
+ *     DiffusionGemma (Gemma-4 MoE block-diffusion) support", Summary; Hugging
+ *     Face card "kingjones777/DiffusionGemma-26B-A4B-it-ROCmFP4-GGUF", header);
+ *   - the router reads the raw residual through its own (1+gamma) RMSNorm,
+ *     and a fused 3-D gate_up projection feeds the experts (Quant-Tuner pull
+ *     request, "Answers to the motivating questions");
+ *   - per expert gate/up 2816->704, down 704->2816, act GELUTanh; optional
+ *     symmetric int4 weights in groups of 128 (auto-round pull request "Add
+ *     quantization support for DiffusionGemma", transformers backend test
+ *     log);
+ *   - the canvas of 256 tokens is denoised in parallel, so each step is a set
+ *     of large batched expert matmuls (the ROCmFP4-GGUF card, section "The
+ *     4-bit is NOT the fastest here").
+ *
+ * For each token t (x_t bf16 [d]):
+ *   u   = x_t / sqrt(mean(x_t^2) + eps) * (1 + gamma)
+ *   z_e = router_w[e] . u (+ router_bias[e])            fp32
+ *   S   = the k largest z_e, ties to the lower index; j order = (z desc, e asc)
+ *   w_j = softmax(z)[S_j] / sum_j' softmax(z)[S_j']
+ *   h   = gelu_tanh(Wgu[S_j][0:f] x_t) * (Wgu[S_j][f:2f] x_t)   (bf16 h)
+ *   y_j = Wd[S_j] h                                              (fp32 y)
+ *   out_t = residual_t + sum_j w_j y_j  (j order, fp32, one rounding to bf16)
+ *
+ * Conventions for every entry point:
+ *   - All tensor arguments are DEVICE pointers on the plan's device, owned by
+ *     the caller, contiguous row-major, 16-byte aligned (moe_forward_host is
+ *     the one exception: its x and out are HOST pointers).
+ *   - bf16 / fp16 data are passed as raw 16-bit words (void*).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on that stream except where stated.
+ *     A plan is used by one stream at a time.
+ *   - On any invalid argument nothing is launched and an error is returned.
+ *     Launch failures return MOE_ERR_CUDA.  Faults the kernels detect
+ *     themselves (a bounded wait that ran out, an index out of range) are
+ *     recorded in a device status word read by moe_plan_sync_status.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_plan_s* moe_plan_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or aliasing      */
+  MOE_ERR_UNSUPPORTED = 2,  /* shape or dtype outside what the kernels cover */
+  MOE_ERR_ALLOC = 3,        /* workspace allocation failed                   */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed          */
+  MOE_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out            */
+  MOE_ERR_DEVICE_CHECK = 6  /* a kernel saw an out-of-range routing index    */
+} moe_status_t;
+
+typedef enum {
+  MOE_W_BF16 = 0,      /* w_gate_up bf16 [E,2f,d]; w_down bf16 [E,d,f]           */
+  MOE_W_INT4_G128 = 1  /* w_gate_up u8 [E,2f,d/2]; w_down u8 [E,d,f/2]; element i
+                          of a row in byte i/2, low nibble for even i, 4-bit two's
+                          complement; value = code * scale[row][i/128] (fp16)  */
+} moe_wdtype_t;
+
+/* Options for moe_plan_set_option. */
+enum {
+  MOE_OPT_EPS = 0,        /* RMSNorm epsilon (default 1e-6)                        */
+  MOE_OPT_TIMEOUT_MS = 1, /* bound of every device-side wait, ms (default 1000)    */
+  MOE_OPT_PROFILE = 2,    /* 1: moe_forward records CUDA events around each kernel */
+  MOE_OPT_TEST_STALL = 3  /* test hook: 1 makes the expert kernel wait on a flag
+                             nothing sets, so the bounded wait runs out and the
+                             call reports MOE_ERR_TIMEOUT (no trap, no hang)     */
+};
+
+/* Kernels of one moe_forward, for moe_plan_profile. */
+enum {
+  MOE_K_ROUTER = 0,   /* norm + logits + softmax + top-k          */
+  MOE_K_PLAN = 1,     /* histogram + scan + stable permutation    */
+  MOE_K_GATHER = 2,   /* x rows in expert order                   */
+  MOE_K_EXPERT = 3,   /* grouped gate_up(+GELU*up) and down GEMMs */
+  MOE_K_COMBINE = 4,  /* weighted k-order sum (+ residual)        */
+  MOE_K_COUNT = 5
+};
+
+/* Create a plan for E experts, top-k, hidden d, per-expert intermediate f.
+ * Limits: 1 <= E <= 256; 1 <= k <= min(E, 32); d % 128 == 0, 128 <= d <= 4096;
+ * f % 64 == 0, 64 <= f <= 4096.  Binds the plan to the current CUDA device.
+ * Returns MOE_ERR_UNSUPPORTED outside the limits, MOE_ERR_INVALID_ARG on a
+ * NULL `out`.  Allocates nothing on the device until the first call. */
+moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, moe_plan_t* out);
+
+/* Set an option (see MOE_OPT_*).  Synchronous, host only. */
+moe_status_t moe_plan_set_option(moe_plan_t plan, int key, double value);
+
+/* Grow the plan-owned workspace to hold max_T tokens (synchronous device
+ * allocation).  moe_forward grows it on demand; call this first when the
+ * calls are to be captured in a CUDA graph. */
+moe_status_t moe_plan_reserve(moe_plan_t plan, int max_T);
+
+/* The whole layer for T tokens (T = 0 is a no-op).
+ *   x              bf16 [T,d]
+ *   router_w       fp32 [E,d]
+ *   router_gamma   fp32 [d]    (applied as 1 + gamma)
+ *   router_bias    fp32 [E] or NULL
+ *   w_gate_up      see moe_wdtype_t (rows [0,f) gate, [f,2f) up)
+ *   w_down         see moe_wdtype_t
+ *   scales_gate_up fp16 [E,2f,ceil(d/128)]  (int4 plans; must be NULL for bf16)
+ *   scales_down    fp16 [E,d,ceil(f/128)]   (int4 plans; must be NULL for bf16)
+ *   residual       bf16 [T,d] or NULL; may alias `out`
+ *   out            bf16 [T,d]; must not overlap x
+ * Asynchronous on `stream`; the plan's workspace holds the routing tables
+ * until the next call. */
+moe_status_t moe_forward(moe_plan_t plan, int T, const void* x, const float* router_w,
+                         const float* router_gamma, const float* router_bias,
+                         const void* w_gate_up, const void* w_down, const void* scales_gate_up,
+                         const void* scales_down, const void* residual, void* out, void* stream);
+
+/* moe_forward with x, residual and out in HOST memory (pinned or pageable):
+ * copies x (and residual) to the plan's device buffers, runs the layer, copies
+ * out back and synchronises `stream` before returning.  Weights and router
+ * tensors are device pointers as in moe_forward. */
+moe_status_t moe_forward_host(moe_plan_t plan, int T, const void* x_host, const float* router_w,
+                              const float* router_gamma, const float* router_bias,
+                              const void* w_gate_up, const void* w_down,
+                              const void* scales_gate_up, const void* scales_down,
+                              const void* residual_host, void* out_host, void* stream);
+
+/* Routing only: idx int32 [T,k] (j order), w fp32 [T,k], gap fp32 [T] or NULL
+ * (gap = z_(k) - z_(k+1), +inf when k == E). */
+moe_status_t moe_route(moe_plan_t plan, int T, const void* x, const float* router_w,
+                       const float* router_gamma, const float* router_bias, int32_t* idx_out,
+                       float* w_out, float* gap_out, void* stream);
+
+/* Device-to-device copies of the last moe_forward's routing tables (NULL to
+ * skip one): offsets int32 [E+1] (expert segment starts in slot order),
+ * perm int32 [T*k] (token of each slot), slot_of int32 [T*k] (slot of
+ * assignment t*k+j).  Asynchronous on `stream`. */
+moe_status_t moe_plan_routing(moe_plan_t plan, int32_t* offsets, int32_t* perm, int32_t* slot_of,
+                              void* stream);
+
+/* Synchronise `stream`, return the device status word (MOE_OK, MOE_ERR_TIMEOUT
+ * or MOE_ERR_DEVICE_CHECK) and clear it. */
+moe_status_t moe_plan_sync_status(moe_plan_t plan, void* stream);
+
+/* With MOE_OPT_PROFILE on: total device time (ms) and number of launches of
+ * kernel `kernel` (MOE_K_*) recorded since the last read; synchronises the
+ * recorded events and clears the record. */
+moe_status_t moe_plan_profile(moe_plan_t plan, int kernel, double* total_ms, int* launches);
+
+/* Release the plan and its workspace (synchronous). NULL is ignored. */
+void moe_plan_destroy(moe_plan_t plan);
+
+/* Static description of a status code. */
+const char* moe_status_str(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */
