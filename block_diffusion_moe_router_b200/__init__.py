@@ -16,6 +16,7 @@ from ._abi import (  # noqa: F401
     MOE_OPT_TIMEOUT_MS, MOE_OPT_PROFILE, MOE_OPT_TEST_STALL, MOE_K_ROUTER, MOE_K_PLAN,
     MOE_K_GATHER, MOE_K_EXPERT, MOE_K_COMBINE, KERNEL_NAMES, MoeError,
     moe_plan_create, moe_plan_set_option, moe_plan_reserve, moe_forward, moe_forward_host,
+    moe_forward_noalloc,
     moe_route, moe_plan_routing, moe_plan_sync_status, moe_plan_profile, moe_plan_destroy,
     moe_status_str,
 )

@@ -37,7 +37,7 @@ KERNEL_NAMES = ["router", "plan", "gather", "expert", "combine"]
 EXPORTS = [
     "moe_plan_create", "moe_plan_set_option", "moe_plan_reserve", "moe_forward",
     "moe_forward_host", "moe_route", "moe_plan_routing", "moe_plan_sync_status",
-    "moe_plan_profile", "moe_plan_destroy", "moe_status_str",
+    "moe_plan_profile", "moe_plan_destroy", "moe_status_str", "moe_forward_noalloc",
 ]
 
 _lock = threading.Lock()
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
             L.moe_plan_profile.restype = I
             L.moe_plan_destroy.argtypes = [P]
             L.moe_plan_destroy.restype = None
+            L.moe_forward_noalloc.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P, P, P]
+            L.moe_forward_noalloc.restype = I
             L.moe_status_str.argtypes = [I]
             L.moe_status_str.restype = ctypes.c_char_p
             _lib = L
@@ -155,6 +157,18 @@ def moe_forward_host(plan, T, x_host, router_w, router_gamma, router_bias, w_gat
                                 _ptr(scales_gate_up), _ptr(scales_down), _ptr(residual_host),
                                 _ptr(out_host), _stream(stream))
     return _check(st, "moe_forward_host", check)
+
+
+def moe_forward_noalloc(plan, T, x, router_w, router_gamma, router_bias, w_gate_up, w_down,
+                        scales_gate_up, scales_down, residual, out, status_out=None, stream=None,
+                        check: bool = True):
+    """moe_forward without any device allocation: intermediates live in the
+    library's fixed 40 MiB device array (see include/moe.h)."""
+    st = lib().moe_forward_noalloc(plan, T, _ptr(x), _ptr(router_w), _ptr(router_gamma),
+                                   _ptr(router_bias), _ptr(w_gate_up), _ptr(w_down),
+                                   _ptr(scales_gate_up), _ptr(scales_down), _ptr(residual),
+                                   _ptr(out), _ptr(status_out), _stream(stream))
+    return _check(st, "moe_forward_noalloc", check)
 
 
 def moe_route(plan, T, x, router_w, router_gamma, router_bias, idx_out, w_out, gap_out,

@@ -512,3 +512,176 @@ void moe_plan_destroy(moe_plan_t p) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// moe_forward_noalloc: the moe_forward launch sequence with every
+// intermediate carved from one file-scope device array, for callers that
+// cannot allocate device memory (a host that pre-assigns all GPU memory, or a
+// loop that must never enter the allocator).  Nothing here calls cudaMalloc,
+// cudaFree or any allocating routine.
+
+static __device__ __align__(256) unsigned char moe_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[128] = {};
+
+// Device address of the array on device `dev` (must be current).  Looked up
+// once per device; in host code the array's name is only a stand-in, so it
+// is never passed to a kernel directly.
+void* noalloc_scratch(int dev) {
+  if (dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, moe_noalloc_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
+                                            const float* router_w, const float* router_gamma,
+                                            const float* router_bias, const void* w_gate_up,
+                                            const void* w_down, const void* scales_gate_up,
+                                            const void* scales_down, const void* residual,
+                                            void* out, int32_t* status_out, void* stream) {
+  moe_status_t st = validate_route(p, T, x, router_w, router_gamma, router_bias);
+  if (st != MOE_OK || T == 0) return st;
+  if (!w_gate_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
+  if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (p->wdtype == MOE_W_BF16) {
+    if (scales_gate_up || scales_down) return MOE_ERR_INVALID_ARG;
+  } else {
+    return MOE_ERR_UNSUPPORTED;
+  }
+  const size_t act = (size_t)T * p->d * 2;
+  if (overlap(out, act, x, act)) return MOE_ERR_INVALID_ARG;
+  if (residual && residual != out && overlap(out, act, residual, act)) return MOE_ERR_INVALID_ARG;
+
+  // Carve the intermediates for T tokens; refuse what does not fit.
+  const size_t A = (size_t)T * p->k;
+  const size_t MC = (size_t)max_chunks(p->E, T, p->k);
+  size_t sz = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = sz;
+    sz += align256(bytes);
+    return o;
+  };
+  const size_t o_ctl = take(sizeof(Ctl));
+  const size_t o_idx = take(A * 4), o_w = take(A * 4), o_gap = take((size_t)T * 4);
+  const size_t o_perm = take(A * 4), o_slot = take(A * 4), o_off = take((size_t)(p->E + 1) * 4);
+  const size_t o_ce = take(MC * 4), o_cc = take(MC * 4), o_rd = take(MC * 4);
+  const size_t o_xp = take(A * p->d * 2), o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
+  if (sz > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
+
+  char* b = static_cast<char*>(noalloc_scratch(p->device));
+  if (!b) return MOE_ERR_CUDA;
+  Ctl* ctl = reinterpret_cast<Ctl*>(b + o_ctl);
+  int32_t* idx = reinterpret_cast<int32_t*>(b + o_idx);
+  float* w = reinterpret_cast<float*>(b + o_w);
+  float* gap = reinterpret_cast<float*>(b + o_gap);
+  int32_t* perm = reinterpret_cast<int32_t*>(b + o_perm);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(b + o_slot);
+  int32_t* offsets = reinterpret_cast<int32_t*>(b + o_off);
+  int32_t* chunk_e = reinterpret_cast<int32_t*>(b + o_ce);
+  int32_t* chunk_c = reinterpret_cast<int32_t*>(b + o_cc);
+  int32_t* ready = reinterpret_cast<int32_t*>(b + o_rd);
+  __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(b + o_xp);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
+  float* y = reinterpret_cast<float*>(b + o_y);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUtensorMap tm_wgu, tm_wd, tm_xp, tm_h;
+  if (!make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) ||
+      !make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM) ||
+      !make_map_bf16(&tm_xp, x_perm, (uint64_t)A, p->d, moe::kBRows) ||
+      !make_map_bf16(&tm_h, h, (uint64_t)A, p->f, moe::kBRows))
+    return MOE_ERR_CUDA;
+
+  // The status word must start at zero; the plan kernel resets the scheduler
+  // counters and chunk tables itself on every call.
+  if (cudaMemsetAsync(ctl, 0, sizeof(Ctl), s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  moe::RouterArgs ra;
+  ra.T = T;
+  ra.E = p->E;
+  ra.k = p->k;
+  ra.d = p->d;
+  ra.eps = p->eps;
+  ra.x = static_cast<const __nv_bfloat16*>(x);
+  ra.router_w = router_w;
+  ra.gamma = router_gamma;
+  ra.bias = router_bias;
+  ra.idx = idx;
+  ra.w = w;
+  ra.gap = gap;
+  ra.ctl = ctl;
+  if (moe_launch_router(ra, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  moe::PlanArgs pa;
+  pa.T = T;
+  pa.E = p->E;
+  pa.k = p->k;
+  pa.d = p->d;
+  pa.f = p->f;
+  pa.idx = idx;
+  pa.offsets = offsets;
+  pa.perm = perm;
+  pa.slot_of = slot_of;
+  pa.chunk_e = chunk_e;
+  pa.chunk_c = chunk_c;
+  pa.ready = ready;
+  pa.ctl = ctl;
+  if (moe_launch_plan(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  moe::GatherArgs ga;
+  ga.rows = (int)A;
+  ga.d = p->d;
+  ga.perm = perm;
+  ga.x = static_cast<const __nv_bfloat16*>(x);
+  ga.x_perm = x_perm;
+  if (moe_launch_gather(ga, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  moe::ExpertArgs ea;
+  ea.T = T;
+  ea.E = p->E;
+  ea.k = p->k;
+  ea.d = p->d;
+  ea.f = p->f;
+  ea.offsets = offsets;
+  ea.chunk_e = chunk_e;
+  ea.chunk_c = chunk_c;
+  ea.ready = ready;
+  ea.h = h;
+  ea.y = y;
+  ea.ctl = ctl;
+  ea.timeout_ns = (uint64_t)p->timeout_ms * 1000000ull;
+  ea.test_stall = p->test_stall;
+  if (moe_launch_expert(ea, tm_wgu, tm_wd, tm_xp, tm_h, p->num_sms, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+
+  moe::CombineArgs ca;
+  ca.T = T;
+  ca.k = p->k;
+  ca.d = p->d;
+  ca.slot_of = slot_of;
+  ca.w = w;
+  ca.y = y;
+  ca.residual = static_cast<const __nv_bfloat16*>(residual);
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  if (moe_launch_combine(ca, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  if (status_out && cudaMemcpyAsync(status_out, &ctl->status, sizeof(int32_t),
+                                    cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}

@@ -130,6 +130,44 @@ moe_status_t moe_forward_host(moe_plan_t plan, int T, const void* x_host, const 
                               const void* scales_gate_up, const void* scales_down,
                               const void* residual_host, void* out_host, void* stream);
 
+/* Size of the fixed device array used by moe_forward_noalloc (40 MiB). */
+#define MOE_NOALLOC_SCRATCH_BYTES (40u * 1024u * 1024u)
+
+/* moe_forward for callers that cannot allocate device memory: a host that
+ * owns and pre-assigns every byte of the GPU (an inference server or plugin
+ * host with its own allocator), or a latency-critical loop that must never
+ * enter the CUDA allocator.  The pages describe no such entry point; it is
+ * this library's addition.
+ *
+ * Same arguments, layouts, results and errors as moe_forward, plus
+ * status_out: a DEVICE int32 (or NULL) that receives this call's device
+ * status word (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK) in stream
+ * order.  The caller still passes every input and output.  All intermediates
+ * (routing tables, gathered rows, h, y, counters) live in one file-scope
+ * __device__ array of MOE_NOALLOC_SCRATCH_BYTES; the call never calls
+ * cudaMalloc, cudaFree or any allocating routine.
+ *   - Limit: the intermediates of T tokens must fit the array (about
+ *     T*k*(6d + 2f) + T*(8k + 4) bytes plus small tables; one 256-token
+ *     canvas of the 2816/704/128/top-8 layer needs 37.5 MB).  A larger call
+ *     returns MOE_ERR_UNSUPPORTED and launches nothing.
+ *   - Set-up: the first call on each device (with that device current) looks
+ *     up the array's device address once; make that first call before any
+ *     stream capture.
+ *   - The array is part of the library's device image: every GPU that loads
+ *     it holds the 40 MiB until the process exits.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents (each call clears the words that must start at zero).
+ *     Calls that overlap on the GPU (other streams, other threads, other
+ *     plans) race on it and must be serialised by the caller.
+ *   - bf16 plans only for now (int4 returns MOE_ERR_UNSUPPORTED, as in
+ *     moe_forward); MOE_OPT_PROFILE is ignored. */
+moe_status_t moe_forward_noalloc(moe_plan_t plan, int T, const void* x, const float* router_w,
+                                 const float* router_gamma, const float* router_bias,
+                                 const void* w_gate_up, const void* w_down,
+                                 const void* scales_gate_up, const void* scales_down,
+                                 const void* residual, void* out, int32_t* status_out,
+                                 void* stream);
+
 /* Routing only: idx int32 [T,k] (j order), w fp32 [T,k], gap fp32 [T] or NULL
  * (gap = z_(k) - z_(k+1), +inf when k == E). */
 moe_status_t moe_route(moe_plan_t plan, int T, const void* x, const float* router_w,
