@@ -47,6 +47,10 @@ def parse():
     p.add_argument("--workload", default="canvas")
     p.add_argument("--sets", type=int, default=0, help="input sets rotated (0: enough to exceed L2)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
+    p.add_argument("--router-ffma", action="store_true", help="FFMA router instead of tensor cores")
+    p.add_argument("--prefetch-mb", type=int, default=None,
+                   help="MiB of gate_up weights pulled into L2 during routing")
     return p.parse_args()
 
 
@@ -172,7 +176,8 @@ def oracle_sample_rate(lay_cpu, k, n_tokens, eps=1e-6):
     oracle.moe_forward(x, lay_cpu["router_w"], lay_cpu["router_gamma"],
                        lay_cpu.get("router_bias"), lay_cpu["w_gate_up"], lay_cpu["w_down"], k,
                        scales_gate_up=lay_cpu.get("scales_gate_up"),
-                       scales_down=lay_cpu.get("scales_down"), eps=eps)
+                       scales_down=lay_cpu.get("scales_down"), eps=eps,
+                       expert_gamma=lay_cpu.get("expert_gamma"))
     return n_tokens / (time.perf_counter() - t0)
 
 
@@ -223,7 +228,8 @@ def run_reference(args):
         oracle.moe_forward(sub["x"], sub["router_w"], sub["router_gamma"],
                            sub.get("router_bias"), sub["w_gate_up"], sub["w_down"], w.k,
                            scales_gate_up=sub.get("scales_gate_up"),
-                           scales_down=sub.get("scales_down"))
+                           scales_down=sub.get("scales_down"),
+                           expert_gamma=sub.get("expert_gamma"))
 
     for _ in range(args.warmup):
         step()
@@ -261,40 +267,67 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     w = inputs.WORKLOADS[args.workload]
-    T = w.T
-    lay = inputs.make_layer(w, device="cuda", with_x=False)
+    T, L = w.T, w.layers
+    lays = [inputs.make_layer(w, layer=l, device="cuda", with_x=False) for l in range(L)]
+    lay = lays[0]
     # rotate the small per-call inputs so that, with the weights, the working
     # set exceeds L2 on every step
-    small = T * w.d * 2 * 2 + w.E * w.d * 4 + w.d * 4
+    small = T * w.d * 2 * 2 + (w.E * w.d * 4 + w.d * 4 if L == 1 else 0)
     nsets = args.sets or max(2, math.ceil(1.1 * L2_BYTES / small))
     xs = [inputs._randn((T, w.d), 1.0, 777000 + 1000 * rank + i, "cuda", torch.bfloat16)
           for i in range(nsets)]
-    rws = [lay["router_w"]] + [lay["router_w"][torch.randperm(w.E, device="cuda")].contiguous()
-                               for _ in range(nsets - 1)]
-    gms = [lay["router_gamma"]] + [lay["router_gamma"].roll(i).contiguous()
-                                   for i in range(1, nsets)]
+    if L == 1:
+        rws = [lay["router_w"]] + [lay["router_w"][torch.randperm(w.E, device="cuda")]
+                                   .contiguous() for _ in range(nsets - 1)]
+        gms = [lay["router_gamma"]] + [lay["router_gamma"].roll(i).contiguous()
+                                       for i in range(1, nsets)]
     outs = [torch.empty((T, w.d), dtype=torch.bfloat16, device="cuda") for _ in range(nsets)]
+    bufs = [torch.empty((T, w.d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     plan = moe.moe_plan_create(w.E, w.k, w.d, w.f, w.wdtype)
     moe.moe_plan_reserve(plan, T)
+    moe.moe_plan_set_option(plan, moe.MOE_OPT_PDL, 0 if args.no_pdl else 1)
+    moe.moe_plan_set_option(plan, moe.MOE_OPT_ROUTER_FFMA, 1 if args.router_ffma else 0)
+    if args.prefetch_mb is not None:
+        moe.moe_plan_set_option(plan, moe.MOE_OPT_L2_PREFETCH_MB, args.prefetch_mb)
     stream = torch.cuda.current_stream()
 
-    def step(i):
-        j = i % nsets
-        moe.moe_forward(plan, T, xs[j], rws[j], gms[j], lay["router_bias"], lay["w_gate_up"],
-                        lay["w_down"], lay["scales_gate_up"], lay["scales_down"], None, outs[j],
-                        stream)
+    def layer_call(l, x, out, residual, rw=None, gm=None):
+        ly = lays[l]
+        moe.moe_forward(plan, T, x, ly["router_w"] if rw is None else rw,
+                        ly["router_gamma"] if gm is None else gm, ly["router_bias"],
+                        ly["w_gate_up"], ly["w_down"], ly["scales_gate_up"], ly["scales_down"],
+                        residual, out, stream, expert_gamma=ly["expert_gamma"])
 
-    # touched experts per set (weights the layer must stream)
-    touched = []
-    for i in range(nsets):
-        step(i)
-        off = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+    def step(i, per_layer=None):
+        j = i % nsets
+        if L == 1:
+            layer_call(0, xs[j], outs[j], None, rws[j], gms[j])
+            if per_layer is not None:
+                per_layer(0)
+            return outs[j]
+        cur = xs[j]
+        for l in range(L):  # x_{l+1} = x_l + MoE_l(x_l)
+            nxt = bufs[l % 2]
+            layer_call(l, cur, nxt, cur)
+            if per_layer is not None:
+                per_layer(l)
+            cur = nxt
+        return cur
+
+    # experts that receive a token (their weights are the bytes the layer
+    # must stream), per layer, averaged over the input sets
+    touched = [0.0] * L
+    off = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+
+    def count(l):
         moe.moe_plan_routing(plan, off, None, None, stream)
-        touched.append(int(((off[1:] - off[:-1]) > 0).sum().item()))
+        touched[l] += float(((off[1:] - off[:-1]) > 0).sum().item()) / nsets
+
+    for i in range(nsets):
+        step(i, count)
     st = moe.moe_plan_sync_status(plan, stream)
     if st != moe.MOE_OK:
         raise RuntimeError(moe.moe_status_str(st))
-    mean_touched = sum(touched) / len(touched)
 
     def barrier():
         if world > 1:
@@ -323,7 +356,7 @@ def run_ours(args):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    for kk in range(moe.MOE_K_COMBINE + 1):  # discard warm-up records
+    for kk in range(len(moe.KERNEL_NAMES)):  # discard warm-up records
         moe.moe_plan_profile(plan, kk)
     with ClockSampler(local) as clk:
         ms = timed(args.steps, profile=True)
@@ -336,16 +369,22 @@ def run_ours(args):
     if st != moe.MOE_OK:
         raise RuntimeError(moe.moe_status_str(st))
 
-    # end to end through moe_forward_host: host x in, host out back, every step
+    # end to end: host x in, host result out, every step, through the C ABI
     x_host = [xs[i].cpu().pin_memory() for i in range(min(nsets, 4))]
     out_host = torch.empty((T, w.d), dtype=torch.bfloat16).pin_memory()
     K2 = args.steps
     barrier()
     t0 = time.perf_counter()
     for i in range(K2):
-        moe.moe_forward_host(plan, T, x_host[i % len(x_host)], rws[0], gms[0], lay["router_bias"],
-                             lay["w_gate_up"], lay["w_down"], lay["scales_gate_up"],
-                             lay["scales_down"], None, out_host, stream)
+        if L == 1:
+            moe.moe_forward_host(plan, T, x_host[i % len(x_host)], rws[0], gms[0],
+                                 lay["router_bias"], lay["w_gate_up"], lay["w_down"],
+                                 lay["scales_gate_up"], lay["scales_down"], None, out_host,
+                                 stream, expert_gamma=lay["expert_gamma"])
+        else:
+            xs[0].copy_(x_host[i % len(x_host)], non_blocking=True)
+            out_host.copy_(step(0), non_blocking=True)
+            stream.synchronize()
     e2e_s = time.perf_counter() - t0
     if world > 1:
         t = torch.tensor([e2e_s], device="cuda", dtype=torch.float64)
@@ -356,11 +395,25 @@ def run_ours(args):
         raise RuntimeError(moe.moe_status_str(st))
 
     hbm, bf16, bf16_sus, basis = peaks()
-    expert_bytes, layer_bytes, flops, wbytes = layer_costs(w, mean_touched, T)
+    expert_bytes, layer_bytes, flops = 0.0, 0.0, 0.0
+    for l in range(L):
+        eb, lb, fl, wbytes = layer_costs(w, touched[l], T)
+        expert_bytes += eb
+        layer_bytes += lb
+        flops += fl
+    expert_bytes /= L  # per expert-kernel launch
     ms_step = ms / args.steps
     k_ms = kern["expert"]
     achieved = expert_bytes / (k_ms * 1e-3) / 1e9 if k_ms else None
-    traffic = recorded_traffic()
+    traffic = recorded_traffic() if args.workload == "canvas" else None
+    desc = {
+        "canvas": "one MoE layer over a T=256 token canvas",
+        "canvas4": "one MoE layer over a T=256 token canvas, int4 w4g128 weights",
+        "encode": "one MoE layer over T=2048 tokens (1792 prompt + 256 canvas)",
+        "stack30": "one denoising step: 30 stacked MoE layers (distinct weights, Zipf(1.1) "
+                   "router bias, residual chained) over a T=256 canvas",
+        "tiny": "tiny MoE layer",
+    }[w.name]
     line = {
         "metric": METRIC,
         "value": world * T * args.steps / (ms * 1e-3),
@@ -375,14 +428,16 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": f"{w.name}: one MoE layer over a T={T} token canvas, d={w.d}, E={w.E}, "
-                        f"top-{w.k}, f={w.f}, bf16 weights",
-            "global_batch": world * T, "seq_len": T,
+            "workload": f"{w.name}: {desc}, d={w.d}, E={w.E}, top-{w.k}, f={w.f}, "
+                        f"{'int4 w4g128' if w.wdtype else 'bf16'} weights",
+            "global_batch": world * T, "seq_len": T, "layers_per_step": L,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "l2": f"weights {wbytes * w.E / 1e9:.2f} GB > L2; x/router/out rotated over "
+            "l2": f"weights {wbytes * w.E * L / 1e9:.2f} GB > L2; x/out rotated over "
                   f"{nsets} sets ({nsets * small / 2**20:.0f} MiB)",
             "timed_region": "per-kernel CUDA events recorded inside the timed steps",
             "ms_per_step_without_events": ms_plain / args.steps,
+            "pdl": not args.no_pdl,
+            "router": "ffma" if (args.router_ffma or w.E > 128) else "tensor cores",
         },
         "roofline": {
             "bound": "hbm", "kernel": "expert (grouped gate_up + down GEMMs)",
@@ -390,19 +445,20 @@ def run_ours(args):
             "frac": (achieved / hbm) if achieved else None, "traffic": traffic,
             "peak_basis": f"{basis} HBM copy bandwidth",
             "alg_bytes_per_launch": expert_bytes,
-            "alg_bytes_rule": f"{mean_touched:.2f} touched experts x {wbytes} B of expert "
-                              f"weights",
+            "alg_bytes_rule": f"{sum(touched) / L:.2f} touched experts per layer x {wbytes} B "
+                              f"of expert weights",
             "kernel_ms": k_ms,
         },
         "layer_roofline": {
-            "alg_bytes": layer_bytes, "flops": flops,
+            "alg_bytes_per_step": layer_bytes, "flops_per_step": flops,
             "t_hbm_ms": layer_bytes / (hbm * 1e9) * 1e3,
             "t_tensor_ms": flops / (bf16 * 1e12) * 1e3,
             "frac_of_roofline": (max(layer_bytes / (hbm * 1e9), flops / (bf16 * 1e12)) * 1e3)
                                 / ms_step,
+            "tensor_frac_of_burst_peak": flops / (ms_step * 1e-3) / (bf16 * 1e12),
         },
         "kernel_ms": kern,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": len(moe.KERNEL_NAMES) * L * args.steps,
         "e2e": {"value": world * T * K2 / e2e_s, "unit": "tokens/s",
                 "h2d_bytes_per_step": T * w.d * 2, "d2h_bytes_per_step": T * w.d * 2},
         "clocks": clk.summary(),
@@ -411,7 +467,11 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         lay_cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in lay.items()}
         lay_cpu["x"] = xs[0].cpu()
-        line["cpu_baseline"] = cpu_baseline(lay_cpu, w)
+        cb = cpu_baseline(lay_cpu, w)
+        if L > 1:
+            cb["value"] /= L
+            cb["sample"] += f"; per step = {L} layers"
+        line["cpu_baseline"] = cb
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

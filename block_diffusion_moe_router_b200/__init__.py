@@ -13,7 +13,8 @@ from . import _abi
 from ._abi import (  # noqa: F401
     MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_ALLOC, MOE_ERR_CUDA,
     MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_CHECK, MOE_W_BF16, MOE_W_INT4_G128, MOE_OPT_EPS,
-    MOE_OPT_TIMEOUT_MS, MOE_OPT_PROFILE, MOE_OPT_TEST_STALL, MOE_K_ROUTER, MOE_K_PLAN,
+    MOE_OPT_TIMEOUT_MS, MOE_OPT_PROFILE, MOE_OPT_TEST_STALL, MOE_OPT_PDL,
+    MOE_OPT_L2_PREFETCH_MB, MOE_OPT_ROUTER_FFMA, MOE_K_ROUTER, MOE_K_PLAN,
     MOE_K_GATHER, MOE_K_EXPERT, MOE_K_COMBINE, KERNEL_NAMES, MoeError,
     moe_plan_create, moe_plan_set_option, moe_plan_reserve, moe_forward, moe_forward_host,
     moe_forward_noalloc,
@@ -41,13 +42,15 @@ class MoeLayer:
             pass
 
     def forward(self, x, router_w, router_gamma, w_gate_up, w_down, router_bias=None,
-                scales_gate_up=None, scales_down=None, residual=None, out=None, stream=None):
+                scales_gate_up=None, scales_down=None, residual=None, out=None, stream=None,
+                expert_gamma=None):
         import torch
         T = x.shape[0]
         if out is None:
             out = torch.empty((T, self.d), dtype=torch.bfloat16, device=x.device)
         moe_forward(self.plan, T, x, router_w, router_gamma, router_bias, w_gate_up, w_down,
-                    scales_gate_up, scales_down, residual, out, stream)
+                    scales_gate_up, scales_down, residual, out, stream,
+                    expert_gamma=expert_gamma)
         return out
 
     def route(self, x, router_w, router_gamma, router_bias=None, stream=None):

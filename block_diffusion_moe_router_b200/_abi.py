@@ -29,6 +29,9 @@ MOE_OPT_EPS = 0
 MOE_OPT_TIMEOUT_MS = 1
 MOE_OPT_PROFILE = 2
 MOE_OPT_TEST_STALL = 3
+MOE_OPT_PDL = 4
+MOE_OPT_L2_PREFETCH_MB = 5
+MOE_OPT_ROUTER_FFMA = 6
 
 MOE_K_ROUTER, MOE_K_PLAN, MOE_K_GATHER, MOE_K_EXPERT, MOE_K_COMBINE = range(5)
 KERNEL_NAMES = ["router", "plan", "gather", "expert", "combine"]
@@ -66,9 +69,9 @@ def lib() -> ctypes.CDLL:
             L.moe_plan_set_option.restype = I
             L.moe_plan_reserve.argtypes = [P, I]
             L.moe_plan_reserve.restype = I
-            L.moe_forward.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P, P]
+            L.moe_forward.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P, P, P]
             L.moe_forward.restype = I
-            L.moe_forward_host.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P, P]
+            L.moe_forward_host.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P, P, P]
             L.moe_forward_host.restype = I
             L.moe_route.argtypes = [P, I, P, P, P, P, P, P, P, P]
             L.moe_route.restype = I
@@ -80,7 +83,7 @@ def lib() -> ctypes.CDLL:
             L.moe_plan_profile.restype = I
             L.moe_plan_destroy.argtypes = [P]
             L.moe_plan_destroy.restype = None
-            L.moe_forward_noalloc.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P, P, P]
+            L.moe_forward_noalloc.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P, P, P, P]
             L.moe_forward_noalloc.restype = I
             L.moe_status_str.argtypes = [I]
             L.moe_status_str.restype = ctypes.c_char_p
@@ -141,9 +144,10 @@ def moe_plan_reserve(plan: int, max_T: int, check: bool = True) -> int:
 
 
 def moe_forward(plan, T, x, router_w, router_gamma, router_bias, w_gate_up, w_down,
-                scales_gate_up, scales_down, residual, out, stream=None, check: bool = True):
+                scales_gate_up, scales_down, residual, out, stream=None, check: bool = True,
+                expert_gamma=None):
     st = lib().moe_forward(plan, T, _ptr(x), _ptr(router_w), _ptr(router_gamma),
-                           _ptr(router_bias), _ptr(w_gate_up), _ptr(w_down),
+                           _ptr(router_bias), _ptr(expert_gamma), _ptr(w_gate_up), _ptr(w_down),
                            _ptr(scales_gate_up), _ptr(scales_down), _ptr(residual), _ptr(out),
                            _stream(stream))
     return _check(st, "moe_forward", check)
@@ -151,9 +155,10 @@ def moe_forward(plan, T, x, router_w, router_gamma, router_bias, w_gate_up, w_do
 
 def moe_forward_host(plan, T, x_host, router_w, router_gamma, router_bias, w_gate_up, w_down,
                      scales_gate_up, scales_down, residual_host, out_host, stream=None,
-                     check: bool = True):
+                     check: bool = True, expert_gamma=None):
     st = lib().moe_forward_host(plan, T, _ptr(x_host), _ptr(router_w), _ptr(router_gamma),
-                                _ptr(router_bias), _ptr(w_gate_up), _ptr(w_down),
+                                _ptr(router_bias), _ptr(expert_gamma), _ptr(w_gate_up),
+                                _ptr(w_down),
                                 _ptr(scales_gate_up), _ptr(scales_down), _ptr(residual_host),
                                 _ptr(out_host), _stream(stream))
     return _check(st, "moe_forward_host", check)
@@ -161,11 +166,12 @@ def moe_forward_host(plan, T, x_host, router_w, router_gamma, router_bias, w_gat
 
 def moe_forward_noalloc(plan, T, x, router_w, router_gamma, router_bias, w_gate_up, w_down,
                         scales_gate_up, scales_down, residual, out, status_out=None, stream=None,
-                        check: bool = True):
+                        check: bool = True, expert_gamma=None):
     """moe_forward without any device allocation: intermediates live in the
     library's fixed 40 MiB device array (see include/moe.h)."""
     st = lib().moe_forward_noalloc(plan, T, _ptr(x), _ptr(router_w), _ptr(router_gamma),
-                                   _ptr(router_bias), _ptr(w_gate_up), _ptr(w_down),
+                                   _ptr(router_bias), _ptr(expert_gamma), _ptr(w_gate_up),
+                                   _ptr(w_down),
                                    _ptr(scales_gate_up), _ptr(scales_down), _ptr(residual),
                                    _ptr(out), _ptr(status_out), _stream(stream))
     return _check(st, "moe_forward_noalloc", check)

@@ -131,6 +131,25 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, int
       : "memory");
 }
 
+// Four rows (r0..r3) of a 2-D tensor, columns [x, x + box width), into four
+// consecutive smem rows; the tensor map's box is one row high.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, int x, int r0, int r1,
+                                            int r2, int r3, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// Bring [p, p + bytes) into L2 (bytes a multiple of 16, p 16-byte aligned).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -229,6 +248,15 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Programmatic dependent launch: wait until the preceding grid in the stream
+// has completed and its memory is visible (a no-op when the kernel was not
+// launched with the attribute), and let the next grid begin launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -245,10 +273,13 @@ struct RouterArgs {
   float* w;
   float* gap;
   Ctl* ctl;
+  const void* l2_prefetch;      // bytes to pull into L2 while routing (or NULL)
+  uint64_t l2_prefetch_bytes;
 };
 
 struct PlanArgs {
   int T, E, k, d, f;
+  int chunk;             // tokens per scheduler chunk (256 bf16, 128 int4)
   const int32_t* idx;    // [T*k]
   int32_t* offsets;      // [E+1]
   int32_t* perm;         // [T*k] slot -> token
@@ -259,24 +290,14 @@ struct PlanArgs {
   Ctl* ctl;
 };
 
+
 struct GatherArgs {
   int rows, d;
+  float eps;
+  const float* gamma2;   // expert-side (1 + gamma2) RMSNorm, or NULL for raw x
   const int32_t* perm;
   const __nv_bfloat16* x;
   __nv_bfloat16* x_perm;
-};
-
-struct ExpertArgs {
-  int T, E, k, d, f;
-  const int32_t* offsets;
-  const int32_t* chunk_e;
-  const int32_t* chunk_c;
-  int32_t* ready;
-  __nv_bfloat16* h;   // [T*k, f]
-  float* y;           // [T*k, d]
-  Ctl* ctl;
-  uint64_t timeout_ns;
-  int test_stall;
 };
 
 struct CombineArgs {
@@ -288,13 +309,58 @@ struct CombineArgs {
   __nv_bfloat16* out;
 };
 
+struct ExpertArgs {
+  int T, E, k, d, f;
+  const int32_t* perm;     // slot -> token
+  const int32_t* offsets;
+  const int32_t* chunk_e;
+  const int32_t* chunk_c;
+  int32_t* ready;
+  const __half* scales_gu;  // int4: [E, 2f, ceil(d/128)]
+  const __half* scales_d;   // int4: [E, d, ceil(f/128)]
+  __nv_bfloat16* h;   // [T*k, f]
+  float* y;           // [T*k, d]
+  Ctl* ctl;
+  uint64_t timeout_ns;
+  int test_stall;
+};
+
+
+// Launch with programmatic stream serialization (when pdl is set) so the
+// kernel's launch and prologue overlap the tail of the previous kernel.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 }  // namespace moe
 
 // Host-side launchers (one per kernel file).
-cudaError_t moe_launch_router(const moe::RouterArgs& a, cudaStream_t s);
-cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s);
-cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s);
+cudaError_t moe_launch_router(const moe::RouterArgs& a, const CUtensorMap& tm_rw, cudaStream_t s,
+                              bool pdl);
+size_t moe_router_smem_bytes(int d);
+int moe_router_tc_splits(int d);
+cudaError_t moe_launch_router_split(const float* rw, const float* gamma, int E, int EP, int d,
+                                    __nv_bfloat16* wsplit, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x,
+                                 const CUtensorMap& tm_w, int EP, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_expert(const moe::ExpertArgs& a, const CUtensorMap& tm_wgu,
                               const CUtensorMap& tm_wd, const CUtensorMap& tm_xp,
-                              const CUtensorMap& tm_h, int num_sms, cudaStream_t s);
-cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s);
+                              const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_expert_w4(const moe::ExpertArgs& a, const CUtensorMap& tm_cgu,
+                                 const CUtensorMap& tm_cd, const CUtensorMap& tm_xp,
+                                 const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);

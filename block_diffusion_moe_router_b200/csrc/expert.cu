@@ -29,83 +29,19 @@
 // Every wait is bounded by %globaltimer; on expiry the kernel records
 // MOE_ERR_TIMEOUT, the roles leave their loops, in-flight TMA copies and
 // UMMAs are drained (again bounded) and TMEM is released.
-#include "common.cuh"
+#include "expert_common.cuh"
 
 namespace moe {
 
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kUnitRing = 4;
 constexpr int kMaxStages = 8;
 constexpr int kRingBytes = 200 * 1024;
-constexpr int kXchgStride = 33;  // floats per exchanged row (bank-conflict padding)
-constexpr int kXchgBytes = 64 * kXchgStride * 4;
+constexpr int kXchgBytes = 64 * kXchgStride * 4;  // gate/up exchange rows
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBarBytes = 8 * (2 * kMaxStages + 4 + 2 * kUnitRing + 1);
 constexpr int kSmemBytes = 1024 + kRingBytes + kXchgBytes + kBarBytes + 256;
-
-enum { kUnitGateUp = 0, kUnitDown = 1, kUnitStop = -1 };
-
-struct UnitInfo {
-  int type;
-  int e;      // expert
-  int m;      // row tile inside the expert's weight
-  int n;      // tokens in this chunk (1..256)
-  int slot0;  // first slot of the chunk
-  int q;      // chunk index (scheduler table)
-};
-
-enum {
-  kWhereUnitEmpty = 1,
-  kWhereStageEmpty,
-  kWhereReady,
-  kWhereUnitFullMma,
-  kWhereTmemEmpty,
-  kWhereStageFull,
-  kWhereUnitFullEpi,
-  kWhereTmemFull,
-  kWhereDrain
-};
-
-__device__ __forceinline__ float gelu_tanh(float g) {
-  // 0.5 g (1 + tanh( sqrt(2/pi) (g + 0.044715 g^3) ))
-  const float c = 0.7978845608028654f;
-  return 0.5f * g * (1.f + tanhf(c * fmaf(0.044715f * g, g * g, g)));
-}
-
-// Spin until *p >= need (acquire), bounded like mbar_wait.
-__device__ bool wait_count(const int* p, int need, volatile int* abort, Ctl* ctl,
-                           uint64_t timeout_ns, int where) {
-  if (ld_acquire_gpu(p) >= need) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 16; ++i) {
-      __nanosleep(64);
-      if (ld_acquire_gpu(p) >= need) return true;
-    }
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > timeout_ns) {
-      record_error(ctl, MOE_ERR_TIMEOUT, where);
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
-// Bounded wait that ignores the abort flag (used only while draining).
-__device__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, Ctl* ctl, uint64_t timeout_ns) {
-  const uint32_t a = smem_u32(bar);
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(a, parity)) {
-    if (globaltimer_ns() - t0 > timeout_ns) {
-      record_error(ctl, MOE_ERR_TIMEOUT, kWhereDrain);
-      return false;
-    }
-  }
-  return true;
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     expert_kernel(const __grid_constant__ CUtensorMap tm_wgu,
@@ -135,16 +71,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int DN = a.d / kBM;
   Ctl* ctl = a.ctl;
 
-  // B-operand rows per stage: the largest chunk, rounded up to the TMA box.
-  const int maxn = max(1, min(kMaxN, ctl->max_chunk));
-  const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
-  const int stage_bytes = kABytes + NB * kBK * 2;
-  const int S = min(kMaxStages, kRingBytes / stage_bytes);
-  const int n_chunks = ctl->n_chunks;
-  const int U = n_chunks * (GU + DN);
-
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
+    for (int i = 0; i < kMaxStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -174,23 +102,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // routing tables: written by the preceding kernels
+  pdl_launch_dependents();
+
+  // B-operand rows per stage: the largest chunk, rounded up to the TMA box.
+  const int maxn = max(1, min(kMaxN, ctl->max_chunk));
+  const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
+  const int stage_bytes = kABytes + NB * kBK * 2;
+  const int S = min(kMaxStages, kRingBytes / stage_bytes);
+  const int n_chunks = ctl->n_chunks;
+  const int U = n_chunks * (GU + DN);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();
-      const uint64_t pol_act = l2_policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      int ur = 0;
-      uint32_t uphase = 0;
-      uint32_t issued = 0, issued_par = 0;  // stages with a copy issued, and its parity
-      while (true) {
-        if (*s_abort) break;
+    // Lane 0 claims units, waits and issues the copies.
+    const uint64_t pol_w = l2_policy_evict_first();
+    const uint64_t pol_act = l2_policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    int ur = 0;
+    uint32_t uphase = 0;
+    uint32_t issued = 0, issued_par = 0;  // stages with a copy issued, and its parity
+    while (true) {
+      UnitInfo ui;
+      ui.type = kUnitStop;
+      ui.e = ui.m = ui.n = ui.slot0 = ui.q = 0;
+      int go = 0;
+      if (lane == 0 && !*s_abort) {
+        go = 1;
         const int u = atomicAdd(&ctl->work_next, 1);
-        UnitInfo ui;
-        ui.type = kUnitStop;
-        ui.e = ui.m = ui.n = ui.slot0 = ui.q = 0;
         if (u < U) {
           int q, m;
           if (u < n_chunks * GU) {
@@ -215,33 +155,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ui.n < 1 || ui.n > NB) {  // corrupt plan: never index outside the ring
             record_error(ctl, MOE_ERR_DEVICE_CHECK, 200);
             *s_abort = 1;
-            break;
+            go = 0;
           }
         }
-        if (ui.type == kUnitDown) {
+        if (go && ui.type == kUnitDown) {
           const int need = GU + (a.test_stall ? (1 << 30) : 0);
-          if (!wait_count(a.ready + ui.q, need, s_abort, ctl, a.timeout_ns, kWhereReady)) break;
-          fence_proxy_async_global();
+          if (wait_count(a.ready + ui.q, need, s_abort, ctl, a.timeout_ns, kWhereReady))
+            fence_proxy_async_global();
+          else
+            go = 0;
         }
-        if (!mbar_wait(&uempty[ur], uphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereUnitEmpty))
-          break;
-        units[ur] = ui;
-        mbar_arrive(&ufull[ur]);
-        if (++ur == kUnitRing) {
-          ur = 0;
-          uphase ^= 1;
+        if (go && mbar_wait(&uempty[ur], uphase ^ 1, s_abort, ctl, a.timeout_ns,
+                            kWhereUnitEmpty)) {
+          units[ur] = ui;
+          mbar_arrive(&ufull[ur]);
+        } else {
+          go = 0;
         }
-        if (ui.type == kUnitStop) break;
-
+      }
+      go = __shfl_sync(0xffffffffu, go, 0);
+      ui.type = __shfl_sync(0xffffffffu, ui.type, 0);
+      ui.n = __shfl_sync(0xffffffffu, ui.n, 0);
+      ui.slot0 = __shfl_sync(0xffffffffu, ui.slot0, 0);
+      if (!go || ui.type == kUnitStop) break;
+      if (++ur == kUnitRing) {
+        ur = 0;
+        uphase ^= 1;
+      }
+      int ok = 1;
+      if (lane == 0) {
         const int nkb = (ui.type == kUnitGateUp) ? a.d / kBK : a.f / kBK;
         const int nbox = (ui.n + kBRows - 1) / kBRows;
         const uint32_t tx = kABytes + nbox * kBRows * kBK * 2;
         const CUtensorMap* tb = (ui.type == kUnitGateUp) ? &tm_xp : &tm_h;
-        bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
                          kWhereStageEmpty)) {
-            ok = false;
+            ok = 0;
             break;
           }
           uint8_t* sa = ring + stage * stage_bytes;
@@ -265,13 +215,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             phase ^= 1;
           }
         }
-        if (!ok) break;
       }
-      // Drain: every issued copy must land before the CTA may exit.
-      for (int s2 = 0; s2 < S; ++s2)
-        if ((issued >> s2) & 1u) mbar_wait_drain(&full[s2], (issued_par >> s2) & 1u, ctl,
-                                                 a.timeout_ns);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
     }
+    // Drain: every issued copy must land before the CTA may exit.
+    if (lane == 0)
+      for (int s2 = 0; s2 < S; ++s2)
+        if ((issued >> s2) & 1u)
+          mbar_wait_drain(&full[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
@@ -326,88 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(drain, 0, ctl, a.timeout_ns);
     }
   } else {
-    // ------------------------------------------------------------ epilogue
-    const int q4 = warp & 3;          // TMEM lane quarter this warp may access
-    const int row = q4 * 32 + lane;   // accumulator row (TMEM lane)
-    const int et = threadIdx.x - 64;  // 0..127
-    int ur = 0;
-    uint32_t uphase = 0;
-    int acc = 0;
-    uint32_t aphase = 0;
-    while (true) {
-      // The leader waits; the decision is broadcast so the 128 threads always
-      // take the same path through the named barriers below.
-      if (et == 0) {
-        bool ok = mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullEpi);
-        if (ok && units[ur].type != kUnitStop)
-          ok = mbar_wait(&tfull[acc], aphase, s_abort, ctl, a.timeout_ns, kWhereTmemFull);
-        *s_bcast = ok ? 1 : 0;
-      }
-      named_barrier(1, 128);
-      const bool ok = *s_bcast != 0;
-      const UnitInfo ui = units[ur];
-      named_barrier(1, 128);
-      if (!ok || ui.type == kUnitStop) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kMaxN);
-      const int nch = (ui.n + 31) / 32;
-      if (ui.type == kUnitGateUp) {
-        __nv_bfloat16* hcol = a.h + (size_t)ui.slot0 * a.f + ui.m * kGuHalf + row;
-        for (int cc = 0; cc < nch; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tbase + cc * 32, v);
-          tmem_wait_ld();
-          if (row >= kGuHalf) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              xchg[(row - kGuHalf) * kXchgStride + i] = __uint_as_float(v[i]);
-          }
-          named_barrier(1, 128);
-          if (row < kGuHalf) {
-            const int cmax = min(32, ui.n - cc * 32);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (i < cmax) {
-                const float g = __uint_as_float(v[i]);
-                const float up = xchg[row * kXchgStride + i];
-                hcol[(size_t)(cc * 32 + i) * a.f] = __float2bfloat16(gelu_tanh(g) * up);
-              }
-            }
-          }
-          named_barrier(1, 128);
-        }
-      } else {
-        float* ycol = a.y + (size_t)ui.slot0 * a.d + ui.m * kBM + row;
-        for (int cc = 0; cc < nch; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tbase + cc * 32, v);
-          tmem_wait_ld();
-          const int cmax = min(32, ui.n - cc * 32);
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __uint_as_float(v[i]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
-      if (ui.type == kUnitGateUp) __threadfence();  // h visible before the chunk counter
-      named_barrier(1, 128);
-      if (et == 0) {
-        if (ui.type == kUnitGateUp) {
-          __threadfence();
-          fence_proxy_async_global();
-          atomicAdd(a.ready + ui.q, 1);
-        }
-        mbar_arrive(&uempty[ur]);
-      }
-      if (++ur == kUnitRing) {
-        ur = 0;
-        uphase ^= 1;
-      }
-      acc ^= 1;
-      if (acc == 0) aphase ^= 1;
-    }
+    epilogue_role(a, units, ufull, uempty, tfull, tempty, xchg, s_abort, s_bcast, tmem_base,
+                  kMaxN, warp, lane);
   }
 
   tc_fence_before();
@@ -424,13 +296,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t moe_launch_expert(const moe::ExpertArgs& a, const CUtensorMap& tm_wgu,
                               const CUtensorMap& tm_wd, const CUtensorMap& tm_xp,
-                              const CUtensorMap& tm_h, int num_sms, cudaStream_t s) {
+                              const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl) {
   static_assert(moe::kSmemBytes <= 232448, "expert kernel smem above the sm_100 limit");
   cudaError_t err = cudaFuncSetAttribute(moe::expert_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          moe::kSmemBytes);
   if (err != cudaSuccess) return err;
-  moe::expert_kernel<<<num_sms, moe::kThreads, moe::kSmemBytes, s>>>(tm_wgu, tm_wd, tm_xp, tm_h,
-                                                                      a);
-  return cudaGetLastError();
+  return moe::launch_pdl(moe::expert_kernel, dim3(num_sms), dim3(moe::kThreads),
+                         (size_t)moe::kSmemBytes, s, pdl, tm_wgu, tm_wd, tm_xp, tm_h, a);
 }

@@ -1,0 +1,178 @@
+// expert_common.cuh -- pieces shared by the bf16 and the int4 expert
+// kernels: the work-unit record, bounded waits, GELU-tanh and the epilogue
+// role (TMEM accumulators -> h = gelu(gate) * up in bf16, or y in fp32).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kXchgStride = 33;  // floats per exchanged row (bank-conflict padding)
+constexpr int kUnitRing = 4;     // work units in flight between the roles
+
+enum { kUnitGateUp = 0, kUnitDown = 1, kUnitStop = -1 };
+
+struct UnitInfo {
+  int type;
+  int e;      // expert
+  int m;      // row tile inside the expert's weight
+  int n;      // tokens in this chunk (1..256)
+  int slot0;  // first slot of the chunk
+  int q;      // chunk index (scheduler table)
+};
+
+enum {
+  kWhereUnitEmpty = 1,
+  kWhereStageEmpty,
+  kWhereReady,
+  kWhereUnitFullMma,
+  kWhereTmemEmpty,
+  kWhereStageFull,
+  kWhereUnitFullEpi,
+  kWhereTmemFull,
+  kWhereDrain
+};
+
+__device__ __forceinline__ float gelu_tanh(float g) {
+  // 0.5 g (1 + tanh( sqrt(2/pi) (g + 0.044715 g^3) ))
+  const float c = 0.7978845608028654f;
+  return 0.5f * g * (1.f + tanhf(c * fmaf(0.044715f * g, g * g, g)));
+}
+
+// Spin until *p >= need (acquire), bounded like mbar_wait.
+__device__ inline bool wait_count(const int* p, int need, volatile int* abort, Ctl* ctl,
+                           uint64_t timeout_ns, int where) {
+  if (ld_acquire_gpu(p) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i) {
+      __nanosleep(64);
+      if (ld_acquire_gpu(p) >= need) return true;
+    }
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      record_error(ctl, MOE_ERR_TIMEOUT, where);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag (used only while draining).
+__device__ inline bool mbar_wait_drain(uint64_t* bar, uint32_t parity, Ctl* ctl, uint64_t timeout_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      record_error(ctl, MOE_ERR_TIMEOUT, kWhereDrain);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Epilogue role (warps 2..5, 128 threads): for each unit, read the fp32
+// accumulator from TMEM (lane = weight row, column = token), and write
+//   gate_up: h[slot][m*64 + r] = gelu_tanh(gate_r) * up_r  (lane r pairs
+//            with lane 64 + r through smem), bf16;
+//   down:    y[slot][m*128 + r], fp32.
+// The leader does the waits and broadcasts the outcome, so the 128 threads
+// always pass the same named barriers.
+__device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInfo* units,
+                                              uint64_t* ufull, uint64_t* uempty, uint64_t* tfull,
+                                              uint64_t* tempty, float* xchg,
+                                              volatile int* s_abort, volatile int* s_bcast,
+                                              uint32_t tmem_base, int acc_cols, int warp,
+                                              int lane) {
+  Ctl* ctl = a.ctl;
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;          // TMEM lane quarter this warp may access
+    const int row = q4 * 32 + lane;   // accumulator row (TMEM lane)
+    const int et = threadIdx.x - 64;  // 0..127
+    int ur = 0;
+    uint32_t uphase = 0;
+    int acc = 0;
+    uint32_t aphase = 0;
+    while (true) {
+      // The leader waits; the decision is broadcast so the 128 threads always
+      // take the same path through the named barriers below.
+      if (et == 0) {
+        bool ok = mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullEpi);
+        if (ok && units[ur].type != kUnitStop)
+          ok = mbar_wait(&tfull[acc], aphase, s_abort, ctl, a.timeout_ns, kWhereTmemFull);
+        *s_bcast = ok ? 1 : 0;
+      }
+      named_barrier(1, 128);
+      const bool ok = *s_bcast != 0;
+      const UnitInfo ui = units[ur];
+      named_barrier(1, 128);
+      if (!ok || ui.type == kUnitStop) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * acc_cols);
+      const int nch = (ui.n + 31) / 32;
+      if (ui.type == kUnitGateUp) {
+        __nv_bfloat16* hcol = a.h + (size_t)ui.slot0 * a.f + ui.m * kGuHalf + row;
+        for (int cc = 0; cc < nch; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tbase + cc * 32, v);
+          tmem_wait_ld();
+          if (row >= kGuHalf) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              xchg[(row - kGuHalf) * kXchgStride + i] = __uint_as_float(v[i]);
+          }
+          named_barrier(1, 128);
+          if (row < kGuHalf) {
+            const int cmax = min(32, ui.n - cc * 32);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i < cmax) {
+                const float g = __uint_as_float(v[i]);
+                const float up = xchg[row * kXchgStride + i];
+                hcol[(size_t)(cc * 32 + i) * a.f] = __float2bfloat16(gelu_tanh(g) * up);
+              }
+            }
+          }
+          named_barrier(1, 128);
+        }
+      } else {
+        float* ycol = a.y + (size_t)ui.slot0 * a.d + ui.m * kBM + row;
+        for (int cc = 0; cc < nch; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tbase + cc * 32, v);
+          tmem_wait_ld();
+          const int cmax = min(32, ui.n - cc * 32);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __uint_as_float(v[i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+      }
+      if (ui.type == kUnitGateUp) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[acc]);
+      }
+      if (ui.type == kUnitGateUp) __threadfence();  // h visible before the chunk counter
+      named_barrier(1, 128);
+      if (et == 0) {
+        if (ui.type == kUnitGateUp) {
+          __threadfence();
+          fence_proxy_async_global();
+          atomicAdd(a.ready + ui.q, 1);
+        }
+        mbar_arrive(&uempty[ur]);
+      }
+      if (++ur == kUnitRing) {
+        ur = 0;
+        uphase ^= 1;
+      }
+      acc ^= 1;
+      if (acc == 0) aphase ^= 1;
+    }
+  }
+
+}  // namespace moe

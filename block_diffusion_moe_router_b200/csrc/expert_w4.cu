@@ -1,0 +1,463 @@
+// expert_w4.cu -- grouped expert GEMMs with symmetric int4 weights in groups
+// of 128 along the input dimension (auto-round pull request "Add
+// quantization support for DiffusionGemma", transformers backend test log:
+// quantization_config bits 4, group_size 128, sym True, data_type int).
+//
+// Same work units, scheduler, B operands and epilogue as the bf16 kernel
+// (expert.cu); what changes is the A operand (the weights):
+//   - TMA brings each 128-wide K stage of packed codes (128 rows x 64 bytes)
+//     into shared memory;
+//   - 8 dequant warps turn the codes into bf16 A values straight in TMEM
+//     (tcgen05.st): per 32-bit word of 8 codes, (code ^ 8) nibbles are placed
+//     in the low mantissa bits of bf16 128.0, so each value reads 136 + code;
+//     subtracting 136 is exact, and one bf16 multiply applies the group scale
+//     (the stage is exactly one group of 128);
+//   - the UMMA reads A from TMEM (kind::f16, A and B both bf16) and B from
+//     shared memory.
+// Weights thus never round-trip through shared memory as bf16: per weight
+// the SM moves half a byte through smem and two bytes into TMEM.
+//
+// TMEM (512 columns): two 128-column fp32 accumulators (a unit holds at most
+// 128 tokens here) and four 64-column A stages.
+#include "expert_common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 448;  // producer, UMMA, 4 epilogue, 8 dequant warps
+constexpr int kDqWarp0 = 6;
+constexpr int kDqWarps = 8;
+constexpr int kChunkN = 128;                 // tokens per unit
+constexpr int kBK4 = 128;                    // K per stage = one scale group
+constexpr int kCodeBytes = kBM * kBK4 / 2;   // 8 KB of codes per stage
+constexpr int kAStages = 4;                  // TMEM A stages
+constexpr int kACols = kBK4 / 2;             // 64 columns of bf16x2 per A stage
+constexpr int kAColBase = 2 * kChunkN;       // A stages after the accumulators
+constexpr int kMaxStages = 8;
+constexpr int kRingBytes = 192 * 1024;
+constexpr int kScaleStride = 32;             // fp16 scales per row kept (d, f <= 4096)
+constexpr int kScaleBytes = kBM * kScaleStride * 2;
+constexpr int kXchgBytes = 64 * kXchgStride * 4;
+constexpr int kBarBytes = 8 * (2 * kMaxStages + 2 * kAStages + 4 + 2 * kUnitRing + 1);
+constexpr int kSmemBytes =
+    1024 + kRingBytes + kScaleBytes + kXchgBytes + kBarBytes + 256;
+static_assert(kAColBase + kAStages * kACols <= kTmemCols, "TMEM budget");
+
+enum { kWhereAFull = 20, kWhereAEmpty, kWhereDqFull };
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Eight packed codes (element i in bits [4i, 4i+4), 4-bit two's complement)
+// -> four bf16x2 words holding elements (0,1), (2,3), (4,5), (6,7), each
+// value code * scale.
+__device__ __forceinline__ void dequant8(uint32_t w, __nv_bfloat162 s2, uint32_t* out) {
+  const uint32_t x = w ^ 0x88888888u;  // code + 8 in every nibble
+  const uint32_t t0 = (x & 0x000F000Fu) | 0x43004300u;  // (e0, e4) as 136 + code
+  const uint32_t t1 = ((x >> 4) & 0x000F000Fu) | 0x43004300u;   // (e1, e5)
+  const uint32_t t2 = ((x >> 8) & 0x000F000Fu) | 0x43004300u;   // (e2, e6)
+  const uint32_t t3 = ((x >> 12) & 0x000F000Fu) | 0x43004300u;  // (e3, e7)
+  uint32_t c[4];
+  c[0] = __byte_perm(t0, t1, 0x5410);
+  c[1] = __byte_perm(t2, t3, 0x5410);
+  c[2] = __byte_perm(t0, t1, 0x7632);
+  c[3] = __byte_perm(t2, t3, 0x7632);
+  const __nv_bfloat162 k136 = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)0x4308),
+                                                 __ushort_as_bfloat16((unsigned short)0x4308));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&c[i]);
+    v = __hmul2(__hsub2(v, k136), s2);  // exact subtraction, one rounding
+    out[i] = *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    expert_w4_kernel(const __grid_constant__ CUtensorMap tm_cgu,
+                     const __grid_constant__ CUtensorMap tm_cd,
+                     const __grid_constant__ CUtensorMap tm_xp,
+                     const __grid_constant__ CUtensorMap tm_h, ExpertArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  __half* sc = reinterpret_cast<__half*>(smem + kRingBytes);  // [128][kScaleStride]
+  float* xchg = reinterpret_cast<float*>(smem + kRingBytes + kScaleBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kScaleBytes + kXchgBytes);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* afull = empty + kMaxStages;
+  uint64_t* aempty = afull + kAStages;
+  uint64_t* tfull = aempty + kAStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* ufull = tempty + 2;
+  uint64_t* uempty = ufull + kUnitRing;
+  uint64_t* drain = uempty + kUnitRing;
+  UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(units + kUnitRing);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_bcast = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile int* s_dqbc = reinterpret_cast<volatile int*>(tmem_slot + 3);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int GU = a.f / kGuHalf;
+  const int DN = a.d / kBM;
+  Ctl* ctl = a.ctl;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMaxStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kDqWarps + 1);  // dequant warps read codes, UMMA reads B
+    }
+    for (int i = 0; i < kAStages; ++i) {
+      mbar_init(&afull[i], kDqWarps);
+      mbar_init(&aempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    for (int i = 0; i < kUnitRing; ++i) {
+      mbar_init(&ufull[i], 1);
+      mbar_init(&uempty[i], 2 + kDqWarps);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_cgu);
+    tma_prefetch_desc(&tm_cd);
+    tma_prefetch_desc(&tm_xp);
+    tma_prefetch_desc(&tm_h);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_launch_dependents();
+
+  const int maxn = max(1, min(kChunkN, ctl->max_chunk));
+  const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
+  const int stage_bytes = kCodeBytes + 2 * NB * kBK * 2;  // codes + two 64-wide B sub-tiles
+  const int S = min(kMaxStages, kRingBytes / stage_bytes);
+  const int n_chunks = ctl->n_chunks;
+  const int U = n_chunks * (GU + DN);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol_w = l2_policy_evict_first();
+    const uint64_t pol_act = l2_policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    int ur = 0;
+    uint32_t uphase = 0;
+    uint32_t issued = 0, issued_par = 0;
+    while (true) {
+      UnitInfo ui;
+      ui.type = kUnitStop;
+      ui.e = ui.m = ui.n = ui.slot0 = ui.q = 0;
+      int go = 0;
+      if (lane == 0 && !*s_abort) {
+        go = 1;
+        const int u = atomicAdd(&ctl->work_next, 1);
+        if (u < U) {
+          int q, m;
+          if (u < n_chunks * GU) {
+            ui.type = kUnitGateUp;
+            q = u / GU;
+            m = u - q * GU;
+          } else {
+            const int v = u - n_chunks * GU;
+            ui.type = kUnitDown;
+            q = v / DN;
+            m = v - q * DN;
+          }
+          const int e = a.chunk_e[q];
+          const int c = a.chunk_c[q];
+          const int seg0 = a.offsets[e];
+          const int ne = a.offsets[e + 1] - seg0;
+          ui.e = e;
+          ui.m = m;
+          ui.q = q;
+          ui.slot0 = seg0 + c * kChunkN;
+          ui.n = min(kChunkN, ne - c * kChunkN);
+          if (ui.n < 1 || ui.n > NB) {
+            record_error(ctl, MOE_ERR_DEVICE_CHECK, 201);
+            *s_abort = 1;
+            go = 0;
+          }
+        }
+        if (go && ui.type == kUnitDown) {
+          const int need = GU + (a.test_stall ? (1 << 30) : 0);
+          if (wait_count(a.ready + ui.q, need, s_abort, ctl, a.timeout_ns, kWhereReady))
+            fence_proxy_async_global();
+          else
+            go = 0;
+        }
+        if (go && mbar_wait(&uempty[ur], uphase ^ 1, s_abort, ctl, a.timeout_ns,
+                            kWhereUnitEmpty)) {
+          units[ur] = ui;
+          mbar_arrive(&ufull[ur]);
+        } else {
+          go = 0;
+        }
+      }
+      go = __shfl_sync(0xffffffffu, go, 0);
+      ui.type = __shfl_sync(0xffffffffu, ui.type, 0);
+      ui.n = __shfl_sync(0xffffffffu, ui.n, 0);
+      ui.slot0 = __shfl_sync(0xffffffffu, ui.slot0, 0);
+      if (!go || ui.type == kUnitStop) break;
+      if (++ur == kUnitRing) {
+        ur = 0;
+        uphase ^= 1;
+      }
+      int ok = 1;
+      if (lane == 0) {
+        const int C = (ui.type == kUnitGateUp) ? a.d : a.f;
+        const int nkb = (C + kBK4 - 1) / kBK4;
+        const int nbox = (ui.n + kBRows - 1) / kBRows;
+        const uint32_t tx = kCodeBytes + 2 * nbox * kBRows * kBK * 2;
+        const CUtensorMap* tb = (ui.type == kUnitGateUp) ? &tm_xp : &tm_h;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
+                         kWhereStageEmpty)) {
+            ok = 0;
+            break;
+          }
+          uint8_t* sa = ring + stage * stage_bytes;
+          uint8_t* sb = sa + kCodeBytes;
+          mbar_arrive_expect_tx(&full[stage], tx);
+          const int cx = kb * (kBK4 / 2);  // byte column of the packed codes
+          if (ui.type == kUnitGateUp) {
+            const int r0 = ui.e * 2 * a.f + ui.m * kGuHalf;
+            tma_load_2d(sa, &tm_cgu, cx, r0, &full[stage], pol_w);
+            tma_load_2d(sa + kCodeBytes / 2, &tm_cgu, cx, r0 + a.f, &full[stage], pol_w);
+          } else {
+            tma_load_2d(sa, &tm_cd, cx, ui.e * a.d + ui.m * kBM, &full[stage], pol_w);
+          }
+          for (int h = 0; h < 2; ++h)
+            for (int bx = 0; bx < nbox; ++bx)
+              tma_load_2d(sb + h * NB * kBK * 2 + bx * kBRows * kBK * 2, tb, kb * kBK4 + h * kBK,
+                          ui.slot0 + bx * kBRows, &full[stage], pol_act);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+    }
+    if (lane == 0)
+      for (int s2 = 0; s2 < S; ++s2)
+        if ((issued >> s2) & 1u)
+          mbar_wait_drain(&full[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int ast = 0;
+      uint32_t aph = 0;
+      int ur = 0;
+      uint32_t uphase = 0;
+      int acc = 0;
+      uint32_t aphase = 0;
+      while (true) {
+        if (!mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullMma)) break;
+        const UnitInfo ui = units[ur];
+        if (ui.type == kUnitStop) break;
+        const int C = (ui.type == kUnitGateUp) ? a.d : a.f;
+        const int nkb = (C + kBK4 - 1) / kBK4;
+        const int N = (ui.n + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(kBM, N);
+        if (!mbar_wait(&tempty[acc], aphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereTmemEmpty))
+          break;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + (uint32_t)(acc * kChunkN);
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, s_abort, ctl, a.timeout_ns, kWhereStageFull) ||
+              !mbar_wait(&afull[ast], aph, s_abort, ctl, a.timeout_ns, kWhereAFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(ring + stage * stage_bytes + kCodeBytes);
+          const uint32_t ta = tmem_base + (uint32_t)(kAColBase + ast * kACols);
+#pragma unroll
+          for (int kk = 0; kk < kBK4 / kUmmaK; ++kk) {
+            const uint32_t b = sb + (kk >> 2) * NB * kBK * 2 + (kk & 3) * kUmmaK * 2;
+            umma_bf16_ts(dt, ta + kk * (kUmmaK / 2), sdesc_k_sw128(b), idesc,
+                         (kb | kk) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          umma_commit(&aempty[ast]);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1;
+          }
+          if (++ast == kAStages) {
+            ast = 0;
+            aph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        mbar_arrive(&uempty[ur]);
+        if (++ur == kUnitRing) {
+          ur = 0;
+          uphase ^= 1;
+        }
+        acc ^= 1;
+        if (acc == 0) aphase ^= 1;
+      }
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, ctl, a.timeout_ns);
+    }
+  } else if (warp < kDqWarp0) {
+    epilogue_role(a, units, ufull, uempty, tfull, tempty, xchg, s_abort, s_bcast, tmem_base,
+                  kChunkN, warp, lane);
+  } else {
+    // ------------------------------------------------------------ dequant warps
+    const int dw = warp - kDqWarp0;        // 0..7
+    const int q4 = warp & 3;               // TMEM lane quarter
+    const int row = q4 * 32 + lane;        // A row == TMEM lane
+    const int half = dw >> 2;              // which 64 of the stage's 128 codes
+    const int dt = threadIdx.x - kDqWarp0 * 32;  // 0..255
+    int stage = 0;
+    uint32_t phase = 0;
+    int ast = 0;
+    uint32_t aph = 0;
+    int ur = 0;
+    uint32_t uphase = 0;
+    while (true) {
+      if (dt == 0) {
+        bool ok = mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereDqFull);
+        *s_dqbc = ok ? 1 : 0;
+      }
+      named_barrier(2, kDqWarps * 32);
+      const bool uok = *s_dqbc != 0;
+      const UnitInfo ui = units[ur];
+      named_barrier(2, kDqWarps * 32);
+      if (!uok || ui.type == kUnitStop) break;
+      // this unit's fp16 scales: A row r -> weight row, one per group of 128
+      const bool gu = ui.type == kUnitGateUp;
+      const int C = gu ? a.d : a.f;
+      const int G = (C + kBK4 - 1) / kBK4;
+      const __half* sg = gu ? a.scales_gu : a.scales_d;
+      for (int i = dt; i < kBM * G; i += kDqWarps * 32) {
+        const int r = i / G;
+        const int g = i - r * G;
+        const int wrow = gu ? (ui.e * 2 * a.f + (r < kGuHalf ? 0 : a.f) + ui.m * kGuHalf +
+                               (r & (kGuHalf - 1)))
+                            : (ui.e * a.d + ui.m * kBM + r);
+        sc[r * kScaleStride + g] = sg[(size_t)wrow * G + g];
+      }
+      named_barrier(2, kDqWarps * 32);
+      bool sok = true;
+      for (int kb = 0; kb < G; ++kb) {
+        if (sok) {
+          sok = mbar_wait(&full[stage], phase, s_abort, ctl, a.timeout_ns, kWhereDqFull) &&
+                mbar_wait(&aempty[ast], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty);
+        }
+        if (sok) {
+          const uint8_t* codes = ring + stage * stage_bytes + row * (kBK4 / 2) + half * 32;
+          const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
+          const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[stage]);  // codes are in registers
+          const float sf = __half2float(sc[row * kScaleStride + kb]);
+          const __nv_bfloat162 s2 = __float2bfloat162_rn(sf);
+          uint32_t v[32];
+          dequant8(c0.x, s2, v + 0);
+          dequant8(c0.y, s2, v + 4);
+          dequant8(c0.z, s2, v + 8);
+          dequant8(c0.w, s2, v + 12);
+          dequant8(c1.x, s2, v + 16);
+          dequant8(c1.y, s2, v + 20);
+          dequant8(c1.z, s2, v + 24);
+          dequant8(c1.w, s2, v + 28);
+          const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) +
+                              (uint32_t)(kAColBase + ast * kACols + half * 32);
+          tmem_st32(ta, v);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&afull[ast]);
+        }
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (++ast == kAStages) {
+          ast = 0;
+          aph ^= 1;
+        }
+      }
+      named_barrier(2, kDqWarps * 32);  // sc[] is rewritten only after every warp is done
+      if (lane == 0) mbar_arrive(&uempty[ur]);
+      if (++ur == kUnitRing) {
+        ur = 0;
+        uphase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+}  // namespace moe
+
+cudaError_t moe_launch_expert_w4(const moe::ExpertArgs& a, const CUtensorMap& tm_cgu,
+                                 const CUtensorMap& tm_cd, const CUtensorMap& tm_xp,
+                                 const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl) {
+  static_assert(moe::kSmemBytes <= 232448, "int4 expert kernel smem above the sm_100 limit");
+  cudaError_t err = cudaFuncSetAttribute(moe::expert_w4_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         moe::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  return moe::launch_pdl(moe::expert_w4_kernel, dim3(num_sms), dim3(moe::kThreads),
+                         (size_t)moe::kSmemBytes, s, pdl, tm_cgu, tm_cd, tm_xp, tm_h, a);
+}

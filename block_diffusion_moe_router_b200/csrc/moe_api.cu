@@ -32,13 +32,16 @@ struct moe_plan_s {
   int timeout_ms;
   int profile;
   int test_stall;
+  int pdl;
+  int prefetch_mb;
+  int router_ffma;
   int cap_T;
   int last_T;
   void* ws;  // one device allocation holding everything below
   Ctl* ctl;
   int32_t *idx, *perm, *slot_of, *offsets, *chunk_e, *chunk_c, *ready;
   float *w, *gap, *y;
-  __nv_bfloat16 *x_perm, *h, *x_dev, *res_dev, *out_dev;
+  __nv_bfloat16 *x_perm, *h, *x_dev, *res_dev, *out_dev, *wsplit;
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> ev_pool;
 };
@@ -80,6 +83,35 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t col
   return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor map over the router weight [E, d]: box = 32 rows x 128
+// columns, no swizzle; rows past E read as zero.
+bool make_map_router(CUtensorMap* m, const float* base, uint64_t E, uint64_t d) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {d, E};
+  cuuint64_t strides[1] = {d * 4};
+  cuuint32_t box[2] = {128, (cuuint32_t)moe::kRouterTE};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols_bytes,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols_bytes, rows};
+  cuuint64_t strides[1] = {cols_bytes};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool overlap(const void* a, size_t na, const void* b, size_t nb) {
@@ -89,7 +121,24 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-int max_chunks(int E, int T, int k) { return E + (T * k) / moe::kMaxN + 1; }
+// Tokens per scheduler chunk: 256 for bf16 weights, 128 for int4 (whose
+// kernel keeps dequantised A stages in TMEM next to the accumulators).
+int chunk_size(moe_plan_t p) { return p->wdtype == MOE_W_BF16 ? moe::kMaxN : 128; }
+
+int max_chunks(int E, int T, int k) { return E + (T * k) / 128 + 1; }
+
+// Experts rounded up to the UMMA N granularity for the tensor-core router.
+int router_ep(int E) { return (E + 15) / 16 * 16; }
+
+bool use_router_tc(moe_plan_t p) { return !p->router_ffma && p->E <= 128; }
+
+// The router weight times (1 + gamma), split into three bf16 parts.
+size_t wsplit_bytes(moe_plan_t p) { return (size_t)3 * router_ep(p->E) * p->d * 2; }
+
+// 2-D byte tensor map over packed int4 codes [rows, cols_bytes]: box = box_rows
+// x 64 bytes (one group of 128 codes), no swizzle.
+bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols_bytes,
+                    uint32_t box_rows);
 
 moe_status_t check_device(moe_plan_t p) {
   int dev = -1;
@@ -113,7 +162,9 @@ moe_status_t ensure_workspace(moe_plan_t p, int T) {
   const size_t o_idx = take(A * 4), o_w = take(A * 4), o_gap = take((size_t)cap * 4);
   const size_t o_perm = take(A * 4), o_slot = take(A * 4), o_off = take((size_t)(p->E + 1) * 4);
   const size_t o_ce = take(MC * 4), o_cc = take(MC * 4), o_rd = take(MC * 4);
-  const size_t o_xp = take(A * p->d * 2), o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
+  const size_t o_xp = take(A * p->d * 2);
+  const size_t o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
+  const size_t o_ws = take(wsplit_bytes(p));
   const size_t o_xd = take((size_t)cap * p->d * 2), o_rs = take((size_t)cap * p->d * 2);
   const size_t o_od = take((size_t)cap * p->d * 2);
   if (p->ws) {
@@ -141,6 +192,7 @@ moe_status_t ensure_workspace(moe_plan_t p, int T) {
   p->chunk_c = reinterpret_cast<int32_t*>(b + o_cc);
   p->ready = reinterpret_cast<int32_t*>(b + o_rd);
   p->x_perm = reinterpret_cast<__nv_bfloat16*>(b + o_xp);
+  p->wsplit = reinterpret_cast<__nv_bfloat16*>(b + o_ws);
   p->h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
   p->y = reinterpret_cast<float*>(b + o_y);
   p->x_dev = reinterpret_cast<__nv_bfloat16*>(b + o_xd);
@@ -193,9 +245,19 @@ moe_status_t validate_route(moe_plan_t p, int T, const void* x, const float* rw,
   return check_device(p);
 }
 
+// Bytes of the fused gate_up weight pulled into L2 during routing.
+uint64_t prefetch_bytes(moe_plan_t p) {
+  const uint64_t all = (uint64_t)p->E * 2 * p->f * p->d * (p->wdtype == MOE_W_BF16 ? 2 : 1) /
+                       (p->wdtype == MOE_W_BF16 ? 1 : 2);
+  const uint64_t want = (uint64_t)p->prefetch_mb << 20;
+  return want < all ? want : all;
+}
+
 moe_status_t launch_router(moe_plan_t p, int T, const void* x, const float* rw,
                            const float* gamma, const float* bias, int32_t* idx, float* w,
-                           float* gap, cudaStream_t s) {
+                           float* gap, cudaStream_t s, const void* pf = nullptr,
+                           uint64_t pf_bytes = 0, Ctl* ctl = nullptr,
+                           __nv_bfloat16* wsplit = nullptr) {
   moe::RouterArgs ra;
   ra.T = T;
   ra.E = p->E;
@@ -209,9 +271,28 @@ moe_status_t launch_router(moe_plan_t p, int T, const void* x, const float* rw,
   ra.idx = idx;
   ra.w = w;
   ra.gap = gap;
-  ra.ctl = p->ctl;
+  ra.ctl = ctl ? ctl : p->ctl;
+  ra.l2_prefetch = pf_bytes ? pf : nullptr;
+  ra.l2_prefetch_bytes = pf_bytes;
+  const bool pdl = p->pdl != 0;
+  if (use_router_tc(p)) {
+    __nv_bfloat16* ws = wsplit ? wsplit : p->wsplit;
+    const int EP = router_ep(p->E);
+    CUtensorMap tm_x, tm_w;
+    if (!make_map_bf16(&tm_x, x, (uint64_t)T, p->d, 128) ||
+        !make_map_bf16(&tm_w, ws, (uint64_t)3 * EP, p->d, (uint32_t)EP))
+      return MOE_ERR_CUDA;
+    ProfScope ps(p, MOE_K_ROUTER, s);
+    if (moe_launch_router_split(rw, gamma, p->E, EP, p->d, ws, p->num_sms, s, pdl) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    return moe_launch_router_tc(ra, tm_x, tm_w, EP, s, pdl) == cudaSuccess ? MOE_OK
+                                                                           : MOE_ERR_CUDA;
+  }
+  CUtensorMap tm_rw;
+  if (!make_map_router(&tm_rw, rw, p->E, p->d)) return MOE_ERR_CUDA;
   ProfScope ps(p, MOE_K_ROUTER, s);
-  return moe_launch_router(ra, s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return moe_launch_router(ra, tm_rw, s, pdl) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
@@ -255,6 +336,9 @@ moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, mo
   p->timeout_ms = 1000;
   p->profile = 0;
   p->test_stall = 0;
+  p->pdl = 1;
+  p->prefetch_mb = 0;
+  p->router_ffma = 0;
   p->cap_T = 0;
   p->last_T = 0;
   p->ws = nullptr;
@@ -278,6 +362,16 @@ moe_status_t moe_plan_set_option(moe_plan_t p, int key, double value) {
       return MOE_OK;
     case MOE_OPT_TEST_STALL:
       p->test_stall = value != 0.0;
+      return MOE_OK;
+    case MOE_OPT_PDL:
+      p->pdl = value != 0.0;
+      return MOE_OK;
+    case MOE_OPT_ROUTER_FFMA:
+      p->router_ffma = value != 0.0;
+      return MOE_OK;
+    case MOE_OPT_L2_PREFETCH_MB:
+      if (!(value >= 0.0 && value <= 4096.0)) return MOE_ERR_INVALID_ARG;
+      p->prefetch_mb = (int)value;
       return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
@@ -307,19 +401,19 @@ moe_status_t moe_route(moe_plan_t p, int T, const void* x, const float* router_w
 
 moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router_w,
                          const float* router_gamma, const float* router_bias,
-                         const void* w_gate_up, const void* w_down, const void* scales_gate_up,
+                         const float* expert_gamma, const void* w_gate_up, const void* w_down, const void* scales_gate_up,
                          const void* scales_down, const void* residual, void* out, void* stream) {
   moe_status_t st = validate_route(p, T, x, router_w, router_gamma, router_bias);
   if (st != MOE_OK || T == 0) return st;
   if (!w_gate_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (expert_gamma && !aligned16(expert_gamma)) return MOE_ERR_INVALID_ARG;
   if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
   if (p->wdtype == MOE_W_BF16) {
     if (scales_gate_up || scales_down) return MOE_ERR_INVALID_ARG;
   } else {
     if (!scales_gate_up || !scales_down) return MOE_ERR_INVALID_ARG;
     if (!aligned16(scales_gate_up) || !aligned16(scales_down)) return MOE_ERR_INVALID_ARG;
-    return MOE_ERR_UNSUPPORTED;  // int4 expert kernels not built yet
   }
   const size_t act = (size_t)T * p->d * 2;
   if (overlap(out, act, x, act)) return MOE_ERR_INVALID_ARG;
@@ -329,14 +423,19 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int A = T * p->k;
-  CUtensorMap tm_wgu, tm_wd, tm_xp, tm_h;
-  if (!make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) ||
-      !make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM) ||
-      !make_map_bf16(&tm_xp, p->x_perm, (uint64_t)A, p->d, moe::kBRows) ||
-      !make_map_bf16(&tm_h, p->h, (uint64_t)A, p->f, moe::kBRows))
-    return MOE_ERR_CUDA;
+  const bool w4 = p->wdtype == MOE_W_INT4_G128;
+  CUtensorMap tm_wgu, tm_wd, tm_x, tm_h;
+  const bool maps_ok =
+      (w4 ? make_map_codes(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d / 2, moe::kGuHalf) &&
+                make_map_codes(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f / 2, moe::kBM)
+          : make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) &&
+                make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM)) &&
+      make_map_bf16(&tm_x, p->x_perm, (uint64_t)A, p->d, moe::kBRows) &&
+      make_map_bf16(&tm_h, p->h, (uint64_t)A, p->f, moe::kBRows);
+  if (!maps_ok) return MOE_ERR_CUDA;
 
-  st = launch_router(p, T, x, router_w, router_gamma, router_bias, p->idx, p->w, p->gap, s);
+  st = launch_router(p, T, x, router_w, router_gamma, router_bias, p->idx, p->w, p->gap, s,
+                     w_gate_up, prefetch_bytes(p));
   if (st != MOE_OK) return st;
 
   moe::PlanArgs pa;
@@ -345,6 +444,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   pa.k = p->k;
   pa.d = p->d;
   pa.f = p->f;
+  pa.chunk = chunk_size(p);
   pa.idx = p->idx;
   pa.offsets = p->offsets;
   pa.perm = p->perm;
@@ -355,18 +455,20 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   pa.ctl = p->ctl;
   {
     ProfScope ps(p, MOE_K_PLAN, s);
-    if (moe_launch_plan(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe_launch_plan(pa, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   moe::GatherArgs ga;
   ga.rows = A;
   ga.d = p->d;
+  ga.eps = p->eps;
+  ga.gamma2 = expert_gamma;
   ga.perm = p->perm;
   ga.x = static_cast<const __nv_bfloat16*>(x);
   ga.x_perm = p->x_perm;
   {
     ProfScope ps(p, MOE_K_GATHER, s);
-    if (moe_launch_gather(ga, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe_launch_gather(ga, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   moe::ExpertArgs ea;
@@ -375,6 +477,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ea.k = p->k;
   ea.d = p->d;
   ea.f = p->f;
+  ea.perm = p->perm;
   ea.offsets = p->offsets;
   ea.chunk_e = p->chunk_e;
   ea.chunk_c = p->chunk_c;
@@ -384,10 +487,14 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ea.ctl = p->ctl;
   ea.timeout_ns = (uint64_t)p->timeout_ms * 1000000ull;
   ea.test_stall = p->test_stall;
+  ea.scales_gu = static_cast<const __half*>(scales_gate_up);
+  ea.scales_d = static_cast<const __half*>(scales_down);
   {
     ProfScope ps(p, MOE_K_EXPERT, s);
-    if (moe_launch_expert(ea, tm_wgu, tm_wd, tm_xp, tm_h, p->num_sms, s) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    const cudaError_t le =
+        w4 ? moe_launch_expert_w4(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0)
+           : moe_launch_expert(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0);
+    if (le != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   moe::CombineArgs ca;
@@ -401,15 +508,16 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ca.out = static_cast<__nv_bfloat16*>(out);
   {
     ProfScope ps(p, MOE_K_COMBINE, s);
-    if (moe_launch_combine(ca, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe_launch_combine(ca, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
   }
+
   p->last_T = T;
   return MOE_OK;
 }
 
 moe_status_t moe_forward_host(moe_plan_t p, int T, const void* x_host, const float* router_w,
                               const float* router_gamma, const float* router_bias,
-                              const void* w_gate_up, const void* w_down,
+                              const float* expert_gamma, const void* w_gate_up, const void* w_down,
                               const void* scales_gate_up, const void* scales_down,
                               const void* residual_host, void* out_host, void* stream) {
   if (!p || T < 0) return MOE_ERR_INVALID_ARG;
@@ -426,7 +534,8 @@ moe_status_t moe_forward_host(moe_plan_t p, int T, const void* x_host, const flo
   if (residual_host &&
       cudaMemcpyAsync(p->res_dev, residual_host, act, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  st = moe_forward(p, T, p->x_dev, router_w, router_gamma, router_bias, w_gate_up, w_down,
+  st = moe_forward(p, T, p->x_dev, router_w, router_gamma, router_bias, expert_gamma, w_gate_up,
+                   w_down,
                    scales_gate_up, scales_down, residual_host ? p->res_dev : nullptr, p->out_dev,
                    stream);
   if (st != MOE_OK) return st;
@@ -548,7 +657,8 @@ void* noalloc_scratch(int dev) {
 
 extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
                                             const float* router_w, const float* router_gamma,
-                                            const float* router_bias, const void* w_gate_up,
+                                            const float* router_bias, const float* expert_gamma,
+                                            const void* w_gate_up,
                                             const void* w_down, const void* scales_gate_up,
                                             const void* scales_down, const void* residual,
                                             void* out, int32_t* status_out, void* stream) {
@@ -556,8 +666,10 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   if (st != MOE_OK || T == 0) return st;
   if (!w_gate_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (expert_gamma && !aligned16(expert_gamma)) return MOE_ERR_INVALID_ARG;
   if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
   if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (expert_gamma && !aligned16(expert_gamma)) return MOE_ERR_INVALID_ARG;
   if (p->wdtype == MOE_W_BF16) {
     if (scales_gate_up || scales_down) return MOE_ERR_INVALID_ARG;
   } else {
@@ -580,7 +692,9 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   const size_t o_idx = take(A * 4), o_w = take(A * 4), o_gap = take((size_t)T * 4);
   const size_t o_perm = take(A * 4), o_slot = take(A * 4), o_off = take((size_t)(p->E + 1) * 4);
   const size_t o_ce = take(MC * 4), o_cc = take(MC * 4), o_rd = take(MC * 4);
-  const size_t o_xp = take(A * p->d * 2), o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
+  const size_t o_xp = take(A * p->d * 2);
+  const size_t o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
+  const size_t o_ws = take(wsplit_bytes(p));
   if (sz > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
 
   char* b = static_cast<char*>(noalloc_scratch(p->device));
@@ -596,14 +710,15 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   int32_t* chunk_c = reinterpret_cast<int32_t*>(b + o_cc);
   int32_t* ready = reinterpret_cast<int32_t*>(b + o_rd);
   __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(b + o_xp);
+  __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(b + o_ws);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
   float* y = reinterpret_cast<float*>(b + o_y);
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  CUtensorMap tm_wgu, tm_wd, tm_xp, tm_h;
+  CUtensorMap tm_wgu, tm_wd, tm_x, tm_h;
   if (!make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) ||
       !make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM) ||
-      !make_map_bf16(&tm_xp, x_perm, (uint64_t)A, p->d, moe::kBRows) ||
+      !make_map_bf16(&tm_x, x_perm, (uint64_t)A, p->d, moe::kBRows) ||
       !make_map_bf16(&tm_h, h, (uint64_t)A, p->f, moe::kBRows))
     return MOE_ERR_CUDA;
 
@@ -611,21 +726,15 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   // counters and chunk tables itself on every call.
   if (cudaMemsetAsync(ctl, 0, sizeof(Ctl), s) != cudaSuccess) return MOE_ERR_CUDA;
 
-  moe::RouterArgs ra;
-  ra.T = T;
-  ra.E = p->E;
-  ra.k = p->k;
-  ra.d = p->d;
-  ra.eps = p->eps;
-  ra.x = static_cast<const __nv_bfloat16*>(x);
-  ra.router_w = router_w;
-  ra.gamma = router_gamma;
-  ra.bias = router_bias;
-  ra.idx = idx;
-  ra.w = w;
-  ra.gap = gap;
-  ra.ctl = ctl;
-  if (moe_launch_router(ra, s) != cudaSuccess) return MOE_ERR_CUDA;
+  {
+    const bool prof = p->profile != 0;
+    p->profile = 0;  // no event records on this path
+    const moe_status_t rs =
+        launch_router(p, T, x, router_w, router_gamma, router_bias, idx, w, gap, s, w_gate_up,
+                      prefetch_bytes(p), ctl, wsplit);
+    p->profile = prof;
+    if (rs != MOE_OK) return rs;
+  }
 
   moe::PlanArgs pa;
   pa.T = T;
@@ -633,6 +742,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   pa.k = p->k;
   pa.d = p->d;
   pa.f = p->f;
+  pa.chunk = chunk_size(p);
   pa.idx = idx;
   pa.offsets = offsets;
   pa.perm = perm;
@@ -641,15 +751,17 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   pa.chunk_c = chunk_c;
   pa.ready = ready;
   pa.ctl = ctl;
-  if (moe_launch_plan(pa, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe_launch_plan(pa, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
 
   moe::GatherArgs ga;
   ga.rows = (int)A;
   ga.d = p->d;
+  ga.eps = p->eps;
+  ga.gamma2 = expert_gamma;
   ga.perm = perm;
   ga.x = static_cast<const __nv_bfloat16*>(x);
   ga.x_perm = x_perm;
-  if (moe_launch_gather(ga, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe_launch_gather(ga, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
 
   moe::ExpertArgs ea;
   ea.T = T;
@@ -657,6 +769,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ea.k = p->k;
   ea.d = p->d;
   ea.f = p->f;
+  ea.perm = perm;
   ea.offsets = offsets;
   ea.chunk_e = chunk_e;
   ea.chunk_c = chunk_c;
@@ -666,7 +779,10 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ea.ctl = ctl;
   ea.timeout_ns = (uint64_t)p->timeout_ms * 1000000ull;
   ea.test_stall = p->test_stall;
-  if (moe_launch_expert(ea, tm_wgu, tm_wd, tm_xp, tm_h, p->num_sms, s) != cudaSuccess)
+  ea.scales_gu = nullptr;
+  ea.scales_d = nullptr;
+  if (moe_launch_expert(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
 
   moe::CombineArgs ca;
@@ -678,7 +794,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ca.y = y;
   ca.residual = static_cast<const __nv_bfloat16*>(residual);
   ca.out = static_cast<__nv_bfloat16*>(out);
-  if (moe_launch_combine(ca, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe_launch_combine(ca, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
 
   if (status_out && cudaMemcpyAsync(status_out, &ctl->status, sizeof(int32_t),
                                     cudaMemcpyDeviceToDevice, s) != cudaSuccess)

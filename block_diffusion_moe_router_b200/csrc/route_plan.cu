@@ -3,7 +3,8 @@
 //   a = t*k + j of expert e gets slot offsets[e] + (number of earlier
 //   assignments with the same expert).  Also the chunk table of the expert
 //   kernel's scheduler (one chunk = up to 256 tokens of one expert) and the
-//   reset of its counters; and the gather of x rows into slot order.
+//   reset of its counters; the gather of x rows into slot order; and the
+//   fixed-order weighted combine.
 //
 // One CTA of 32 warps does the counting sort: warp w owns a contiguous range
 // of assignments, ranks equal experts inside each 32-wide step with
@@ -17,11 +18,15 @@ namespace {
 
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
+constexpr int kRegIters = 16;  // 32-wide steps per warp held in registers (16K assignments)
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   __shared__ int cnt[kPlanWarps][kMaxE];  // per-warp counts, then per-warp bases
+  __shared__ int tot[kMaxE];
   __shared__ int off[kMaxE + 1];
   __shared__ int cst[kMaxE + 1];
+  __shared__ int wsum[2][kMaxE / 32];
+  __shared__ int s_maxc;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -29,62 +34,128 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   const int A = a.T * a.k;
 
   for (int i = tid; i < kPlanWarps * kMaxE; i += kPlanThreads) (&cnt[0][0])[i] = 0;
+  if (tid == 0) s_maxc = 0;
+  pdl_wait();  // idx comes from the router
+  pdl_launch_dependents();
   __syncthreads();
 
   const int per = (A + kPlanWarps - 1) / kPlanWarps;
   const int lo = min(A, warp * per);
   const int hi = min(A, lo + per);
 
-  // ---- local ranks (stored in slot_of until the bases are known)
-  for (int base = lo; base < hi; base += 32) {
-    const int as = base + lane;
-    const bool act = as < hi;
-    const unsigned mask = __ballot_sync(0xffffffffu, act);
-    if (act) {
-      int e = a.idx[as];
-      if (e < 0 || e >= E) {
-        record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 100);
-        e = 0;
+  // ---- local ranks.  With at most kRegIters 32-wide steps per warp the
+  // expert ids and ranks stay in registers; longer ranges keep the rank in
+  // slot_of until the bases are known.
+  const int iters = (hi - lo + 31) / 32;
+  const bool in_regs = iters <= kRegIters;
+  int e_r[kRegIters], r_r[kRegIters];
+  if (in_regs) {
+    int e_next = (lo + lane < hi) ? __ldg(a.idx + lo + lane) : 0;
+#pragma unroll
+    for (int it = 0; it < kRegIters; ++it) {
+      if (it >= iters) break;  // warp-uniform
+      const int as = lo + 32 * it + lane;
+      const bool act = as < hi;
+      int e = e_next;
+      if (as + 32 < hi) e_next = __ldg(a.idx + as + 32);  // prefetch the next step
+      const unsigned mask = __ballot_sync(0xffffffffu, act);
+      int rk = 0;
+      if (act) {
+        if (e < 0 || e >= E) {
+          record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 100);
+          e = 0;
+        }
+        const unsigned peers = __match_any_sync(mask, e);
+        const int r = __popc(peers & ((1u << lane) - 1u));
+        const int b = cnt[warp][e];
+        __syncwarp(mask);
+        if (r == 0) cnt[warp][e] = b + __popc(peers);
+        rk = b + r;
       }
-      const unsigned peers = __match_any_sync(mask, e);
-      const int r = __popc(peers & ((1u << lane) - 1u));
-      const int b = cnt[warp][e];
-      __syncwarp(mask);
-      if (r == 0) cnt[warp][e] = b + __popc(peers);
-      a.slot_of[as] = b + r;
+      __syncwarp();
+      e_r[it] = e;
+      r_r[it] = rk;
     }
-    __syncwarp();
+  } else {
+    for (int base = lo; base < hi; base += 32) {
+      const int as = base + lane;
+      const bool act = as < hi;
+      const unsigned mask = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        int e = __ldg(a.idx + as);
+        if (e < 0 || e >= E) {
+          record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 100);
+          e = 0;
+        }
+        const unsigned peers = __match_any_sync(mask, e);
+        const int r = __popc(peers & ((1u << lane) - 1u));
+        const int b = cnt[warp][e];
+        __syncwarp(mask);
+        if (r == 0) cnt[warp][e] = b + __popc(peers);
+        a.slot_of[as] = b + r;
+      }
+      __syncwarp();
+    }
   }
   __syncthreads();
 
   // ---- per-expert totals; per-warp bases inside each expert's segment
   if (tid < E) {
     int run = 0;
+#pragma unroll 8
     for (int w = 0; w < kPlanWarps; ++w) {
       const int c = cnt[w][tid];
       cnt[w][tid] = run;
       run += c;
     }
-    off[tid] = run;  // total, scanned below
+    tot[tid] = run;
+    atomicMax(&s_maxc, min(run, a.chunk));
+  }
+  __syncthreads();
+  // ---- exclusive scans of the totals (slots) and of the chunk counts,
+  // warp-level inclusive scans then a scan of the warp sums (E <= 256)
+  {
+    const int n = (tid < E) ? tot[tid] : 0;
+    const int c = (n + a.chunk - 1) / a.chunk;
+    int sn = n, sc = c;
+    if (tid < kMaxE) {
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yn = __shfl_up_sync(0xffffffffu, sn, o);
+        const int yc = __shfl_up_sync(0xffffffffu, sc, o);
+        if (lane >= o) {
+          sn += yn;
+          sc += yc;
+        }
+      }
+      if (lane == 31) {
+        wsum[0][warp] = sn;
+        wsum[1][warp] = sc;
+      }
+    }
+    __syncthreads();
+    if (tid < kMaxE) {
+      int bn = 0, bc = 0;
+      for (int w = 0; w < warp; ++w) {
+        bn += wsum[0][w];
+        bc += wsum[1][w];
+      }
+      if (tid < E) {
+        off[tid + 1] = bn + sn;
+        cst[tid + 1] = bc + sc;
+      }
+      if (tid == 0) {
+        off[0] = 0;
+        cst[0] = 0;
+      }
+    }
   }
   __syncthreads();
   if (tid == 0) {
-    int o = 0, q = 0, mx = 0;
-    for (int e = 0; e < E; ++e) {
-      const int n = off[e];
-      off[e] = o;
-      cst[e] = q;
-      o += n;
-      q += (n + kMaxN - 1) / kMaxN;
-      mx = max(mx, min(n, kMaxN));
-    }
-    off[E] = o;
-    cst[E] = q;
-    a.ctl->n_chunks = q;
-    a.ctl->max_chunk = mx;
+    a.ctl->n_chunks = cst[E];
+    a.ctl->max_chunk = s_maxc;
     a.ctl->work_next = 0;
   }
-  __syncthreads();
   if (tid <= E) a.offsets[tid] = off[tid];
   if (tid < E) {
     for (int q = cst[tid]; q < cst[tid + 1]; ++q) {
@@ -95,61 +166,156 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   }
 
   // ---- final slots
-  for (int as = lo + lane; as < hi; as += 32) {
-    int e = a.idx[as];
-    if (e < 0 || e >= E) e = 0;
-    const int slot = off[e] + cnt[warp][e] + a.slot_of[as];
-    a.slot_of[as] = slot;
-    a.perm[slot] = as / a.k;
+  if (in_regs) {
+#pragma unroll
+    for (int it = 0; it < kRegIters; ++it) {
+      if (it >= iters) break;
+      const int as = lo + 32 * it + lane;
+      if (as < hi) {
+        const int slot = off[e_r[it]] + cnt[warp][e_r[it]] + r_r[it];
+        a.slot_of[as] = slot;
+        a.perm[slot] = as / a.k;
+      }
+    }
+  } else {
+    for (int as = lo + lane; as < hi; as += 32) {
+      int e = __ldg(a.idx + as);
+      if (e < 0 || e >= E) e = 0;
+      const int slot = off[e] + cnt[warp][e] + a.slot_of[as];
+      a.slot_of[as] = slot;
+      a.perm[slot] = as / a.k;
+    }
   }
 }
 
-// x rows in slot order: x_perm[s] = x[perm[s]] (one warp per row, 16-byte moves)
+// x rows in slot order: x_perm[s] = x[perm[s]], or, with gamma2, the
+// expert-side norm bf16(x / sqrt(mean(x^2) + eps) * (1 + gamma2)) of that row
+// (the model's pre-FFN norm, whose only consumer is the fused gate_up).  One
+// warp per row, 16-byte moves, every load of the row issued before any use.
+constexpr int kGatherVec = 16;  // uint4 per lane held in registers (d <= 4096)
+
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= a.rows) return;
   const int t = __ldg(a.perm + row);
   const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d);
   uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (size_t)row * a.d);
-  for (int i = lane; i < a.d / 8; i += 32) dst[i] = __ldg(src + i);
+  const int n = a.d / 8;
+  uint4 v[kGatherVec];
+#pragma unroll
+  for (int j = 0; j < kGatherVec; ++j)
+    if (lane + 32 * j < n) v[j] = __ldg(src + lane + 32 * j);
+  if (a.gamma2) {
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kGatherVec; ++j) {
+      if (lane + 32 * j < n) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h2[q]);
+          ss = fmaf(f.x, f.x, ss);
+          ss = fmaf(f.y, f.y, ss);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = 1.0f / sqrtf(ss / (float)a.d + a.eps);
+    const float4* g4 = reinterpret_cast<const float4*>(a.gamma2);
+#pragma unroll
+    for (int j = 0; j < kGatherVec; ++j) {
+      const int i = lane + 32 * j;
+      if (i < n) {
+        const float4 ga = __ldg(g4 + 2 * i), gb = __ldg(g4 + 2 * i + 1);
+        const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[j]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h2[q]);
+          h2[q] = __floats2bfloat162_rn((f.x * inv) * (1.f + g[2 * q]),
+                                        (f.y * inv) * (1.f + g[2 * q + 1]));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kGatherVec; ++j)
+    if (lane + 32 * j < n) dst[lane + 32 * j] = v[j];
 }
 
-// out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32)
-__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+// out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32, one
+// rounding).  One CTA per token; each thread owns up to kCombCols float4
+// columns and issues all k loads of a column before accumulating.
+constexpr int kCombThreads = 256;
+constexpr int kCombCols = 3;   // 3 * 256 * 4 >= 2816; larger d loops
+constexpr int kCombK = 8;      // loads in flight per column
+
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   __shared__ int sl[kMaxK];
   __shared__ float wt[kMaxK];
+  pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   if (threadIdx.x < a.k) {
     sl[threadIdx.x] = a.slot_of[(size_t)t * a.k + threadIdx.x];
     wt[threadIdx.x] = a.w[(size_t)t * a.k + threadIdx.x];
   }
   __syncthreads();
-  for (int i = threadIdx.x * 4; i < a.d; i += blockDim.x * 4) {
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < a.k; ++j) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(a.y + (size_t)sl[j] * a.d + i));
-      const float wj = wt[j];
-      s.x = fmaf(wj, v.x, s.x);
-      s.y = fmaf(wj, v.y, s.y);
-      s.z = fmaf(wj, v.z, s.z);
-      s.w = fmaf(wj, v.w, s.w);
+  const int nc4 = a.d / 4;
+  for (int c0 = threadIdx.x; c0 < nc4; c0 += kCombThreads * kCombCols) {
+    float4 acc[kCombCols];
+#pragma unroll
+    for (int c = 0; c < kCombCols; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < a.k; j0 += kCombK) {
+      float4 v[kCombCols][kCombK];
+#pragma unroll
+      for (int c = 0; c < kCombCols; ++c) {
+        const int col = c0 + c * kCombThreads;
+#pragma unroll
+        for (int j = 0; j < kCombK; ++j)
+          if (col < nc4 && j0 + j < a.k)
+            v[c][j] = __ldg(reinterpret_cast<const float4*>(a.y + (size_t)sl[j0 + j] * a.d) + col);
+      }
+#pragma unroll
+      for (int c = 0; c < kCombCols; ++c) {
+#pragma unroll
+        for (int j = 0; j < kCombK; ++j) {
+          if (j0 + j < a.k) {
+            const float wj = wt[j0 + j];
+            acc[c].x = fmaf(wj, v[c][j].x, acc[c].x);
+            acc[c].y = fmaf(wj, v[c][j].y, acc[c].y);
+            acc[c].z = fmaf(wj, v[c][j].z, acc[c].z);
+            acc[c].w = fmaf(wj, v[c][j].w, acc[c].w);
+          }
+        }
+      }
     }
-    if (a.residual) {
-      const uint2 r = *reinterpret_cast<const uint2*>(a.residual + (size_t)t * a.d + i);
-      const float2 r0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-      const float2 r1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-      s.x = r0.x + s.x;
-      s.y = r0.y + s.y;
-      s.z = r1.x + s.z;
-      s.w = r1.y + s.w;
+#pragma unroll
+    for (int c = 0; c < kCombCols; ++c) {
+      const int col = c0 + c * kCombThreads;
+      if (col >= nc4) continue;
+      float4 s4 = acc[c];
+      const size_t o = (size_t)t * a.d + 4 * col;
+      if (a.residual) {
+        const uint2 r = *reinterpret_cast<const uint2*>(a.residual + o);
+        const float2 r0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+        const float2 r1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+        s4.x = r0.x + s4.x;
+        s4.y = r0.y + s4.y;
+        s4.z = r1.x + s4.z;
+        s4.w = r1.y + s4.w;
+      }
+      __nv_bfloat162 o0 = __floats2bfloat162_rn(s4.x, s4.y);
+      __nv_bfloat162 o1 = __floats2bfloat162_rn(s4.z, s4.w);
+      uint2 ov;
+      ov.x = *reinterpret_cast<uint32_t*>(&o0);
+      ov.y = *reinterpret_cast<uint32_t*>(&o1);
+      *reinterpret_cast<uint2*>(a.out + o) = ov;
     }
-    __nv_bfloat162 o0 = __floats2bfloat162_rn(s.x, s.y);
-    __nv_bfloat162 o1 = __floats2bfloat162_rn(s.z, s.w);
-    uint2 o;
-    o.x = *reinterpret_cast<uint32_t*>(&o0);
-    o.y = *reinterpret_cast<uint32_t*>(&o1);
-    *reinterpret_cast<uint2*>(a.out + (size_t)t * a.d + i) = o;
   }
 }
 
@@ -157,19 +323,17 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
 
 }  // namespace moe
 
-cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s) {
-  moe::plan_kernel<<<1, moe::kPlanThreads, 0, s>>>(a);
-  return cudaGetLastError();
+cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s, bool pdl) {
+  return moe::launch_pdl(moe::plan_kernel, dim3(1), dim3(moe::kPlanThreads), 0, s, pdl, a);
 }
 
-cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s) {
+cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl) {
   if (a.rows == 0) return cudaSuccess;
-  moe::gather_kernel<<<(a.rows + 7) / 8, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  static_assert(moe::kGatherVec * 32 * 8 >= 4096, "gather holds a whole row in registers");
+  return moe::launch_pdl(moe::gather_kernel, dim3((a.rows + 7) / 8), dim3(256), 0, s, pdl, a);
 }
 
-cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s) {
+cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s, bool pdl) {
   if (a.T == 0) return cudaSuccess;
-  moe::combine_kernel<<<a.T, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return moe::launch_pdl(moe::combine_kernel, dim3(a.T), dim3(moe::kCombThreads), 0, s, pdl, a);
 }

@@ -1,0 +1,366 @@
+// router_tc.cu -- the MoE router on tcgen05 tensor cores (E <= 128).
+//
+// Same result as the FFMA router (router.cu): the router's own (1+gamma)
+// RMSNorm of the raw residual, fp32 logits against router_w (+ bias),
+// softmax, top-k with the lower index winning ties, renormalised weights
+// (Quant-Tuner pull request "Add DiffusionGemma (Gemma-4 MoE block-diffusion)
+// support", "Answers to the motivating questions"; top-8 of 128 from its
+// Summary).
+//
+// Exactness of the tensor-core logits: the logit is
+//   z_e = (sum_i x_i * W'_ei) / rms(x),  W'_ei = router_w[e][i] * (1 + gamma_i)
+// with x already bf16.  W' (fp32, 24-bit significand) is split exactly into
+// three bf16 terms hi + mid + lo (each captures the next 8 bits), so every
+// product x_i * part is exact in fp32 and the UMMA accumulates in fp32: the
+// logits carry fp32 accumulation error only, as an FFMA dot product would.
+//
+// Work split: a CTA owns 128 tokens (UMMA M) x all experts (UMMA N = E
+// rounded up to 16) over a slice of the hidden dimension; the 8 (or fewer)
+// CTAs that share a token tile form a cluster along the hidden dimension.
+// Each accumulates its partial logits in TMEM (plus the partial sum of x^2,
+// read from the staged x tiles), writes them to its smem, and after a
+// cluster barrier rank r sums its ceil(128 / cluster) tokens over the
+// cluster in rank order (deterministic), then one warp per token runs the
+// top-k.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace moe {
+
+namespace {
+
+constexpr int kTThreads = 192;   // producer, UMMA, 4 epilogue warps
+constexpr int kTM = 128;         // tokens per CTA
+constexpr int kTStages = 3;
+constexpr int kXTile = kTM * kBK * 2;          // 16 KB
+constexpr int kMaxEP = 128;                    // experts (N) handled here
+constexpr int kWTile = kMaxEP * kBK * 2;       // 16 KB per split part
+constexpr int kTStage = kXTile + 3 * kWTile;   // 64 KB
+constexpr int kPartStride = kMaxEP + 1;        // floats per token row of a partial
+constexpr int kMaxCluster = 8;
+constexpr int kTSmem = 1024 + kTStages * kTStage + 1024;
+static_assert((kTM * kPartStride + kTM + kTM * kMaxEP + kTM) * 4 <= kTStages * kTStage,
+              "partials and reduced logits reuse the ring");
+
+// W'[e][i] = router_w[e][i] * (1 + gamma[i]) split into three bf16 parts,
+// wsplit[p][e][i], rows e >= E zero.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ rw,
+                                                           const float* __restrict__ gamma, int E,
+                                                           int EP, int d,
+                                                           __nv_bfloat16* __restrict__ wsplit) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t n = (size_t)EP * d;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int e = (int)(i / d);
+    const int k = (int)(i - (size_t)e * d);
+    float v = 0.f;
+    if (e < E) v = __ldg(rw + i) * (1.f + __ldg(gamma + k));
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    wsplit[i] = hi;
+    wsplit[n + i] = mid;
+    wsplit[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
+__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+__global__ void __launch_bounds__(kTThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                     const __grid_constant__ CUtensorMap tm_w, RouterArgs a, int EP, int nsplit) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  // After the main loop the ring is reused: partial logits, partial x^2,
+  // then this rank's reduced logits (kept apart from what other ranks read).
+  float* part = reinterpret_cast<float*>(smem);          // [kTM][kPartStride]
+  float* ssq = part + kTM * kPartStride;                  // [kTM]
+  float* zall = ssq + kTM;                                // [kTM][kMaxEP] (this rank's rows)
+  float* inv_rms = zall + kTM * kMaxEP;                   // [kTM]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTStages * kTStage);
+  uint64_t* empty = full + kTStages;
+  uint64_t* sqd = empty + kTStages;   // x tile's sum of squares taken
+  uint64_t* tfull = sqd + kTStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rank = blockIdx.y;  // K slice == rank in the cluster
+  const int t0 = blockIdx.x * kTM;
+  const int nst = a.d / kBK;
+  const int kb0 = rank * nst / nsplit;
+  const int kb1 = (rank + 1) * nst / nsplit;
+  const uint64_t timeout_ns = 1000000000ull;
+  Ctl* ctl = a.ctl;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&sqd[i], 4);
+    }
+    mbar_init(tfull, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kMaxEP);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // x and the split weight come from earlier kernels
+  pdl_launch_dependents();
+
+  float my_ssq = 0.f;
+  if (warp == 0) {
+    if (lane == 0) {  // ---------------------------------------------- producer
+      const uint64_t pol = l2_policy_evict_last();
+      const uint32_t tx = kXTile + 3 * EP * kBK * 2;
+      uint32_t issued = 0, par = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const int i = kb - kb0;
+        const int st = i % kTStages;
+        // refill only after the UMMAs and the x^2 readers are done with it
+        if (i >= kTStages &&
+            (!mbar_wait(&empty[st], ((i / kTStages) - 1) & 1, s_abort, ctl, timeout_ns, 401) ||
+             !mbar_wait(&sqd[st], ((i / kTStages) - 1) & 1, s_abort, ctl, timeout_ns, 406)))
+          break;
+        uint8_t* sx = ring + st * kTStage;
+        mbar_arrive_expect_tx(&full[st], tx);
+        tma_load_2d(sx, &tm_x, kb * kBK, t0, &full[st], pol);
+        for (int p = 0; p < 3; ++p)
+          tma_load_2d(sx + kXTile + p * kWTile, &tm_w, kb * kBK, p * EP, &full[st], pol);
+        issued |= 1u << st;
+        par = (par & ~(1u << st)) | ((uint32_t)((i / kTStages) & 1) << st);
+      }
+      for (int st = 0; st < kTStages; ++st) {  // drain
+        if (!((issued >> st) & 1u)) continue;
+        const uint32_t b = smem_u32(&full[st]);
+        const uint64_t tq = globaltimer_ns();
+        while (!mbar_try_wait(b, (par >> st) & 1u))
+          if (globaltimer_ns() - tq > timeout_ns) {
+            record_error(ctl, MOE_ERR_TIMEOUT, 402);
+            break;
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---------------------------------------------- UMMA issuer
+      const uint32_t idesc = idesc_bf16_f32(kTM, EP);
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const int i = kb - kb0;
+        const int st = i % kTStages;
+        if (!mbar_wait(&full[st], (i / kTStages) & 1, s_abort, ctl, timeout_ns, 403)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sx = smem_u32(ring + st * kTStage);
+#pragma unroll
+        for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+#pragma unroll
+          for (int p = 0; p < 3; ++p)
+            umma_bf16(tmem_base, sdesc_k_sw128(sx + kk * kUmmaK * 2),
+                      sdesc_k_sw128(sx + kXTile + p * kWTile + kk * kUmmaK * 2), idesc,
+                      (i | kk | p) ? 1u : 0u);
+        umma_commit(&empty[st]);
+      }
+      umma_commit(tfull);  // also drains every issued UMMA
+      (void)ok;
+    }
+  } else {
+    // ---------------------------------------------------------- x^2 partials
+    // Each epilogue thread owns one token row of the staged x tiles (128-byte
+    // swizzled rows): 16-byte chunk c of row r sits at chunk c ^ (r % 8).
+    const int r = (warp & 3) * 32 + lane;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      const int i = kb - kb0;
+      const int st = i % kTStages;
+      if (!mbar_wait(&full[st], (i / kTStages) & 1, s_abort, ctl, timeout_ns, 404)) break;
+      const uint8_t* row = ring + st * kTStage + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 pk = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) * 16));
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&pk);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h2[q]);
+          my_ssq = fmaf(f.x, f.x, my_ssq);
+          my_ssq = fmaf(f.y, f.y, my_ssq);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sqd[st]);
+    }
+  }
+  __syncthreads();
+
+  // ---- partial logits: TMEM -> smem (the ring is free: every UMMA and every
+  // copy has completed once tfull fires)
+  if (warp >= 2) {
+    const bool ok = mbar_wait(tfull, 0, s_abort, ctl, timeout_ns, 405);
+    tc_fence_after();
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    if (ok) {
+      for (int c0 = 0; c0 < EP; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q4 * 32) << 16) + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) part[r * kPartStride + c0 + j] = __uint_as_float(v[j]);
+      }
+    }
+    ssq[r] = my_ssq;
+  }
+  tc_fence_before();
+  cluster.sync();
+
+  // ---- rank r reduces its share of the tile's tokens over the cluster, in
+  // rank order (ceil split: the last rank may take fewer)
+  const int tpr = (kTM + nsplit - 1) / nsplit;
+  const int tb = rank * tpr;
+  const int tcount = max(0, min(tpr, kTM - tb));
+  for (int idx = threadIdx.x; idx < tcount * EP; idx += kTThreads) {
+    const int tl = idx / EP;
+    const int e = idx - tl * EP;
+    float sacc = 0.f;
+    for (int q = 0; q < nsplit; ++q) {
+      const float* rp = cluster.map_shared_rank(part, q);
+      sacc += rp[(tb + tl) * kPartStride + e];
+    }
+    zall[tl * kMaxEP + e] = sacc;
+  }
+  if (threadIdx.x < tcount) {
+    float s2 = 0.f;
+    for (int q = 0; q < nsplit; ++q) s2 += cluster.map_shared_rank(ssq, q)[tb + threadIdx.x];
+    inv_rms[threadIdx.x] = 1.0f / sqrtf(s2 / (float)a.d + a.eps);
+  }
+  cluster.sync();  // remote partials stay alive until every rank has read them
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kMaxEP);
+  }
+
+  // ---- top-k: one warp per token, lane holds experts lane + 32c
+  const int E = a.E;
+  for (int tl = warp; tl < tcount; tl += kTThreads / 32) {
+    const int t = t0 + tb + tl;
+    if (t >= a.T) break;
+    float v[kMaxEP / 32];
+#pragma unroll
+    for (int c = 0; c < kMaxEP / 32; ++c) {
+      const int ee = lane + 32 * c;
+      float z = -INFINITY;
+      if (ee < E) {
+        z = zall[tl * kMaxEP + ee] * inv_rms[tl];
+        if (a.bias) z += __ldg(a.bias + ee);
+        if (z != z) z = -INFINITY;
+      }
+      v[c] = z;
+    }
+    uint32_t taken = 0;
+    float my_sel = -INFINITY;
+    float next_v = -INFINITY;
+    const int rounds = (a.k < E) ? a.k + 1 : a.k;
+    for (int j = 0; j < rounds; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int c = 0; c < kMaxEP / 32; ++c) {
+        const int ee = lane + 32 * c;
+        if (ee < E && !((taken >> c) & 1u) && better(v[c], ee, bv, bi)) {
+          bv = v[c];
+          bi = ee;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if (j < a.k) {
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (lane == j) my_sel = bv;
+        if (lane == 0) a.idx[(size_t)t * a.k + j] = bi;
+      } else {
+        next_v = bv;
+      }
+    }
+    const float top = __shfl_sync(0xffffffffu, my_sel, 0);
+    const float ex = (lane < a.k) ? expf(my_sel - top) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < a.k) a.w[(size_t)t * a.k + lane] = ex / sum;
+    const float last = __shfl_sync(0xffffffffu, my_sel, a.k - 1);
+    if (lane == 0 && a.gap) a.gap[t] = (a.k < E) ? (last - next_v) : INFINITY;
+  }
+}
+
+}  // namespace
+
+}  // namespace moe
+
+int moe_router_tc_splits(int d) {
+  const int nst = d / moe::kBK;
+  return nst < moe::kMaxCluster ? nst : moe::kMaxCluster;
+}
+
+cudaError_t moe_launch_router_split(const float* rw, const float* gamma, int E, int EP, int d,
+                                    __nv_bfloat16* wsplit, int num_sms, cudaStream_t s,
+                                    bool pdl) {
+  const size_t n = (size_t)EP * d;
+  int blocks = (int)((n + 255) / 256);
+  if (blocks > 4 * num_sms) blocks = 4 * num_sms;
+  return moe::launch_pdl(moe::router_split_kernel, dim3(blocks), dim3(256), 0, s, pdl, rw, gamma,
+                         E, EP, d, wsplit);
+}
+
+cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x,
+                                 const CUtensorMap& tm_w, int EP, cudaStream_t s, bool pdl) {
+  const int nsplit = moe_router_tc_splits(a.d);
+  cudaError_t err = cudaFuncSetAttribute(moe::router_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         moe::kTSmem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.T + moe::kTM - 1) / moe::kTM, nsplit, 1);
+  cfg.blockDim = dim3(moe::kTThreads, 1, 1);
+  cfg.dynamicSmemBytes = moe::kTSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = nsplit;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, moe::router_tc_kernel, tm_x, tm_w, a, EP, nsplit);
+}

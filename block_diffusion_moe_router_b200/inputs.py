@@ -13,7 +13,8 @@ per-expert intermediate 704, symmetric int4 weights in groups of 128):
   canvas4  T=256,  d=2816, E=128, k=8, f=704, int4 w4g128 weights + fp16 scales
   encode   T=2048, d=2816, E=128, k=8, f=704, bf16 weights (prompt + canvas)
   stack30  30 layers of `canvas`, distinct weights, Zipf(1.1)-skewed router bias,
-           residual carried between layers
+           residual carried between layers, experts reading the (1+gamma2)
+           RMSNorm of x (the model's pre-FFN norm; gamma2 ~ N(0, 0.1^2))
 
 Distributions: x ~ N(0,1) rounded to bf16; router W ~ N(0, 1/d) (variance 1/d,
 so logits have unit scale) in fp32; gamma ~ N(0, 0.1^2) in fp32; expert weights
@@ -25,6 +26,7 @@ Layouts (all row-major, contiguous):
   router_w     [E, d]            fp32
   router_gamma [d]               fp32 (applied as 1 + gamma)
   router_bias  [E]               fp32 or None
+  expert_gamma [d]               fp32 or None (experts read rmsnorm(x)*(1+gamma2))
   w_gate_up    [E, 2f, d]        bf16 (rows [0,f) gate, [f,2f) up)
                [E, 2f, d/2]      uint8 for int4 (element i in byte i/2, low
                                  nibble for even i, 4-bit two's complement)
@@ -59,6 +61,7 @@ class Workload:
     layers: int = 1
     zipf_s: float = 0.0   # > 0: router bias drawn so expert load is Zipf(s)-skewed
     residual: bool = False
+    expert_norm: bool = False  # experts read the (1+gamma2) RMSNorm of x
     act_wid: Optional[int] = None  # take x / router tensors from another workload's seeds
 
     @property
@@ -77,11 +80,12 @@ WORKLOADS = {
                         wdtype=WDTYPE_INT4, act_wid=1),
     "encode": Workload("encode", 3, T=2048, d=2816, E=128, k=8, f=704),
     "stack30": Workload("stack30", 4, T=256, d=2816, E=128, k=8, f=704,
-                        layers=30, zipf_s=1.1, residual=True),
+                        layers=30, zipf_s=1.1, residual=True, expert_norm=True),
 }
 
 # tensor ids inside the seed formula
-_TID_X, _TID_RW, _TID_GAMMA, _TID_WGU, _TID_WD, _TID_SGU, _TID_SD, _TID_BIAS = range(8)
+(_TID_X, _TID_RW, _TID_GAMMA, _TID_WGU, _TID_WD, _TID_SGU, _TID_SD, _TID_BIAS,
+ _TID_EGAMMA) = range(9)
 
 
 def seed_for(wid: int, layer: int, tensor_id: int) -> int:
@@ -157,6 +161,8 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T: Optional[int] = Non
                                  torch.float32)
     out["router_bias"] = (zipf_bias(w.E, w.zipf_s, seed_for(w.wid, layer, _TID_BIAS), device)
                           if w.zipf_s > 0 else None)
+    out["expert_gamma"] = (_randn((w.d,), 0.1, seed_for(w.wid, layer, _TID_EGAMMA), device,
+                                  torch.float32) if w.expert_norm else None)
     if w.wdtype == WDTYPE_BF16:
         out["w_gate_up"] = _randn((w.E, 2 * w.f, w.d), 0.02, seed_for(w.wid, layer, _TID_WGU),
                                   device, torch.bfloat16)
@@ -175,7 +181,7 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T: Optional[int] = Non
 
 
 def make_small(T, d, E, k, f, seed, wdtype=WDTYPE_BF16, bias=False, residual=False,
-               device="cpu", w_std=0.02, gamma_std=0.1) -> dict:
+               device="cpu", w_std=0.02, gamma_std=0.1, expert_norm=False) -> dict:
     """A small random layer of arbitrary shape for tests (same distributions)."""
     base = 100000 + 1000 * seed
     out = {
@@ -184,6 +190,8 @@ def make_small(T, d, E, k, f, seed, wdtype=WDTYPE_BF16, bias=False, residual=Fal
         "router_gamma": _randn((d,), gamma_std, base + 3, device, torch.float32),
         "router_bias": _randn((E,), 1.0, base + 4, device, torch.float32) if bias else None,
         "residual": _randn((T, d), 1.0, base + 5, device, torch.bfloat16) if residual else None,
+        "expert_gamma": (_randn((d,), gamma_std, base + 10, device, torch.float32)
+                         if expert_norm else None),
     }
     if wdtype == WDTYPE_BF16:
         out["w_gate_up"] = _randn((E, 2 * f, d), w_std, base + 6, device, torch.bfloat16)

@@ -19,10 +19,11 @@
  *
  * For each token t (x_t bf16 [d]):
  *   u   = x_t / sqrt(mean(x_t^2) + eps) * (1 + gamma)
+ *   xe  = x_t, or bf16(x_t / sqrt(mean(x_t^2) + eps) * (1 + expert_gamma))
  *   z_e = router_w[e] . u (+ router_bias[e])            fp32
  *   S   = the k largest z_e, ties to the lower index; j order = (z desc, e asc)
  *   w_j = softmax(z)[S_j] / sum_j' softmax(z)[S_j']
- *   h   = gelu_tanh(Wgu[S_j][0:f] x_t) * (Wgu[S_j][f:2f] x_t)   (bf16 h)
+ *   h   = gelu_tanh(Wgu[S_j][0:f] xe) * (Wgu[S_j][f:2f] xe)     (bf16 h)
  *   y_j = Wd[S_j] h                                              (fp32 y)
  *   out_t = residual_t + sum_j w_j y_j  (j order, fp32, one rounding to bf16)
  *
@@ -72,18 +73,27 @@ enum {
   MOE_OPT_EPS = 0,        /* RMSNorm epsilon (default 1e-6)                        */
   MOE_OPT_TIMEOUT_MS = 1, /* bound of every device-side wait, ms (default 1000)    */
   MOE_OPT_PROFILE = 2,    /* 1: moe_forward records CUDA events around each kernel */
-  MOE_OPT_TEST_STALL = 3  /* test hook: 1 makes the expert kernel wait on a flag
+  MOE_OPT_TEST_STALL = 3, /* test hook: 1 makes the expert kernel wait on a flag
                              nothing sets, so the bounded wait runs out and the
                              call reports MOE_ERR_TIMEOUT (no trap, no hang)     */
+  MOE_OPT_PDL = 4,        /* 1 (default): launch each kernel with programmatic
+                             dependent launch so it overlaps the previous one's
+                             tail; 0: plain stream-ordered launches              */
+  MOE_OPT_ROUTER_FFMA = 6, /* 1: use the FFMA router even when E <= 128 (default 0:
+                             tensor-core router for E <= 128, FFMA above)       */
+  MOE_OPT_L2_PREFETCH_MB = 5 /* MiB of the gate_up weight (from its start) the
+                             router pulls into L2 while routing runs, so the
+                             expert kernel's first wave finds it there
+                             (default 0 = off)                                   */
 };
 
 /* Kernels of one moe_forward, for moe_plan_profile. */
 enum {
-  MOE_K_ROUTER = 0,   /* norm + logits + softmax + top-k          */
-  MOE_K_PLAN = 1,     /* histogram + scan + stable permutation    */
-  MOE_K_GATHER = 2,   /* x rows in expert order                   */
-  MOE_K_EXPERT = 3,   /* grouped gate_up(+GELU*up) and down GEMMs */
-  MOE_K_COMBINE = 4,  /* weighted k-order sum (+ residual)        */
+  MOE_K_ROUTER = 0,   /* norm + logits + softmax + top-k                         */
+  MOE_K_PLAN = 1,     /* histogram + scan + stable permutation                   */
+  MOE_K_GATHER = 2,   /* x rows in slot order                                    */
+  MOE_K_EXPERT = 3,   /* grouped gate_up(+GELU*up) and down GEMMs               */
+  MOE_K_COMBINE = 4,  /* weighted k-order sum (+ residual)                       */
   MOE_K_COUNT = 5
 };
 
@@ -107,6 +117,12 @@ moe_status_t moe_plan_reserve(moe_plan_t plan, int max_T);
  *   router_w       fp32 [E,d]
  *   router_gamma   fp32 [d]    (applied as 1 + gamma)
  *   router_bias    fp32 [E] or NULL
+ *   expert_gamma   fp32 [d] or NULL: the experts then read the expert-side
+ *                  RMSNorm x / sqrt(mean(x^2) + eps) * (1 + expert_gamma)
+ *                  (rounded to bf16), the model's pre-FFN norm whose only
+ *                  consumer is the fused gate_up (Quant-Tuner pull request,
+ *                  "Answers to the motivating questions"); NULL: raw x.
+ *                  The router and the residual always see the raw x.
  *   w_gate_up      see moe_wdtype_t (rows [0,f) gate, [f,2f) up)
  *   w_down         see moe_wdtype_t
  *   scales_gate_up fp16 [E,2f,ceil(d/128)]  (int4 plans; must be NULL for bf16)
@@ -117,7 +133,7 @@ moe_status_t moe_plan_reserve(moe_plan_t plan, int max_T);
  * until the next call. */
 moe_status_t moe_forward(moe_plan_t plan, int T, const void* x, const float* router_w,
                          const float* router_gamma, const float* router_bias,
-                         const void* w_gate_up, const void* w_down, const void* scales_gate_up,
+                         const float* expert_gamma, const void* w_gate_up, const void* w_down, const void* scales_gate_up,
                          const void* scales_down, const void* residual, void* out, void* stream);
 
 /* moe_forward with x, residual and out in HOST memory (pinned or pageable):
@@ -126,7 +142,7 @@ moe_status_t moe_forward(moe_plan_t plan, int T, const void* x, const float* rou
  * tensors are device pointers as in moe_forward. */
 moe_status_t moe_forward_host(moe_plan_t plan, int T, const void* x_host, const float* router_w,
                               const float* router_gamma, const float* router_bias,
-                              const void* w_gate_up, const void* w_down,
+                              const float* expert_gamma, const void* w_gate_up, const void* w_down,
                               const void* scales_gate_up, const void* scales_down,
                               const void* residual_host, void* out_host, void* stream);
 
@@ -147,8 +163,8 @@ moe_status_t moe_forward_host(moe_plan_t plan, int T, const void* x_host, const 
  * __device__ array of MOE_NOALLOC_SCRATCH_BYTES; the call never calls
  * cudaMalloc, cudaFree or any allocating routine.
  *   - Limit: the intermediates of T tokens must fit the array (about
- *     T*k*(6d + 2f) + T*(8k + 4) bytes plus small tables; one 256-token
- *     canvas of the 2816/704/128/top-8 layer needs 37.5 MB).  A larger call
+ *     T*k*(6d + 2f) + T*(16k + 4) bytes plus small tables; one
+ *     256-token canvas of the 2816/704/128/top-8 layer needs 37.5 MB).  A larger call
  *     returns MOE_ERR_UNSUPPORTED and launches nothing.
  *   - Set-up: the first call on each device (with that device current) looks
  *     up the array's device address once; make that first call before any
@@ -163,7 +179,7 @@ moe_status_t moe_forward_host(moe_plan_t plan, int T, const void* x_host, const 
  *     moe_forward); MOE_OPT_PROFILE is ignored. */
 moe_status_t moe_forward_noalloc(moe_plan_t plan, int T, const void* x, const float* router_w,
                                  const float* router_gamma, const float* router_bias,
-                                 const void* w_gate_up, const void* w_down,
+                                 const float* expert_gamma, const void* w_gate_up, const void* w_down,
                                  const void* scales_gate_up, const void* scales_down,
                                  const void* residual, void* out, int32_t* status_out,
                                  void* stream);

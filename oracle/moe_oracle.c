@@ -27,7 +27,9 @@
  *    w_j = p[S_j] / sum_{j'} p[S_j'];  gap = z_(k) - z_(k+1);
  *  - gated form: out = down(gelu_tanh(gate(x)) * up(x)), gate = rows [0,f)
  *    of the fused gate_up weight, up = rows [f,2f);
- *  - the experts read x as given (any expert-side pre-norm is the caller's);
+ *  - the experts read x as given, or, with an expert gamma, the expert-side
+ *    (1+gamma2) RMSNorm of x ([QT] Answers: pre_feedforward_layernorm_2 is
+ *    the only consumer of the fused gate_up; the router does not see it);
  *  - RMSNorm: u_i = x_i / sqrt(mean_i x_i^2 + eps) * (1 + gamma_i);
  *  - router bias (optional) is added to the logits before the softmax;
  *  - int4: element i of a row sits in byte i/2, low nibble for even i, 4-bit
@@ -242,15 +244,17 @@ void oracle_route(int T, int E, int k, int d, const uint16_t* x, const float* ro
 
 /* The whole layer for T tokens, one token at a time over its k selected
  * experts.  forced_idx [T,k] (or NULL) replaces the selected set S (the j
- * order is then the given order); residual [T,d] bf16 (or NULL) is added.
+ * order is then the given order); residual [T,d] bf16 (or NULL) is added;
+ * expert_gamma [d] (or NULL) applies the expert-side (1+gamma2) RMSNorm to
+ * the experts' input (the residual is still the raw x).
  * Outputs: out [T,d] (double), idx [T,k], w [T,k], gap [T] (NULL allowed
  * for w and gap). */
 void oracle_moe_forward(int T, int E, int k, int d, int f, int wdtype, const uint16_t* x,
                         const float* router_w, const float* gamma, const float* bias,
-                        double eps, const void* w_gu, const void* w_d, const uint16_t* s_gu,
-                        const uint16_t* s_d, const uint16_t* residual,
-                        const int32_t* forced_idx, double* out, int32_t* idx_out,
-                        double* w_out, double* gap_out) {
+                        const float* expert_gamma, double eps, const void* w_gu,
+                        const void* w_d, const uint16_t* s_gu, const uint16_t* s_d,
+                        const uint16_t* residual, const int32_t* forced_idx, double* out,
+                        int32_t* idx_out, double* w_out, double* gap_out) {
 #pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_get_threads())
   for (int t = 0; t < T; t++) {
     double* xs = (double*)malloc(sizeof(double) * (size_t)d);
@@ -262,6 +266,11 @@ void oracle_moe_forward(int T, int E, int k, int d, int f, int wdtype, const uin
     double gap = 0.0;
     route_token(E, k, d, x + (size_t)t * d, router_w, gamma, bias, eps,
                 forced_idx ? forced_idx + (size_t)t * k : NULL, xs, u, z, idx, w, &gap);
+    /* the experts' input: x itself, or its expert-side (1+gamma2) RMSNorm */
+    if (expert_gamma) {
+      oracle_rmsnorm_plus_one(d, xs, expert_gamma, eps, u);
+      memcpy(xs, u, sizeof(double) * (size_t)d);
+    }
     double* o = out + (size_t)t * d;
     for (int m = 0; m < d; m++)
       o[m] = residual ? bf16_to_double(residual[(size_t)t * d + m]) : 0.0;

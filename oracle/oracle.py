@@ -52,8 +52,8 @@ def lib():
             L.oracle_select_topk.argtypes = [I, I, P, P, P]
             L.oracle_route_weights.argtypes = [I, I, P, P, P]
             L.oracle_route.argtypes = [I, I, I, I, P, P, P, P, D, P, P, P, P]
-            L.oracle_moe_forward.argtypes = [I, I, I, I, I, I, P, P, P, P, D, P, P, P, P, P, P,
-                                             P, P, P, P]
+            L.oracle_moe_forward.argtypes = [I, I, I, I, I, I, P, P, P, P, P, D, P, P, P, P, P,
+                                             P, P, P, P, P]
             L.oracle_expert_ffn.argtypes = [I, I, I, P, P, P, P, I, P, P, P]
             L.oracle_weight_row.argtypes = [I, P, P, I, I, I, I, P]
             L.oracle_decode_bf16.argtypes = [I, P, P]
@@ -152,8 +152,9 @@ def route(x, router_w, router_gamma, router_bias, k: int, eps: float = 1e-6):
 
 def moe_forward(x, router_w, router_gamma, router_bias, w_gate_up, w_down, k: int,
                 scales_gate_up=None, scales_down=None, residual=None, forced_idx=None,
-                eps: float = 1e-6):
-    """The whole layer: (out [T,d] float64, idx [T,k], w [T,k], gap [T])."""
+                eps: float = 1e-6, expert_gamma=None):
+    """The whole layer: (out [T,d] float64, idx [T,k], w [T,k], gap [T]).
+    expert_gamma (or None): the experts read rmsnorm(x) * (1 + expert_gamma)."""
     x = _np(x)
     rw = _np(router_w, np.float32)
     g = _np(router_gamma, np.float32)
@@ -164,6 +165,7 @@ def moe_forward(x, router_w, router_gamma, router_bias, w_gate_up, w_down, k: in
     sd = _np(scales_down)
     res = _np(residual)
     fi = _np(forced_idx, np.int32)
+    eg = _np(expert_gamma, np.float32)
     T, d = x.shape
     E = rw.shape[0]
     wdtype = W_INT4 if wgu.dtype == np.uint8 else W_BF16
@@ -175,9 +177,9 @@ def moe_forward(x, router_w, router_gamma, router_bias, w_gate_up, w_down, k: in
     idx = np.empty((T, k), np.int32)
     w = np.empty((T, k), np.float64)
     gap = np.empty(T, np.float64)
-    lib().oracle_moe_forward(T, E, k, d, f, wdtype, _p(x), _p(rw), _p(g), _p(b), float(eps),
-                             _p(wgu), _p(wd), _p(sgu), _p(sd), _p(res), _p(fi), _p(out),
-                             _p(idx), _p(w), _p(gap))
+    lib().oracle_moe_forward(T, E, k, d, f, wdtype, _p(x), _p(rw), _p(g), _p(b), _p(eg),
+                             float(eps), _p(wgu), _p(wd), _p(sgu), _p(sd), _p(res), _p(fi),
+                             _p(out), _p(idx), _p(w), _p(gap))
     return out, idx, w, gap
 
 

@@ -63,7 +63,8 @@ def oracle_rows_for_sets(lay, k, rows, sets, eps=1e-6):
                                       sub.get("router_bias"), sub["w_gate_up"], sub["w_down"], k,
                                       scales_gate_up=sub.get("scales_gate_up"),
                                       scales_down=sub.get("scales_down"),
-                                      residual=sub.get("residual"), forced_idx=forced, eps=eps)
+                                      residual=sub.get("residual"), forced_idx=forced, eps=eps,
+                                      expert_gamma=sub.get("expert_gamma"))
     return out
 
 

@@ -63,7 +63,7 @@ def test_null_plan_calls_are_rejected(abi):
     lib = abi.lib()
     assert lib.moe_plan_set_option(None, 0, 1e-6) == abi.MOE_ERR_INVALID_ARG
     assert lib.moe_plan_reserve(None, 16) == abi.MOE_ERR_INVALID_ARG
-    assert lib.moe_forward(None, 4, *([None] * 11)) == abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward(None, 4, *([None] * 12)) == abi.MOE_ERR_INVALID_ARG
     assert lib.moe_route(None, 4, *([None] * 8)) == abi.MOE_ERR_INVALID_ARG
     assert lib.moe_plan_sync_status(None, None) == abi.MOE_ERR_INVALID_ARG
     lib.moe_plan_destroy(None)

@@ -7,7 +7,8 @@ import torch
 import oracle
 from block_diffusion_moe_router_b200 import inputs
 import block_diffusion_moe_router_b200 as moe
-from parity_util import (TOL_BF16, check_routing, oracle_rows_for_sets, rel_l2, stable_tables)
+from parity_util import (TOL_BF16, TOL_INT4, check_routing, oracle_rows_for_sets, rel_l2,
+                         stable_tables)
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +28,8 @@ def run_gpu(layer, lay_gpu, T, residual=None, out=None):
     out = layer.forward(x, lay_gpu["router_w"], lay_gpu["router_gamma"], lay_gpu["w_gate_up"],
                         lay_gpu["w_down"], router_bias=lay_gpu.get("router_bias"),
                         scales_gate_up=lay_gpu.get("scales_gate_up"),
-                        scales_down=lay_gpu.get("scales_down"), residual=residual, out=out)
+                        scales_down=lay_gpu.get("scales_down"), residual=residual, out=out,
+                        expert_gamma=lay_gpu.get("expert_gamma"))
     st = layer.sync_status()
     assert st == moe.MOE_OK, moe.moe_status_str(st)
     return out
@@ -38,7 +40,10 @@ def full_check(lay_cpu, lay_gpu, E, k, d, f, rows=None, residual=None, tol=TOL_B
     """Runs route + forward on the GPU and compares with the oracle (all rows
     or the sampled `rows`)."""
     T = lay_gpu["x"].shape[0]
-    layer = moe.MoeLayer(E, k, d, f, lay_gpu.get("wdtype", moe.MOE_W_BF16))
+    int4 = lay_gpu["w_gate_up"].dtype == torch.uint8
+    if int4 and tol == TOL_BF16:
+        tol = TOL_INT4
+    layer = moe.MoeLayer(E, k, d, f, moe.MOE_W_INT4_G128 if int4 else moe.MOE_W_BF16)
     try:
         gidx, gw, ggap = layer.route(lay_gpu["x"], lay_gpu["router_w"], lay_gpu["router_gamma"],
                                      lay_gpu.get("router_bias"))
@@ -56,7 +61,8 @@ def full_check(lay_cpu, lay_gpu, E, k, d, f, rows=None, residual=None, tol=TOL_B
                                              sub["w_down"], k,
                                              scales_gate_up=sub.get("scales_gate_up"),
                                              scales_down=sub.get("scales_down"),
-                                             residual=res_cpu, eps=EPS)
+                                             residual=res_cpu, eps=EPS,
+                                             expert_gamma=sub.get("expert_gamma"))
     _, _, _, z = oracle.route(sub["x"], sub["router_w"], sub["router_gamma"],
                               sub.get("router_bias"), k, eps=EPS)
     gidx_s = gidx.cpu().numpy()[sel]
@@ -76,7 +82,7 @@ def full_check(lay_cpu, lay_gpu, E, k, d, f, rows=None, residual=None, tol=TOL_B
     assert np.all(np.isinf(gg[~fin]))
     np.testing.assert_allclose(gg[fin], ogap[fin], rtol=1e-3, atol=2e-5)
     # routing tables bit-exact (when the sets agree everywhere)
-    if check_tables and rows is None and len(mism) == 0:
+    if check_tables and rows is None and len(mism) == 0 and not int4:
         off, perm, slot_of = stable_tables(oidx, E)
         assert np.array_equal(tables[0], off)
         assert np.array_equal(tables[1], perm)
@@ -106,6 +112,32 @@ def test_canvas_full_layer(canvas):
     w, lay_cpu, lay_gpu = canvas
     err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f)
     print("canvas rel-L2", err)
+
+
+@pytest.mark.parametrize("ffma", [0, 1])
+def test_router_paths_canvas(canvas, ffma):
+    """Both routers (tensor-core split-bf16 logits, FFMA fp32 logits) on the
+    canvas: exact indices on unflagged tokens, weights and gaps close."""
+    w, lay_cpu, lay_gpu = canvas
+    layer = moe.MoeLayer(w.E, w.k, w.d, w.f)
+    try:
+        moe.moe_plan_set_option(layer.plan, moe.MOE_OPT_ROUTER_FFMA, ffma)
+        gidx, gw, ggap = layer.route(lay_gpu["x"], lay_gpu["router_w"], lay_gpu["router_gamma"])
+        assert layer.sync_status() == moe.MOE_OK
+    finally:
+        layer.close()
+    oidx, ow, ogap, z = oracle.route(lay_cpu["x"], lay_cpu["router_w"], lay_cpu["router_gamma"],
+                                     None, w.k, eps=EPS)
+    check_routing(gidx.cpu().numpy(), gw.cpu().numpy(), oidx, ow, ogap, z, w.k)
+    np.testing.assert_allclose(ggap.cpu().numpy(), ogap, rtol=1e-3, atol=2e-5)
+
+
+def test_router_more_than_128_experts():
+    """E = 200 (> 128) takes the FFMA router; top-8 still exact."""
+    T, E, k, d, f = 40, 200, 8, 256, 64
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=200, bias=True)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f)
+    print("E=200 rel-L2", err)
 
 
 def test_canvas_deterministic(canvas):
@@ -156,6 +188,38 @@ def test_stack30_layer_zipf_bias_and_residual():
     print("stack30 layer delta rel-L2", err)
 
 
+def test_canvas4_int4_full_layer():
+    """T=256 canvas with symmetric int4 w4g128 expert weights (fp16 scales):
+    every token against the oracle's exact code * scale arithmetic."""
+    w = inputs.WORKLOADS["canvas4"]
+    lay_gpu = inputs.make_layer(w, device="cuda")
+    lay_cpu = _cpu(lay_gpu)
+    err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f)
+    print("canvas4 int4 rel-L2", err)
+
+
+@pytest.mark.parametrize("T,E,k,d,f,bias", [
+    (17, 16, 2, 256, 64, True),      # f=64: the only K stage of down is half out of bounds
+    (300, 33, 3, 384, 192, False),   # f=192: last group of 64; E not a multiple of 32
+])
+def test_int4_edge_shapes(T, E, k, d, f, bias):
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=T + E + 1, bias=bias,
+                            wdtype=inputs.WDTYPE_INT4)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f)
+    print("int4", (T, E, k, d, f), "rel-L2", err)
+
+
+def test_int4_hot_expert_chunks():
+    """int4 units hold 128 tokens: one expert with 600 tokens spans 5 chunks."""
+    T, E, k, d, f = 600, 16, 2, 256, 128
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=78, bias=True,
+                            wdtype=inputs.WDTYPE_INT4)
+    lay["router_bias"] = torch.zeros(E)
+    lay["router_bias"][3] = 50.0
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f)
+    print("int4 hot expert rel-L2", err)
+
+
 # ------------------------------------------------------------------ edge cases
 
 
@@ -165,11 +229,45 @@ def test_stack30_layer_zipf_bias_and_residual():
     (40, 8, 8, 256, 128, False),     # E == k: every expert used
     (9, 1, 1, 128, 64, False),       # dense gated FFN
     (300, 33, 3, 384, 192, True),    # E not a multiple of 32, f not of 128
+    (2200, 16, 8, 128, 64, False),   # > 16K assignments: plan kernel's long-range path
 ])
 def test_edge_shapes(T, E, k, d, f, bias):
     lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=T + E, bias=bias)
     err, _ = full_check(lay, _cuda(lay), E, k, d, f)
     print((T, E, k, d, f), "rel-L2", err)
+
+
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4])
+def test_expert_side_norm(wd):
+    """Experts read the (1+gamma2) RMSNorm of x (applied while gathering the
+    rows); router and residual see the raw x."""
+    T, E, k, d, f = 70, 16, 4, 384, 128
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=90 + wd, bias=True, residual=True,
+                            expert_norm=True, wdtype=wd)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f, residual=_cuda(lay)["residual"])
+    print("expert norm", wd, "rel-L2", err)
+
+
+def test_awq_fold_invariance_on_gpu():
+    """Per-channel power-of-two scales folded into (1+gamma2) and their
+    inverse into the gate_up columns give bit-identical routing and output."""
+    T, E, k, d, f = 64, 16, 2, 256, 64
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=23, expert_norm=True)
+    lay["expert_gamma"] = torch.round(lay["expert_gamma"] * 256) / 256
+    s = torch.pow(2.0, torch.randint(-3, 4, (d,), generator=torch.Generator().manual_seed(6))
+                  .double())
+    lay2 = dict(lay)
+    lay2["expert_gamma"] = ((1.0 + lay["expert_gamma"].double()) * s - 1.0).float()
+    lay2["w_gate_up"] = (lay["w_gate_up"].double() / s).to(torch.bfloat16)
+    outs = []
+    for ly in (lay, lay2):
+        g = _cuda(ly)
+        layer = moe.MoeLayer(E, k, d, f)
+        try:
+            outs.append(run_gpu(layer, g, T).clone())
+        finally:
+            layer.close()
+    assert torch.equal(outs[0], outs[1])
 
 
 def test_hot_expert_multi_chunk():
@@ -218,7 +316,7 @@ def test_invalid_arguments_launch_nothing():
     layer = moe.MoeLayer(E, k, d, f)
     out = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
     args = [lay["x"], lay["router_w"], lay["router_gamma"], None, lay["w_gate_up"],
-            lay["w_down"], None, None, None, out]
+            lay["w_down"], None, None, None, out]  # expert_gamma passed by keyword (None)
 
     def call(*a, T_=T):
         return moe.moe_forward(layer.plan, T_, *a, check=False)
@@ -266,3 +364,55 @@ def test_bounded_wait_reports_timeout_and_context_survives():
         assert torch.equal(again, good)
     finally:
         layer.close()
+
+
+def test_stack30_denoising_step_teacher_forced():
+    """The 30-layer denoising step (distinct weights, Zipf(1.1)-skewed router
+    bias, residual chained: x_{l+1} = x_l + MoE_l(x_l)).  Every layer is
+    checked teacher-forced: the oracle gets the GPU's bf16 input of that
+    layer, on 16 sampled tokens, and the layer's output delta must match."""
+    w = inputs.WORKLOADS["stack30"]
+    x0 = inputs.make_layer(w, device="cuda")["x"]
+    layer = moe.MoeLayer(w.E, w.k, w.d, w.f)
+    xs = [x0]
+    loads = []
+    try:
+        for l in range(w.layers):
+            lay = inputs.make_layer(w, layer=l, device="cuda", with_x=False)
+            nxt = torch.empty_like(x0)
+            layer.forward(xs[-1], lay["router_w"], lay["router_gamma"], lay["w_gate_up"],
+                          lay["w_down"], router_bias=lay["router_bias"], residual=xs[-1],
+                          out=nxt, expert_gamma=lay["expert_gamma"])
+            off, _, _ = layer.routing_tables(w.T)
+            loads.append((off[1:] - off[:-1]).cpu())
+            xs.append(nxt)
+            del lay
+        assert layer.sync_status() == moe.MOE_OK
+    finally:
+        layer.close()
+    rows = np.random.default_rng(30).choice(w.T, 16, replace=False)
+    worst = 0.0
+    for l in range(w.layers):
+        lay = _cpu(inputs.make_layer(w, layer=l, device="cuda", with_x=False))
+        xin = xs[l].cpu()[rows]
+        ref, oidx, ow, ogap = oracle.moe_forward(xin, lay["router_w"], lay["router_gamma"],
+                                                 lay["router_bias"], lay["w_gate_up"],
+                                                 lay["w_down"], w.k, residual=xin,
+                                                 expert_gamma=lay["expert_gamma"])
+        got = xs[l + 1].cpu()[rows].double().numpy()
+        delta_ref = ref - xin.double().numpy()
+        delta_got = got - xin.double().numpy()
+        # out = bf16(x + delta) is checked with the parity tolerance; the delta
+        # itself carries that one rounding of a value ~5x larger (|x| ~ 1,
+        # |delta| ~ 0.2), so its own rel-L2 is bounded at 2e-2
+        err = rel_l2(got, ref)
+        assert err <= TOL_BF16, f"layer {l}: rel-L2 {err}"
+        derr = rel_l2(delta_got, delta_ref)
+        assert derr <= 2e-2, f"layer {l}: delta rel-L2 {derr}"
+        worst = max(worst, err)
+        del lay
+    # the Zipf-skewed bias concentrates load: the busiest expert of each layer
+    # takes several times the mean share
+    ratio = max(float(c.max()) / float(c.float().mean()) for c in loads)
+    assert ratio > 2.0
+    print("stack30 worst layer rel-L2", worst, "max load / mean", ratio)

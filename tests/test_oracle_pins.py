@@ -40,6 +40,9 @@ def brute_force(lay, k, eps=EPS):
     E = lay["router_w"].shape[0]
     f = lay["w_gate_up"].shape[1] // 2
     u = F.rms_norm(x, (d,), weight=1.0 + lay["router_gamma"].double(), eps=eps)
+    # the experts' input: x, or its expert-side (1+gamma2) RMSNorm
+    xe = x if lay.get("expert_gamma") is None else F.rms_norm(
+        x, (d,), weight=1.0 + lay["expert_gamma"].double(), eps=eps)
     b = lay["router_bias"].double() if lay.get("router_bias") is not None else None
     z = F.linear(u, lay["router_w"].double(), b)
     p = torch.softmax(z, dim=-1)
@@ -58,8 +61,8 @@ def brute_force(lay, k, eps=EPS):
     if lay.get("residual") is not None:
         out += lay["residual"].double()
     for e in range(E):
-        g = F.linear(x, Wgu[e, :f])
-        v = F.linear(x, Wgu[e, f:])
+        g = F.linear(xe, Wgu[e, :f])
+        v = F.linear(xe, Wgu[e, f:])
         h = F.gelu(g, approximate="tanh") * v
         y = F.linear(h, Wd[e])
         out += w[:, e:e + 1] * y
@@ -71,7 +74,8 @@ def run_oracle(lay, k, forced=None):
                               lay.get("router_bias"), lay["w_gate_up"], lay["w_down"], k,
                               scales_gate_up=lay.get("scales_gate_up"),
                               scales_down=lay.get("scales_down"),
-                              residual=lay.get("residual"), forced_idx=forced, eps=EPS)
+                              residual=lay.get("residual"), forced_idx=forced, eps=EPS,
+                              expert_gamma=lay.get("expert_gamma"))
 
 
 def rel(a, b):
@@ -198,16 +202,18 @@ def test_tie_break_duplicated_router_rows():
 # ---------------------------------------------------------------- whole layer
 
 
-@pytest.mark.parametrize("seed,E,k,bias,residual,wd", [
-    (0, 16, 2, False, False, inputs.WDTYPE_BF16),
-    (1, 8, 3, True, True, inputs.WDTYPE_BF16),
-    (2, 16, 4, True, False, inputs.WDTYPE_INT4),
-    (3, 5, 5, False, True, inputs.WDTYPE_INT4),
+@pytest.mark.parametrize("seed,E,k,bias,residual,wd,enorm", [
+    (0, 16, 2, False, False, inputs.WDTYPE_BF16, False),
+    (1, 8, 3, True, True, inputs.WDTYPE_BF16, False),
+    (2, 16, 4, True, False, inputs.WDTYPE_INT4, False),
+    (3, 5, 5, False, True, inputs.WDTYPE_INT4, False),
+    (4, 16, 2, True, True, inputs.WDTYPE_BF16, True),
+    (5, 8, 3, False, False, inputs.WDTYPE_INT4, True),
 ])
-def test_layer_matches_brute_force(seed, E, k, bias, residual, wd):
+def test_layer_matches_brute_force(seed, E, k, bias, residual, wd, enorm):
     d, f = 256, 64
     lay = inputs.make_small(T=9, d=d, E=E, k=k, f=f, seed=seed, wdtype=wd, bias=bias,
-                            residual=residual)
+                            residual=residual, expert_norm=enorm)
     ref, sel, wref, z = brute_force(lay, k)
     out, idx, w, gap = run_oracle(lay, k)
     assert np.array_equal(idx, sel)
@@ -250,6 +256,47 @@ def test_E1_k1_is_dense_gated_gelu_ffn():
                        * F.linear(x, Wgu[:128]), Wd).numpy()
     assert rel(out, ref) < 1e-13
     assert rel(out, swapped) > 1e-2
+
+
+def test_expert_norm_dense_form():
+    """E = k = 1 with the expert-side norm: out = FFN(rms_norm(x) * (1 + g2))
+    (library rms_norm), and the router still reads the raw x."""
+    lay = inputs.make_small(T=5, d=256, E=1, k=1, f=64, seed=21, expert_norm=True)
+    out, idx, w, _ = run_oracle(lay, 1)
+    x = lay["x"].double()
+    xe = F.rms_norm(x, (256,), weight=1.0 + lay["expert_gamma"].double(), eps=EPS)
+    Wgu = lay["w_gate_up"].double()[0]
+    Wd = lay["w_down"].double()[0]
+    ref = F.linear(F.gelu(F.linear(xe, Wgu[:64]), approximate="tanh") * F.linear(xe, Wgu[64:]),
+                   Wd).numpy()
+    assert rel(out, ref) < 1e-13
+    raw = F.linear(F.gelu(F.linear(x, Wgu[:64]), approximate="tanh") * F.linear(x, Wgu[64:]),
+                   Wd).numpy()
+    assert rel(out, raw) > 1e-2
+
+
+def test_awq_fold_invariance():
+    """Folding per-channel scales s into the expert-side norm ((1+g2) * s)
+    and their inverse into the fused gate_up columns (W / s) leaves routing
+    and output unchanged (powers of two keep the bf16 weights exact)."""
+    d, f, E, k = 256, 64, 8, 2
+    lay = inputs.make_small(T=11, d=d, E=E, k=k, f=f, seed=22, expert_norm=True, bias=True)
+    # gamma2 on a 2^-8 grid keeps (1 + gamma2) * s - 1 exact in fp32
+    lay["expert_gamma"] = torch.round(lay["expert_gamma"] * 256) / 256
+    g = torch.Generator().manual_seed(5)
+    s = torch.pow(2.0, torch.randint(-3, 4, (d,), generator=g).double())
+    lay2 = dict(lay)
+    lay2["expert_gamma"] = ((1.0 + lay["expert_gamma"].double()) * s - 1.0).float()
+    # (1 + g2') must equal (1 + g2) * s exactly in fp32 for an exact fold
+    assert torch.equal((1.0 + lay2["expert_gamma"]).double(),
+                       (1.0 + lay["expert_gamma"]).double() * s)
+    lay2["w_gate_up"] = (lay["w_gate_up"].double() / s).to(torch.bfloat16)
+    assert torch.equal(lay2["w_gate_up"].double() * s, lay["w_gate_up"].double())
+    out1, idx1, w1, _ = run_oracle(lay, k)
+    out2, idx2, w2, _ = run_oracle(lay2, k)
+    assert np.array_equal(idx1, idx2)
+    np.testing.assert_array_equal(w1, w2)
+    assert rel(out2, out1) < 1e-13
 
 
 def test_token_permutation_equivariance():

@@ -33,7 +33,7 @@ def _call_noalloc(plan, T, lay, x, out, status):
     P = ctypes.c_void_p
     return _abi.lib().moe_forward_noalloc(
         P(plan), T, P(x.data_ptr()), P(lay["router_w"].data_ptr()),
-        P(lay["router_gamma"].data_ptr()), None, P(lay["w_gate_up"].data_ptr()),
+        P(lay["router_gamma"].data_ptr()), None, None, P(lay["w_gate_up"].data_ptr()),
         P(lay["w_down"].data_ptr()), None, None, None, P(out.data_ptr()),
         P(status.data_ptr()), P(torch.cuda.current_stream().cuda_stream))
 
