@@ -48,7 +48,9 @@ def parse():
     p.add_argument("--sets", type=int, default=0, help="input sets rotated (0: enough to exceed L2)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
-    p.add_argument("--router-ffma", action="store_true", help="FFMA router instead of tensor cores")
+    p.add_argument("--y-bf16", action="store_true", help="keep the expert outputs y in bf16")
+    p.add_argument("--router", choices=["auto", "ffma", "tc"], default="auto",
+                   help="router path (auto: tensor cores from 1024 tokens)")
     p.add_argument("--prefetch-mb", type=int, default=None,
                    help="MiB of gate_up weights pulled into L2 during routing")
     return p.parse_args()
@@ -153,7 +155,8 @@ class ClockSampler:
 
 def layer_costs(w, touched: float, T: int):
     """Algorithmic bytes and FLOPs of one layer call: weights of the experts
-    that receive a token (streamed once), x in, router tensors, out."""
+    that receive a token (streamed once), x in, router tensors, out.  The
+    expert kernel's share is those weights."""
     if w.wdtype == 0:
         wbytes = 3 * w.f * w.d * 2
     else:
@@ -195,14 +198,8 @@ def cpu_baseline(lay_cpu, w, budget_s=12.0):
 # ---------------------------------------------------------------- arms
 
 
-def dist_env():
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return rank, world, local
-
-
 def run_reference(args):
+    from block_diffusion_moe_router_b200.replicas import dist_env
     rank, world, _ = dist_env()
     if rank != 0:
         return
@@ -256,16 +253,13 @@ def run_reference(args):
 
 def run_ours(args):
     import torch
-    import torch.distributed as dist
     import block_diffusion_moe_router_b200 as moe
     from block_diffusion_moe_router_b200 import inputs
+    from block_diffusion_moe_router_b200 import replicas as rep
 
-    rank, world, local = dist_env()
+    rank, world, local = rep.dist_env()
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    rep.init("nccl", torch.device("cuda", local), timeout_s=120)
     w = inputs.WORKLOADS[args.workload]
     T, L = w.T, w.layers
     lays = [inputs.make_layer(w, layer=l, device="cuda", with_x=False) for l in range(L)]
@@ -274,7 +268,7 @@ def run_ours(args):
     # set exceeds L2 on every step
     small = T * w.d * 2 * 2 + (w.E * w.d * 4 + w.d * 4 if L == 1 else 0)
     nsets = args.sets or max(2, math.ceil(1.1 * L2_BYTES / small))
-    xs = [inputs._randn((T, w.d), 1.0, 777000 + 1000 * rank + i, "cuda", torch.bfloat16)
+    xs = [inputs._randn((T, w.d), 1.0, rep.replica_seed(rank, i), "cuda", torch.bfloat16)
           for i in range(nsets)]
     if L == 1:
         rws = [lay["router_w"]] + [lay["router_w"][torch.randperm(w.E, device="cuda")]
@@ -286,9 +280,11 @@ def run_ours(args):
     plan = moe.moe_plan_create(w.E, w.k, w.d, w.f, w.wdtype)
     moe.moe_plan_reserve(plan, T)
     moe.moe_plan_set_option(plan, moe.MOE_OPT_PDL, 0 if args.no_pdl else 1)
-    moe.moe_plan_set_option(plan, moe.MOE_OPT_ROUTER_FFMA, 1 if args.router_ffma else 0)
+    moe.moe_plan_set_option(plan, moe.MOE_OPT_ROUTER,
+                            {"auto": 0, "ffma": 1, "tc": 2}[args.router])
     if args.prefetch_mb is not None:
         moe.moe_plan_set_option(plan, moe.MOE_OPT_L2_PREFETCH_MB, args.prefetch_mb)
+    moe.moe_plan_set_option(plan, moe.MOE_OPT_Y_BF16, 1 if args.y_bf16 else 0)
     stream = torch.cuda.current_stream()
 
     def layer_call(l, x, out, residual, rw=None, gm=None):
@@ -329,29 +325,23 @@ def run_ours(args):
     if st != moe.MOE_OK:
         raise RuntimeError(moe.moe_status_str(st))
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def timed(K, profile):
+    def timed(K, profile, per_step=False):
         moe.moe_plan_set_option(plan, moe.MOE_OPT_PROFILE, 1 if profile else 0)
-        barrier()
+        rep.barrier()
         torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1 if per_step else 2)]
+        ev[0].record(stream)
         for i in range(K):
             step(i)
-        e1.record(stream)
+            if per_step:
+                ev[i + 1].record(stream)
+        ev[-1].record(stream)
         torch.cuda.synchronize()
-        barrier()
-        ms = e0.elapsed_time(e1)
+        rep.barrier()
         moe.moe_plan_set_option(plan, moe.MOE_OPT_PROFILE, 0)
-        if world > 1:
-            t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        if per_step:
+            return [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+        return rep.max_over_ranks(ev[0].elapsed_time(ev[-1]), "cuda")
 
     for i in range(args.warmup):
         step(i)
@@ -365,6 +355,9 @@ def run_ours(args):
         tot, n = moe.moe_plan_profile(plan, kk)
         kern[name] = (tot / n) if n else None
     ms_plain = timed(args.steps, profile=False)
+    per_step = sorted(timed(args.steps, profile=False, per_step=True))
+    pct = {f"p{q}": per_step[min(len(per_step) - 1, int(q / 100 * len(per_step)))]
+           for q in (10, 50, 90)}
     st = moe.moe_plan_sync_status(plan, stream)
     if st != moe.MOE_OK:
         raise RuntimeError(moe.moe_status_str(st))
@@ -373,8 +366,11 @@ def run_ours(args):
     x_host = [xs[i].cpu().pin_memory() for i in range(min(nsets, 4))]
     out_host = torch.empty((T, w.d), dtype=torch.bfloat16).pin_memory()
     K2 = args.steps
-    barrier()
-    t0 = time.perf_counter()
+    rep.barrier()
+    torch.cuda.synchronize()
+    h0 = torch.cuda.Event(enable_timing=True)
+    h1 = torch.cuda.Event(enable_timing=True)
+    h0.record(stream)
     for i in range(K2):
         if L == 1:
             moe.moe_forward_host(plan, T, x_host[i % len(x_host)], rws[0], gms[0],
@@ -385,11 +381,9 @@ def run_ours(args):
             xs[0].copy_(x_host[i % len(x_host)], non_blocking=True)
             out_host.copy_(step(0), non_blocking=True)
             stream.synchronize()
-    e2e_s = time.perf_counter() - t0
-    if world > 1:
-        t = torch.tensor([e2e_s], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    h1.record(stream)
+    torch.cuda.synchronize()
+    e2e_s = rep.max_over_ranks(h0.elapsed_time(h1), "cuda") * 1e-3
     st = moe.moe_plan_sync_status(plan, stream)
     if st != moe.MOE_OK:
         raise RuntimeError(moe.moe_status_str(st))
@@ -416,7 +410,7 @@ def run_ours(args):
     }[w.name]
     line = {
         "metric": METRIC,
-        "value": world * T * args.steps / (ms * 1e-3),
+        "value": rep.job_rate(T, world, args.steps, ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -436,8 +430,11 @@ def run_ours(args):
                   f"{nsets} sets ({nsets * small / 2**20:.0f} MiB)",
             "timed_region": "per-kernel CUDA events recorded inside the timed steps",
             "ms_per_step_without_events": ms_plain / args.steps,
+            "step_ms_percentiles_rank0": pct,
             "pdl": not args.no_pdl,
-            "router": "ffma" if (args.router_ffma or w.E > 128) else "tensor cores",
+            "y_dtype": "bf16" if args.y_bf16 else "fp32",
+            "router": ("tensor cores" if (args.router == "tc" or (args.router == "auto" and T >= 1024))
+                       and w.E <= 128 else "ffma"),
         },
         "roofline": {
             "bound": "hbm", "kernel": "expert (grouped gate_up + down GEMMs)",
@@ -459,7 +456,7 @@ def run_ours(args):
         },
         "kernel_ms": kern,
         "gpu_launches": len(moe.KERNEL_NAMES) * L * args.steps,
-        "e2e": {"value": world * T * K2 / e2e_s, "unit": "tokens/s",
+        "e2e": {"value": rep.job_rate(T, world, K2, e2e_s * 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * w.d * 2, "d2h_bytes_per_step": T * w.d * 2},
         "clocks": clk.summary(),
     }
@@ -474,9 +471,8 @@ def run_ours(args):
         line["cpu_baseline"] = cb
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    rep.barrier()
+    rep.shutdown()
 
 
 def main():

@@ -31,7 +31,8 @@ MOE_OPT_PROFILE = 2
 MOE_OPT_TEST_STALL = 3
 MOE_OPT_PDL = 4
 MOE_OPT_L2_PREFETCH_MB = 5
-MOE_OPT_ROUTER_FFMA = 6
+MOE_OPT_ROUTER = 6
+MOE_OPT_Y_BF16 = 7
 
 MOE_K_ROUTER, MOE_K_PLAN, MOE_K_GATHER, MOE_K_EXPERT, MOE_K_COMBINE = range(5)
 KERNEL_NAMES = ["router", "plan", "gather", "expert", "combine"]

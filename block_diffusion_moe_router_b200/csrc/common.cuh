@@ -143,6 +143,19 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, int
       : "memory");
 }
 
+// One 128-byte line into L2 (fire and forget, through the load/store unit).
+__device__ __forceinline__ void prefetch_l2_line(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
+// Spread the prefetch of [base, base + bytes) over every thread of the grid.
+__device__ __forceinline__ void prefetch_l2_grid(const void* base, uint64_t bytes) {
+  const uint64_t nthr = (uint64_t)gridDim.x * gridDim.y * blockDim.x;
+  const uint64_t tid = ((uint64_t)blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
+  const char* b = static_cast<const char*>(base);
+  for (uint64_t o = tid * 128; o < bytes; o += nthr * 128) prefetch_l2_line(b + o);
+}
+
 // Bring [p, p + bytes) into L2 (bytes a multiple of 16, p 16-byte aligned).
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
@@ -304,7 +317,8 @@ struct CombineArgs {
   int T, k, d;
   const int32_t* slot_of;
   const float* w;
-  const float* y;
+  const void* y;       // fp32 or bf16 [T*k, d]
+  int y_bf16;
   const __nv_bfloat16* residual;
   __nv_bfloat16* out;
 };
@@ -319,7 +333,8 @@ struct ExpertArgs {
   const __half* scales_gu;  // int4: [E, 2f, ceil(d/128)]
   const __half* scales_d;   // int4: [E, d, ceil(f/128)]
   __nv_bfloat16* h;   // [T*k, f]
-  float* y;           // [T*k, d]
+  void* y;            // [T*k, d], fp32 or (y_bf16) bf16
+  int y_bf16;
   Ctl* ctl;
   uint64_t timeout_ns;
   int test_stall;

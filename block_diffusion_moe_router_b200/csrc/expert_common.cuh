@@ -137,15 +137,23 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
           named_barrier(1, 128);
         }
       } else {
-        float* ycol = a.y + (size_t)ui.slot0 * a.d + ui.m * kBM + row;
+        const size_t y0 = (size_t)ui.slot0 * a.d + ui.m * kBM + row;
         for (int cc = 0; cc < nch; ++cc) {
           uint32_t v[32];
           tmem_ld32(tbase + cc * 32, v);
           tmem_wait_ld();
           const int cmax = min(32, ui.n - cc * 32);
+          if (a.y_bf16) {
+            __nv_bfloat16* ycol = static_cast<__nv_bfloat16*>(a.y) + y0;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __uint_as_float(v[i]);
+            for (int i = 0; i < 32; ++i)
+              if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __float2bfloat16(__uint_as_float(v[i]));
+          } else {
+            float* ycol = static_cast<float*>(a.y) + y0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __uint_as_float(v[i]);
+          }
         }
         tc_fence_before();
         __syncwarp();

@@ -5,7 +5,8 @@
 //
 // Same work units, scheduler, B operands and epilogue as the bf16 kernel
 // (expert.cu); what changes is the A operand (the weights):
-//   - TMA brings each 128-wide K stage of packed codes (128 rows x 64 bytes)
+//   - TMA brings each 128-wide K stage of packed codes (128 rows x 64 bytes,
+//     64-byte swizzled so the dequant warps read them without bank conflicts)
 //     into shared memory;
 //   - 8 dequant warps turn the codes into bf16 A values straight in TMEM
 //     (tcgen05.st): per 32-bit word of 8 codes, (code ^ 8) nibbles are placed
@@ -27,7 +28,8 @@ namespace {
 
 constexpr int kThreads = 448;  // producer, UMMA, 4 epilogue, 8 dequant warps
 constexpr int kDqWarp0 = 6;
-constexpr int kDqWarps = 8;
+constexpr int kDqGroups = 2;              // dequant groups, each owning every other stage
+constexpr int kDqWarps = 4 * kDqGroups;   // a group is one warp per TMEM lane quarter
 constexpr int kChunkN = 128;                 // tokens per unit
 constexpr int kBK4 = 128;                    // K per stage = one scale group
 constexpr int kCodeBytes = kBM * kBK4 / 2;   // 8 KB of codes per stage
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  __half* sc = reinterpret_cast<__half*>(smem + kRingBytes);  // [128][kScaleStride]
+  __half* sc = reinterpret_cast<__half*>(smem + kRingBytes);  // [kScaleStride][128]
   float* xchg = reinterpret_cast<float*>(smem + kRingBytes + kScaleBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kScaleBytes + kXchgBytes);
   uint64_t* empty = full + kMaxStages;
@@ -133,10 +135,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMaxStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kDqWarps + 1);  // dequant warps read codes, UMMA reads B
+      mbar_init(&empty[i], 4 + 1);  // one dequant group reads codes, UMMA reads B
     }
     for (int i = 0; i < kAStages; ++i) {
-      mbar_init(&afull[i], kDqWarps);
+      mbar_init(&afull[i], 4);
       mbar_init(&aempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -354,11 +356,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                   kChunkN, warp, lane);
   } else {
     // ------------------------------------------------------------ dequant warps
-    const int dw = warp - kDqWarp0;        // 0..7
+    // Group g (one warp per TMEM lane quarter) takes the stages kb with
+    // kb % kDqGroups == g, a whole 128-code row per thread, so the groups
+    // work on different stages at once.  Inside a group the TMEM stores of
+    // one stage stay in flight while the next stage is loaded and decoded;
+    // the stage is signalled full once they have landed.
+    const int dw = warp - kDqWarp0;        // 0..kDqWarps-1
     const int q4 = warp & 3;               // TMEM lane quarter
     const int row = q4 * 32 + lane;        // A row == TMEM lane
-    const int half = dw >> 2;              // which 64 of the stage's 128 codes
-    const int dt = threadIdx.x - kDqWarp0 * 32;  // 0..255
+    const int grp = dw >> 2;
+    const int dt = threadIdx.x - kDqWarp0 * 32;
+    const int sw = (row >> 1) & 3;
     int stage = 0;
     uint32_t phase = 0;
     int ast = 0;
@@ -386,39 +394,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wrow = gu ? (ui.e * 2 * a.f + (r < kGuHalf ? 0 : a.f) + ui.m * kGuHalf +
                                (r & (kGuHalf - 1)))
                             : (ui.e * a.d + ui.m * kBM + r);
-        sc[r * kScaleStride + g] = sg[(size_t)wrow * G + g];
+        sc[g * kBM + r] = sg[(size_t)wrow * G + g];  // group-major: conflict-free reads
       }
       named_barrier(2, kDqWarps * 32);
       bool sok = true;
+      bool pend = false;
+      int pend_ast = 0;
       for (int kb = 0; kb < G; ++kb) {
-        if (sok) {
+        if (kb % kDqGroups == grp && sok) {
           sok = mbar_wait(&full[stage], phase, s_abort, ctl, a.timeout_ns, kWhereDqFull) &&
                 mbar_wait(&aempty[ast], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty);
-        }
-        if (sok) {
-          const uint8_t* codes = ring + stage * stage_bytes + row * (kBK4 / 2) + half * 32;
-          const uint4 c0 = *reinterpret_cast<const uint4*>(codes);
-          const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[stage]);  // codes are in registers
-          const float sf = __half2float(sc[row * kScaleStride + kb]);
-          const __nv_bfloat162 s2 = __float2bfloat162_rn(sf);
-          uint32_t v[32];
-          dequant8(c0.x, s2, v + 0);
-          dequant8(c0.y, s2, v + 4);
-          dequant8(c0.z, s2, v + 8);
-          dequant8(c0.w, s2, v + 12);
-          dequant8(c1.x, s2, v + 16);
-          dequant8(c1.y, s2, v + 20);
-          dequant8(c1.z, s2, v + 24);
-          dequant8(c1.w, s2, v + 28);
-          const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) +
-                              (uint32_t)(kAColBase + ast * kACols + half * 32);
-          tmem_st32(ta, v);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&afull[ast]);
+          if (sok) {
+            // codes tile: 64-byte rows written by TMA with 64-byte swizzling,
+            // i.e. 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
+            const uint8_t* crow = ring + stage * stage_bytes + row * (kBK4 / 2);
+            uint4 cw[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              cw[c] = *reinterpret_cast<const uint4*>(crow + ((c ^ sw) << 4));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);  // codes are in registers
+            const float sf = __half2float(sc[kb * kBM + row]);
+            const __nv_bfloat162 s2 = __float2bfloat162_rn(sf);
+            const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) +
+                                (uint32_t)(kAColBase + ast * kACols);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t v[32];
+              dequant8(cw[2 * h].x, s2, v + 0);
+              dequant8(cw[2 * h].y, s2, v + 4);
+              dequant8(cw[2 * h].z, s2, v + 8);
+              dequant8(cw[2 * h].w, s2, v + 12);
+              dequant8(cw[2 * h + 1].x, s2, v + 16);
+              dequant8(cw[2 * h + 1].y, s2, v + 20);
+              dequant8(cw[2 * h + 1].z, s2, v + 24);
+              dequant8(cw[2 * h + 1].w, s2, v + 28);
+              if (h == 0 && pend) {  // the previous stage's stores have landed
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&afull[pend_ast]);
+                pend = false;
+              }
+              tmem_st32(ta + h * 32, v);
+            }
+            pend = true;
+            pend_ast = ast;
+          }
         }
         if (++stage == S) {
           stage = 0;
@@ -428,6 +450,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ast = 0;
           aph ^= 1;
         }
+      }
+      if (pend) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[pend_ast]);
       }
       named_barrier(2, kDqWarps * 32);  // sc[] is rewritten only after every warp is done
       if (lane == 0) mbar_arrive(&uempty[ur]);

@@ -34,7 +34,8 @@ struct moe_plan_s {
   int test_stall;
   int pdl;
   int prefetch_mb;
-  int router_ffma;
+  int y_bf16;
+  int router_sel;
   int cap_T;
   int last_T;
   void* ws;  // one device allocation holding everything below
@@ -107,7 +108,7 @@ bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -130,13 +131,19 @@ int max_chunks(int E, int T, int k) { return E + (T * k) / 128 + 1; }
 // Experts rounded up to the UMMA N granularity for the tensor-core router.
 int router_ep(int E) { return (E + 15) / 16 * 16; }
 
-bool use_router_tc(moe_plan_t p) { return !p->router_ffma && p->E <= 128; }
+// Router path: the tensor-core router needs E <= 128; automatic selection
+// takes it from 1024 tokens up, where its split-K GEMM outruns the FFMA
+// router (below that both are latency-bound and the FFMA one is shorter).
+bool use_router_tc(moe_plan_t p, int T) {
+  if (p->E > 128 || p->router_sel == 1) return false;
+  return p->router_sel == 2 || T >= 1024;
+}
 
 // The router weight times (1 + gamma), split into three bf16 parts.
 size_t wsplit_bytes(moe_plan_t p) { return (size_t)3 * router_ep(p->E) * p->d * 2; }
 
 // 2-D byte tensor map over packed int4 codes [rows, cols_bytes]: box = box_rows
-// x 64 bytes (one group of 128 codes), no swizzle.
+// x 64 bytes (one group of 128 codes), 64-byte swizzle.
 bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols_bytes,
                     uint32_t box_rows);
 
@@ -275,7 +282,7 @@ moe_status_t launch_router(moe_plan_t p, int T, const void* x, const float* rw,
   ra.l2_prefetch = pf_bytes ? pf : nullptr;
   ra.l2_prefetch_bytes = pf_bytes;
   const bool pdl = p->pdl != 0;
-  if (use_router_tc(p)) {
+  if (use_router_tc(p, T)) {
     __nv_bfloat16* ws = wsplit ? wsplit : p->wsplit;
     const int EP = router_ep(p->E);
     CUtensorMap tm_x, tm_w;
@@ -338,7 +345,8 @@ moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, mo
   p->test_stall = 0;
   p->pdl = 1;
   p->prefetch_mb = 0;
-  p->router_ffma = 0;
+  p->y_bf16 = 0;
+  p->router_sel = 0;
   p->cap_T = 0;
   p->last_T = 0;
   p->ws = nullptr;
@@ -366,12 +374,16 @@ moe_status_t moe_plan_set_option(moe_plan_t p, int key, double value) {
     case MOE_OPT_PDL:
       p->pdl = value != 0.0;
       return MOE_OK;
-    case MOE_OPT_ROUTER_FFMA:
-      p->router_ffma = value != 0.0;
+    case MOE_OPT_ROUTER:
+      if (!(value == 0.0 || value == 1.0 || value == 2.0)) return MOE_ERR_INVALID_ARG;
+      p->router_sel = (int)value;
       return MOE_OK;
     case MOE_OPT_L2_PREFETCH_MB:
       if (!(value >= 0.0 && value <= 4096.0)) return MOE_ERR_INVALID_ARG;
       p->prefetch_mb = (int)value;
+      return MOE_OK;
+    case MOE_OPT_Y_BF16:
+      p->y_bf16 = value != 0.0;
       return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
@@ -484,6 +496,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ea.ready = p->ready;
   ea.h = p->h;
   ea.y = p->y;
+  ea.y_bf16 = p->y_bf16;
   ea.ctl = p->ctl;
   ea.timeout_ns = (uint64_t)p->timeout_ms * 1000000ull;
   ea.test_stall = p->test_stall;
@@ -504,6 +517,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ca.slot_of = p->slot_of;
   ca.w = p->w;
   ca.y = p->y;
+  ca.y_bf16 = p->y_bf16;
   ca.residual = static_cast<const __nv_bfloat16*>(residual);
   ca.out = static_cast<__nv_bfloat16*>(out);
   {
@@ -776,6 +790,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ea.ready = ready;
   ea.h = h;
   ea.y = y;
+  ea.y_bf16 = p->y_bf16;
   ea.ctl = ctl;
   ea.timeout_ns = (uint64_t)p->timeout_ms * 1000000ull;
   ea.test_stall = p->test_stall;
@@ -792,6 +807,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ca.slot_of = slot_of;
   ca.w = w;
   ca.y = y;
+  ca.y_bf16 = p->y_bf16;
   ca.residual = static_cast<const __nv_bfloat16*>(residual);
   ca.out = static_cast<__nv_bfloat16*>(out);
   if (moe_launch_combine(ca, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;

@@ -50,14 +50,18 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   const bool in_regs = iters <= kRegIters;
   int e_r[kRegIters], r_r[kRegIters];
   if (in_regs) {
-    int e_next = (lo + lane < hi) ? __ldg(a.idx + lo + lane) : 0;
+    // every load of the warp's range in flight before the first use
+#pragma unroll
+    for (int it = 0; it < kRegIters; ++it) {
+      const int as = lo + 32 * it + lane;
+      e_r[it] = (it < iters && as < hi) ? __ldg(a.idx + as) : 0;
+    }
 #pragma unroll
     for (int it = 0; it < kRegIters; ++it) {
       if (it >= iters) break;  // warp-uniform
       const int as = lo + 32 * it + lane;
       const bool act = as < hi;
-      int e = e_next;
-      if (as + 32 < hi) e_next = __ldg(a.idx + as + 32);  // prefetch the next step
+      int e = e_r[it];
       const unsigned mask = __ballot_sync(0xffffffffu, act);
       int rk = 0;
       if (act) {
@@ -248,13 +252,26 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
 }
 
 // out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32, one
-// rounding).  One CTA per token; each thread owns up to kCombCols float4
-// columns and issues all k loads of a column before accumulating.
+// rounding).  One CTA per token; each thread owns up to kCombCols columns of
+// 4 values and issues all k loads of a column before accumulating.  y is fp32
+// or bf16 (widened exactly on load).
 constexpr int kCombThreads = 256;
 constexpr int kCombCols = 3;   // 3 * 256 * 4 >= 2816; larger d loops
 constexpr int kCombK = 8;      // loads in flight per column
 
+__device__ __forceinline__ float4 load_y4(const float* y, size_t i4) {
+  return __ldg(reinterpret_cast<const float4*>(y) + i4);
+}
+__device__ __forceinline__ float4 load_y4(const __nv_bfloat16* y, size_t i4) {
+  const uint2 r = __ldg(reinterpret_cast<const uint2*>(y) + i4);
+  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+template <typename YT>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
+  const YT* y = static_cast<const YT*>(a.y);
   __shared__ int sl[kMaxK];
   __shared__ float wt[kMaxK];
   pdl_wait();
@@ -278,7 +295,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
 #pragma unroll
         for (int j = 0; j < kCombK; ++j)
           if (col < nc4 && j0 + j < a.k)
-            v[c][j] = __ldg(reinterpret_cast<const float4*>(a.y + (size_t)sl[j0 + j] * a.d) + col);
+            v[c][j] = load_y4(y, ((size_t)sl[j0 + j] * a.d) / 4 + col);
       }
 #pragma unroll
       for (int c = 0; c < kCombCols; ++c) {
@@ -335,5 +352,9 @@ cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl
 
 cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s, bool pdl) {
   if (a.T == 0) return cudaSuccess;
-  return moe::launch_pdl(moe::combine_kernel, dim3(a.T), dim3(moe::kCombThreads), 0, s, pdl, a);
+  if (a.y_bf16)
+    return moe::launch_pdl(moe::combine_kernel<__nv_bfloat16>, dim3(a.T), dim3(moe::kCombThreads),
+                           0, s, pdl, a);
+  return moe::launch_pdl(moe::combine_kernel<float>, dim3(a.T), dim3(moe::kCombThreads), 0, s,
+                         pdl, a);
 }

@@ -100,17 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Pull the first wave of expert weights into L2 while routing runs: HBM is
   // otherwise idle until the expert kernel starts.  Safe before the wait: a
   // prefetch only moves lines into the coherent L2.
-  if (a.l2_prefetch && threadIdx.x == kCompWarps * 32) {
-    const uint64_t nct = (uint64_t)gridDim.x * gridDim.y;
-    const uint64_t id = (uint64_t)blockIdx.y * gridDim.x + blockIdx.x;
-    const uint64_t per = ((a.l2_prefetch_bytes + nct - 1) / nct + 15) & ~15ull;
-    const uint64_t beg = id * per;
-    const uint64_t lim = a.l2_prefetch_bytes & ~15ull;
-    const uint64_t end = (beg + per < lim) ? beg + per : lim;
-    const char* base = static_cast<const char*>(a.l2_prefetch);
-    for (uint64_t o = beg; o < end; o += 65536)
-      prefetch_l2_bulk(base + o, (uint32_t)((end - o < 65536) ? end - o : 65536));
-  }
+  if (a.l2_prefetch) prefetch_l2_grid(a.l2_prefetch, a.l2_prefetch_bytes);
   __syncthreads();
   pdl_wait();  // x (and the weights) may come from the previous kernel
   pdl_launch_dependents();

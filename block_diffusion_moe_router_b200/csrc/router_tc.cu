@@ -18,10 +18,10 @@
 // rounded up to 16) over a slice of the hidden dimension; the 8 (or fewer)
 // CTAs that share a token tile form a cluster along the hidden dimension.
 // Each accumulates its partial logits in TMEM (plus the partial sum of x^2,
-// read from the staged x tiles), writes them to its smem, and after a
-// cluster barrier rank r sums its ceil(128 / cluster) tokens over the
-// cluster in rank order (deterministic), then one warp per token runs the
-// top-k.
+// read from the staged x tiles) and pushes every token row to the rank that
+// owns it (ceil(128 / cluster) tokens per rank) with distributed-shared-
+// memory stores; each rank sums its slots in rank order (deterministic) and
+// one warp per token runs the top-k.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -39,11 +39,11 @@ constexpr int kXTile = kTM * kBK * 2;          // 16 KB
 constexpr int kMaxEP = 128;                    // experts (N) handled here
 constexpr int kWTile = kMaxEP * kBK * 2;       // 16 KB per split part
 constexpr int kTStage = kXTile + 3 * kWTile;   // 64 KB
-constexpr int kPartStride = kMaxEP + 1;        // floats per token row of a partial
 constexpr int kMaxCluster = 8;
+constexpr int kRecvRows = kTM + kMaxCluster;   // >= nsplit * ceil(kTM / nsplit)
 constexpr int kTSmem = 1024 + kTStages * kTStage + 1024;
-static_assert((kTM * kPartStride + kTM + kTM * kMaxEP + kTM) * 4 <= kTStages * kTStage,
-              "partials and reduced logits reuse the ring");
+static_assert((kRecvRows * kMaxEP + kRecvRows + kTM * kMaxEP + kTM) * 4 <= kTStages * kTStage,
+              "receive buffers and reduced logits reuse the ring");
 
 // W'[e][i] = router_w[e][i] * (1 + gamma[i]) split into three bf16 parts,
 // wsplit[p][e][i], rows e >= E zero.
@@ -81,12 +81,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  // After the main loop the ring is reused: partial logits, partial x^2,
-  // then this rank's reduced logits (kept apart from what other ranks read).
-  float* part = reinterpret_cast<float*>(smem);          // [kTM][kPartStride]
-  float* ssq = part + kTM * kPartStride;                  // [kTM]
-  float* zall = ssq + kTM;                                // [kTM][kMaxEP] (this rank's rows)
-  float* inv_rms = zall + kTM * kMaxEP;                   // [kTM]
+  // After the main loop the ring is reused: the receive buffer for the
+  // partial logits of this rank's tokens from every rank, their x^2
+  // partials, then this rank's reduced logits.
+  float* recv = reinterpret_cast<float*>(smem);          // [nsplit*tpr <= kRecvRows][kMaxEP]
+  float* recv_ssq = recv + kRecvRows * kMaxEP;            // [kRecvRows]
+  float* zall = recv_ssq + kRecvRows;                     // [tpr][kMaxEP]
+  float* inv_rms = zall + kTM * kMaxEP;                   // [tpr]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTStages * kTStage);
   uint64_t* empty = full + kTStages;
   uint64_t* sqd = empty + kTStages;   // x tile's sum of squares taken
@@ -123,6 +124,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
   }
+  // first-wave expert weights into L2 while routing runs (see router.cu)
+  if (a.l2_prefetch) prefetch_l2_grid(a.l2_prefetch, a.l2_prefetch_bytes);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -166,14 +169,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {  // ---------------------------------------------- UMMA issuer
       const uint32_t idesc = idesc_bf16_f32(kTM, EP);
-      bool ok = true;
       for (int kb = kb0; kb < kb1; ++kb) {
         const int i = kb - kb0;
         const int st = i % kTStages;
-        if (!mbar_wait(&full[st], (i / kTStages) & 1, s_abort, ctl, timeout_ns, 403)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait(&full[st], (i / kTStages) & 1, s_abort, ctl, timeout_ns, 403)) break;
         tc_fence_after();
         const uint32_t sx = smem_u32(ring + st * kTStage);
 #pragma unroll
@@ -186,7 +185,6 @@ __global__ void __launch_bounds__(kTThreads, 1)
         umma_commit(&empty[st]);
       }
       umma_commit(tfull);  // also drains every issued UMMA
-      (void)ok;
     }
   } else {
     // ---------------------------------------------------------- x^2 partials
@@ -215,52 +213,62 @@ __global__ void __launch_bounds__(kTThreads, 1)
   }
   __syncthreads();
 
-  // ---- partial logits: TMEM -> smem (the ring is free: every UMMA and every
-  // copy has completed once tfull fires)
-  if (warp >= 2) {
-    const bool ok = mbar_wait(tfull, 0, s_abort, ctl, timeout_ns, 405);
-    tc_fence_after();
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    if (ok) {
-      for (int c0 = 0; c0 < EP; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q4 * 32) << 16) + c0, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) part[r * kPartStride + c0 + j] = __uint_as_float(v[j]);
-      }
-    }
-    ssq[r] = my_ssq;
-  }
-  tc_fence_before();
-  cluster.sync();
-
-  // ---- rank r reduces its share of the tile's tokens over the cluster, in
-  // rank order (ceil split: the last rank may take fewer)
-  const int tpr = (kTM + nsplit - 1) / nsplit;
+  // ---- partial logits.  Rank r of the cluster owns tokens [r*tpr, r*tpr +
+  // tpr) of the tile.  Every CTA pushes each of its partial rows straight into
+  // the owner's receive buffer with distributed-shared-memory stores (which
+  // pipeline, unlike remote loads), then each rank sums its slots in rank
+  // order.  The first cluster barrier makes sure every CTA is done with its
+  // stage ring (the receive buffers live there) before anyone writes.
+  const int tpr = (kTM + nsplit - 1) / nsplit;  // ceil split: the last rank may take fewer
   const int tb = rank * tpr;
   const int tcount = max(0, min(tpr, kTM - tb));
-  for (int idx = threadIdx.x; idx < tcount * EP; idx += kTThreads) {
-    const int tl = idx / EP;
-    const int e = idx - tl * EP;
-    float sacc = 0.f;
-    for (int q = 0; q < nsplit; ++q) {
-      const float* rp = cluster.map_shared_rank(part, q);
-      sacc += rp[(tb + tl) * kPartStride + e];
+  bool tmem_ok = true;
+  if (warp >= 2) {
+    tmem_ok = mbar_wait(tfull, 0, s_abort, ctl, timeout_ns, 405);
+    tc_fence_after();
+  }
+  cluster.sync();
+  if (warp >= 2) {
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;     // token row of the tile
+    const int owner = r / tpr;
+    const int tl = r - owner * tpr;
+    float* dst = cluster.map_shared_rank(recv, owner) + (size_t)(rank * tpr + tl) * kMaxEP;
+    for (int c0 = 0; c0 < EP; c0 += 32) {
+      uint32_t v[32];
+      tmem_ld32(tmem_base + ((uint32_t)(q4 * 32) << 16) + c0, v);
+      tmem_wait_ld();
+      if (!tmem_ok) {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) v[jj] = 0u;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 32; jj += 4)
+        *reinterpret_cast<float4*>(dst + c0 + jj) =
+            make_float4(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
+                        __uint_as_float(v[jj + 2]), __uint_as_float(v[jj + 3]));
     }
-    zall[tl * kMaxEP + e] = sacc;
+    cluster.map_shared_rank(recv_ssq, owner)[rank * tpr + tl] = my_ssq;
   }
-  if (threadIdx.x < tcount) {
-    float s2 = 0.f;
-    for (int q = 0; q < nsplit; ++q) s2 += cluster.map_shared_rank(ssq, q)[tb + threadIdx.x];
-    inv_rms[threadIdx.x] = 1.0f / sqrtf(s2 / (float)a.d + a.eps);
-  }
-  cluster.sync();  // remote partials stay alive until every rank has read them
+  tc_fence_before();
+  cluster.sync();  // every push has landed
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kMaxEP);
   }
+  for (int idx = threadIdx.x; idx < tcount * EP; idx += kTThreads) {
+    const int tl = idx / EP;
+    const int e = idx - tl * EP;
+    float sacc = 0.f;
+    for (int q = 0; q < nsplit; ++q) sacc += recv[(size_t)(q * tpr + tl) * kMaxEP + e];
+    zall[tl * kMaxEP + e] = sacc;
+  }
+  if (threadIdx.x < tcount) {
+    float s2 = 0.f;
+    for (int q = 0; q < nsplit; ++q) s2 += recv_ssq[q * tpr + threadIdx.x];
+    inv_rms[threadIdx.x] = 1.0f / sqrtf(s2 / (float)a.d + a.eps);
+  }
+  __syncthreads();
 
   // ---- top-k: one warp per token, lane holds experts lane + 32c
   const int E = a.E;

@@ -79,12 +79,16 @@ enum {
   MOE_OPT_PDL = 4,        /* 1 (default): launch each kernel with programmatic
                              dependent launch so it overlaps the previous one's
                              tail; 0: plain stream-ordered launches              */
-  MOE_OPT_ROUTER_FFMA = 6, /* 1: use the FFMA router even when E <= 128 (default 0:
-                             tensor-core router for E <= 128, FFMA above)       */
-  MOE_OPT_L2_PREFETCH_MB = 5 /* MiB of the gate_up weight (from its start) the
+  MOE_OPT_ROUTER = 6,     /* router path: 0 (default) automatic -- tensor cores
+                             when E <= 128 and T >= 1024, FFMA otherwise;
+                             1 FFMA; 2 tensor cores (E <= 128)                   */
+  MOE_OPT_L2_PREFETCH_MB = 5, /* MiB of the gate_up weight (from its start) the
                              router pulls into L2 while routing runs, so the
                              expert kernel's first wave finds it there
                              (default 0 = off)                                   */
+  MOE_OPT_Y_BF16 = 7      /* 1: the per-slot expert outputs y are kept in bf16
+                             (one more rounding before the fp32 combine, half
+                             the bytes); 0 (default): fp32                       */
 };
 
 /* Kernels of one moe_forward, for moe_plan_profile. */

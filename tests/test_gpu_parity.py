@@ -36,15 +36,17 @@ def run_gpu(layer, lay_gpu, T, residual=None, out=None):
 
 
 def full_check(lay_cpu, lay_gpu, E, k, d, f, rows=None, residual=None, tol=TOL_BF16,
-               check_tables=True):
+               check_tables=True, options=None):
     """Runs route + forward on the GPU and compares with the oracle (all rows
-    or the sampled `rows`)."""
+    or the sampled `rows`); `options` are plan options set before the calls."""
     T = lay_gpu["x"].shape[0]
     int4 = lay_gpu["w_gate_up"].dtype == torch.uint8
     if int4 and tol == TOL_BF16:
         tol = TOL_INT4
     layer = moe.MoeLayer(E, k, d, f, moe.MOE_W_INT4_G128 if int4 else moe.MOE_W_BF16)
     try:
+        for key, val in (options or {}).items():
+            moe.moe_plan_set_option(layer.plan, key, val)
         gidx, gw, ggap = layer.route(lay_gpu["x"], lay_gpu["router_w"], lay_gpu["router_gamma"],
                                      lay_gpu.get("router_bias"))
         out = run_gpu(layer, lay_gpu, T, residual=residual)
@@ -114,14 +116,32 @@ def test_canvas_full_layer(canvas):
     print("canvas rel-L2", err)
 
 
-@pytest.mark.parametrize("ffma", [0, 1])
-def test_router_paths_canvas(canvas, ffma):
+def test_canvas_y_bf16(canvas):
+    """Expert outputs kept in bf16 before the combine: same tolerance."""
+    w, lay_cpu, lay_gpu = canvas
+    err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f, options={moe.MOE_OPT_Y_BF16: 1})
+    print("canvas y-bf16 rel-L2", err)
+
+
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4])
+def test_y_bf16_ragged_residual(wd):
+    """bf16 y with a residual, ragged T and both weight formats."""
+    lay = inputs.make_small(T=77, d=384, E=24, k=5, f=192, seed=61, wdtype=wd, bias=True,
+                            residual=True)
+    res = lay.pop("residual")
+    err, _ = full_check(lay, _cuda(lay), 24, 5, 384, 192, residual=res.cuda(),
+                        options={moe.MOE_OPT_Y_BF16: 1})
+    print("ragged y-bf16 rel-L2", err)
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_router_paths_canvas(canvas, path):
     """Both routers (tensor-core split-bf16 logits, FFMA fp32 logits) on the
     canvas: exact indices on unflagged tokens, weights and gaps close."""
     w, lay_cpu, lay_gpu = canvas
     layer = moe.MoeLayer(w.E, w.k, w.d, w.f)
     try:
-        moe.moe_plan_set_option(layer.plan, moe.MOE_OPT_ROUTER_FFMA, ffma)
+        moe.moe_plan_set_option(layer.plan, moe.MOE_OPT_ROUTER, path)
         gidx, gw, ggap = layer.route(lay_gpu["x"], lay_gpu["router_w"], lay_gpu["router_gamma"])
         assert layer.sync_status() == moe.MOE_OK
     finally:
