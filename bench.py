@@ -48,7 +48,8 @@ def parse():
     p.add_argument("--sets", type=int, default=0, help="input sets rotated (0: enough to exceed L2)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-pdl", action="store_true", help="plain stream-ordered launches")
-    p.add_argument("--y-bf16", action="store_true", help="keep the expert outputs y in bf16")
+    p.add_argument("--y-fp32", action="store_true",
+                   help="keep the expert outputs y in fp32 (default bf16)")
     p.add_argument("--router", choices=["auto", "ffma", "tc"], default="auto",
                    help="router path (auto: tensor cores from 1024 tokens)")
     p.add_argument("--prefetch-mb", type=int, default=None,
@@ -284,7 +285,7 @@ def run_ours(args):
                             {"auto": 0, "ffma": 1, "tc": 2}[args.router])
     if args.prefetch_mb is not None:
         moe.moe_plan_set_option(plan, moe.MOE_OPT_L2_PREFETCH_MB, args.prefetch_mb)
-    moe.moe_plan_set_option(plan, moe.MOE_OPT_Y_BF16, 1 if args.y_bf16 else 0)
+    moe.moe_plan_set_option(plan, moe.MOE_OPT_Y_BF16, 0 if args.y_fp32 else 1)
     stream = torch.cuda.current_stream()
 
     def layer_call(l, x, out, residual, rw=None, gm=None):
@@ -432,7 +433,7 @@ def run_ours(args):
             "ms_per_step_without_events": ms_plain / args.steps,
             "step_ms_percentiles_rank0": pct,
             "pdl": not args.no_pdl,
-            "y_dtype": "bf16" if args.y_bf16 else "fp32",
+            "y_dtype": "fp32" if args.y_fp32 else "bf16",
             "router": ("tensor cores" if (args.router == "tc" or (args.router == "auto" and T >= 1024))
                        and w.E <= 128 else "ffma"),
         },

@@ -341,6 +341,65 @@ struct ExpertArgs {
 };
 
 
+// ---------------------------------------------------------------- top-k
+// Order-preserving map of a float to an unsigned key (-0 is folded into +0
+// first, so equal floats get equal keys).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t b = __float_as_uint(f == 0.f ? 0.f : f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Top-k of one token's logits, held C per lane (lane l: experts l + 32c, NaN
+// already mapped to -inf).  Selection order is (logit desc, index asc); each
+// round takes the warp's best by two redux.sync reductions (largest key,
+// then lowest index among the lanes holding it).  Writes idx[j] and the
+// routing weights w[j] = exp(z_j - z_0) / sum (softmax over the selected
+// logits, i.e. the full softmax renormalised over the set), and gap =
+// z_(k) - z_(k+1) (+inf when k == E).
+template <int C>
+__device__ __forceinline__ void warp_topk(const float (&v)[C], int E, int k, int lane,
+                                          int32_t* idx, float* w, float* gap) {
+  uint32_t taken = 0;
+  float my_sel = -INFINITY;
+  float next_v = -INFINITY;
+  const int rounds = (k < E) ? k + 1 : k;
+  for (int j = 0; j < rounds; ++j) {
+    float bv = -INFINITY;
+    int bc = -1;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      const int ee = lane + 32 * c;
+      if (ee < E && !((taken >> c) & 1u) && (bc < 0 || v[c] > bv)) {
+        bv = v[c];
+        bc = c;
+      }
+    }
+    const uint32_t key = (bc < 0) ? 0u : float_key(bv);
+    const uint32_t m = __reduce_max_sync(0xffffffffu, key);
+    const uint32_t cand = (bc >= 0 && key == m) ? (uint32_t)(lane + 32 * bc) : 0xffffffffu;
+    const int bi = (int)__reduce_min_sync(0xffffffffu, cand);
+    const float val = key_float(m);
+    if (j < k) {
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (lane == j) my_sel = val;
+      if (lane == 0) idx[j] = bi;
+    } else {
+      next_v = val;
+    }
+  }
+  const float top = __shfl_sync(0xffffffffu, my_sel, 0);
+  const float ex = (lane < k) ? expf(my_sel - top) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < k) w[lane] = ex / sum;
+  const float last = __shfl_sync(0xffffffffu, my_sel, k - 1);
+  if (lane == 0 && gap) *gap = (k < E) ? (last - next_v) : INFINITY;
+}
+
 // Launch with programmatic stream serialization (when pdl is set) so the
 // kernel's launch and prologue overlap the tail of the previous kernel.
 template <typename... KArgs, typename... Args>
@@ -365,7 +424,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 cudaError_t moe_launch_router(const moe::RouterArgs& a, const CUtensorMap& tm_rw, cudaStream_t s,
                               bool pdl);
 size_t moe_router_smem_bytes(int d);
-int moe_router_tc_splits(int d);
+int moe_router_tc_splits(int d, int T);
 cudaError_t moe_launch_router_split(const float* rw, const float* gamma, int E, int EP, int d,
                                     __nv_bfloat16* wsplit, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x,

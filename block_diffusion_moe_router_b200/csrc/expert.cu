@@ -18,13 +18,18 @@
 // the expert are N (16..256), so every weight byte is streamed from HBM once
 // per chunk, and at 256 tokens per canvas one chunk covers every expert.
 //
-// Roles (192 threads): warp 0 = TMA producer (also the scheduler: it claims
-// units from a global counter), warp 1 = UMMA issuer (owns the TMEM
-// allocation), warps 2..5 = epilogue (TMEM -> registers -> global).  Smem
-// holds a ring of A/B stages sized at run time from the largest chunk; TMEM
+// Roles (224 threads): warp 0 = scheduler (claims units from a global
+// counter) and weight (A) producer, warp 1 = UMMA issuer (owns the TMEM
+// allocation), warps 2..5 = epilogue (TMEM -> registers -> global), warp 6 =
+// activation (B) producer.  Weights and activations have rings of their own,
+// sized at run time from the largest chunk: the weight ring is deep, since
+// its tiles come from HBM and are the bytes the kernel exists to stream,
+// while the activation tiles come from L2.  So the weights of a unit keep
+// streaming while its activations are still being produced: a down unit's
+// W_d tiles are fetched before every gate_up unit of its chunk has published
+// h, and only its h tiles wait (per-chunk counter, acquire/release).  TMEM
 // holds two 256-column fp32 accumulators so the epilogue of one unit overlaps
-// the MMAs of the next.  A down unit may start only when all gate_up units of
-// its chunk have published h (per-chunk counter, acquire/release).
+// the MMAs of the next.
 //
 // Every wait is bounded by %globaltimer; on expiry the kernel records
 // MOE_ERR_TIMEOUT, the roles leave their loops, in-flight TMA copies and
@@ -35,12 +40,14 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kMaxStages = 8;
+constexpr int kThreads = 224;
+constexpr int kMaxA = 12;  // weight stages
+constexpr int kMaxB = 8;   // activation stages
+constexpr int kMinB = 3;
 constexpr int kRingBytes = 200 * 1024;
 constexpr int kXchgBytes = 64 * kXchgStride * 4;  // gate/up exchange rows
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
-constexpr int kBarBytes = 8 * (2 * kMaxStages + 4 + 2 * kUnitRing + 1);
+constexpr int kBarBytes = 8 * (2 * kMaxA + 2 * kMaxB + 4 + 2 * kUnitRing + 1);
 constexpr int kSmemBytes = 1024 + kRingBytes + kXchgBytes + kBarBytes + 256;
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -53,9 +60,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
   float* xchg = reinterpret_cast<float*>(smem + kRingBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kXchgBytes);
-  uint64_t* empty = full + kMaxStages;
-  uint64_t* tfull = empty + kMaxStages;
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + kRingBytes + kXchgBytes);
+  uint64_t* emptyA = fullA + kMaxA;
+  uint64_t* fullB = emptyA + kMaxA;
+  uint64_t* emptyB = fullB + kMaxB;
+  uint64_t* tfull = emptyB + kMaxB;
   uint64_t* tempty = tfull + 2;
   uint64_t* ufull = tempty + 2;
   uint64_t* uempty = ufull + kUnitRing;
@@ -72,9 +81,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   Ctl* ctl = a.ctl;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMaxStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+    for (int i = 0; i < kMaxA; ++i) {
+      mbar_init(&fullA[i], 1);
+      mbar_init(&emptyA[i], 1);
+    }
+    for (int i = 0; i < kMaxB; ++i) {
+      mbar_init(&fullB[i], 1);
+      mbar_init(&emptyB[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
@@ -82,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(&ufull[i], 1);
-      mbar_init(&uempty[i], 2);  // UMMA issuer + epilogue leader
+      mbar_init(&uempty[i], 3);  // UMMA issuer, epilogue leader, B producer
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -106,10 +119,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
 
   // B-operand rows per stage: the largest chunk, rounded up to the TMA box.
+  // The activation ring takes kMinB..kMaxB stages (as many as fit a quarter
+  // of the ring: small chunks get a deep one, to hide L2 latency), the
+  // weights the rest.
   const int maxn = max(1, min(kMaxN, ctl->max_chunk));
   const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
-  const int stage_bytes = kABytes + NB * kBK * 2;
-  const int S = min(kMaxStages, kRingBytes / stage_bytes);
+  const int b_bytes = NB * kBK * 2;
+  const int SB = min(kMaxB, max(kMinB, (kRingBytes / 4) / b_bytes));
+  const int SA = min(kMaxA, (kRingBytes - SB * b_bytes) / kABytes);
+  uint8_t* ringA = ring;
+  uint8_t* ringB = ring + SA * kABytes;
   const int n_chunks = ctl->n_chunks;
   const int U = n_chunks * (GU + DN);
 
@@ -117,7 +136,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     // Lane 0 claims units, waits and issues the copies.
     const uint64_t pol_w = l2_policy_evict_first();
-    const uint64_t pol_act = l2_policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     int ur = 0;
@@ -158,13 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             go = 0;
           }
         }
-        if (go && ui.type == kUnitDown) {
-          const int need = GU + (a.test_stall ? (1 << 30) : 0);
-          if (wait_count(a.ready + ui.q, need, s_abort, ctl, a.timeout_ns, kWhereReady))
-            fence_proxy_async_global();
-          else
-            go = 0;
-        }
         if (go && mbar_wait(&uempty[ur], uphase ^ 1, s_abort, ctl, a.timeout_ns,
                             kWhereUnitEmpty)) {
           units[ur] = ui;
@@ -185,32 +196,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       int ok = 1;
       if (lane == 0) {
         const int nkb = (ui.type == kUnitGateUp) ? a.d / kBK : a.f / kBK;
-        const int nbox = (ui.n + kBRows - 1) / kBRows;
-        const uint32_t tx = kABytes + nbox * kBRows * kBK * 2;
-        const CUtensorMap* tb = (ui.type == kUnitGateUp) ? &tm_xp : &tm_h;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
+          if (!mbar_wait(&emptyA[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
                          kWhereStageEmpty)) {
             ok = 0;
             break;
           }
-          uint8_t* sa = ring + stage * stage_bytes;
-          uint8_t* sb = sa + kABytes;
-          mbar_arrive_expect_tx(&full[stage], tx);
+          uint8_t* sa = ringA + stage * kABytes;
+          mbar_arrive_expect_tx(&fullA[stage], kABytes);
           const int kx = kb * kBK;
           if (ui.type == kUnitGateUp) {
             const int r0 = ui.e * 2 * a.f + ui.m * kGuHalf;
-            tma_load_2d(sa, &tm_wgu, kx, r0, &full[stage], pol_w);
-            tma_load_2d(sa + kGuHalf * kBK * 2, &tm_wgu, kx, r0 + a.f, &full[stage], pol_w);
+            tma_load_2d(sa, &tm_wgu, kx, r0, &fullA[stage], pol_w);
+            tma_load_2d(sa + kGuHalf * kBK * 2, &tm_wgu, kx, r0 + a.f, &fullA[stage], pol_w);
           } else {
-            tma_load_2d(sa, &tm_wd, kx, ui.e * a.d + ui.m * kBM, &full[stage], pol_w);
+            tma_load_2d(sa, &tm_wd, kx, ui.e * a.d + ui.m * kBM, &fullA[stage], pol_w);
           }
-          for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d(sb + bx * kBRows * kBK * 2, tb, kx, ui.slot0 + bx * kBRows, &full[stage],
-                        pol_act);
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == S) {
+          if (++stage == SA) {
             stage = 0;
             phase ^= 1;
           }
@@ -221,14 +225,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // Drain: every issued copy must land before the CTA may exit.
     if (lane == 0)
-      for (int s2 = 0; s2 < S; ++s2)
+      for (int s2 = 0; s2 < SA; ++s2)
         if ((issued >> s2) & 1u)
-          mbar_wait_drain(&full[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
+          mbar_wait_drain(&fullA[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      int sa_i = 0, sb_i = 0;
+      uint32_t pa = 0, pb = 0;
       int ur = 0;
       uint32_t uphase = 0;
       int acc = 0;
@@ -246,21 +250,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t dt = tmem_base + (uint32_t)(acc * kMaxN);
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, s_abort, ctl, a.timeout_ns, kWhereStageFull)) {
+          if (!mbar_wait(&fullA[sa_i], pa, s_abort, ctl, a.timeout_ns, kWhereStageFull) ||
+              !mbar_wait(&fullB[sb_i], pb, s_abort, ctl, a.timeout_ns, kWhereStageFull)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(ring + stage * stage_bytes);
-          const uint32_t sb = sa + kABytes;
+          const uint32_t sa = smem_u32(ringA + sa_i * kABytes);
+          const uint32_t sb = smem_u32(ringB + sb_i * b_bytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk)
             umma_bf16(dt, sdesc_k_sw128(sa + kk * kUmmaK * 2), sdesc_k_sw128(sb + kk * kUmmaK * 2),
                       idesc, (kb | kk) ? 1u : 0u);
-          umma_commit(&empty[stage]);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1;
+          umma_commit(&emptyA[sa_i]);
+          umma_commit(&emptyB[sb_i]);
+          if (++sa_i == SA) {
+            sa_i = 0;
+            pa ^= 1;
+          }
+          if (++sb_i == SB) {
+            sb_i = 0;
+            pb ^= 1;
           }
         }
         if (!ok) break;
@@ -276,6 +286,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Drain: all issued UMMAs complete before TMEM is released.
       umma_commit(drain);
       mbar_wait_drain(drain, 0, ctl, a.timeout_ns);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ B producer
+    // Follows the unit ring; a down unit's h tiles wait for every gate_up
+    // unit of the chunk.
+    if (lane == 0) {
+      const uint64_t pol_act = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int ur = 0;
+      uint32_t uphase = 0;
+      uint32_t issued = 0, issued_par = 0;
+      while (true) {
+        if (!mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullB)) break;
+        const UnitInfo ui = units[ur];
+        if (ui.type == kUnitStop) break;
+        if (ui.type == kUnitDown) {
+          const int need = GU + (a.test_stall ? (1 << 30) : 0);
+          if (!wait_count(a.ready + ui.q, need, s_abort, ctl, a.timeout_ns, kWhereReady)) break;
+          fence_proxy_async_global();
+        }
+        const int nkb = (ui.type == kUnitGateUp) ? a.d / kBK : a.f / kBK;
+        const int nbox = (ui.n + kBRows - 1) / kBRows;
+        const uint32_t tx = nbox * kBRows * kBK * 2;
+        const CUtensorMap* tb = (ui.type == kUnitGateUp) ? &tm_xp : &tm_h;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&emptyB[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
+                         kWhereStageEmpty)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = ringB + stage * b_bytes;
+          mbar_arrive_expect_tx(&fullB[stage], tx);
+          for (int bx = 0; bx < nbox; ++bx)
+            tma_load_2d(sb + bx * kBRows * kBK * 2, tb, kb * kBK, ui.slot0 + bx * kBRows,
+                        &fullB[stage], pol_act);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == SB) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mbar_arrive(&uempty[ur]);
+        if (++ur == kUnitRing) {
+          ur = 0;
+          uphase ^= 1;
+        }
+      }
+      for (int s2 = 0; s2 < SB; ++s2)
+        if ((issued >> s2) & 1u)
+          mbar_wait_drain(&fullB[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
     }
   } else {
     epilogue_role(a, units, ufull, uempty, tfull, tempty, xchg, s_abort, s_bcast, tmem_base,

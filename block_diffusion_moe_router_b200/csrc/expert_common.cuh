@@ -30,7 +30,8 @@ enum {
   kWhereStageFull,
   kWhereUnitFullEpi,
   kWhereTmemFull,
-  kWhereDrain
+  kWhereDrain,
+  kWhereUnitFullB
 };
 
 __device__ __forceinline__ float gelu_tanh(float g) {

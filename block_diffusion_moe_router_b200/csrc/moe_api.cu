@@ -345,7 +345,7 @@ moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, mo
   p->test_stall = 0;
   p->pdl = 1;
   p->prefetch_mb = 0;
-  p->y_bf16 = 0;
+  p->y_bf16 = 1;
   p->router_sel = 0;
   p->cap_T = 0;
   p->last_T = 0;

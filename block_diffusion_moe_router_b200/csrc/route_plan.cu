@@ -7,9 +7,10 @@
 //   fixed-order weighted combine.
 //
 // One CTA of 32 warps does the counting sort: warp w owns a contiguous range
-// of assignments, ranks equal experts inside each 32-wide step with
-// __match_any_sync, and per-(warp, expert) counts are scanned in warp order,
-// so the result is independent of timing (bitwise deterministic).
+// of assignments, ranks equal experts inside each 32-wide step (the lanes
+// with the same id, found with one ballot per id bit), and per-(warp,
+// expert) counts are scanned in warp order, so the result is independent of
+// timing (bitwise deterministic).
 #include "common.cuh"
 
 namespace moe {
@@ -19,8 +20,25 @@ namespace {
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kRegIters = 16;  // 32-wide steps per warp held in registers (16K assignments)
+constexpr int kPermSmem = kPlanWarps * 32 * kRegIters;  // perm staged in smem up to this many
+
+// Lanes of `mask` whose expert id equals this lane's: one ballot per bit of
+// the id (ids < 2^nbits), each narrowing the set to the lanes that agree on
+// that bit.  Cheaper than a match instruction and just as exact.
+__device__ __forceinline__ unsigned peer_lanes(unsigned mask, int e, int nbits) {
+  unsigned peers = mask;
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    if (b < nbits) {
+      const unsigned ones = __ballot_sync(0xffffffffu, (e >> b) & 1);
+      peers &= ((e >> b) & 1) ? ones : ~ones;
+    }
+  }
+  return peers;
+}
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+  extern __shared__ int s_perm[];  // [T*k] when the register path is taken
   __shared__ int cnt[kPlanWarps][kMaxE];  // per-warp counts, then per-warp bases
   __shared__ int tot[kMaxE];
   __shared__ int off[kMaxE + 1];
@@ -32,6 +50,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   const int lane = tid & 31;
   const int E = a.E;
   const int A = a.T * a.k;
+  const int nbits = E > 1 ? 32 - __clz(E - 1) : 0;  // bits of an expert id (E <= 256)
 
   for (int i = tid; i < kPlanWarps * kMaxE; i += kPlanThreads) (&cnt[0][0])[i] = 0;
   if (tid == 0) s_maxc = 0;
@@ -47,7 +66,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   // expert ids and ranks stay in registers; longer ranges keep the rank in
   // slot_of until the bases are known.
   const int iters = (hi - lo + 31) / 32;
-  const bool in_regs = iters <= kRegIters;
+  // uniform over the CTA: A <= kPermSmem gives every warp <= kRegIters steps
+  const bool in_regs = A <= kPermSmem;
   int e_r[kRegIters], r_r[kRegIters];
   if (in_regs) {
     // every load of the warp's range in flight before the first use
@@ -63,13 +83,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
       const bool act = as < hi;
       int e = e_r[it];
       const unsigned mask = __ballot_sync(0xffffffffu, act);
+      if (act && (e < 0 || e >= E)) {
+        record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 100);
+        e = 0;
+      }
+      const unsigned peers = peer_lanes(mask, e, nbits);  // all lanes take part
       int rk = 0;
       if (act) {
-        if (e < 0 || e >= E) {
-          record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 100);
-          e = 0;
-        }
-        const unsigned peers = __match_any_sync(mask, e);
         const int r = __popc(peers & ((1u << lane) - 1u));
         const int b = cnt[warp][e];
         __syncwarp(mask);
@@ -85,13 +105,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
       const int as = base + lane;
       const bool act = as < hi;
       const unsigned mask = __ballot_sync(0xffffffffu, act);
+      int e = act ? __ldg(a.idx + as) : 0;
+      if (act && (e < 0 || e >= E)) {
+        record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 100);
+        e = 0;
+      }
+      const unsigned peers = peer_lanes(mask, e, nbits);  // all lanes take part
       if (act) {
-        int e = __ldg(a.idx + as);
-        if (e < 0 || e >= E) {
-          record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 100);
-          e = 0;
-        }
-        const unsigned peers = __match_any_sync(mask, e);
         const int r = __popc(peers & ((1u << lane) - 1u));
         const int b = cnt[warp][e];
         __syncwarp(mask);
@@ -169,7 +189,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
     }
   }
 
-  // ---- final slots
+  // ---- final slots.  perm is a scatter; on the register path it is built
+  // in shared memory and written out in order (coalesced), since every
+  // store of this single CTA goes through one SM.
   if (in_regs) {
 #pragma unroll
     for (int it = 0; it < kRegIters; ++it) {
@@ -178,9 +200,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
       if (as < hi) {
         const int slot = off[e_r[it]] + cnt[warp][e_r[it]] + r_r[it];
         a.slot_of[as] = slot;
-        a.perm[slot] = as / a.k;
+        s_perm[slot] = as / a.k;
       }
     }
+    __syncthreads();
+    for (int i = tid; i < A; i += kPlanThreads) a.perm[i] = s_perm[i];
   } else {
     for (int as = lo + lane; as < hi; as += 32) {
       int e = __ldg(a.idx + as);
@@ -252,28 +276,41 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
 }
 
 // out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32, one
-// rounding).  One CTA per token; each thread owns up to kCombCols columns of
-// 4 values and issues all k loads of a column before accumulating.  y is fp32
-// or bf16 (widened exactly on load).
+// rounding).  A CTA covers kCombThreads 16-byte column groups of one token
+// (grid: tokens x column blocks), so many small CTAs are resident per SM;
+// each thread issues the loads of up to kCombK contributions before
+// accumulating them.  y is fp32 (4 values per load) or bf16 (8 values per
+// load, widened exactly).
 constexpr int kCombThreads = 256;
-constexpr int kCombCols = 3;   // 3 * 256 * 4 >= 2816; larger d loops
-constexpr int kCombK = 8;      // loads in flight per column
+constexpr int kCombK = 8;  // loads in flight per thread
 
-__device__ __forceinline__ float4 load_y4(const float* y, size_t i4) {
-  return __ldg(reinterpret_cast<const float4*>(y) + i4);
+template <typename YT>
+struct YVec {
+  static constexpr int n = 16 / (int)sizeof(YT);  // values per 16-byte load
+};
+
+__device__ __forceinline__ void widen(const uint4& r, const float*, float (&v)[4]) {
+  v[0] = __uint_as_float(r.x);
+  v[1] = __uint_as_float(r.y);
+  v[2] = __uint_as_float(r.z);
+  v[3] = __uint_as_float(r.w);
 }
-__device__ __forceinline__ float4 load_y4(const __nv_bfloat16* y, size_t i4) {
-  const uint2 r = __ldg(reinterpret_cast<const uint2*>(y) + i4);
-  const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-  const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-  return make_float4(lo.x, lo.y, hi.x, hi.y);
+__device__ __forceinline__ void widen(const uint4& r, const __nv_bfloat16*, float (&v)[8]) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
 }
 
 template <typename YT>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
-  const YT* y = static_cast<const YT*>(a.y);
+  constexpr int V = YVec<YT>::n;
   __shared__ int sl[kMaxK];
   __shared__ float wt[kMaxK];
+  const YT* y = static_cast<const YT*>(a.y);
   pdl_wait();
   pdl_launch_dependents();
   const int t = blockIdx.x;
@@ -282,57 +319,50 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     wt[threadIdx.x] = a.w[(size_t)t * a.k + threadIdx.x];
   }
   __syncthreads();
-  const int nc4 = a.d / 4;
-  for (int c0 = threadIdx.x; c0 < nc4; c0 += kCombThreads * kCombCols) {
-    float4 acc[kCombCols];
+  const int ncol = a.d / V;  // 16-byte column groups per row
+  const int col = blockIdx.y * kCombThreads + threadIdx.x;
+  if (col >= ncol) return;
+  float acc[V];
 #pragma unroll
-    for (int c = 0; c < kCombCols; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < a.k; j0 += kCombK) {
-      float4 v[kCombCols][kCombK];
+  for (int i = 0; i < V; ++i) acc[i] = 0.f;
+  for (int j0 = 0; j0 < a.k; j0 += kCombK) {
+    uint4 r[kCombK];
 #pragma unroll
-      for (int c = 0; c < kCombCols; ++c) {
-        const int col = c0 + c * kCombThreads;
+    for (int j = 0; j < kCombK; ++j)
+      if (j0 + j < a.k)
+        r[j] = __ldg(reinterpret_cast<const uint4*>(y + (size_t)sl[j0 + j] * a.d) + col);
 #pragma unroll
-        for (int j = 0; j < kCombK; ++j)
-          if (col < nc4 && j0 + j < a.k)
-            v[c][j] = load_y4(y, ((size_t)sl[j0 + j] * a.d) / 4 + col);
-      }
+    for (int j = 0; j < kCombK; ++j) {
+      if (j0 + j < a.k) {
+        float v[V];
+        widen(r[j], y, v);
+        const float wj = wt[j0 + j];
 #pragma unroll
-      for (int c = 0; c < kCombCols; ++c) {
-#pragma unroll
-        for (int j = 0; j < kCombK; ++j) {
-          if (j0 + j < a.k) {
-            const float wj = wt[j0 + j];
-            acc[c].x = fmaf(wj, v[c][j].x, acc[c].x);
-            acc[c].y = fmaf(wj, v[c][j].y, acc[c].y);
-            acc[c].z = fmaf(wj, v[c][j].z, acc[c].z);
-            acc[c].w = fmaf(wj, v[c][j].w, acc[c].w);
-          }
-        }
+        for (int i = 0; i < V; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
       }
     }
+  }
+  const size_t o = (size_t)t * a.d + (size_t)V * col;
+  if (a.residual) {
 #pragma unroll
-    for (int c = 0; c < kCombCols; ++c) {
-      const int col = c0 + c * kCombThreads;
-      if (col >= nc4) continue;
-      float4 s4 = acc[c];
-      const size_t o = (size_t)t * a.d + 4 * col;
-      if (a.residual) {
-        const uint2 r = *reinterpret_cast<const uint2*>(a.residual + o);
-        const float2 r0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-        const float2 r1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-        s4.x = r0.x + s4.x;
-        s4.y = r0.y + s4.y;
-        s4.z = r1.x + s4.z;
-        s4.w = r1.y + s4.w;
-      }
-      __nv_bfloat162 o0 = __floats2bfloat162_rn(s4.x, s4.y);
-      __nv_bfloat162 o1 = __floats2bfloat162_rn(s4.z, s4.w);
-      uint2 ov;
-      ov.x = *reinterpret_cast<uint32_t*>(&o0);
-      ov.y = *reinterpret_cast<uint32_t*>(&o1);
-      *reinterpret_cast<uint2*>(a.out + o) = ov;
+    for (int i = 0; i < V; i += 4) {
+      const uint2 rr = *reinterpret_cast<const uint2*>(a.residual + o + i);
+      const float2 r0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rr.x));
+      const float2 r1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rr.y));
+      acc[i] = r0.x + acc[i];
+      acc[i + 1] = r0.y + acc[i + 1];
+      acc[i + 2] = r1.x + acc[i + 2];
+      acc[i + 3] = r1.y + acc[i + 3];
     }
+  }
+#pragma unroll
+  for (int i = 0; i < V; i += 4) {
+    __nv_bfloat162 o0 = __floats2bfloat162_rn(acc[i], acc[i + 1]);
+    __nv_bfloat162 o1 = __floats2bfloat162_rn(acc[i + 2], acc[i + 3]);
+    uint2 ov;
+    ov.x = *reinterpret_cast<uint32_t*>(&o0);
+    ov.y = *reinterpret_cast<uint32_t*>(&o1);
+    *reinterpret_cast<uint2*>(a.out + o + i) = ov;
   }
 }
 
@@ -341,7 +371,15 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
 }  // namespace moe
 
 cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s, bool pdl) {
-  return moe::launch_pdl(moe::plan_kernel, dim3(1), dim3(moe::kPlanThreads), 0, s, pdl, a);
+  // in_regs (every warp's range fits kRegIters steps) <=> T*k <= kPermSmem
+  const int A = a.T * a.k;
+  const size_t smem = A <= moe::kPermSmem ? (size_t)A * sizeof(int) : 0;
+  if (smem > 0) {
+    const cudaError_t err = cudaFuncSetAttribute(
+        moe::plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+  }
+  return moe::launch_pdl(moe::plan_kernel, dim3(1), dim3(moe::kPlanThreads), smem, s, pdl, a);
 }
 
 cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl) {
@@ -352,9 +390,11 @@ cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl
 
 cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s, bool pdl) {
   if (a.T == 0) return cudaSuccess;
+  const int per = a.y_bf16 ? 8 : 4;  // values per 16-byte column group
+  const dim3 grid(a.T, (a.d / per + moe::kCombThreads - 1) / moe::kCombThreads);
   if (a.y_bf16)
-    return moe::launch_pdl(moe::combine_kernel<__nv_bfloat16>, dim3(a.T), dim3(moe::kCombThreads),
-                           0, s, pdl, a);
-  return moe::launch_pdl(moe::combine_kernel<float>, dim3(a.T), dim3(moe::kCombThreads), 0, s,
-                         pdl, a);
+    return moe::launch_pdl(moe::combine_kernel<__nv_bfloat16>, grid, dim3(moe::kCombThreads), 0,
+                           s, pdl, a);
+  return moe::launch_pdl(moe::combine_kernel<float>, grid, dim3(moe::kCombThreads), 0, s, pdl,
+                         a);
 }

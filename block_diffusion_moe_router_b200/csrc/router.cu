@@ -35,15 +35,12 @@ namespace {
 constexpr int kCompWarps = 8;
 constexpr int kThreads = (kCompWarps + 1) * 32;
 constexpr int kChunk = 128;  // hidden columns per stage
-constexpr int kStages = 4;
+constexpr int kMaxStages = 8;
+constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA on sm_100
 constexpr int kExpPerWarp = kRouterTE / kCompWarps;  // 4
 constexpr int kXVec = 16;  // uint4 of an x row per lane (d <= 4096)
 static_assert(kCompWarps == kRouterTT, "one warp per token while staging x");
 static_assert(kRouterTT * kExpPerWarp == 32, "one reduced logit per lane");
-
-__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
-  return v > bv || (v == bv && i < bi);
-}
 
 struct RouterSmem {
   float* us;       // [TT][d]   x * (1 + gamma), fp32
@@ -57,17 +54,29 @@ struct RouterSmem {
   int* abort;
 };
 
-__device__ RouterSmem carve(float* sm, int d) {
+// Floats of everything but the weight ring.
+__host__ __device__ inline int router_fixed_floats(int d) {
+  return kRouterTT * d + d + kRouterTT * kRouterTE + kRouterTT * kMaxE + kRouterTT;
+}
+// Weight-ring depth: as many 16 KB chunks as the rest of shared memory holds
+// (the ring's bytes in flight are what hide the L2 latency), at most 8.
+__host__ __device__ inline int router_stages(int d) {
+  const int avail = kSmemLimit - 1024 - 16 - 2 * kMaxStages * 8 - 4 * router_fixed_floats(d);
+  const int st = avail / (kRouterTE * kChunk * 4);
+  return st < kMaxStages ? st : kMaxStages;
+}
+
+__device__ RouterSmem carve(float* sm, int d, int S) {
   RouterSmem s;
   s.wst = sm;                                      // 1024-aligned (TMA destination)
-  s.us = s.wst + kStages * kRouterTE * kChunk;
+  s.us = s.wst + S * kRouterTE * kChunk;
   s.g1 = s.us + kRouterTT * d;
   s.zloc = s.g1 + d;
   s.zall = s.zloc + kRouterTT * kRouterTE;
   s.inv_rms = s.zall + kRouterTT * kMaxE;
   s.full = reinterpret_cast<uint64_t*>(s.inv_rms + kRouterTT);
-  s.empty = s.full + kStages;
-  s.abort = reinterpret_cast<int*>(s.empty + kStages);
+  s.empty = s.full + kMaxStages;
+  s.abort = reinterpret_cast<int*>(s.empty + kMaxStages);
   return s;
 }
 
@@ -79,7 +88,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        ~uintptr_t(1023));
   const int d = a.d;
   const int E = a.E;
-  RouterSmem s = carve(sm, d);
+  const int S = router_stages(d);
+  RouterSmem s = carve(sm, d, S);
   cg::cluster_group cluster = cg::this_cluster();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -90,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = s.abort;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < S; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], kCompWarps);
     }
@@ -112,18 +122,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol = l2_policy_evict_last();
       uint32_t issued = 0, par = 0;
       for (int c = 0; c < nch; ++c) {
-        const int st = c % kStages;
-        if (c >= kStages &&
-            !mbar_wait(&s.empty[st], ((c / kStages) - 1) & 1, abort, a.ctl, timeout_ns, 301))
+        const int st = c % S;
+        if (c >= S &&
+            !mbar_wait(&s.empty[st], ((c / S) - 1) & 1, abort, a.ctl, timeout_ns, 301))
           break;
         mbar_arrive_expect_tx(&s.full[st], kRouterTE * kChunk * 4);
         tma_load_2d(s.wst + st * kRouterTE * kChunk, &tm_rw, c * kChunk, eg * kRouterTE,
                     &s.full[st], pol);
         issued |= 1u << st;
-        par = (par & ~(1u << st)) | ((uint32_t)((c / kStages) & 1) << st);
+        par = (par & ~(1u << st)) | ((uint32_t)((c / S) & 1) << st);
       }
       // every issued copy lands before the CTA can leave
-      for (int st = 0; st < kStages; ++st) {
+      for (int st = 0; st < S; ++st) {
         if (!((issued >> st) & 1u)) continue;
         const uint32_t b = smem_u32(&s.full[st]);
         const uint64_t t_0 = globaltimer_ns();
@@ -136,6 +146,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- compute warps
+    // this warp's x row: its loads go out first, so they overlap the (1 + gamma)
+    // staging below
+    const int t = t0 + warp;
+    const int n8 = d / 8;  // <= 512
+    uint4 pk[kXVec];
+    if (t < a.T) {
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * d);
+#pragma unroll
+      for (int j = 0; j < kXVec; ++j)
+        if (lane + 32 * j < n8) pk[j] = __ldg(src + lane + 32 * j);
+    }
     {  // (1 + gamma) once for the CTA, every load in flight together
       const float4* g4 = reinterpret_cast<const float4*>(a.gamma);
       for (int i = threadIdx.x; i < d / 4; i += kCompWarps * 32) {
@@ -146,16 +167,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     named_barrier(1, kCompWarps * 32);
     {  // u = x * (1 + gamma) for the token of this warp; 1/rms from x itself
-      const int t = t0 + warp;
       float* row = s.us + warp * d;
       float ss = 0.f;
-      const int n8 = d / 8;  // <= 512
       if (t < a.T) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * d);
-        uint4 pk[kXVec];
-#pragma unroll
-        for (int j = 0; j < kXVec; ++j)
-          if (lane + 32 * j < n8) pk[j] = __ldg(src + lane + 32 * j);
 #pragma unroll
         for (int j = 0; j < kXVec; ++j) {
           const int i = lane + 32 * j;
@@ -188,8 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < kRouterTT * kExpPerWarp; ++i) acc[i] = 0.f;
     for (int c = 0; c < nch; ++c) {
-      const int st = c % kStages;
-      if (!mbar_wait(&s.full[st], (c / kStages) & 1, abort, a.ctl, timeout_ns, 303)) break;
+      const int st = c % S;
+      if (!mbar_wait(&s.full[st], (c / S) & 1, abort, a.ctl, timeout_ns, 303)) break;
       const float* wchunk = s.wst + st * kRouterTE * kChunk;
       float4 wv[kExpPerWarp];
 #pragma unroll
@@ -257,50 +271,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int c = 0; c < kMaxE / 32; ++c) {
     const int ee = lane + 32 * c;
-    v[c] = (ee < E) ? s.zall[warp * E + ee] : -INFINITY;
+    const float z = (ee < E) ? s.zall[warp * E + ee] : -INFINITY;
+    v[c] = (z != z) ? -INFINITY : z;
   }
-  uint32_t taken = 0;
-  float my_sel = -INFINITY;
-  float next_v = -INFINITY;
-  const int rounds = (a.k < E) ? a.k + 1 : a.k;
-  for (int j = 0; j < rounds; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int c = 0; c < kMaxE / 32; ++c) {
-      const int ee = lane + 32 * c;
-      if (ee < E && !((taken >> c) & 1u) && better(v[c], ee, bv, bi)) {
-        bv = v[c];
-        bi = ee;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (better(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (j < a.k) {
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (lane == j) my_sel = bv;
-      if (lane == 0) a.idx[(size_t)t * a.k + j] = bi;
-    } else {
-      next_v = bv;
-    }
-  }
-  // w_j = exp(z_j - z_0) / sum_j' exp(z_j' - z_0): the full softmax restricted
-  // to the selected set and renormalised.
-  const float top = __shfl_sync(0xffffffffu, my_sel, 0);
-  const float ex = (lane < a.k) ? expf(my_sel - top) : 0.f;
-  float sum = ex;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane < a.k) a.w[(size_t)t * a.k + lane] = ex / sum;
-  const float last = __shfl_sync(0xffffffffu, my_sel, a.k - 1);
-  if (lane == 0 && a.gap) a.gap[t] = (a.k < E) ? (last - next_v) : INFINITY;
+  warp_topk(v, E, a.k, lane, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k,
+            a.gap ? a.gap + t : nullptr);
 }
 
 }  // namespace
@@ -308,10 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace moe
 
 size_t moe_router_smem_bytes(int d) {
-  return sizeof(float) * ((size_t)moe::kStages * moe::kRouterTE * moe::kChunk +
-                          (size_t)moe::kRouterTT * d + d + moe::kRouterTT * moe::kRouterTE +
-                          moe::kRouterTT * moe::kMaxE + moe::kRouterTT) +
-         2 * moe::kStages * sizeof(uint64_t) + 16 + 1024;
+  return sizeof(float) * ((size_t)moe::router_stages(d) * moe::kRouterTE * moe::kChunk +
+                          (size_t)moe::router_fixed_floats(d)) +
+         2 * moe::kMaxStages * sizeof(uint64_t) + 16 + 1024;
 }
 
 cudaError_t moe_launch_router(const moe::RouterArgs& a, const CUtensorMap& tm_rw, cudaStream_t s,

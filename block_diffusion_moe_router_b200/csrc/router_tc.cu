@@ -24,6 +24,8 @@
 // one warp per token runs the top-k.
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace cg = cooperative_groups;
@@ -68,10 +70,6 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
     wsplit[n + i] = mid;
     wsplit[2 * n + i] = __float2bfloat16_rn(r2);
   }
-}
-
-__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
-  return v > bv || (v == bv && i < bi);
 }
 
 __global__ void __launch_bounds__(kTThreads, 1)
@@ -256,12 +254,20 @@ __global__ void __launch_bounds__(kTThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, kMaxEP);
   }
-  for (int idx = threadIdx.x; idx < tcount * EP; idx += kTThreads) {
-    const int tl = idx / EP;
-    const int e = idx - tl * EP;
-    float sacc = 0.f;
-    for (int q = 0; q < nsplit; ++q) sacc += recv[(size_t)(q * tpr + tl) * kMaxEP + e];
-    zall[tl * kMaxEP + e] = sacc;
+  // rank-order sums, four experts per thread (EP is a multiple of 16)
+  const int EP4 = EP / 4;
+  for (int idx = threadIdx.x; idx < tcount * EP4; idx += kTThreads) {
+    const int tl = idx / EP4;
+    const int e = 4 * (idx - tl * EP4);
+    float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < nsplit; ++q) {
+      const float4 r = *reinterpret_cast<const float4*>(recv + (size_t)(q * tpr + tl) * kMaxEP + e);
+      sacc.x += r.x;
+      sacc.y += r.y;
+      sacc.z += r.z;
+      sacc.w += r.w;
+    }
+    *reinterpret_cast<float4*>(zall + tl * kMaxEP + e) = sacc;
   }
   if (threadIdx.x < tcount) {
     float s2 = 0.f;
@@ -287,46 +293,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
       }
       v[c] = z;
     }
-    uint32_t taken = 0;
-    float my_sel = -INFINITY;
-    float next_v = -INFINITY;
-    const int rounds = (a.k < E) ? a.k + 1 : a.k;
-    for (int j = 0; j < rounds; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int c = 0; c < kMaxEP / 32; ++c) {
-        const int ee = lane + 32 * c;
-        if (ee < E && !((taken >> c) & 1u) && better(v[c], ee, bv, bi)) {
-          bv = v[c];
-          bi = ee;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (better(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if (j < a.k) {
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == j) my_sel = bv;
-        if (lane == 0) a.idx[(size_t)t * a.k + j] = bi;
-      } else {
-        next_v = bv;
-      }
-    }
-    const float top = __shfl_sync(0xffffffffu, my_sel, 0);
-    const float ex = (lane < a.k) ? expf(my_sel - top) : 0.f;
-    float sum = ex;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane < a.k) a.w[(size_t)t * a.k + lane] = ex / sum;
-    const float last = __shfl_sync(0xffffffffu, my_sel, a.k - 1);
-    if (lane == 0 && a.gap) a.gap[t] = (a.k < E) ? (last - next_v) : INFINITY;
+    warp_topk(v, E, a.k, lane, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k,
+              a.gap ? a.gap + t : nullptr);
   }
 }
 
@@ -334,9 +302,56 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
 }  // namespace moe
 
-int moe_router_tc_splits(int d) {
+namespace {
+
+// Clusters of each size that can be resident at once on this device (a
+// cluster must fit inside one GPC, so the count is not simply SMs / size).
+constexpr int kMaxDevices = 64;
+int g_max_clusters[kMaxDevices][moe::kMaxCluster + 1];
+bool g_max_clusters_ok[kMaxDevices];
+std::mutex g_max_clusters_mu;
+
+int max_active_clusters(int ns) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lock(g_max_clusters_mu);
+  if (!g_max_clusters_ok[dev]) {
+    if (cudaFuncSetAttribute(moe::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             moe::kTSmem) != cudaSuccess)
+      return 0;
+    for (int c = 1; c <= moe::kMaxCluster; ++c) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1, c, 1);
+      cfg.blockDim = dim3(moe::kTThreads, 1, 1);
+      cfg.dynamicSmemBytes = moe::kTSmem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 1;
+      attr.val.clusterDim.y = c;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, moe::router_tc_kernel, &cfg) != cudaSuccess) n = 0;
+      g_max_clusters[dev][c] = n;
+    }
+    g_max_clusters_ok[dev] = true;
+  }
+  return g_max_clusters[dev][ns];
+}
+
+}  // namespace
+
+// Hidden-dimension split (= cluster size): as many as there are K stages up
+// to the cluster limit, lowered while the token tiles would not all be
+// resident in one wave of clusters.
+int moe_router_tc_splits(int d, int T) {
   const int nst = d / moe::kBK;
-  return nst < moe::kMaxCluster ? nst : moe::kMaxCluster;
+  const int cap = nst < moe::kMaxCluster ? nst : moe::kMaxCluster;
+  const int tiles = (T + moe::kTM - 1) / moe::kTM;
+  for (int c = cap; c >= 1; --c)
+    if (tiles <= max_active_clusters(c)) return c;
+  return cap;
 }
 
 cudaError_t moe_launch_router_split(const float* rw, const float* gamma, int E, int EP, int d,
@@ -351,7 +366,7 @@ cudaError_t moe_launch_router_split(const float* rw, const float* gamma, int E, 
 
 cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x,
                                  const CUtensorMap& tm_w, int EP, cudaStream_t s, bool pdl) {
-  const int nsplit = moe_router_tc_splits(a.d);
+  const int nsplit = moe_router_tc_splits(a.d, a.T);
   cudaError_t err = cudaFuncSetAttribute(moe::router_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          moe::kTSmem);

@@ -86,9 +86,9 @@ enum {
                              router pulls into L2 while routing runs, so the
                              expert kernel's first wave finds it there
                              (default 0 = off)                                   */
-  MOE_OPT_Y_BF16 = 7      /* 1: the per-slot expert outputs y are kept in bf16
-                             (one more rounding before the fp32 combine, half
-                             the bytes); 0 (default): fp32                       */
+  MOE_OPT_Y_BF16 = 7      /* 1 (default): the per-slot expert outputs y are kept
+                             in bf16 (one more rounding before the fp32
+                             combine, half the bytes); 0: fp32                   */
 };
 
 /* Kernels of one moe_forward, for moe_plan_profile. */

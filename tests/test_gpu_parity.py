@@ -116,22 +116,23 @@ def test_canvas_full_layer(canvas):
     print("canvas rel-L2", err)
 
 
-def test_canvas_y_bf16(canvas):
-    """Expert outputs kept in bf16 before the combine: same tolerance."""
+def test_canvas_y_fp32(canvas):
+    """Expert outputs kept in fp32 before the combine (the default is bf16)."""
     w, lay_cpu, lay_gpu = canvas
-    err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f, options={moe.MOE_OPT_Y_BF16: 1})
-    print("canvas y-bf16 rel-L2", err)
+    err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f, options={moe.MOE_OPT_Y_BF16: 0})
+    print("canvas y-fp32 rel-L2", err)
 
 
 @pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4])
-def test_y_bf16_ragged_residual(wd):
-    """bf16 y with a residual, ragged T and both weight formats."""
+@pytest.mark.parametrize("ybf16", [0, 1])
+def test_y_dtype_ragged_residual(wd, ybf16):
+    """Both y precisions with a residual, ragged T and both weight formats."""
     lay = inputs.make_small(T=77, d=384, E=24, k=5, f=192, seed=61, wdtype=wd, bias=True,
                             residual=True)
     res = lay.pop("residual")
     err, _ = full_check(lay, _cuda(lay), 24, 5, 384, 192, residual=res.cuda(),
-                        options={moe.MOE_OPT_Y_BF16: 1})
-    print("ragged y-bf16 rel-L2", err)
+                        options={moe.MOE_OPT_Y_BF16: ybf16})
+    print("ragged y-bf16" if ybf16 else "ragged y-fp32", "rel-L2", err)
 
 
 @pytest.mark.parametrize("path", [1, 2])
