@@ -35,6 +35,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "expert_kernel_canvas.txt")
 EXPERT_SOURCES = ["block_diffusion_moe_router_b200/csrc/expert.cu",
+                  "block_diffusion_moe_router_b200/csrc/expert_common.cuh",
                   "block_diffusion_moe_router_b200/csrc/common.cuh"]
 
 
@@ -152,6 +153,18 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
                 "samples": len(self.samples),
                 "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+
+
+def router_on_tensor_cores(w, T: int, router: str) -> bool:
+    """The library's router choice (MOE_OPT_ROUTER): tensor cores for E <= 128
+    when asked, or automatically from T >= 1024."""
+    return w.E <= 128 and (router == "tc" or (router == "auto" and T >= 1024))
+
+
+def launches_per_layer(w, T: int, router: str) -> int:
+    """Kernels one moe_forward launches: router (+ its weight split on the
+    tensor-core path), route plan, gather, expert GEMMs, combine."""
+    return (2 if router_on_tensor_cores(w, T, router) else 1) + 4
 
 
 def layer_costs(w, touched: float, T: int):
@@ -434,8 +447,7 @@ def run_ours(args):
             "step_ms_percentiles_rank0": pct,
             "pdl": not args.no_pdl,
             "y_dtype": "fp32" if args.y_fp32 else "bf16",
-            "router": ("tensor cores" if (args.router == "tc" or (args.router == "auto" and T >= 1024))
-                       and w.E <= 128 else "ffma"),
+            "router": "tensor cores" if router_on_tensor_cores(w, T, args.router) else "ffma",
         },
         "roofline": {
             "bound": "hbm", "kernel": "expert (grouped gate_up + down GEMMs)",
@@ -456,7 +468,7 @@ def run_ours(args):
             "tensor_frac_of_burst_peak": flops / (ms_step * 1e-3) / (bf16 * 1e12),
         },
         "kernel_ms": kern,
-        "gpu_launches": len(moe.KERNEL_NAMES) * L * args.steps,
+        "gpu_launches": launches_per_layer(w, T, args.router) * L * args.steps,
         "e2e": {"value": rep.job_rate(T, world, K2, e2e_s * 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * w.d * 2, "d2h_bytes_per_step": T * w.d * 2},
         "clocks": clk.summary(),

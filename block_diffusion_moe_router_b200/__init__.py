@@ -15,7 +15,7 @@ from ._abi import (  # noqa: F401
     MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_CHECK, MOE_W_BF16, MOE_W_INT4_G128, MOE_OPT_EPS,
     MOE_OPT_TIMEOUT_MS, MOE_OPT_PROFILE, MOE_OPT_TEST_STALL, MOE_OPT_PDL,
     MOE_OPT_L2_PREFETCH_MB, MOE_OPT_ROUTER, MOE_OPT_Y_BF16, MOE_K_ROUTER, MOE_K_PLAN,
-    MOE_K_GATHER, MOE_K_EXPERT, MOE_K_COMBINE, KERNEL_NAMES, MoeError,
+    MOE_K_EXPERT, MOE_K_COMBINE, KERNEL_NAMES, MoeError,
     moe_plan_create, moe_plan_set_option, moe_plan_reserve, moe_forward, moe_forward_host,
     moe_forward_noalloc,
     moe_route, moe_plan_routing, moe_plan_sync_status, moe_plan_profile, moe_plan_destroy,

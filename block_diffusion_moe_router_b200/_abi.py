@@ -34,8 +34,8 @@ MOE_OPT_L2_PREFETCH_MB = 5
 MOE_OPT_ROUTER = 6
 MOE_OPT_Y_BF16 = 7
 
-MOE_K_ROUTER, MOE_K_PLAN, MOE_K_GATHER, MOE_K_EXPERT, MOE_K_COMBINE = range(5)
-KERNEL_NAMES = ["router", "plan", "gather", "expert", "combine"]
+MOE_K_ROUTER, MOE_K_PLAN, MOE_K_EXPERT, MOE_K_COMBINE = range(4)
+KERNEL_NAMES = ["router", "plan_gather", "expert", "combine"]
 
 # Every function include/moe.h declares.
 EXPORTS = [

@@ -465,10 +465,6 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   pa.chunk_c = p->chunk_c;
   pa.ready = p->ready;
   pa.ctl = p->ctl;
-  {
-    ProfScope ps(p, MOE_K_PLAN, s);
-    if (moe_launch_plan(pa, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
-  }
 
   moe::GatherArgs ga;
   ga.rows = A;
@@ -478,9 +474,10 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ga.perm = p->perm;
   ga.x = static_cast<const __nv_bfloat16*>(x);
   ga.x_perm = p->x_perm;
-  {
-    ProfScope ps(p, MOE_K_GATHER, s);
-    if (moe_launch_gather(ga, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
+  {  // one launch (plan + gather) when T*k fits the fused kernel, else two
+    ProfScope ps(p, MOE_K_PLAN, s);
+    if (moe_launch_plan_gather(pa, ga, p->num_sms, s, p->pdl != 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
 
   moe::ExpertArgs ea;
@@ -765,7 +762,6 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   pa.chunk_c = chunk_c;
   pa.ready = ready;
   pa.ctl = ctl;
-  if (moe_launch_plan(pa, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
 
   moe::GatherArgs ga;
   ga.rows = (int)A;
@@ -775,7 +771,8 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ga.perm = perm;
   ga.x = static_cast<const __nv_bfloat16*>(x);
   ga.x_perm = x_perm;
-  if (moe_launch_gather(ga, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe_launch_plan_gather(pa, ga, p->num_sms, s, p->pdl != 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
 
   moe::ExpertArgs ea;
   ea.T = T;

@@ -37,8 +37,10 @@ __device__ __forceinline__ unsigned peer_lanes(unsigned mask, int e, int nbits) 
   return peers;
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
-  extern __shared__ int s_perm[];  // [T*k] when the register path is taken
+// The counting sort.  A `writer` CTA stores the tables (offsets, perm,
+// slot_of, chunk table, scheduler counters); with A <= kPermSmem the whole
+// perm is also left in s_perm.
+__device__ __forceinline__ void plan_body(const PlanArgs& a, int* s_perm, bool writer) {
   __shared__ int cnt[kPlanWarps][kMaxE];  // per-warp counts, then per-warp bases
   __shared__ int tot[kMaxE];
   __shared__ int off[kMaxE + 1];
@@ -175,13 +177,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
     }
   }
   __syncthreads();
-  if (tid == 0) {
+  if (writer && tid == 0) {
     a.ctl->n_chunks = cst[E];
     a.ctl->max_chunk = s_maxc;
     a.ctl->work_next = 0;
   }
-  if (tid <= E) a.offsets[tid] = off[tid];
-  if (tid < E) {
+  if (writer && tid <= E) a.offsets[tid] = off[tid];
+  if (writer && tid < E) {
     for (int q = cst[tid]; q < cst[tid + 1]; ++q) {
       a.chunk_e[q] = tid;
       a.chunk_c[q] = q - cst[tid];
@@ -199,12 +201,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
       const int as = lo + 32 * it + lane;
       if (as < hi) {
         const int slot = off[e_r[it]] + cnt[warp][e_r[it]] + r_r[it];
-        a.slot_of[as] = slot;
+        if (writer) a.slot_of[as] = slot;
         s_perm[slot] = as / a.k;
       }
     }
     __syncthreads();
-    for (int i = tid; i < A; i += kPlanThreads) a.perm[i] = s_perm[i];
+    if (writer)
+      for (int i = tid; i < A; i += kPlanThreads) a.perm[i] = s_perm[i];
   } else {
     for (int as = lo + lane; as < hi; as += 32) {
       int e = __ldg(a.idx + as);
@@ -216,63 +219,88 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
   }
 }
 
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+  extern __shared__ int s_perm[];  // [T*k] when the register path is taken
+  plan_body(a, s_perm, true);
+}
+
 // x rows in slot order: x_perm[s] = x[perm[s]], or, with gamma2, the
 // expert-side norm bf16(x / sqrt(mean(x^2) + eps) * (1 + gamma2)) of that row
 // (the model's pre-FFN norm, whose only consumer is the fused gate_up).  One
 // warp per row, 16-byte moves, every load of the row issued before any use.
 constexpr int kGatherVec = 16;  // uint4 per lane held in registers (d <= 4096)
 
-__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= a.rows) return;
-  const int t = __ldg(a.perm + row);
+// One row (warp-wide, lane owns 16-byte pieces lane + 32j), in passes of
+// VEC pieces per lane with every load of a pass issued before any use.  With
+// the expert norm, the row's sum of squares is taken first (an extra read
+// when the row needs more than one pass).
+template <int VEC>
+__device__ __forceinline__ void gather_row(const GatherArgs& a, int row, int t, int lane) {
   const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d);
   uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (size_t)row * a.d);
   const int n = a.d / 8;
-  uint4 v[kGatherVec];
-#pragma unroll
-  for (int j = 0; j < kGatherVec; ++j)
-    if (lane + 32 * j < n) v[j] = __ldg(src + lane + 32 * j);
+  const bool one_pass = n <= 32 * VEC;
+  float inv = 1.f;
+  uint4 v[VEC];
   if (a.gamma2) {
     float ss = 0.f;
+    for (int p0 = 0; p0 < n; p0 += 32 * VEC) {
 #pragma unroll
-    for (int j = 0; j < kGatherVec; ++j) {
-      if (lane + 32 * j < n) {
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
+      for (int j = 0; j < VEC; ++j)
+        if (p0 + lane + 32 * j < n) v[j] = __ldg(src + p0 + lane + 32 * j);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(h2[q]);
-          ss = fmaf(f.x, f.x, ss);
-          ss = fmaf(f.y, f.y, ss);
+      for (int j = 0; j < VEC; ++j) {
+        if (p0 + lane + 32 * j < n) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[j]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(h2[q]);
+            ss = fmaf(f.x, f.x, ss);
+            ss = fmaf(f.y, f.y, ss);
+          }
         }
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float inv = 1.0f / sqrtf(ss / (float)a.d + a.eps);
-    const float4* g4 = reinterpret_cast<const float4*>(a.gamma2);
+    inv = 1.0f / sqrtf(ss / (float)a.d + a.eps);
+  }
+  for (int p0 = 0; p0 < n; p0 += 32 * VEC) {
+    if (!(a.gamma2 && one_pass)) {  // a single-pass row is still in v
 #pragma unroll
-    for (int j = 0; j < kGatherVec; ++j) {
-      const int i = lane + 32 * j;
-      if (i < n) {
-        const float4 ga = __ldg(g4 + 2 * i), gb = __ldg(g4 + 2 * i + 1);
-        const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-        __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[j]);
+      for (int j = 0; j < VEC; ++j)
+        if (p0 + lane + 32 * j < n) v[j] = __ldg(src + p0 + lane + 32 * j);
+    }
+    if (a.gamma2) {
+      const float4* g4 = reinterpret_cast<const float4*>(a.gamma2);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(h2[q]);
-          h2[q] = __floats2bfloat162_rn((f.x * inv) * (1.f + g[2 * q]),
-                                        (f.y * inv) * (1.f + g[2 * q + 1]));
+      for (int j = 0; j < VEC; ++j) {
+        const int i = p0 + lane + 32 * j;
+        if (i < n) {
+          const float4 ga = __ldg(g4 + 2 * i), gb = __ldg(g4 + 2 * i + 1);
+          const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[j]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(h2[q]);
+            h2[q] = __floats2bfloat162_rn((f.x * inv) * (1.f + g[2 * q]),
+                                          (f.y * inv) * (1.f + g[2 * q + 1]));
+          }
         }
       }
     }
-  }
 #pragma unroll
-  for (int j = 0; j < kGatherVec; ++j)
-    if (lane + 32 * j < n) dst[lane + 32 * j] = v[j];
+    for (int j = 0; j < VEC; ++j)
+      if (p0 + lane + 32 * j < n) dst[p0 + lane + 32 * j] = v[j];
+  }
+}
+
+__global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= a.rows) return;
+  gather_row<kGatherVec>(a, row, __ldg(a.perm + row), threadIdx.x & 31);
 }
 
 // out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32, one
@@ -380,6 +408,14 @@ cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s, bool pdl) {
     if (err != cudaSuccess) return err;
   }
   return moe::launch_pdl(moe::plan_kernel, dim3(1), dim3(moe::kPlanThreads), smem, s, pdl, a);
+}
+
+cudaError_t moe_launch_plan_gather(const moe::PlanArgs& a, const moe::GatherArgs& g, int num_sms,
+                                   cudaStream_t s, bool pdl) {
+  (void)num_sms;
+  const cudaError_t err = moe_launch_plan(a, s, pdl);
+  if (err != cudaSuccess) return err;
+  return moe_launch_gather(g, s, pdl);
 }
 
 cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl) {

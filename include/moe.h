@@ -94,11 +94,11 @@ enum {
 /* Kernels of one moe_forward, for moe_plan_profile. */
 enum {
   MOE_K_ROUTER = 0,   /* norm + logits + softmax + top-k                         */
-  MOE_K_PLAN = 1,     /* histogram + scan + stable permutation                   */
-  MOE_K_GATHER = 2,   /* x rows in slot order                                    */
-  MOE_K_EXPERT = 3,   /* grouped gate_up(+GELU*up) and down GEMMs               */
-  MOE_K_COMBINE = 4,  /* weighted k-order sum (+ residual)                       */
-  MOE_K_COUNT = 5
+  MOE_K_PLAN = 1,     /* histogram + scan + stable permutation, then the gather
+                         of x rows in slot order                                */
+  MOE_K_EXPERT = 2,   /* grouped gate_up(+GELU*up) and down GEMMs               */
+  MOE_K_COMBINE = 3,  /* weighted k-order sum (+ residual)                       */
+  MOE_K_COUNT = 4
 };
 
 /* Create a plan for E experts, top-k, hidden d, per-expert intermediate f.
