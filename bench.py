@@ -52,7 +52,7 @@ def parse():
     p.add_argument("--y-fp32", action="store_true",
                    help="keep the expert outputs y in fp32 (default bf16)")
     p.add_argument("--router", choices=["auto", "ffma", "tc"], default="auto",
-                   help="router path (auto: tensor cores from 1024 tokens)")
+                   help="router path (auto: tensor cores when E <= 128)")
     p.add_argument("--prefetch-mb", type=int, default=None,
                    help="MiB of gate_up weights pulled into L2 during routing")
     return p.parse_args()
@@ -157,14 +157,14 @@ class ClockSampler:
 
 def router_on_tensor_cores(w, T: int, router: str) -> bool:
     """The library's router choice (MOE_OPT_ROUTER): tensor cores for E <= 128
-    when asked, or automatically from T >= 1024."""
-    return w.E <= 128 and (router == "tc" or (router == "auto" and T >= 1024))
+    unless the FFMA router is asked for."""
+    return w.E <= 128 and router != "ffma"
 
 
 def launches_per_layer(w, T: int, router: str) -> int:
-    """Kernels one moe_forward launches: router (+ its weight split on the
-    tensor-core path), route plan, gather, expert GEMMs, combine."""
-    return (2 if router_on_tensor_cores(w, T, router) else 1) + 4
+    """Kernels one moe_forward launches: router, route plan, gather, expert
+    GEMMs, combine."""
+    return 5
 
 
 def layer_costs(w, touched: float, T: int):

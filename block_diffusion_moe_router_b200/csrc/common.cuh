@@ -143,24 +143,29 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, int
       : "memory");
 }
 
-// One 128-byte line into L2 (fire and forget, through the load/store unit).
-__device__ __forceinline__ void prefetch_l2_line(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
-}
-
-// Spread the prefetch of [base, base + bytes) over every thread of the grid.
-__device__ __forceinline__ void prefetch_l2_grid(const void* base, uint64_t bytes) {
-  const uint64_t nthr = (uint64_t)gridDim.x * gridDim.y * blockDim.x;
-  const uint64_t tid = ((uint64_t)blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
-  const char* b = static_cast<const char*>(base);
-  for (uint64_t o = tid * 128; o < bytes; o += nthr * 128) prefetch_l2_line(b + o);
-}
-
 // Bring [p, p + bytes) into L2 (bytes a multiple of 16, p 16-byte aligned).
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
                "r"(bytes)
                : "memory");
+}
+
+// The calling CTA's share of [base, base + bytes) into L2, issued by one
+// thread as 64 KB bulk prefetches (bytes and base 16-byte aligned).  A
+// prefetch only fills the coherent L2, so it is safe before the grid
+// dependency wait.
+__device__ __forceinline__ void prefetch_l2_grid(const void* base, uint64_t bytes) {
+  if (threadIdx.x != 0) return;
+  const uint64_t nblk = (uint64_t)gridDim.x * gridDim.y;
+  const uint64_t me = (uint64_t)blockIdx.y * gridDim.x + blockIdx.x;
+  const uint64_t share = ((bytes + nblk - 1) / nblk + 15) & ~uint64_t(15);
+  const uint64_t lo = me * share;
+  const uint64_t hi = lo + share < bytes ? lo + share : bytes;
+  const char* b = static_cast<const char*>(base);
+  for (uint64_t o = lo; o < hi; o += 65536) {
+    const uint64_t n = hi - o < 65536 ? hi - o : 65536;
+    prefetch_l2_bulk(b + o, (uint32_t)n);
+  }
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -362,30 +367,55 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 template <int C>
 __device__ __forceinline__ void warp_topk(const float (&v)[C], int E, int k, int lane,
                                           int32_t* idx, float* w, float* gap) {
-  uint32_t taken = 0;
+  // Each lane first orders its C candidates (logit desc, index asc; the
+  // indices lane + 32c rise with c, so an odd-even transposition sort that
+  // swaps only on a strictly larger key keeps equal keys in index order).
+  // Every round then compares lane heads only: the warp maximum of the key,
+  // the lowest index among the lanes holding it, and that lane pops its head.
+  uint32_t key[C];
+  int id[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    const int ee = lane + 32 * c;
+    key[c] = ee < E ? float_key(v[c]) : 0u;
+    id[c] = ee < E ? ee : 0x7fffffff;
+  }
+#pragma unroll
+  for (int pass = 0; pass < C; ++pass) {
+#pragma unroll
+    for (int c = pass & 1; c + 1 < C; c += 2) {
+      const bool sw = key[c + 1] > key[c];
+      const uint32_t ka = sw ? key[c + 1] : key[c], kb = sw ? key[c] : key[c + 1];
+      const int ia = sw ? id[c + 1] : id[c], ib = sw ? id[c] : id[c + 1];
+      key[c] = ka;
+      key[c + 1] = kb;
+      id[c] = ia;
+      id[c + 1] = ib;
+    }
+  }
   float my_sel = -INFINITY;
+  int my_idx = 0;
   float next_v = -INFINITY;
   const int rounds = (k < E) ? k + 1 : k;
   for (int j = 0; j < rounds; ++j) {
-    float bv = -INFINITY;
-    int bc = -1;
-#pragma unroll
-    for (int c = 0; c < C; ++c) {
-      const int ee = lane + 32 * c;
-      if (ee < E && !((taken >> c) & 1u) && (bc < 0 || v[c] > bv)) {
-        bv = v[c];
-        bc = c;
-      }
-    }
-    const uint32_t key = (bc < 0) ? 0u : float_key(bv);
-    const uint32_t m = __reduce_max_sync(0xffffffffu, key);
-    const uint32_t cand = (bc >= 0 && key == m) ? (uint32_t)(lane + 32 * bc) : 0xffffffffu;
+    const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+    const uint32_t cand = (key[0] == m) ? (uint32_t)id[0] : 0xffffffffu;
     const int bi = (int)__reduce_min_sync(0xffffffffu, cand);
     const float val = key_float(m);
     if (j < k) {
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (lane == j) my_sel = val;
-      if (lane == 0) idx[j] = bi;
+      if (id[0] == bi) {  // pop the head
+#pragma unroll
+        for (int c = 0; c + 1 < C; ++c) {
+          key[c] = key[c + 1];
+          id[c] = id[c + 1];
+        }
+        key[C - 1] = 0u;
+        id[C - 1] = 0x7fffffff;
+      }
+      if (lane == j) {
+        my_sel = val;
+        my_idx = bi;
+      }
     } else {
       next_v = val;
     }
@@ -395,7 +425,10 @@ __device__ __forceinline__ void warp_topk(const float (&v)[C], int E, int k, int
   float sum = ex;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane < k) w[lane] = ex / sum;
+  if (lane < k) {
+    idx[lane] = my_idx;
+    w[lane] = ex / sum;
+  }
   const float last = __shfl_sync(0xffffffffu, my_sel, k - 1);
   if (lane == 0 && gap) *gap = (k < E) ? (last - next_v) : INFINITY;
 }
@@ -425,10 +458,8 @@ cudaError_t moe_launch_router(const moe::RouterArgs& a, const CUtensorMap& tm_rw
                               bool pdl);
 size_t moe_router_smem_bytes(int d);
 int moe_router_tc_splits(int d, int T);
-cudaError_t moe_launch_router_split(const float* rw, const float* gamma, int E, int EP, int d,
-                                    __nv_bfloat16* wsplit, int num_sms, cudaStream_t s, bool pdl);
-cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x,
-                                 const CUtensorMap& tm_w, int EP, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x, int EP,
+                                 cudaStream_t s, bool pdl);
 cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_plan_gather(const moe::PlanArgs& a, const moe::GatherArgs& g, int num_sms,

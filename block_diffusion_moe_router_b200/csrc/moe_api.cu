@@ -42,7 +42,7 @@ struct moe_plan_s {
   Ctl* ctl;
   int32_t *idx, *perm, *slot_of, *offsets, *chunk_e, *chunk_c, *ready;
   float *w, *gap, *y;
-  __nv_bfloat16 *x_perm, *h, *x_dev, *res_dev, *out_dev, *wsplit;
+  __nv_bfloat16 *x_perm, *h, *x_dev, *res_dev, *out_dev;
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> ev_pool;
 };
@@ -131,16 +131,12 @@ int max_chunks(int E, int T, int k) { return E + (T * k) / 128 + 1; }
 // Experts rounded up to the UMMA N granularity for the tensor-core router.
 int router_ep(int E) { return (E + 15) / 16 * 16; }
 
-// Router path: the tensor-core router needs E <= 128; automatic selection
-// takes it from 1024 tokens up, where its split-K GEMM outruns the FFMA
-// router (below that both are latency-bound and the FFMA one is shorter).
+// Router path: the tensor-core router (E <= 128) unless the FFMA router is
+// asked for; E > 128 always takes the FFMA router.
 bool use_router_tc(moe_plan_t p, int T) {
-  if (p->E > 128 || p->router_sel == 1) return false;
-  return p->router_sel == 2 || T >= 1024;
+  (void)T;
+  return p->E <= 128 && p->router_sel != 1;
 }
-
-// The router weight times (1 + gamma), split into three bf16 parts.
-size_t wsplit_bytes(moe_plan_t p) { return (size_t)3 * router_ep(p->E) * p->d * 2; }
 
 // 2-D byte tensor map over packed int4 codes [rows, cols_bytes]: box = box_rows
 // x 64 bytes (one group of 128 codes), 64-byte swizzle.
@@ -171,7 +167,6 @@ moe_status_t ensure_workspace(moe_plan_t p, int T) {
   const size_t o_ce = take(MC * 4), o_cc = take(MC * 4), o_rd = take(MC * 4);
   const size_t o_xp = take(A * p->d * 2);
   const size_t o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
-  const size_t o_ws = take(wsplit_bytes(p));
   const size_t o_xd = take((size_t)cap * p->d * 2), o_rs = take((size_t)cap * p->d * 2);
   const size_t o_od = take((size_t)cap * p->d * 2);
   if (p->ws) {
@@ -199,7 +194,6 @@ moe_status_t ensure_workspace(moe_plan_t p, int T) {
   p->chunk_c = reinterpret_cast<int32_t*>(b + o_cc);
   p->ready = reinterpret_cast<int32_t*>(b + o_rd);
   p->x_perm = reinterpret_cast<__nv_bfloat16*>(b + o_xp);
-  p->wsplit = reinterpret_cast<__nv_bfloat16*>(b + o_ws);
   p->h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
   p->y = reinterpret_cast<float*>(b + o_y);
   p->x_dev = reinterpret_cast<__nv_bfloat16*>(b + o_xd);
@@ -263,8 +257,7 @@ uint64_t prefetch_bytes(moe_plan_t p) {
 moe_status_t launch_router(moe_plan_t p, int T, const void* x, const float* rw,
                            const float* gamma, const float* bias, int32_t* idx, float* w,
                            float* gap, cudaStream_t s, const void* pf = nullptr,
-                           uint64_t pf_bytes = 0, Ctl* ctl = nullptr,
-                           __nv_bfloat16* wsplit = nullptr) {
+                           uint64_t pf_bytes = 0, Ctl* ctl = nullptr) {
   moe::RouterArgs ra;
   ra.T = T;
   ra.E = p->E;
@@ -283,18 +276,11 @@ moe_status_t launch_router(moe_plan_t p, int T, const void* x, const float* rw,
   ra.l2_prefetch_bytes = pf_bytes;
   const bool pdl = p->pdl != 0;
   if (use_router_tc(p, T)) {
-    __nv_bfloat16* ws = wsplit ? wsplit : p->wsplit;
     const int EP = router_ep(p->E);
-    CUtensorMap tm_x, tm_w;
-    if (!make_map_bf16(&tm_x, x, (uint64_t)T, p->d, 128) ||
-        !make_map_bf16(&tm_w, ws, (uint64_t)3 * EP, p->d, (uint32_t)EP))
-      return MOE_ERR_CUDA;
+    CUtensorMap tm_x;
+    if (!make_map_bf16(&tm_x, x, (uint64_t)T, p->d, 128)) return MOE_ERR_CUDA;
     ProfScope ps(p, MOE_K_ROUTER, s);
-    if (moe_launch_router_split(rw, gamma, p->E, EP, p->d, ws, p->num_sms, s, pdl) !=
-        cudaSuccess)
-      return MOE_ERR_CUDA;
-    return moe_launch_router_tc(ra, tm_x, tm_w, EP, s, pdl) == cudaSuccess ? MOE_OK
-                                                                           : MOE_ERR_CUDA;
+    return moe_launch_router_tc(ra, tm_x, EP, s, pdl) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
   CUtensorMap tm_rw;
   if (!make_map_router(&tm_rw, rw, p->E, p->d)) return MOE_ERR_CUDA;
@@ -705,7 +691,6 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   const size_t o_ce = take(MC * 4), o_cc = take(MC * 4), o_rd = take(MC * 4);
   const size_t o_xp = take(A * p->d * 2);
   const size_t o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
-  const size_t o_ws = take(wsplit_bytes(p));
   if (sz > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
 
   char* b = static_cast<char*>(noalloc_scratch(p->device));
@@ -721,7 +706,6 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   int32_t* chunk_c = reinterpret_cast<int32_t*>(b + o_cc);
   int32_t* ready = reinterpret_cast<int32_t*>(b + o_rd);
   __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(b + o_xp);
-  __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(b + o_ws);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
   float* y = reinterpret_cast<float*>(b + o_y);
 
@@ -742,7 +726,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
     p->profile = 0;  // no event records on this path
     const moe_status_t rs =
         launch_router(p, T, x, router_w, router_gamma, router_bias, idx, w, gap, s, w_gate_up,
-                      prefetch_bytes(p), ctl, wsplit);
+                      prefetch_bytes(p), ctl);
     p->profile = prof;
     if (rs != MOE_OK) return rs;
   }

@@ -11,17 +11,27 @@
 //   z_e = (sum_i x_i * W'_ei) / rms(x),  W'_ei = router_w[e][i] * (1 + gamma_i)
 // with x already bf16.  W' (fp32, 24-bit significand) is split exactly into
 // three bf16 terms hi + mid + lo (each captures the next 8 bits), so every
-// product x_i * part is exact in fp32 and the UMMA accumulates in fp32: the
-// logits carry fp32 accumulation error only, as an FFMA dot product would.
+// product x_i * part is exact in fp32, and all three parts accumulate into
+// the same fp32 TMEM accumulator: the logits carry fp32 accumulation error
+// only, as an FFMA dot product would.
 //
 // Work split: a CTA owns 128 tokens (UMMA M) x all experts (UMMA N = E
-// rounded up to 16) over a slice of the hidden dimension; the 8 (or fewer)
-// CTAs that share a token tile form a cluster along the hidden dimension.
-// Each accumulates its partial logits in TMEM (plus the partial sum of x^2,
-// read from the staged x tiles) and pushes every token row to the rank that
-// owns it (ceil(128 / cluster) tokens per rank) with distributed-shared-
-// memory stores; each rank sums its slots in rank order (deterministic) and
-// one warp per token runs the top-k.
+// rounded up to 16) over a slice of the hidden dimension; the KS (<= 16)
+// CTAs that share a token tile form one cluster along the hidden dimension.
+// Roles per CTA (320 threads):
+//   warp 0      TMA producer: x tile [128 x 64] bf16 (128-byte swizzle) per
+//               64-column step, three stages;
+//   warp 1      UMMA issuer (owns the TMEM accumulator, 128 columns);
+//   warps 2..9  load the fp32 router_w rows of the step (one step ahead, in
+//               registers), split them times (1 + gamma) into the three
+//               bf16 parts, written straight into the swizzled K-major
+//               layout the UMMA reads (two buffers), and take the x^2
+//               partials of the x tile;
+//               afterwards they read the accumulator and push every token
+//               row to the cluster rank that owns it (ceil(128 / KS) tokens
+//               per rank) with distributed-shared-memory stores;
+//   all warps   each rank sums its slots in rank order (deterministic) and
+//               one warp per token runs the top-k.
 #include <cooperative_groups.h>
 
 #include <mutex>
@@ -34,85 +44,121 @@ namespace moe {
 
 namespace {
 
-constexpr int kTThreads = 192;   // producer, UMMA, 4 epilogue warps
-constexpr int kTM = 128;         // tokens per CTA
-constexpr int kTStages = 3;
-constexpr int kXTile = kTM * kBK * 2;          // 16 KB
-constexpr int kMaxEP = 128;                    // experts (N) handled here
-constexpr int kWTile = kMaxEP * kBK * 2;       // 16 KB per split part
-constexpr int kTStage = kXTile + 3 * kWTile;   // 64 KB
-constexpr int kMaxCluster = 8;
-constexpr int kRecvRows = kTM + kMaxCluster;   // >= nsplit * ceil(kTM / nsplit)
-constexpr int kTSmem = 1024 + kTStages * kTStage + 1024;
-static_assert((kRecvRows * kMaxEP + kRecvRows + kTM * kMaxEP + kTM) * 4 <= kTStages * kTStage,
-              "receive buffers and reduced logits reuse the ring");
+constexpr int kTThreads = 320;  // producer, UMMA, 8 converter / epilogue warps
+constexpr int kConvWarps = 8;
+constexpr int kTM = 128;        // tokens per CTA
+constexpr int kMaxEP = 128;     // experts (N) handled here
+constexpr int kXTile = kTM * kBK * 2;           // 16 KB bf16
+constexpr int kWPart = kMaxEP * kBK * 2;        // 16 KB per bf16 part
+constexpr int kXStages = 3;                     // x tiles (TMA)
+constexpr int kWBufs = 2;                       // split router_w buffers (3 parts each)
+constexpr int kWsOff = kXStages * kXTile;
+constexpr int kRingBytes = kWsOff + kWBufs * 3 * kWPart;  // 144 KB
+constexpr int kRowsPerThread = kMaxEP / 16;     // fp32 router_w rows a converter thread splits
+constexpr int kMaxCluster = 16;
+constexpr int kRecvRows = kTM + kMaxCluster;    // >= KS * ceil(kTM / KS)
+// One exchanged token row: EP partial logits (padded to 128) and the two x^2
+// partials (padded to four floats, so every block is a multiple of 16 bytes).
+constexpr int kRowFloats = kMaxEP + 4;
+constexpr int kRowBytes = kRowFloats * 4;       // 528
+constexpr int kRecvOff = kRingBytes;
+constexpr int kRecvBytes = kRecvRows * kRowBytes;
+constexpr int kBarOff = kRecvOff + kRecvBytes;
+constexpr int kTSmem = 1024 + kBarOff + 256;
+// after the main loop: the outgoing rows (staging) and this rank's reduced
+// logits reuse the stage ring and the part buffer
+constexpr int kZallOff = (kRecvRows * kRowBytes + 1023) / 1024 * 1024;
+static_assert(kZallOff + (kTM * kMaxEP + kTM) * 4 <= kRingBytes,
+              "staging rows and reduced logits fit in the ring");
+static_assert(kTSmem <= 232448, "router smem above the sm_100 limit");
 
-// W'[e][i] = router_w[e][i] * (1 + gamma[i]) split into three bf16 parts,
-// wsplit[p][e][i], rows e >= E zero.
-__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ rw,
-                                                           const float* __restrict__ gamma, int E,
-                                                           int EP, int d,
-                                                           __nv_bfloat16* __restrict__ wsplit) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const size_t n = (size_t)EP * d;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * blockDim.x) {
-    const int e = (int)(i / d);
-    const int k = (int)(i - (size_t)e * d);
-    float v = 0.f;
-    if (e < E) v = __ldg(rw + i) * (1.f + __ldg(gamma + k));
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    const float r1 = v - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);
-    wsplit[i] = hi;
-    wsplit[n + i] = mid;
-    wsplit[2 * n + i] = __float2bfloat16_rn(r2);
-  }
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// v = w * g split into bf16 hi + mid + lo (exact: each residual is exact in
+// fp32 and the last one fits 8 bits), packed two per 32-bit word.
+__device__ __forceinline__ void split3(float v0, float v1, uint32_t& hi, uint32_t& mid,
+                                       uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+  const float2 hf = __bfloat1622float2(h);
+  const float r0 = v0 - hf.x, r1 = v1 - hf.y;
+  const __nv_bfloat162 m = __floats2bfloat162_rn(r0, r1);
+  const float2 mf = __bfloat1622float2(m);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(r0 - mf.x, r1 - mf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  mid = *reinterpret_cast<const uint32_t*>(&m);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Bulk copy of `bytes` from this CTA's shared memory into a peer CTA's
+// (both addresses as the peer sees them), completing on the peer's mbarrier.
+__device__ __forceinline__ void bulk_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                             uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst_cluster), "r"(src), "r"(bytes), "r"(bar_cluster)
+      : "memory");
 }
 
 __global__ void __launch_bounds__(kTThreads, 1)
-    router_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                     const __grid_constant__ CUtensorMap tm_w, RouterArgs a, int EP, int nsplit) {
+    router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, RouterArgs a, int EP, int KS) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  // After the main loop the ring is reused: the receive buffer for the
-  // partial logits of this rank's tokens from every rank, their x^2
-  // partials, then this rank's reduced logits.
-  float* recv = reinterpret_cast<float*>(smem);          // [nsplit*tpr <= kRecvRows][kMaxEP]
-  float* recv_ssq = recv + kRecvRows * kMaxEP;            // [kRecvRows]
-  float* zall = recv_ssq + kRecvRows;                     // [tpr][kMaxEP]
-  float* inv_rms = zall + kTM * kMaxEP;                   // [tpr]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTStages * kTStage);
-  uint64_t* empty = full + kTStages;
-  uint64_t* sqd = empty + kTStages;   // x tile's sum of squares taken
-  uint64_t* tfull = sqd + kTStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull + 1);
+  uint8_t* wsp = smem + kWsOff;                                 // bf16 parts hi, mid, lo
+  float* stage_rows = reinterpret_cast<float*>(smem);           // [128][kRowFloats] outgoing
+  float* recv = reinterpret_cast<float*>(smem + kRecvOff);      // [KS*tpr][kRowFloats] incoming
+  float* zall = reinterpret_cast<float*>(smem + kZallOff);      // [tpr][kMaxEP]
+  float* inv_rms = zall + kTM * kMaxEP;                         // [tpr]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  uint64_t* empty = full + kXStages;
+  uint64_t* conv = empty + kXStages;
+  uint64_t* wfree = conv + kWBufs;
+  uint64_t* tfull = wfree + kWBufs;
+  uint64_t* rbar = tfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   cg::cluster_group cluster = cg::this_cluster();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int rank = blockIdx.y;  // K slice == rank in the cluster
+  const int rank = (int)cluster.block_rank();  // K slice
   const int t0 = blockIdx.x * kTM;
   const int nst = a.d / kBK;
-  const int kb0 = rank * nst / nsplit;
-  const int kb1 = (rank + 1) * nst / nsplit;
+  const int kb0 = rank * nst / KS;
+  const int kb1 = (rank + 1) * nst / KS;
+  const int nk = kb1 - kb0;
+  // Rank r owns tokens [r*tpr, r*tpr + tpr) of the tile (the last ranks may
+  // own fewer, or none).
+  const int tpr = (kTM + KS - 1) / KS;
+  const int tb = rank * tpr;
+  const int tcount = max(0, min(tpr, kTM - tb));
   const uint64_t timeout_ns = 1000000000ull;
   Ctl* ctl = a.ctl;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kTStages; ++i) {
+    for (int i = 0; i < kXStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
-      mbar_init(&sqd[i], 4);
+    }
+    for (int i = 0; i < kWBufs; ++i) {
+      mbar_init(&conv[i], kConvWarps);
+      mbar_init(&wfree[i], 1);
     }
     mbar_init(tfull, 1);
+    mbar_init(rbar, 1);
     *s_abort = 0;
     fence_mbar_init();
+    // every rank sends this one its rows of our tokens (tx may run ahead of
+    // this: an mbarrier's transaction count may go negative)
+    mbar_arrive_expect_tx(rbar, (uint32_t)(KS * tcount * kRowBytes));
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kMaxEP);
@@ -120,40 +166,37 @@ __global__ void __launch_bounds__(kTThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_w);
   }
-  // first-wave expert weights into L2 while routing runs (see router.cu)
+  // Pull the first expert weights into L2 while routing runs: HBM is
+  // otherwise idle until the expert kernel starts.
   if (a.l2_prefetch) prefetch_l2_grid(a.l2_prefetch, a.l2_prefetch_bytes);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Peers may target this CTA's barrier only once it is initialised: arrive
+  // now, wait just before the first remote copy.
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // x and the split weight come from earlier kernels
+  pdl_wait();  // x, router_w and gamma may come from the previous kernel
   pdl_launch_dependents();
 
   float my_ssq = 0.f;
   if (warp == 0) {
     if (lane == 0) {  // ---------------------------------------------- producer
       const uint64_t pol = l2_policy_evict_last();
-      const uint32_t tx = kXTile + 3 * EP * kBK * 2;
       uint32_t issued = 0, par = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        const int i = kb - kb0;
-        const int st = i % kTStages;
-        // refill only after the UMMAs and the x^2 readers are done with it
-        if (i >= kTStages &&
-            (!mbar_wait(&empty[st], ((i / kTStages) - 1) & 1, s_abort, ctl, timeout_ns, 401) ||
-             !mbar_wait(&sqd[st], ((i / kTStages) - 1) & 1, s_abort, ctl, timeout_ns, 406)))
+      for (int i = 0; i < nk; ++i) {
+        const int st = i % kXStages;
+        // refill only after the UMMAs of the step that last used the stage
+        if (i >= kXStages &&
+            !mbar_wait(&empty[st], ((i / kXStages) - 1) & 1, s_abort, ctl, timeout_ns, 401))
           break;
-        uint8_t* sx = ring + st * kTStage;
-        mbar_arrive_expect_tx(&full[st], tx);
-        tma_load_2d(sx, &tm_x, kb * kBK, t0, &full[st], pol);
-        for (int p = 0; p < 3; ++p)
-          tma_load_2d(sx + kXTile + p * kWTile, &tm_w, kb * kBK, p * EP, &full[st], pol);
+        mbar_arrive_expect_tx(&full[st], kXTile);
+        tma_load_2d(smem + st * kXTile, &tm_x, (kb0 + i) * kBK, t0, &full[st], pol);
         issued |= 1u << st;
-        par = (par & ~(1u << st)) | ((uint32_t)((i / kTStages) & 1) << st);
+        par = (par & ~(1u << st)) | ((uint32_t)((i / kXStages) & 1) << st);
       }
-      for (int st = 0; st < kTStages; ++st) {  // drain
+      for (int st = 0; st < kXStages; ++st) {  // every issued copy lands before exit
         if (!((issued >> st) & 1u)) continue;
         const uint32_t b = smem_u32(&full[st]);
         const uint64_t tq = globaltimer_ns();
@@ -167,72 +210,124 @@ __global__ void __launch_bounds__(kTThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {  // ---------------------------------------------- UMMA issuer
       const uint32_t idesc = idesc_bf16_f32(kTM, EP);
-      for (int kb = kb0; kb < kb1; ++kb) {
-        const int i = kb - kb0;
-        const int st = i % kTStages;
-        if (!mbar_wait(&full[st], (i / kTStages) & 1, s_abort, ctl, timeout_ns, 403)) break;
+      for (int i = 0; i < nk; ++i) {
+        const int st = i % kXStages;
+        const int wb = i % kWBufs;
+        if (!mbar_wait(&full[st], (i / kXStages) & 1, s_abort, ctl, timeout_ns, 403) ||
+            !mbar_wait(&conv[wb], (i / kWBufs) & 1, s_abort, ctl, timeout_ns, 403))
+          break;
         tc_fence_after();
-        const uint32_t sx = smem_u32(ring + st * kTStage);
+        const uint32_t sx = smem_u32(smem + st * kXTile);
+        const uint32_t sw = smem_u32(wsp + wb * 3 * kWPart);
 #pragma unroll
         for (int kk = 0; kk < kBK / kUmmaK; ++kk)
 #pragma unroll
           for (int p = 0; p < 3; ++p)
             umma_bf16(tmem_base, sdesc_k_sw128(sx + kk * kUmmaK * 2),
-                      sdesc_k_sw128(sx + kXTile + p * kWTile + kk * kUmmaK * 2), idesc,
+                      sdesc_k_sw128(sw + p * kWPart + kk * kUmmaK * 2), idesc,
                       (i | kk | p) ? 1u : 0u);
-        umma_commit(&empty[st]);
+        umma_commit(&empty[st]);  // the x tile
+        umma_commit(&wfree[wb]);  // the part buffer
       }
-      umma_commit(tfull);  // also drains every issued UMMA
+      umma_commit(tfull);  // arrives once every issued UMMA is done
     }
   } else {
-    // ---------------------------------------------------------- x^2 partials
-    // Each epilogue thread owns one token row of the staged x tiles (128-byte
-    // swizzled rows): 16-byte chunk c of row r sits at chunk c ^ (r % 8).
-    const int r = (warp & 3) * 32 + lane;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      const int i = kb - kb0;
-      const int st = i % kTStages;
-      if (!mbar_wait(&full[st], (i / kTStages) & 1, s_abort, ctl, timeout_ns, 404)) break;
-      const uint8_t* row = ring + st * kTStage + r * 128;
+    // ------------------------------------------------ converters (256 threads)
+    // Split: thread c owns fp32 column group j = c % 16 (4 columns) of rows
+    // n = c / 16 + 16 r (three steps of them in flight).  The bf16 parts land in 128-byte K-major rows whose 16-byte
+    // chunk q sits at q ^ (n % 8) (the 128-byte swizzle).  x^2: the thread
+    // owns row c % 128, half c / 128 of the x tile's 64 columns.
+    const int c = threadIdx.x - 64;
+    const int j = c & 15;
+    const int n0 = c >> 4;
+    const int xr = c & (kTM - 1);
+    const int xh = c >> 7;
+    const int E = a.E;
+    // fp32 router_w rows in registers, three steps in flight: step i sits in
+    // slot i % 3 and its slot is refilled with step i + 3 once split
+    float4 w0[kRowsPerThread], w1[kRowsPerThread], w2[kRowsPerThread];
+    auto load_rows = [&](float4 (&dst)[kRowsPerThread], int i) {
+      if (i >= nk) return;
+      const int kb = kb0 + i;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 pk = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) * 16));
+      for (int r = 0; r < kRowsPerThread; ++r) {
+        const int n = n0 + 16 * r;
+        dst[r] = (n < E) ? __ldg(reinterpret_cast<const float4*>(a.router_w + (size_t)n * a.d +
+                                                                  kb * kBK) + j)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    // split step i (rows in wr) into part buffer i % 2, then the x^2 of its x
+    // tile; false when a wait gave up
+    auto step = [&](const float4 (&wr)[kRowsPerThread], int i) -> bool {
+      const int st = i % kXStages;
+      const int wb = i % kWBufs;
+      const float4 g = __ldg(reinterpret_cast<const float4*>(a.gamma + (kb0 + i) * kBK) + j);
+      const float g0 = 1.f + g.x, g1 = 1.f + g.y, g2 = 1.f + g.z, g3 = 1.f + g.w;
+      // the part buffer is free once the UMMAs two steps back are done
+      if (i >= kWBufs &&
+          !mbar_wait(&wfree[wb], ((i / kWBufs) - 1) & 1, s_abort, ctl, timeout_ns, 406))
+        return false;
+      uint8_t* wp = wsp + wb * 3 * kWPart;
+#pragma unroll
+      for (int r = 0; r < kRowsPerThread; ++r) {
+        const int n = n0 + 16 * r;
+        if (n < EP) {
+          uint32_t h0, m0, l0, h1, m1, l1;
+          split3(wr[r].x * g0, wr[r].y * g1, h0, m0, l0);
+          split3(wr[r].z * g2, wr[r].w * g3, h1, m1, l1);
+          const int off = n * 128 + (((j >> 1) ^ (n & 7)) << 4) + ((j & 1) << 3);
+          *reinterpret_cast<uint2*>(wp + off) = make_uint2(h0, h1);
+          *reinterpret_cast<uint2*>(wp + kWPart + off) = make_uint2(m0, m1);
+          *reinterpret_cast<uint2*>(wp + 2 * kWPart + off) = make_uint2(l0, l1);
+        }
+      }
+      if (!mbar_wait(&full[st], (i / kXStages) & 1, s_abort, ctl, timeout_ns, 404)) return false;
+      const uint8_t* row = smem + st * kXTile + xr * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 pk = *reinterpret_cast<const uint4*>(row + (((xh * 4 + q) ^ (xr & 7)) << 4));
         const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&pk);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(h2[q]);
+        for (int u = 0; u < 4; ++u) {
+          const float2 f = __bfloat1622float2(h2[u]);
           my_ssq = fmaf(f.x, f.x, my_ssq);
           my_ssq = fmaf(f.y, f.y, my_ssq);
         }
       }
+      fence_async_smem();  // generic-proxy stores -> visible to the UMMA
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sqd[st]);
+      if (lane == 0) mbar_arrive(&conv[wb]);
+      return true;
+    };
+    load_rows(w0, 0);
+    load_rows(w1, 1);
+    load_rows(w2, 2);
+#pragma unroll 1
+    for (int i = 0; i < nk; i += 3) {
+      if (!step(w0, i)) break;
+      load_rows(w0, i + 3);
+      if (i + 1 >= nk || !step(w1, i + 1)) break;
+      load_rows(w1, i + 4);
+      if (i + 2 >= nk || !step(w2, i + 2)) break;
+      load_rows(w2, i + 5);
     }
   }
-  __syncthreads();
 
-  // ---- partial logits.  Rank r of the cluster owns tokens [r*tpr, r*tpr +
-  // tpr) of the tile.  Every CTA pushes each of its partial rows straight into
-  // the owner's receive buffer with distributed-shared-memory stores (which
-  // pipeline, unlike remote loads), then each rank sums its slots in rank
-  // order.  The first cluster barrier makes sure every CTA is done with its
-  // stage ring (the receive buffers live there) before anyone writes.
-  const int tpr = (kTM + nsplit - 1) / nsplit;  // ceil split: the last rank may take fewer
-  const int tb = rank * tpr;
-  const int tcount = max(0, min(tpr, kTM - tb));
-  bool tmem_ok = true;
+  // ---- exchange.  Each converter thread copies its accumulator row (and its
+  // x^2 partial) into the staging rows; row r of the tile goes to rank
+  // r / tpr, where it lands as row (rank * tpr + r % tpr) of the receive
+  // buffer.  The rows for one owner are contiguous, so one bulk copy per
+  // owner moves them (completing on the owner's barrier); each rank then sums
+  // its slots in rank order, which keeps the result deterministic.
   if (warp >= 2) {
-    tmem_ok = mbar_wait(tfull, 0, s_abort, ctl, timeout_ns, 405);
+    const bool tmem_ok = mbar_wait(tfull, 0, s_abort, ctl, timeout_ns, 405);
     tc_fence_after();
-  }
-  cluster.sync();
-  if (warp >= 2) {
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;     // token row of the tile
-    const int owner = r / tpr;
-    const int tl = r - owner * tpr;
-    float* dst = cluster.map_shared_rank(recv, owner) + (size_t)(rank * tpr + tl) * kMaxEP;
-    for (int c0 = 0; c0 < EP; c0 += 32) {
+    const int c = threadIdx.x - 64;
+    const int q4 = warp & 3;       // TMEM lane quarter this warp may read
+    const int r = q4 * 32 + lane;  // token row of the tile
+    float* dst = stage_rows + (size_t)r * kRowFloats;
+    for (int c0 = ((warp - 2) >> 2) * 32; c0 < EP; c0 += 64) {
       uint32_t v[32];
       tmem_ld32(tmem_base + ((uint32_t)(q4 * 32) << 16) + c0, v);
       tmem_wait_ld();
@@ -246,32 +341,61 @@ __global__ void __launch_bounds__(kTThreads, 1)
             make_float4(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
                         __uint_as_float(v[jj + 2]), __uint_as_float(v[jj + 3]));
     }
-    cluster.map_shared_rank(recv_ssq, owner)[rank * tpr + tl] = my_ssq;
+    stage_rows[(size_t)(c & (kTM - 1)) * kRowFloats + kMaxEP + (c >> 7)] = my_ssq;
+    fence_async_smem();  // staging rows -> visible to the bulk copies
   }
   tc_fence_before();
-  cluster.sync();  // every push has landed
+  __syncthreads();
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (threadIdx.x == 0) {
+    const uint32_t src0 = smem_u32(stage_rows);
+    const uint32_t dst0 = smem_u32(recv) + (uint32_t)(rank * tpr * kRowBytes);
+    const uint32_t bar0 = smem_u32(rbar);
+    for (int q = 0; q < KS; ++q) {
+      const int rows = min(tpr, kTM - q * tpr);
+      if (rows <= 0) break;
+      bulk_to_peer(mapa_shared(dst0, q), src0 + (uint32_t)(q * tpr * kRowBytes),
+                   (uint32_t)(rows * kRowBytes), mapa_shared(bar0, q));
+    }
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kMaxEP);
   }
+  if (threadIdx.x == 32) {  // every rank's rows of our tokens have landed
+    const uint32_t b = smem_u32(rbar);
+    const uint64_t tq = globaltimer_ns();
+    while (!mbar_try_wait(b, 0))
+      if (globaltimer_ns() - tq > timeout_ns) {
+        record_error(ctl, MOE_ERR_TIMEOUT, 407);
+        break;
+      }
+  }
+  __syncthreads();
+
   // rank-order sums, four experts per thread (EP is a multiple of 16)
   const int EP4 = EP / 4;
   for (int idx = threadIdx.x; idx < tcount * EP4; idx += kTThreads) {
     const int tl = idx / EP4;
     const int e = 4 * (idx - tl * EP4);
-    float4 sacc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int q = 0; q < nsplit; ++q) {
-      const float4 r = *reinterpret_cast<const float4*>(recv + (size_t)(q * tpr + tl) * kMaxEP + e);
-      sacc.x += r.x;
-      sacc.y += r.y;
-      sacc.z += r.z;
-      sacc.w += r.w;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q = 0; q < KS; ++q) {
+      const float4 r =
+          *reinterpret_cast<const float4*>(recv + (size_t)(q * tpr + tl) * kRowFloats + e);
+      s.x += r.x;
+      s.y += r.y;
+      s.z += r.z;
+      s.w += r.w;
     }
-    *reinterpret_cast<float4*>(zall + tl * kMaxEP + e) = sacc;
+    *reinterpret_cast<float4*>(zall + tl * kMaxEP + e) = s;
   }
   if (threadIdx.x < tcount) {
     float s2 = 0.f;
-    for (int q = 0; q < nsplit; ++q) s2 += recv_ssq[q * tpr + threadIdx.x];
+    for (int q = 0; q < KS; ++q) {
+      const float* rr = recv + (size_t)(q * tpr + threadIdx.x) * kRowFloats + kMaxEP;
+      s2 += rr[0] + rr[1];
+    }
     inv_rms[threadIdx.x] = 1.0f / sqrtf(s2 / (float)a.d + a.eps);
   }
   __syncthreads();
@@ -283,19 +407,21 @@ __global__ void __launch_bounds__(kTThreads, 1)
     if (t >= a.T) break;
     float v[kMaxEP / 32];
 #pragma unroll
-    for (int c = 0; c < kMaxEP / 32; ++c) {
-      const int ee = lane + 32 * c;
+    for (int cc = 0; cc < kMaxEP / 32; ++cc) {
+      const int ee = lane + 32 * cc;
       float z = -INFINITY;
       if (ee < E) {
         z = zall[tl * kMaxEP + ee] * inv_rms[tl];
         if (a.bias) z += __ldg(a.bias + ee);
         if (z != z) z = -INFINITY;
       }
-      v[c] = z;
+      v[cc] = z;
     }
     warp_topk(v, E, a.k, lane, a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k,
               a.gap ? a.gap + t : nullptr);
   }
+  if (threadIdx.x == 0)  // the outgoing copies have read the staging rows
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 }  // namespace
@@ -311,14 +437,23 @@ int g_max_clusters[kMaxDevices][moe::kMaxCluster + 1];
 bool g_max_clusters_ok[kMaxDevices];
 std::mutex g_max_clusters_mu;
 
+cudaError_t set_attrs() {
+  cudaError_t err = cudaFuncSetAttribute(
+      moe::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, moe::kTSmem);
+  if (err != cudaSuccess) return err;
+  return cudaFuncSetAttribute(moe::router_tc_kernel,
+                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+}
+
 int max_active_clusters(int ns) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
   std::lock_guard<std::mutex> lock(g_max_clusters_mu);
   if (!g_max_clusters_ok[dev]) {
-    if (cudaFuncSetAttribute(moe::router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             moe::kTSmem) != cudaSuccess)
+    if (set_attrs() != cudaSuccess) {
+      cudaGetLastError();
       return 0;
+    }
     for (int c = 1; c <= moe::kMaxCluster; ++c) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(1, c, 1);
@@ -332,7 +467,10 @@ int max_active_clusters(int ns) {
       cfg.attrs = &attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, moe::router_tc_kernel, &cfg) != cudaSuccess) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, moe::router_tc_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
       g_max_clusters[dev][c] = n;
     }
     g_max_clusters_ok[dev] = true;
@@ -342,48 +480,36 @@ int max_active_clusters(int ns) {
 
 }  // namespace
 
-// Hidden-dimension split (= cluster size): as many as there are K stages up
-// to the cluster limit, lowered while the token tiles would not all be
-// resident in one wave of clusters.
+// Hidden-dimension split (= cluster size): as many 64-column steps as there
+// are, up to 16, lowered while the token tiles would not all be resident in
+// one wave of clusters.
 int moe_router_tc_splits(int d, int T) {
   const int nst = d / moe::kBK;
   const int cap = nst < moe::kMaxCluster ? nst : moe::kMaxCluster;
   const int tiles = (T + moe::kTM - 1) / moe::kTM;
   for (int c = cap; c >= 1; --c)
     if (tiles <= max_active_clusters(c)) return c;
-  return cap;
+  return 1;
 }
 
-cudaError_t moe_launch_router_split(const float* rw, const float* gamma, int E, int EP, int d,
-                                    __nv_bfloat16* wsplit, int num_sms, cudaStream_t s,
-                                    bool pdl) {
-  const size_t n = (size_t)EP * d;
-  int blocks = (int)((n + 255) / 256);
-  if (blocks > 4 * num_sms) blocks = 4 * num_sms;
-  return moe::launch_pdl(moe::router_split_kernel, dim3(blocks), dim3(256), 0, s, pdl, rw, gamma,
-                         E, EP, d, wsplit);
-}
-
-cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x,
-                                 const CUtensorMap& tm_w, int EP, cudaStream_t s, bool pdl) {
-  const int nsplit = moe_router_tc_splits(a.d, a.T);
-  cudaError_t err = cudaFuncSetAttribute(moe::router_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         moe::kTSmem);
+cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x, int EP,
+                                 cudaStream_t s, bool pdl) {
+  const int KS = moe_router_tc_splits(a.d, a.T);
+  cudaError_t err = set_attrs();
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((a.T + moe::kTM - 1) / moe::kTM, nsplit, 1);
+  cfg.gridDim = dim3((a.T + moe::kTM - 1) / moe::kTM, KS, 1);
   cfg.blockDim = dim3(moe::kTThreads, 1, 1);
   cfg.dynamicSmemBytes = moe::kTSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = nsplit;
+  attr[0].val.clusterDim.y = KS;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, moe::router_tc_kernel, tm_x, tm_w, a, EP, nsplit);
+  return cudaLaunchKernelEx(&cfg, moe::router_tc_kernel, tm_x, a, EP, KS);
 }

@@ -80,8 +80,8 @@ enum {
                              dependent launch so it overlaps the previous one's
                              tail; 0: plain stream-ordered launches              */
   MOE_OPT_ROUTER = 6,     /* router path: 0 (default) automatic -- tensor cores
-                             when E <= 128 and T >= 1024, FFMA otherwise;
-                             1 FFMA; 2 tensor cores (E <= 128)                   */
+                             when E <= 128, FFMA otherwise; 1 FFMA; 2 tensor
+                             cores (E <= 128)                                    */
   MOE_OPT_L2_PREFETCH_MB = 5, /* MiB of the gate_up weight (from its start) the
                              router pulls into L2 while routing runs, so the
                              expert kernel's first wave finds it there
