@@ -461,10 +461,10 @@ int moe_router_tc_splits(int d, int T);
 cudaError_t moe_launch_router_tc(const moe::RouterArgs& a, const CUtensorMap& tm_x, int EP,
                                  cudaStream_t s, bool pdl);
 cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s, bool pdl);
-cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_gather(const moe::GatherArgs& a, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_plan_gather(const moe::PlanArgs& a, const moe::GatherArgs& g, int num_sms,
                                    cudaStream_t s, bool pdl);
-cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_combine(const moe::CombineArgs& a, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_expert(const moe::ExpertArgs& a, const CUtensorMap& tm_wgu,
                               const CUtensorMap& tm_wd, const CUtensorMap& tm_xp,
                               const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);

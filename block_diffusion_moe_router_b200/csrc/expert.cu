@@ -18,8 +18,8 @@
 // the expert are N (16..256), so every weight byte is streamed from HBM once
 // per chunk, and at 256 tokens per canvas one chunk covers every expert.
 //
-// Roles (224 threads): warp 0 = scheduler (claims units from a global
-// counter) and weight (A) producer, warp 1 = UMMA issuer (owns the TMEM
+// Roles (224 threads): warp 0 = scheduler (claims units: its CTA index
+// first, then from a global counter) and weight (A) producer, warp 1 = UMMA issuer (owns the TMEM
 // allocation), warps 2..5 = epilogue (TMEM -> registers -> global), warp 6 =
 // activation (B) producer.  Weights and activations have rings of their own,
 // sized at run time from the largest chunk: the weight ring is deep, since
@@ -45,10 +45,9 @@ constexpr int kMaxA = 12;  // weight stages
 constexpr int kMaxB = 8;   // activation stages
 constexpr int kMinB = 3;
 constexpr int kRingBytes = 200 * 1024;
-constexpr int kXchgBytes = 64 * kXchgStride * 4;  // gate/up exchange rows
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
 constexpr int kBarBytes = 8 * (2 * kMaxA + 2 * kMaxB + 4 + 2 * kUnitRing + 1);
-constexpr int kSmemBytes = 1024 + kRingBytes + kXchgBytes + kBarBytes + 256;
+constexpr int kSmemBytes = 1024 + kRingBytes + kEpiBytes + kBarBytes + 256;
 
 __global__ void __launch_bounds__(kThreads, 1)
     expert_kernel(const __grid_constant__ CUtensorMap tm_wgu,
@@ -60,7 +59,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
   float* xchg = reinterpret_cast<float*>(smem + kRingBytes);
-  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + kRingBytes + kXchgBytes);
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + kRingBytes + kEpiBytes);
   uint64_t* emptyA = fullA + kMaxA;
   uint64_t* fullB = emptyA + kMaxA;
   uint64_t* emptyB = fullB + kMaxB;
@@ -141,6 +140,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int ur = 0;
     uint32_t uphase = 0;
     uint32_t issued = 0, issued_par = 0;  // stages with a copy issued, and its parity
+    // The first unit of CTA b is unit b; later ones come from the counter
+    // (offset by the grid), so every unit is claimed exactly once.
+    bool first_claim = true;
     while (true) {
       UnitInfo ui;
       ui.type = kUnitStop;
@@ -148,7 +150,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int go = 0;
       if (lane == 0 && !*s_abort) {
         go = 1;
-        const int u = atomicAdd(&ctl->work_next, 1);
+        const int u = first_claim ? (int)blockIdx.x
+                                  : (int)gridDim.x + atomicAdd(&ctl->work_next, 1);
+        first_claim = false;
         if (u < U) {
           int q, m;
           if (u < n_chunks * GU) {

@@ -8,6 +8,11 @@
 namespace moe {
 
 constexpr int kXchgStride = 33;  // floats per exchanged row (bank-conflict padding)
+// Epilogue scratch: the gate/up exchange rows, then a [32 tokens x 128
+// columns] bf16 tile through which h and y are written out as 16-byte rows.
+constexpr int kXchgBytes = 64 * kXchgStride * 4;
+constexpr int kTileBytes = 32 * 128 * 2;
+constexpr int kEpiBytes = kXchgBytes + kTileBytes;
 constexpr int kUnitRing = 4;     // work units in flight between the roles
 
 enum { kUnitGateUp = 0, kUnitDown = 1, kUnitStop = -1 };
@@ -74,12 +79,15 @@ __device__ inline bool mbar_wait_drain(uint64_t* bar, uint32_t parity, Ctl* ctl,
 }
 
 // Epilogue role (warps 2..5, 128 threads): for each unit, read the fp32
-// accumulator from TMEM (lane = weight row, column = token), and write
+// accumulator from TMEM (lane = weight row, column = token), 32 tokens at a
+// time, and write
 //   gate_up: h[slot][m*64 + r] = gelu_tanh(gate_r) * up_r  (lane r pairs
 //            with lane 64 + r through smem), bf16;
-//   down:    y[slot][m*128 + r], fp32.
-// The leader does the waits and broadcasts the outcome, so the 128 threads
-// always pass the same named barriers.
+//   down:    y[slot][m*128 + r], bf16 (or fp32 when y_bf16 is off).
+// The bf16 values are transposed through a smem tile so that every global
+// store is a 16-byte piece of one token's row (coalesced rows instead of
+// 2-byte column scatters).  The leader does the waits and broadcasts the
+// outcome, so the 128 threads always pass the same named barriers.
 __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInfo* units,
                                               uint64_t* ufull, uint64_t* uempty, uint64_t* tfull,
                                               uint64_t* tempty, float* xchg,
@@ -87,101 +95,114 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
                                               uint32_t tmem_base, int acc_cols, int warp,
                                               int lane) {
   Ctl* ctl = a.ctl;
-    // ------------------------------------------------------------ epilogue
-    const int q4 = warp & 3;          // TMEM lane quarter this warp may access
-    const int row = q4 * 32 + lane;   // accumulator row (TMEM lane)
-    const int et = threadIdx.x - 64;  // 0..127
-    int ur = 0;
-    uint32_t uphase = 0;
-    int acc = 0;
-    uint32_t aphase = 0;
-    while (true) {
-      // The leader waits; the decision is broadcast so the 128 threads always
-      // take the same path through the named barriers below.
-      if (et == 0) {
-        bool ok = mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullEpi);
-        if (ok && units[ur].type != kUnitStop)
-          ok = mbar_wait(&tfull[acc], aphase, s_abort, ctl, a.timeout_ns, kWhereTmemFull);
-        *s_bcast = ok ? 1 : 0;
-      }
-      named_barrier(1, 128);
-      const bool ok = *s_bcast != 0;
-      const UnitInfo ui = units[ur];
-      named_barrier(1, 128);
-      if (!ok || ui.type == kUnitStop) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * acc_cols);
-      const int nch = (ui.n + 31) / 32;
-      if (ui.type == kUnitGateUp) {
-        __nv_bfloat16* hcol = a.h + (size_t)ui.slot0 * a.f + ui.m * kGuHalf + row;
-        for (int cc = 0; cc < nch; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tbase + cc * 32, v);
-          tmem_wait_ld();
-          if (row >= kGuHalf) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              xchg[(row - kGuHalf) * kXchgStride + i] = __uint_as_float(v[i]);
-          }
-          named_barrier(1, 128);
-          if (row < kGuHalf) {
-            const int cmax = min(32, ui.n - cc * 32);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (i < cmax) {
-                const float g = __uint_as_float(v[i]);
-                const float up = xchg[row * kXchgStride + i];
-                hcol[(size_t)(cc * 32 + i) * a.f] = __float2bfloat16(gelu_tanh(g) * up);
-              }
-            }
-          }
-          named_barrier(1, 128);
-        }
-      } else {
-        const size_t y0 = (size_t)ui.slot0 * a.d + ui.m * kBM + row;
-        for (int cc = 0; cc < nch; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tbase + cc * 32, v);
-          tmem_wait_ld();
-          const int cmax = min(32, ui.n - cc * 32);
-          if (a.y_bf16) {
-            __nv_bfloat16* ycol = static_cast<__nv_bfloat16*>(a.y) + y0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __float2bfloat16(__uint_as_float(v[i]));
-          } else {
-            float* ycol = static_cast<float*>(a.y) + y0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __uint_as_float(v[i]);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
-      }
-      if (ui.type == kUnitGateUp) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
-      }
-      if (ui.type == kUnitGateUp) __threadfence();  // h visible before the chunk counter
-      named_barrier(1, 128);
-      if (et == 0) {
-        if (ui.type == kUnitGateUp) {
-          __threadfence();
-          fence_proxy_async_global();
-          atomicAdd(a.ready + ui.q, 1);
-        }
-        mbar_arrive(&uempty[ur]);
-      }
-      if (++ur == kUnitRing) {
-        ur = 0;
-        uphase ^= 1;
-      }
-      acc ^= 1;
-      if (acc == 0) aphase ^= 1;
+  __nv_bfloat16* tile =
+      reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(xchg) + kXchgBytes);
+  const int q4 = warp & 3;          // TMEM lane quarter this warp may access
+  const int row = q4 * 32 + lane;   // accumulator row (TMEM lane)
+  const int et = threadIdx.x - 64;  // 0..127
+  int ur = 0;
+  uint32_t uphase = 0;
+  int acc = 0;
+  uint32_t aphase = 0;
+  while (true) {
+    // The leader waits; the decision is broadcast so the 128 threads always
+    // take the same path through the named barriers below.
+    if (et == 0) {
+      bool ok = mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullEpi);
+      if (ok && units[ur].type != kUnitStop)
+        ok = mbar_wait(&tfull[acc], aphase, s_abort, ctl, a.timeout_ns, kWhereTmemFull);
+      *s_bcast = ok ? 1 : 0;
     }
+    named_barrier(1, 128);
+    const bool ok = *s_bcast != 0;
+    const UnitInfo ui = units[ur];
+    named_barrier(1, 128);
+    if (!ok || ui.type == kUnitStop) break;
+    tc_fence_after();
+    const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * acc_cols);
+    const int nch = (ui.n + 31) / 32;
+    if (ui.type == kUnitGateUp) {
+      for (int cc = 0; cc < nch; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tbase + cc * 32, v);
+        tmem_wait_ld();
+        if (row >= kGuHalf) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            xchg[(row - kGuHalf) * kXchgStride + i] = __uint_as_float(v[i]);
+        }
+        named_barrier(1, 128);
+        const int cmax = min(32, ui.n - cc * 32);
+        if (row < kGuHalf) {  // tile[token][r], 64 columns
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float g = __uint_as_float(v[i]);
+            const float up = xchg[row * kXchgStride + i];
+            tile[i * kGuHalf + row] = __float2bfloat16(gelu_tanh(g) * up);
+          }
+        }
+        named_barrier(1, 128);
+        // 32 tokens x 128 bytes: eight 16-byte pieces per token
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int pc = et + 128 * k;
+          const int tok = pc >> 3, piece = pc & 7;
+          if (tok < cmax)
+            *reinterpret_cast<uint4*>(a.h + (size_t)(ui.slot0 + cc * 32 + tok) * a.f +
+                                      ui.m * kGuHalf + piece * 8) =
+                *reinterpret_cast<const uint4*>(tile + tok * kGuHalf + piece * 8);
+        }
+      }
+    } else {
+      const size_t y0 = (size_t)ui.slot0 * a.d + ui.m * kBM;
+      for (int cc = 0; cc < nch; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tbase + cc * 32, v);
+        tmem_wait_ld();
+        const int cmax = min(32, ui.n - cc * 32);
+        if (a.y_bf16) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) tile[i * kBM + row] = __float2bfloat16(__uint_as_float(v[i]));
+          named_barrier(1, 128);
+          // 32 tokens x 256 bytes: sixteen 16-byte pieces per token
+          __nv_bfloat16* y = static_cast<__nv_bfloat16*>(a.y) + y0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int pc = et + 128 * k;
+            const int tok = pc >> 4, piece = pc & 15;
+            if (tok < cmax)
+              *reinterpret_cast<uint4*>(y + (size_t)(cc * 32 + tok) * a.d + piece * 8) =
+                  *reinterpret_cast<const uint4*>(tile + tok * kBM + piece * 8);
+          }
+          named_barrier(1, 128);
+        } else {
+          float* ycol = static_cast<float*>(a.y) + y0 + row;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __uint_as_float(v[i]);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tempty[acc]);
+    if (ui.type == kUnitGateUp) __threadfence();  // h visible before the chunk counter
+    named_barrier(1, 128);
+    if (et == 0) {
+      if (ui.type == kUnitGateUp) {
+        __threadfence();
+        fence_proxy_async_global();
+        atomicAdd(a.ready + ui.q, 1);
+      }
+      mbar_arrive(&uempty[ur]);
+    }
+    if (++ur == kUnitRing) {
+      ur = 0;
+      uphase ^= 1;
+    }
+    acc ^= 1;
+    if (acc == 0) aphase ^= 1;
   }
+}
 
 }  // namespace moe

@@ -40,10 +40,9 @@ constexpr int kMaxStages = 8;
 constexpr int kRingBytes = 192 * 1024;
 constexpr int kScaleStride = 32;             // fp16 scales per row kept (d, f <= 4096)
 constexpr int kScaleBytes = kBM * kScaleStride * 2;
-constexpr int kXchgBytes = 64 * kXchgStride * 4;
 constexpr int kBarBytes = 8 * (2 * kMaxStages + 2 * kAStages + 4 + 2 * kUnitRing + 1);
 constexpr int kSmemBytes =
-    1024 + kRingBytes + kScaleBytes + kXchgBytes + kBarBytes + 256;
+    1024 + kRingBytes + kScaleBytes + kEpiBytes + kBarBytes + 256;
 static_assert(kAColBase + kAStages * kACols <= kTmemCols, "TMEM budget");
 
 enum { kWhereAFull = 20, kWhereAEmpty, kWhereDqFull };
@@ -111,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ring = smem;
   __half* sc = reinterpret_cast<__half*>(smem + kRingBytes);  // [kScaleStride][128]
   float* xchg = reinterpret_cast<float*>(smem + kRingBytes + kScaleBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kScaleBytes + kXchgBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kScaleBytes + kEpiBytes);
   uint64_t* empty = full + kMaxStages;
   uint64_t* afull = empty + kMaxStages;
   uint64_t* aempty = afull + kAStages;
@@ -186,6 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int ur = 0;
     uint32_t uphase = 0;
     uint32_t issued = 0, issued_par = 0;
+    // The first unit of CTA b is unit b; later ones come from the counter
+    // (offset by the grid), so every unit is claimed exactly once.
+    bool first_claim = true;
     while (true) {
       UnitInfo ui;
       ui.type = kUnitStop;
@@ -193,7 +195,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int go = 0;
       if (lane == 0 && !*s_abort) {
         go = 1;
-        const int u = atomicAdd(&ctl->work_next, 1);
+        const int u = first_claim ? (int)blockIdx.x
+                                  : (int)gridDim.x + atomicAdd(&ctl->work_next, 1);
+        first_claim = false;
         if (u < U) {
           int q, m;
           if (u < n_chunks * GU) {

@@ -460,7 +460,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ga.perm = p->perm;
   ga.x = static_cast<const __nv_bfloat16*>(x);
   ga.x_perm = p->x_perm;
-  {  // one launch (plan + gather) when T*k fits the fused kernel, else two
+  {
     ProfScope ps(p, MOE_K_PLAN, s);
     if (moe_launch_plan_gather(pa, ga, p->num_sms, s, p->pdl != 0) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -505,7 +505,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ca.out = static_cast<__nv_bfloat16*>(out);
   {
     ProfScope ps(p, MOE_K_COMBINE, s);
-    if (moe_launch_combine(ca, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe_launch_combine(ca, p->num_sms, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   p->last_T = T;
@@ -791,7 +791,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ca.y_bf16 = p->y_bf16;
   ca.residual = static_cast<const __nv_bfloat16*>(residual);
   ca.out = static_cast<__nv_bfloat16*>(out);
-  if (moe_launch_combine(ca, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe_launch_combine(ca, p->num_sms, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
 
   if (status_out && cudaMemcpyAsync(status_out, &ctl->status, sizeof(int32_t),
                                     cudaMemcpyDeviceToDevice, s) != cudaSuccess)

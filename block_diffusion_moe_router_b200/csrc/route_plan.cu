@@ -11,6 +11,8 @@
 // with the same id, found with one ballot per id bit), and per-(warp,
 // expert) counts are scanned in warp order, so the result is independent of
 // timing (bitwise deterministic).
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -56,8 +58,9 @@ __device__ __forceinline__ void plan_body(const PlanArgs& a, int* s_perm, bool w
 
   for (int i = tid; i < kPlanWarps * kMaxE; i += kPlanThreads) (&cnt[0][0])[i] = 0;
   if (tid == 0) s_maxc = 0;
-  pdl_wait();  // idx comes from the router
+  // The gather may launch at once: it waits for this grid to complete.
   pdl_launch_dependents();
+  pdl_wait();  // idx comes from the router
   __syncthreads();
 
   const int per = (A + kPlanWarps - 1) / kPlanWarps;
@@ -296,25 +299,30 @@ __device__ __forceinline__ void gather_row(const GatherArgs& a, int row, int t, 
 }
 
 __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
-  pdl_wait();
+  // The expert kernel may launch at once (its prologue then overlaps this
+  // grid); it waits for this grid to complete before reading the tables.
   pdl_launch_dependents();
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= a.rows) return;
-  gather_row<kGatherVec>(a, row, __ldg(a.perm + row), threadIdx.x & 31);
+  pdl_wait();
+  // grid-stride over rows: at most a few CTAs per SM, all resident at once
+  for (int row = blockIdx.x * 8 + (threadIdx.x >> 5); row < a.rows; row += gridDim.x * 8)
+    gather_row<kGatherVec>(a, row, __ldg(a.perm + row), threadIdx.x & 31);
 }
 
 // out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32, one
-// rounding).  A CTA covers kCombThreads 16-byte column groups of one token
-// (grid: tokens x column blocks), so many small CTAs are resident per SM;
-// each thread issues the loads of up to kCombK contributions before
-// accumulating them.  y is fp32 (4 values per load) or bf16 (8 values per
-// load, widened exactly).
-constexpr int kCombThreads = 256;
-constexpr int kCombK = 8;  // loads in flight per thread
+// rounding).  One token per CTA step (grid-stride over tokens, a few CTAs per
+// SM, so the whole grid is resident at once); a thread owns up to kCombCols
+// 16-byte column groups of the row and issues the loads of up to kCombK
+// contributions per column group before accumulating them.  slot_of and w of
+// the token are read by every thread (the same addresses: one L1 line).  y is
+// fp32 (4 values per load) or bf16 (8 values per load, widened exactly).
+constexpr int kCombThreads = 128;
+constexpr int kCombK = 8;         // contributions in flight per column group
+constexpr int kCombMaxD = 4096;   // d a CTA of kCombThreads covers
 
 template <typename YT>
 struct YVec {
-  static constexpr int n = 16 / (int)sizeof(YT);  // values per 16-byte load
+  static constexpr int n = 16 / (int)sizeof(YT);             // values per 16-byte load
+  static constexpr int cols = kCombMaxD / (kCombThreads * n);  // column groups per thread
 };
 
 __device__ __forceinline__ void widen(const uint4& r, const float*, float (&v)[4]) {
@@ -336,61 +344,72 @@ __device__ __forceinline__ void widen(const uint4& r, const __nv_bfloat16*, floa
 template <typename YT>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   constexpr int V = YVec<YT>::n;
-  __shared__ int sl[kMaxK];
-  __shared__ float wt[kMaxK];
+  constexpr int kCombCols = YVec<YT>::cols;
   const YT* y = static_cast<const YT*>(a.y);
   pdl_wait();
   pdl_launch_dependents();
-  const int t = blockIdx.x;
-  if (threadIdx.x < a.k) {
-    sl[threadIdx.x] = a.slot_of[(size_t)t * a.k + threadIdx.x];
-    wt[threadIdx.x] = a.w[(size_t)t * a.k + threadIdx.x];
-  }
-  __syncthreads();
   const int ncol = a.d / V;  // 16-byte column groups per row
-  const int col = blockIdx.y * kCombThreads + threadIdx.x;
-  if (col >= ncol) return;
-  float acc[V];
+  for (int t = blockIdx.x; t < a.T; t += gridDim.x) {
+    float acc[kCombCols][V];
 #pragma unroll
-  for (int i = 0; i < V; ++i) acc[i] = 0.f;
-  for (int j0 = 0; j0 < a.k; j0 += kCombK) {
-    uint4 r[kCombK];
+    for (int q = 0; q < kCombCols; ++q)
 #pragma unroll
-    for (int j = 0; j < kCombK; ++j)
-      if (j0 + j < a.k)
-        r[j] = __ldg(reinterpret_cast<const uint4*>(y + (size_t)sl[j0 + j] * a.d) + col);
+      for (int i = 0; i < V; ++i) acc[q][i] = 0.f;
+    for (int j0 = 0; j0 < a.k; j0 += kCombK) {
+      int sl[kCombK];
+      float wt[kCombK];
 #pragma unroll
-    for (int j = 0; j < kCombK; ++j) {
-      if (j0 + j < a.k) {
-        float v[V];
-        widen(r[j], y, v);
-        const float wj = wt[j0 + j];
+      for (int j = 0; j < kCombK; ++j) {
+        sl[j] = (j0 + j < a.k) ? __ldg(a.slot_of + (size_t)t * a.k + j0 + j) : 0;
+        wt[j] = (j0 + j < a.k) ? __ldg(a.w + (size_t)t * a.k + j0 + j) : 0.f;
+      }
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = fmaf(wj, v[i], acc[i]);
+      for (int q = 0; q < kCombCols; ++q) {
+        const int col = threadIdx.x + kCombThreads * q;
+        if (col >= ncol) break;
+        uint4 r[kCombK];
+#pragma unroll
+        for (int j = 0; j < kCombK; ++j)
+          if (j0 + j < a.k)
+            r[j] = __ldg(reinterpret_cast<const uint4*>(y + (size_t)sl[j] * a.d) + col);
+#pragma unroll
+        for (int j = 0; j < kCombK; ++j) {
+          if (j0 + j < a.k) {
+            float v[V];
+            widen(r[j], y, v);
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[q][i] = fmaf(wt[j], v[i], acc[q][i]);
+          }
+        }
       }
     }
-  }
-  const size_t o = (size_t)t * a.d + (size_t)V * col;
-  if (a.residual) {
 #pragma unroll
-    for (int i = 0; i < V; i += 4) {
-      const uint2 rr = *reinterpret_cast<const uint2*>(a.residual + o + i);
-      const float2 r0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rr.x));
-      const float2 r1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rr.y));
-      acc[i] = r0.x + acc[i];
-      acc[i + 1] = r0.y + acc[i + 1];
-      acc[i + 2] = r1.x + acc[i + 2];
-      acc[i + 3] = r1.y + acc[i + 3];
+    for (int q = 0; q < kCombCols; ++q) {
+      const int col = threadIdx.x + kCombThreads * q;
+      if (col >= ncol) break;
+      const size_t o = (size_t)t * a.d + (size_t)V * col;
+      if (a.residual) {
+#pragma unroll
+        for (int i = 0; i < V; i += 4) {
+          const uint2 rr = *reinterpret_cast<const uint2*>(a.residual + o + i);
+          const float2 r0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rr.x));
+          const float2 r1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rr.y));
+          acc[q][i] = r0.x + acc[q][i];
+          acc[q][i + 1] = r0.y + acc[q][i + 1];
+          acc[q][i + 2] = r1.x + acc[q][i + 2];
+          acc[q][i + 3] = r1.y + acc[q][i + 3];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < V; i += 4) {
+        __nv_bfloat162 o0 = __floats2bfloat162_rn(acc[q][i], acc[q][i + 1]);
+        __nv_bfloat162 o1 = __floats2bfloat162_rn(acc[q][i + 2], acc[q][i + 3]);
+        uint2 ov;
+        ov.x = *reinterpret_cast<uint32_t*>(&o0);
+        ov.y = *reinterpret_cast<uint32_t*>(&o1);
+        *reinterpret_cast<uint2*>(a.out + o + i) = ov;
+      }
     }
-  }
-#pragma unroll
-  for (int i = 0; i < V; i += 4) {
-    __nv_bfloat162 o0 = __floats2bfloat162_rn(acc[i], acc[i + 1]);
-    __nv_bfloat162 o1 = __floats2bfloat162_rn(acc[i + 2], acc[i + 3]);
-    uint2 ov;
-    ov.x = *reinterpret_cast<uint32_t*>(&o0);
-    ov.y = *reinterpret_cast<uint32_t*>(&o1);
-    *reinterpret_cast<uint2*>(a.out + o + i) = ov;
   }
 }
 
@@ -415,19 +434,20 @@ cudaError_t moe_launch_plan_gather(const moe::PlanArgs& a, const moe::GatherArgs
   (void)num_sms;
   const cudaError_t err = moe_launch_plan(a, s, pdl);
   if (err != cudaSuccess) return err;
-  return moe_launch_gather(g, s, pdl);
+  return moe_launch_gather(g, num_sms, s, pdl);
 }
 
-cudaError_t moe_launch_gather(const moe::GatherArgs& a, cudaStream_t s, bool pdl) {
+cudaError_t moe_launch_gather(const moe::GatherArgs& a, int num_sms, cudaStream_t s, bool pdl) {
   if (a.rows == 0) return cudaSuccess;
   static_assert(moe::kGatherVec * 32 * 8 >= 4096, "gather holds a whole row in registers");
-  return moe::launch_pdl(moe::gather_kernel, dim3((a.rows + 7) / 8), dim3(256), 0, s, pdl, a);
+  const int blocks = std::min((a.rows + 7) / 8, 4 * std::max(num_sms, 1));
+  return moe::launch_pdl(moe::gather_kernel, dim3(blocks), dim3(256), 0, s, pdl, a);
 }
 
-cudaError_t moe_launch_combine(const moe::CombineArgs& a, cudaStream_t s, bool pdl) {
+cudaError_t moe_launch_combine(const moe::CombineArgs& a, int num_sms, cudaStream_t s, bool pdl) {
   if (a.T == 0) return cudaSuccess;
-  const int per = a.y_bf16 ? 8 : 4;  // values per 16-byte column group
-  const dim3 grid(a.T, (a.d / per + moe::kCombThreads - 1) / moe::kCombThreads);
+  if (a.d > moe::kCombMaxD) return cudaErrorInvalidValue;
+  const dim3 grid(std::min(a.T, 8 * std::max(num_sms, 1)));
   if (a.y_bf16)
     return moe::launch_pdl(moe::combine_kernel<__nv_bfloat16>, grid, dim3(moe::kCombThreads), 0,
                            s, pdl, a);

@@ -245,8 +245,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const int E = a.E;
     // fp32 router_w rows in registers, three steps in flight: step i sits in
     // slot i % 3 and its slot is refilled with step i + 3 once split
-    float4 w0[kRowsPerThread], w1[kRowsPerThread], w2[kRowsPerThread];
-    auto load_rows = [&](float4 (&dst)[kRowsPerThread], int i) {
+    // (slot entry kRowsPerThread holds the step's four gamma values)
+    float4 w0[kRowsPerThread + 1], w1[kRowsPerThread + 1], w2[kRowsPerThread + 1];
+    auto load_rows = [&](float4 (&dst)[kRowsPerThread + 1], int i) {
       if (i >= nk) return;
       const int kb = kb0 + i;
 #pragma unroll
@@ -256,13 +257,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
                                                                   kb * kBK) + j)
                          : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      dst[kRowsPerThread] = __ldg(reinterpret_cast<const float4*>(a.gamma + kb * kBK) + j);
     };
     // split step i (rows in wr) into part buffer i % 2, then the x^2 of its x
     // tile; false when a wait gave up
-    auto step = [&](const float4 (&wr)[kRowsPerThread], int i) -> bool {
+    auto step = [&](const float4 (&wr)[kRowsPerThread + 1], int i) -> bool {
       const int st = i % kXStages;
       const int wb = i % kWBufs;
-      const float4 g = __ldg(reinterpret_cast<const float4*>(a.gamma + (kb0 + i) * kBK) + j);
+      const float4 g = wr[kRowsPerThread];
       const float g0 = 1.f + g.x, g1 = 1.f + g.y, g2 = 1.f + g.z, g3 = 1.f + g.w;
       // the part buffer is free once the UMMAs two steps back are done
       if (i >= kWBufs &&
