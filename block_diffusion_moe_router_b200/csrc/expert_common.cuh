@@ -97,6 +97,7 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
   Ctl* ctl = a.ctl;
   __nv_bfloat16* tile =
       reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(xchg) + kXchgBytes);
+  const uint64_t pol_keep = l2_policy_evict_last();  // h and y are read back soon
   const int q4 = warp & 3;          // TMEM lane quarter this warp may access
   const int row = q4 * 32 + lane;   // accumulator row (TMEM lane)
   const int et = threadIdx.x - 64;  // 0..127
@@ -148,9 +149,10 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
           const int pc = et + 128 * k;
           const int tok = pc >> 3, piece = pc & 7;
           if (tok < cmax)
-            *reinterpret_cast<uint4*>(a.h + (size_t)(ui.slot0 + cc * 32 + tok) * a.f +
-                                      ui.m * kGuHalf + piece * 8) =
-                *reinterpret_cast<const uint4*>(tile + tok * kGuHalf + piece * 8);
+            st_global_hint(a.h + (size_t)(ui.slot0 + cc * 32 + tok) * a.f + ui.m * kGuHalf +
+                               piece * 8,
+                           *reinterpret_cast<const uint4*>(tile + tok * kGuHalf + piece * 8),
+                           pol_keep);
         }
       }
     } else {
@@ -171,8 +173,9 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
             const int pc = et + 128 * k;
             const int tok = pc >> 4, piece = pc & 15;
             if (tok < cmax)
-              *reinterpret_cast<uint4*>(y + (size_t)(cc * 32 + tok) * a.d + piece * 8) =
-                  *reinterpret_cast<const uint4*>(tile + tok * kBM + piece * 8);
+              st_global_hint(y + (size_t)(cc * 32 + tok) * a.d + piece * 8,
+                             *reinterpret_cast<const uint4*>(tile + tok * kBM + piece * 8),
+                             pol_keep);
           }
           named_barrier(1, 128);
         } else {

@@ -292,9 +292,10 @@ __device__ __forceinline__ void gather_row(const GatherArgs& a, int row, int t, 
         }
       }
     }
+    const uint64_t pol_keep = l2_policy_evict_last();  // the expert kernel reads it next
 #pragma unroll
     for (int j = 0; j < VEC; ++j)
-      if (p0 + lane + 32 * j < n) dst[p0 + lane + 32 * j] = v[j];
+      if (p0 + lane + 32 * j < n) st_global_hint(dst + p0 + lane + 32 * j, v[j], pol_keep);
   }
 }
 
@@ -349,6 +350,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   pdl_wait();
   pdl_launch_dependents();
   const int ncol = a.d / V;  // 16-byte column groups per row
+  const uint64_t pol_drop = l2_policy_evict_first();
   for (int t = blockIdx.x; t < a.T; t += gridDim.x) {
     float acc[kCombCols][V];
 #pragma unroll
@@ -370,8 +372,9 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
         uint4 r[kCombK];
 #pragma unroll
         for (int j = 0; j < kCombK; ++j)
-          if (j0 + j < a.k)
-            r[j] = __ldg(reinterpret_cast<const uint4*>(y + (size_t)sl[j] * a.d) + col);
+          if (j0 + j < a.k)  // read once: let it leave L2
+            r[j] = ld_global_hint(reinterpret_cast<const uint4*>(y + (size_t)sl[j] * a.d) + col,
+                                  pol_drop);
 #pragma unroll
         for (int j = 0; j < kCombK; ++j) {
           if (j0 + j < a.k) {
