@@ -118,13 +118,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
 
   // B-operand rows per stage: the largest chunk, rounded up to the TMA box.
-  // The activation ring takes kMinB..kMaxB stages (as many as fit a quarter
-  // of the ring: small chunks get a deep one, to hide L2 latency), the
-  // weights the rest.
+  // The activation ring takes kMinB..kMaxB stages (as many as fit half of
+  // the ring: at 2048 tokens a chunk's B stage is larger than its A stage
+  // and its L2 latency must be hidden too), the weights the rest.
   const int maxn = max(1, min(kMaxN, ctl->max_chunk));
   const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
   const int b_bytes = NB * kBK * 2;
-  const int SB = min(kMaxB, max(kMinB, (kRingBytes / 4) / b_bytes));
+  const int SB = min(kMaxB, max(kMinB, (kRingBytes / 2) / b_bytes));
   const int SA = min(kMaxA, (kRingBytes - SB * b_bytes) / kABytes);
   uint8_t* ringA = ring;
   uint8_t* ringB = ring + SA * kABytes;

@@ -6,14 +6,19 @@
 //   reset of its counters; the gather of x rows into slot order; and the
 //   fixed-order weighted combine.
 //
-// One CTA of 32 warps does the counting sort: warp w owns a contiguous range
-// of assignments, ranks equal experts inside each 32-wide step (the lanes
-// with the same id, found with one ballot per id bit), and per-(warp,
-// expert) counts are scanned in warp order, so the result is independent of
-// timing (bitwise deterministic).
+// A cluster of CTAs of 32 warps (one per 2048 assignments, up to 16) does the
+// counting sort: each warp owns a contiguous range of assignments, ranks
+// equal experts inside each 32-wide step (the lanes with the same id, found
+// with one ballot per id bit), and per-(warp, expert) and per-(CTA, expert)
+// counts are scanned in order, so the result is independent of timing
+// (bitwise deterministic).
 #include <algorithm>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace moe {
 
@@ -22,7 +27,9 @@ namespace {
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kRegIters = 16;  // 32-wide steps per warp held in registers (16K assignments)
-constexpr int kPermSmem = kPlanWarps * 32 * kRegIters;  // perm staged in smem up to this many
+constexpr int kRegRange = kPlanWarps * 32 * kRegIters;  // per-CTA range kept in registers
+constexpr int kPlanMaxCluster = 16;
+constexpr int kPlanPerCta = 2048;  // assignments per CTA before another joins the cluster
 
 // Lanes of `mask` whose expert id equals this lane's: one ballot per bit of
 // the id (ids < 2^nbits), each narrowing the set to the lanes that agree on
@@ -39,16 +46,24 @@ __device__ __forceinline__ unsigned peer_lanes(unsigned mask, int e, int nbits) 
   return peers;
 }
 
-// The counting sort.  A `writer` CTA stores the tables (offsets, perm,
-// slot_of, chunk table, scheduler counters); with A <= kPermSmem the whole
-// perm is also left in s_perm.
-__device__ __forceinline__ void plan_body(const PlanArgs& a, int* s_perm, bool writer) {
+// The counting sort, on a cluster of NC CTAs: CTA r owns assignments
+// [r*A/NC, (r+1)*A/NC), warp w of it a contiguous sub-range.  Ranks inside a
+// warp's 32-wide steps come from ballots; per-(warp, expert) counts are
+// scanned in warp order, per-(CTA, expert) totals in rank order through
+// distributed shared memory, so every slot is independent of timing.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
+  extern __shared__ int s_perm[];  // [A] on a single CTA: perm built here, written in order
   __shared__ int cnt[kPlanWarps][kMaxE];  // per-warp counts, then per-warp bases
+  __shared__ int ctot[kMaxE];             // this CTA's per-expert totals (read by peers)
+  __shared__ int base[kMaxE];             // the expert's assignments in lower ranks
   __shared__ int tot[kMaxE];
   __shared__ int off[kMaxE + 1];
   __shared__ int cst[kMaxE + 1];
   __shared__ int wsum[2][kMaxE / 32];
   __shared__ int s_maxc;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int NC = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -63,16 +78,18 @@ __device__ __forceinline__ void plan_body(const PlanArgs& a, int* s_perm, bool w
   pdl_wait();  // idx comes from the router
   __syncthreads();
 
-  const int per = (A + kPlanWarps - 1) / kPlanWarps;
-  const int lo = min(A, warp * per);
-  const int hi = min(A, lo + per);
+  const int clo = (int)((long long)A * rank / NC);
+  const int chi = (int)((long long)A * (rank + 1) / NC);
+  const int per = (chi - clo + kPlanWarps - 1) / kPlanWarps;
+  const int lo = min(chi, clo + warp * per);
+  const int hi = min(chi, lo + per);
 
   // ---- local ranks.  With at most kRegIters 32-wide steps per warp the
   // expert ids and ranks stay in registers; longer ranges keep the rank in
   // slot_of until the bases are known.
   const int iters = (hi - lo + 31) / 32;
-  // uniform over the CTA: A <= kPermSmem gives every warp <= kRegIters steps
-  const bool in_regs = A <= kPermSmem;
+  // uniform over the CTA: a range of <= kRegRange gives every warp <= kRegIters steps
+  const bool in_regs = chi - clo <= kRegRange;
   int e_r[kRegIters], r_r[kRegIters];
   if (in_regs) {
     // every load of the warp's range in flight before the first use
@@ -106,8 +123,8 @@ __device__ __forceinline__ void plan_body(const PlanArgs& a, int* s_perm, bool w
       r_r[it] = rk;
     }
   } else {
-    for (int base = lo; base < hi; base += 32) {
-      const int as = base + lane;
+    for (int b0 = lo; b0 < hi; b0 += 32) {
+      const int as = b0 + lane;
       const bool act = as < hi;
       const unsigned mask = __ballot_sync(0xffffffffu, act);
       int e = act ? __ldg(a.idx + as) : 0;
@@ -128,7 +145,7 @@ __device__ __forceinline__ void plan_body(const PlanArgs& a, int* s_perm, bool w
   }
   __syncthreads();
 
-  // ---- per-expert totals; per-warp bases inside each expert's segment
+  // ---- per-expert bases: warps of this CTA, then the CTAs of the cluster
   if (tid < E) {
     int run = 0;
 #pragma unroll 8
@@ -137,8 +154,22 @@ __device__ __forceinline__ void plan_body(const PlanArgs& a, int* s_perm, bool w
       cnt[w][tid] = run;
       run += c;
     }
-    tot[tid] = run;
-    atomicMax(&s_maxc, min(run, a.chunk));
+    ctot[tid] = run;
+  }
+  if (NC > 1)
+    cluster.sync();
+  else
+    __syncthreads();
+  if (tid < E) {
+    int b = 0, t = 0;
+    for (int q = 0; q < NC; ++q) {
+      const int c = (q == rank) ? ctot[tid] : *cluster.map_shared_rank(&ctot[tid], q);
+      if (q < rank) b += c;
+      t += c;
+    }
+    base[tid] = b;
+    tot[tid] = t;
+    atomicMax(&s_maxc, min(t, a.chunk));
   }
   __syncthreads();
   // ---- exclusive scans of the totals (slots) and of the chunk counts,
@@ -180,51 +211,55 @@ __device__ __forceinline__ void plan_body(const PlanArgs& a, int* s_perm, bool w
     }
   }
   __syncthreads();
-  if (writer && tid == 0) {
-    a.ctl->n_chunks = cst[E];
-    a.ctl->max_chunk = s_maxc;
-    a.ctl->work_next = 0;
-  }
-  if (writer && tid <= E) a.offsets[tid] = off[tid];
-  if (writer && tid < E) {
-    for (int q = cst[tid]; q < cst[tid + 1]; ++q) {
-      a.chunk_e[q] = tid;
-      a.chunk_c[q] = q - cst[tid];
-      a.ready[q] = 0;
+  if (rank == 0) {
+    if (tid == 0) {
+      a.ctl->n_chunks = cst[E];
+      a.ctl->max_chunk = s_maxc;
+      a.ctl->work_next = 0;
+    }
+    if (tid <= E) a.offsets[tid] = off[tid];
+    if (tid < E) {
+      for (int q = cst[tid]; q < cst[tid + 1]; ++q) {
+        a.chunk_e[q] = tid;
+        a.chunk_c[q] = q - cst[tid];
+        a.ready[q] = 0;
+      }
     }
   }
 
-  // ---- final slots.  perm is a scatter; on the register path it is built
-  // in shared memory and written out in order (coalesced), since every
-  // store of this single CTA goes through one SM.
+  // ---- final slots.  perm is a scatter; a single CTA builds it in shared
+  // memory and writes it out in order (coalesced), since every store then
+  // goes through one SM.
   if (in_regs) {
+    const bool staged = NC == 1;
 #pragma unroll
     for (int it = 0; it < kRegIters; ++it) {
       if (it >= iters) break;
       const int as = lo + 32 * it + lane;
       if (as < hi) {
-        const int slot = off[e_r[it]] + cnt[warp][e_r[it]] + r_r[it];
-        if (writer) a.slot_of[as] = slot;
-        s_perm[slot] = as / a.k;
+        const int e = e_r[it];
+        const int slot = off[e] + base[e] + cnt[warp][e] + r_r[it];
+        a.slot_of[as] = slot;
+        if (staged)
+          s_perm[slot] = as / a.k;
+        else
+          a.perm[slot] = as / a.k;
       }
     }
-    __syncthreads();
-    if (writer)
+    if (staged) {
+      __syncthreads();
       for (int i = tid; i < A; i += kPlanThreads) a.perm[i] = s_perm[i];
+    }
   } else {
     for (int as = lo + lane; as < hi; as += 32) {
       int e = __ldg(a.idx + as);
       if (e < 0 || e >= E) e = 0;
-      const int slot = off[e] + cnt[warp][e] + a.slot_of[as];
+      const int slot = off[e] + base[e] + cnt[warp][e] + a.slot_of[as];
       a.slot_of[as] = slot;
       a.perm[slot] = as / a.k;
     }
   }
-}
-
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
-  extern __shared__ int s_perm[];  // [T*k] when the register path is taken
-  plan_body(a, s_perm, true);
+  if (NC > 1) cluster.sync();  // peers may still be reading ctot
 }
 
 // x rows in slot order: x_perm[s] = x[perm[s]], or, with gamma2, the
@@ -421,15 +456,36 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
 }  // namespace moe
 
 cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s, bool pdl) {
-  // in_regs (every warp's range fits kRegIters steps) <=> T*k <= kPermSmem
   const int A = a.T * a.k;
-  const size_t smem = A <= moe::kPermSmem ? (size_t)A * sizeof(int) : 0;
+  int nc = (A + moe::kPlanPerCta - 1) / moe::kPlanPerCta;
+  nc = std::max(1, std::min(nc, moe::kPlanMaxCluster));
+  if (nc > 8) {
+    const cudaError_t err = cudaFuncSetAttribute(
+        moe::plan_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (err != cudaSuccess) return err;
+  }
+  // a single CTA stages perm in shared memory (the whole range is in registers)
+  const size_t smem = (nc == 1 && A <= moe::kRegRange) ? (size_t)A * sizeof(int) : 0;
   if (smem > 0) {
     const cudaError_t err = cudaFuncSetAttribute(
         moe::plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
   }
-  return moe::launch_pdl(moe::plan_kernel, dim3(1), dim3(moe::kPlanThreads), smem, s, pdl, a);
+  if (nc == 1) return moe::launch_pdl(moe::plan_kernel, dim3(1), dim3(moe::kPlanThreads), smem, s, pdl, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nc);
+  cfg.blockDim = dim3(moe::kPlanThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nc;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, moe::plan_kernel, a);
 }
 
 cudaError_t moe_launch_plan_gather(const moe::PlanArgs& a, const moe::GatherArgs& g, int num_sms,

@@ -250,7 +250,9 @@ def test_int4_hot_expert_chunks():
     (40, 8, 8, 256, 128, False),     # E == k: every expert used
     (9, 1, 1, 128, 64, False),       # dense gated FFN
     (300, 33, 3, 384, 192, True),    # E not a multiple of 32, f not of 128
-    (2200, 16, 8, 128, 64, False),   # > 16K assignments: plan kernel's long-range path
+    (2200, 16, 8, 128, 64, False),   # > 16K assignments: a 9-CTA plan cluster
+    (2048, 128, 8, 128, 64, False),  # the encode routing shape: an 8-CTA plan cluster
+    (5000, 64, 8, 128, 64, True),    # 40K assignments: the 16-CTA plan cluster
 ])
 def test_edge_shapes(T, E, k, d, f, bias):
     lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=T + E, bias=bias)
