@@ -37,10 +37,13 @@ constexpr int kAStages = 4;                  // TMEM A stages
 constexpr int kACols = kBK4 / 2;             // 64 columns of bf16x2 per A stage
 constexpr int kAColBase = 2 * kChunkN;       // A stages after the accumulators
 constexpr int kMaxStages = 8;
-constexpr int kRingBytes = 192 * 1024;
+constexpr int kRingBytes = 168 * 1024;
 constexpr int kScaleStride = 32;             // fp16 scales per row kept (d, f <= 4096)
-constexpr int kScaleBytes = kBM * kScaleStride * 2;
-constexpr int kBarBytes = 8 * (2 * kMaxStages + 2 * kAStages + 4 + 2 * kUnitRing + 1);
+// One scale slot per unit-ring entry: the unit's 128 rows x G scales,
+// row-major as they sit in global memory (two 64-row blocks for gate_up).
+constexpr int kScaleSlot = kBM * kScaleStride * 2;
+constexpr int kScaleBytes = kUnitRing * kScaleSlot;
+constexpr int kBarBytes = 8 * (2 * kMaxStages + 2 * kAStages + 4 + 3 * kUnitRing + 1);
 constexpr int kSmemBytes =
     1024 + kRingBytes + kScaleBytes + kEpiBytes + kBarBytes + 256;
 static_assert(kAColBase + kAStages * kACols <= kTmemCols, "TMEM budget");
@@ -57,6 +60,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Untiled bulk copy global -> this CTA's shared memory (16-byte aligned
+// addresses, size a multiple of 16), completing `bytes` on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -108,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  __half* sc = reinterpret_cast<__half*>(smem + kRingBytes);  // [kScaleStride][128]
+  __half* sc = reinterpret_cast<__half*>(smem + kRingBytes);  // [kUnitRing][128][G]
   float* xchg = reinterpret_cast<float*>(smem + kRingBytes + kScaleBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kScaleBytes + kEpiBytes);
   uint64_t* empty = full + kMaxStages;
@@ -118,7 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* ufull = tempty + 2;
   uint64_t* uempty = ufull + kUnitRing;
-  uint64_t* drain = uempty + kUnitRing;
+  uint64_t* sfull = uempty + kUnitRing;  // the unit's scales have landed
+  uint64_t* drain = sfull + kUnitRing;
   UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 1);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(units + kUnitRing);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -147,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(&ufull[i], 1);
       mbar_init(&uempty[i], 2 + kDqWarps);
+      mbar_init(&sfull[i], 1);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -185,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int ur = 0;
     uint32_t uphase = 0;
     uint32_t issued = 0, issued_par = 0;
+    uint32_t sissued = 0, spar = 0;  // scale slots with a copy issued, and its parity
     // The first unit of CTA b is unit b; later ones come from the counter
     // (offset by the grid), so every unit is claimed exactly once.
     bool first_claim = true;
@@ -234,6 +250,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (go && mbar_wait(&uempty[ur], uphase ^ 1, s_abort, ctl, a.timeout_ns,
                             kWhereUnitEmpty)) {
+          if (ui.type != kUnitStop) {
+            // the unit's scales into its slot by bulk copy (rows are G
+            // contiguous fp16; 64-row blocks are multiples of 16 bytes)
+            __half* slot = sc + ur * (kScaleSlot / 2);
+            if (ui.type == kUnitGateUp) {
+              const int G = (a.d + kBK4 - 1) / kBK4;
+              const uint32_t blk = 64u * G * 2;
+              const size_t r0 = (size_t)ui.e * 2 * a.f + (size_t)ui.m * kGuHalf;
+              mbar_arrive_expect_tx(&sfull[ur], 2 * blk);
+              bulk_g2s(slot, a.scales_gu + r0 * G, blk, &sfull[ur]);
+              bulk_g2s(slot + 64 * G, a.scales_gu + (r0 + a.f) * G, blk, &sfull[ur]);
+            } else {
+              const int G = (a.f + kBK4 - 1) / kBK4;
+              const uint32_t blk = 128u * G * 2;
+              const size_t r0 = (size_t)ui.e * a.d + (size_t)ui.m * kBM;
+              mbar_arrive_expect_tx(&sfull[ur], blk);
+              bulk_g2s(slot, a.scales_d + r0 * G, blk, &sfull[ur]);
+            }
+            sissued |= 1u << ur;
+            spar = (spar & ~(1u << ur)) | (uphase << ur);
+          }
           units[ur] = ui;
           mbar_arrive(&ufull[ur]);
         } else {
@@ -288,10 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
     }
-    if (lane == 0)
+    if (lane == 0) {
       for (int s2 = 0; s2 < S; ++s2)
         if ((issued >> s2) & 1u)
           mbar_wait_drain(&full[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
+      for (int s2 = 0; s2 < kUnitRing; ++s2)
+        if ((sissued >> s2) & 1u)
+          mbar_wait_drain(&sfull[s2], (spar >> s2) & 1u, ctl, a.timeout_ns);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
@@ -380,6 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (true) {
       if (dt == 0) {
         bool ok = mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereDqFull);
+        if (ok && units[ur].type != kUnitStop)
+          ok = mbar_wait(&sfull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereDqFull);
         *s_dqbc = ok ? 1 : 0;
       }
       named_barrier(2, kDqWarps * 32);
@@ -387,20 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const UnitInfo ui = units[ur];
       named_barrier(2, kDqWarps * 32);
       if (!uok || ui.type == kUnitStop) break;
-      // this unit's fp16 scales: A row r -> weight row, one per group of 128
+      // this unit's fp16 scales (row-major [128][G], landed by the producer)
       const bool gu = ui.type == kUnitGateUp;
       const int C = gu ? a.d : a.f;
       const int G = (C + kBK4 - 1) / kBK4;
-      const __half* sg = gu ? a.scales_gu : a.scales_d;
-      for (int i = dt; i < kBM * G; i += kDqWarps * 32) {
-        const int r = i / G;
-        const int g = i - r * G;
-        const int wrow = gu ? (ui.e * 2 * a.f + (r < kGuHalf ? 0 : a.f) + ui.m * kGuHalf +
-                               (r & (kGuHalf - 1)))
-                            : (ui.e * a.d + ui.m * kBM + r);
-        sc[g * kBM + r] = sg[(size_t)wrow * G + g];  // group-major: conflict-free reads
-      }
-      named_barrier(2, kDqWarps * 32);
+      const __half* srow = sc + ur * (kScaleSlot / 2) + row * G;
       bool sok = true;
       bool pend = false;
       int pend_ast = 0;
@@ -418,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               cw[c] = *reinterpret_cast<const uint4*>(crow + ((c ^ sw) << 4));
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);  // codes are in registers
-            const float sf = __half2float(sc[kb * kBM + row]);
+            const float sf = __half2float(srow[kb]);
             const __nv_bfloat162 s2 = __float2bfloat162_rn(sf);
             const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) +
                                 (uint32_t)(kAColBase + ast * kACols);
@@ -461,8 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&afull[pend_ast]);
       }
-      named_barrier(2, kDqWarps * 32);  // sc[] is rewritten only after every warp is done
-      if (lane == 0) mbar_arrive(&uempty[ur]);
+      if (lane == 0) mbar_arrive(&uempty[ur]);  // this unit's slot (scales) is free
       if (++ur == kUnitRing) {
         ur = 0;
         uphase ^= 1;
