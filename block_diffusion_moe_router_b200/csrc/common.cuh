@@ -318,8 +318,7 @@ struct PlanArgs {
   int32_t* offsets;      // [E+1]
   int32_t* perm;         // [T*k] slot -> token
   int32_t* slot_of;      // [T*k] assignment -> slot
-  int32_t* chunk_e;      // [max_chunks] chunk -> expert
-  int32_t* chunk_c;      // [max_chunks] chunk -> chunk index within expert
+  int4* chunk_info;      // [max_chunks] chunk -> {expert, first slot, tokens, index in expert}
   int32_t* ready;        // [max_chunks] gate_up tiles finished per chunk
   Ctl* ctl;
 };
@@ -348,8 +347,7 @@ struct ExpertArgs {
   int T, E, k, d, f;
   const int32_t* perm;     // slot -> token
   const int32_t* offsets;
-  const int32_t* chunk_e;
-  const int32_t* chunk_c;
+  const int4* chunk_info;  // [max_chunks] {expert, first slot, tokens, index in expert}
   int32_t* ready;
   const __half* scales_gu;  // int4: [E, 2f, ceil(d/128)]
   const __half* scales_d;   // int4: [E, d, ceil(f/128)]

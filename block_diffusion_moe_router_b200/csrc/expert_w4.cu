@@ -202,8 +202,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t issued = 0, issued_par = 0;
     uint32_t sissued = 0, spar = 0;  // scale slots with a copy issued, and its parity
     // The first unit of CTA b is unit b; later ones come from the counter
-    // (offset by the grid), so every unit is claimed exactly once.
-    bool first_claim = true;
+    // (offset by the grid), so every unit is claimed exactly once.  The next
+    // claim is issued as soon as a unit is taken, so the atomic's round trip
+    // overlaps this unit's copies.
+    int u_next = (int)blockIdx.x;
     while (true) {
       UnitInfo ui;
       ui.type = kUnitStop;
@@ -211,9 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int go = 0;
       if (lane == 0 && !*s_abort) {
         go = 1;
-        const int u = first_claim ? (int)blockIdx.x
-                                  : (int)gridDim.x + atomicAdd(&ctl->work_next, 1);
-        first_claim = false;
+        const int u = u_next;
+        if (u < U) u_next = (int)gridDim.x + atomicAdd(&ctl->work_next, 1);
         if (u < U) {
           int q, m;
           if (u < n_chunks * GU) {
@@ -226,15 +227,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             q = v / DN;
             m = v - q * DN;
           }
-          const int e = a.chunk_e[q];
-          const int c = a.chunk_c[q];
-          const int seg0 = a.offsets[e];
-          const int ne = a.offsets[e + 1] - seg0;
-          ui.e = e;
+          const int4 ci = a.chunk_info[q];  // one load: expert, first slot, tokens
+          ui.e = ci.x;
           ui.m = m;
           ui.q = q;
-          ui.slot0 = seg0 + c * kChunkN;
-          ui.n = min(kChunkN, ne - c * kChunkN);
+          ui.slot0 = ci.y;
+          ui.n = ci.z;
           if (ui.n < 1 || ui.n > NB) {
             record_error(ctl, MOE_ERR_DEVICE_CHECK, 201);
             *s_abort = 1;

@@ -40,7 +40,8 @@ struct moe_plan_s {
   int last_T;
   void* ws;  // one device allocation holding everything below
   Ctl* ctl;
-  int32_t *idx, *perm, *slot_of, *offsets, *chunk_e, *chunk_c, *ready;
+  int32_t *idx, *perm, *slot_of, *offsets, *ready;
+  int4* chunk_info;
   float *w, *gap, *y;
   __nv_bfloat16 *x_perm, *h, *x_dev, *res_dev, *out_dev;
   std::vector<ProfRec> prof;
@@ -164,7 +165,7 @@ moe_status_t ensure_workspace(moe_plan_t p, int T) {
   const size_t o_ctl = take(sizeof(Ctl));
   const size_t o_idx = take(A * 4), o_w = take(A * 4), o_gap = take((size_t)cap * 4);
   const size_t o_perm = take(A * 4), o_slot = take(A * 4), o_off = take((size_t)(p->E + 1) * 4);
-  const size_t o_ce = take(MC * 4), o_cc = take(MC * 4), o_rd = take(MC * 4);
+  const size_t o_ci = take(MC * 16), o_rd = take(MC * 4);
   const size_t o_xp = take(A * p->d * 2);
   const size_t o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
   const size_t o_xd = take((size_t)cap * p->d * 2), o_rs = take((size_t)cap * p->d * 2);
@@ -190,8 +191,7 @@ moe_status_t ensure_workspace(moe_plan_t p, int T) {
   p->perm = reinterpret_cast<int32_t*>(b + o_perm);
   p->slot_of = reinterpret_cast<int32_t*>(b + o_slot);
   p->offsets = reinterpret_cast<int32_t*>(b + o_off);
-  p->chunk_e = reinterpret_cast<int32_t*>(b + o_ce);
-  p->chunk_c = reinterpret_cast<int32_t*>(b + o_cc);
+  p->chunk_info = reinterpret_cast<int4*>(b + o_ci);
   p->ready = reinterpret_cast<int32_t*>(b + o_rd);
   p->x_perm = reinterpret_cast<__nv_bfloat16*>(b + o_xp);
   p->h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
@@ -447,8 +447,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   pa.offsets = p->offsets;
   pa.perm = p->perm;
   pa.slot_of = p->slot_of;
-  pa.chunk_e = p->chunk_e;
-  pa.chunk_c = p->chunk_c;
+  pa.chunk_info = p->chunk_info;
   pa.ready = p->ready;
   pa.ctl = p->ctl;
 
@@ -474,8 +473,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ea.f = p->f;
   ea.perm = p->perm;
   ea.offsets = p->offsets;
-  ea.chunk_e = p->chunk_e;
-  ea.chunk_c = p->chunk_c;
+  ea.chunk_info = p->chunk_info;
   ea.ready = p->ready;
   ea.h = p->h;
   ea.y = p->y;
@@ -688,7 +686,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   const size_t o_ctl = take(sizeof(Ctl));
   const size_t o_idx = take(A * 4), o_w = take(A * 4), o_gap = take((size_t)T * 4);
   const size_t o_perm = take(A * 4), o_slot = take(A * 4), o_off = take((size_t)(p->E + 1) * 4);
-  const size_t o_ce = take(MC * 4), o_cc = take(MC * 4), o_rd = take(MC * 4);
+  const size_t o_ci = take(MC * 16), o_rd = take(MC * 4);
   const size_t o_xp = take(A * p->d * 2);
   const size_t o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
   if (sz > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
@@ -702,8 +700,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   int32_t* perm = reinterpret_cast<int32_t*>(b + o_perm);
   int32_t* slot_of = reinterpret_cast<int32_t*>(b + o_slot);
   int32_t* offsets = reinterpret_cast<int32_t*>(b + o_off);
-  int32_t* chunk_e = reinterpret_cast<int32_t*>(b + o_ce);
-  int32_t* chunk_c = reinterpret_cast<int32_t*>(b + o_cc);
+  int4* chunk_info = reinterpret_cast<int4*>(b + o_ci);
   int32_t* ready = reinterpret_cast<int32_t*>(b + o_rd);
   __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(b + o_xp);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
@@ -742,8 +739,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   pa.offsets = offsets;
   pa.perm = perm;
   pa.slot_of = slot_of;
-  pa.chunk_e = chunk_e;
-  pa.chunk_c = chunk_c;
+  pa.chunk_info = chunk_info;
   pa.ready = ready;
   pa.ctl = ctl;
 
@@ -766,8 +762,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ea.f = p->f;
   ea.perm = perm;
   ea.offsets = offsets;
-  ea.chunk_e = chunk_e;
-  ea.chunk_c = chunk_c;
+  ea.chunk_info = chunk_info;
   ea.ready = ready;
   ea.h = h;
   ea.y = y;

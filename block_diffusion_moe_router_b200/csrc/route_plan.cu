@@ -220,8 +220,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
     if (tid <= E) a.offsets[tid] = off[tid];
     if (tid < E) {
       for (int q = cst[tid]; q < cst[tid + 1]; ++q) {
-        a.chunk_e[q] = tid;
-        a.chunk_c[q] = q - cst[tid];
+        const int c = q - cst[tid];
+        a.chunk_info[q] = make_int4(tid, off[tid] + c * a.chunk, min(a.chunk, tot[tid] - c * a.chunk), c);
         a.ready[q] = 0;
       }
     }
