@@ -344,6 +344,154 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherArgs a) {
     gather_row<kGatherVec>(a, row, __ldg(a.perm + row), threadIdx.x & 31);
 }
 
+
+// Plan and gather in one launch for one canvas (T <= 256 tokens, T*k <=
+// 2048 assignments): every CTA runs the whole counting sort redundantly in
+// shared memory, CTA 0 alone writes the tables out, and each CTA then
+// gathers its share of rows straight from its own copy of perm.  This saves
+// the plan kernel's launch and one hand-off on the layer's critical path.
+//
+// Stable ranks from a token bitmap: thread t owns token t; bit t of row e is
+// set when token t chose expert e (a token's k experts are distinct).  The
+// rank of (t, e) among expert e's assignments in (t, j) order is the number
+// of set bits of row e below t: a per-word exclusive prefix of the row's
+// popcounts plus one masked popcount.
+constexpr int kSmallT = 256;   // tokens (= threads)
+constexpr int kSmallA = 2048;  // assignments
+constexpr int kSmallK = 8;     // experts per token
+constexpr int kSmallWords = kSmallT / 32;
+
+__global__ void __launch_bounds__(kSmallT) plan_gather_small_kernel(PlanArgs a, GatherArgs g) {
+  // word-major, so that lanes holding different experts hit different banks
+  __shared__ uint32_t bits[kSmallWords][kMaxE];  // 8 KB at E = 256
+  __shared__ int pre[kSmallWords][kMaxE];        // exclusive prefix popcounts per row
+  __shared__ int tot[kMaxE];
+  __shared__ int off[kMaxE + 1];
+  __shared__ int cst[kMaxE + 1];
+  __shared__ int wsum[2][kMaxE / 32];
+  __shared__ int s_maxc;
+  __shared__ int s_bad;
+  __shared__ int s_perm[kSmallA];
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int E = a.E;
+  const int T = a.T;
+  const int K = a.k;
+  const int A = T * K;
+  const bool writer = blockIdx.x == 0;
+
+  for (int i = tid; i < kMaxE * kSmallWords; i += kSmallT) (&bits[0][0])[i] = 0u;
+  if (tid == 0) {
+    s_maxc = 0;
+    s_bad = 0;
+  }
+  // The expert kernel may launch at once: it waits for this grid to complete.
+  pdl_launch_dependents();
+  pdl_wait();  // idx comes from the router
+  __syncthreads();
+
+  int ev[kSmallK];
+  const bool own = tid < T;
+  if (own) {
+#pragma unroll
+    for (int j = 0; j < kSmallK; ++j) {
+      if (j < K) {
+        int e = __ldg(a.idx + tid * K + j);
+        if (e < 0 || e >= E) {
+          s_bad = 1;
+          e = 0;
+        }
+        ev[j] = e;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kSmallK; ++j)
+      if (j < K) atomicOr(&bits[warp][ev[j]], 1u << lane);
+  }
+  __syncthreads();
+  if (tid < E) {  // row popcounts: exclusive prefix over the words, total
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kSmallWords; ++w) {
+      pre[w][tid] = run;
+      run += __popc(bits[w][tid]);
+    }
+    tot[tid] = run;
+    atomicMax(&s_maxc, min(run, a.chunk));
+  }
+  __syncthreads();
+  {  // exclusive scans of the totals and of the chunk counts (E <= 256 = threads)
+    const int n = (tid < E) ? tot[tid] : 0;
+    const int c = (n + a.chunk - 1) / a.chunk;
+    int sn = n, sc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yn = __shfl_up_sync(0xffffffffu, sn, o);
+      const int yc = __shfl_up_sync(0xffffffffu, sc, o);
+      if (lane >= o) {
+        sn += yn;
+        sc += yc;
+      }
+    }
+    if (lane == 31) {
+      wsum[0][warp] = sn;
+      wsum[1][warp] = sc;
+    }
+    __syncthreads();
+    int bn = 0, bc = 0;
+    for (int w = 0; w < warp; ++w) {
+      bn += wsum[0][w];
+      bc += wsum[1][w];
+    }
+    if (tid < E) {
+      off[tid + 1] = bn + sn;
+      cst[tid + 1] = bc + sc;
+    }
+    if (tid == 0) {
+      off[0] = 0;
+      cst[0] = 0;
+    }
+  }
+  __syncthreads();
+  if (writer) {
+    if (tid == 0) {
+      // a repeated expert in a token's set (or an id out of range) breaks
+      // the count; slots stay in range, the status word reports it
+      if (s_bad || off[E] != A) record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 101);
+      a.ctl->n_chunks = cst[E];
+      a.ctl->max_chunk = s_maxc;
+      a.ctl->work_next = 0;
+    }
+    if (tid <= E) a.offsets[tid] = off[tid];
+    if (tid < E) {
+      for (int q = cst[tid]; q < cst[tid + 1]; ++q) {
+        const int c = q - cst[tid];
+        a.chunk_info[q] =
+            make_int4(tid, off[tid] + c * a.chunk, min(a.chunk, tot[tid] - c * a.chunk), c);
+        a.ready[q] = 0;
+      }
+    }
+  }
+  if (own) {
+    const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+    for (int j = 0; j < kSmallK; ++j) {
+      if (j >= K) break;
+      const int e = ev[j];
+      const int slot = min(A - 1, off[e] + pre[warp][e] + __popc(bits[warp][e] & below));
+      if (writer) a.slot_of[tid * K + j] = slot;
+      s_perm[slot] = tid;
+    }
+  }
+  __syncthreads();
+  if (writer)
+    for (int i = tid; i < A; i += kSmallT) a.perm[i] = s_perm[i];
+  // this CTA's rows of x_perm (a warp per row)
+  for (int row = blockIdx.x * (kSmallT / 32) + warp; row < A; row += gridDim.x * (kSmallT / 32))
+    gather_row<kGatherVec>(g, row, s_perm[row], lane);
+}
+
 // out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32, one
 // rounding).  One token per CTA step (grid-stride over tokens, a few CTAs per
 // SM, so the whole grid is resident at once); a thread owns up to kCombCols
@@ -382,7 +530,21 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   constexpr int V = YVec<YT>::n;
   constexpr int kCombCols = YVec<YT>::cols;
   const YT* y = static_cast<const YT*>(a.y);
-  pdl_wait();
+  // slot_of and w of the CTA's first token before the wait: they come from
+  // the router and the plan, which completed before the expert kernel (this
+  // grid's predecessor) could let this grid launch.
+  int sl0[kCombK];
+  float wt0[kCombK];
+  {
+    const int t = blockIdx.x;
+#pragma unroll
+    for (int j = 0; j < kCombK; ++j) {
+      const bool in = t < a.T && j < a.k;
+      sl0[j] = in ? __ldg(a.slot_of + (size_t)t * a.k + j) : 0;
+      wt0[j] = in ? __ldg(a.w + (size_t)t * a.k + j) : 0.f;
+    }
+  }
+  pdl_wait();  // y comes from the expert kernel
   pdl_launch_dependents();
   const int ncol = a.d / V;  // 16-byte column groups per row
   const uint64_t pol_drop = l2_policy_evict_first();
@@ -395,10 +557,11 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
     for (int j0 = 0; j0 < a.k; j0 += kCombK) {
       int sl[kCombK];
       float wt[kCombK];
+      const bool pre = t == (int)blockIdx.x && j0 == 0;
 #pragma unroll
       for (int j = 0; j < kCombK; ++j) {
-        sl[j] = (j0 + j < a.k) ? __ldg(a.slot_of + (size_t)t * a.k + j0 + j) : 0;
-        wt[j] = (j0 + j < a.k) ? __ldg(a.w + (size_t)t * a.k + j0 + j) : 0.f;
+        sl[j] = pre ? sl0[j] : (j0 + j < a.k) ? __ldg(a.slot_of + (size_t)t * a.k + j0 + j) : 0;
+        wt[j] = pre ? wt0[j] : (j0 + j < a.k) ? __ldg(a.w + (size_t)t * a.k + j0 + j) : 0.f;
       }
 #pragma unroll
       for (int q = 0; q < kCombCols; ++q) {
@@ -490,7 +653,12 @@ cudaError_t moe_launch_plan(const moe::PlanArgs& a, cudaStream_t s, bool pdl) {
 
 cudaError_t moe_launch_plan_gather(const moe::PlanArgs& a, const moe::GatherArgs& g, int num_sms,
                                    cudaStream_t s, bool pdl) {
-  (void)num_sms;
+  const int A = a.T * a.k;
+  if (a.T <= moe::kSmallT && a.k <= moe::kSmallK && g.rows == A) {  // one launch
+    const int blocks = std::max(1, std::min((A + 7) / 8, 4 * std::max(num_sms, 1)));
+    return moe::launch_pdl(moe::plan_gather_small_kernel, dim3(blocks), dim3(moe::kSmallT), 0, s,
+                           pdl, a, g);
+  }
   const cudaError_t err = moe_launch_plan(a, s, pdl);
   if (err != cudaSuccess) return err;
   return moe_launch_gather(g, num_sms, s, pdl);
