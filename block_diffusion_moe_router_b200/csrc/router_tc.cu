@@ -10,8 +10,8 @@
 // Exactness of the tensor-core logits: the logit is
 //   z_e = (sum_i x_i * W'_ei) / rms(x),  W'_ei = router_w[e][i] * (1 + gamma_i)
 // with x already bf16.  W' (fp32, 24-bit significand) is split exactly into
-// three bf16 terms hi + mid + lo (each captures the next 8 bits), so every
-// product x_i * part is exact in fp32, and all three parts accumulate into
+// three bf16 terms hi + mid + lo (successive 8-bit pieces of the significand),
+// so every product x_i * part is exact in fp32, and all three parts accumulate into
 // the same fp32 TMEM accumulator: the logits carry fp32 accumulation error
 // only, as an FFMA dot product would.
 //
@@ -76,19 +76,25 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// v = w * g split into bf16 hi + mid + lo (exact: each residual is exact in
-// fp32 and the last one fits 8 bits), packed two per 32-bit word.
+// v = w * g split into bf16 hi + mid + lo, packed two per 32-bit word, by
+// truncation: hi keeps the top 16 bits of v's fp32 pattern (sign, exponent,
+// 7 mantissa bits), r = v - hi is exact and holds the remaining 16 bits of
+// significand, mid = trunc(r) its top 8, and lo = r - mid has at most 8
+// significant bits, so it is already a bf16 value.  hi + mid + lo == v
+// exactly, with only logic ops and subtractions on the dependency chain.
+__device__ __forceinline__ float trunc_bf16(float v) {
+  return __uint_as_float(__float_as_uint(v) & 0xFFFF0000u);
+}
+__device__ __forceinline__ uint32_t pack_hi16(float a, float b) {  // (a, b) as bf16x2
+  return __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x7632);
+}
 __device__ __forceinline__ void split3(float v0, float v1, uint32_t& hi, uint32_t& mid,
                                        uint32_t& lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-  const float2 hf = __bfloat1622float2(h);
-  const float r0 = v0 - hf.x, r1 = v1 - hf.y;
-  const __nv_bfloat162 m = __floats2bfloat162_rn(r0, r1);
-  const float2 mf = __bfloat1622float2(m);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(r0 - mf.x, r1 - mf.y);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  mid = *reinterpret_cast<const uint32_t*>(&m);
-  lo = *reinterpret_cast<const uint32_t*>(&l);
+  const float r0 = v0 - trunc_bf16(v0), r1 = v1 - trunc_bf16(v1);
+  const float q0 = r0 - trunc_bf16(r0), q1 = r1 - trunc_bf16(r1);
+  hi = pack_hi16(v0, v1);
+  mid = pack_hi16(r0, r1);
+  lo = pack_hi16(q0, q1);
 }
 
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, int rank) {
