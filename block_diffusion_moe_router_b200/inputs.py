@@ -11,6 +11,7 @@ per-expert intermediate 704, symmetric int4 weights in groups of 128):
   tiny     T=16,   d=256,  E=16,  k=2, f=64,  bf16 weights
   canvas   T=256,  d=2816, E=128, k=8, f=704, bf16 weights
   canvas4  T=256,  d=2816, E=128, k=8, f=704, int4 w4g128 weights + fp16 scales
+  canvas8  T=256,  d=2816, E=128, k=8, f=704, fp8 E4M3 weights + fp32 row scales
   encode   T=2048, d=2816, E=128, k=8, f=704, bf16 weights (prompt + canvas)
   stack30  30 layers of `canvas`, distinct weights, Zipf(1.1)-skewed router bias,
            residual carried between layers, experts reading the (1+gamma2)
@@ -19,7 +20,11 @@ per-expert intermediate 704, symmetric int4 weights in groups of 128):
 Distributions: x ~ N(0,1) rounded to bf16; router W ~ N(0, 1/d) (variance 1/d,
 so logits have unit scale) in fp32; gamma ~ N(0, 0.1^2) in fp32; expert weights
 ~ N(0, 0.02^2) rounded to bf16; int4 codes uniform on [-8, 7] and scales
-U(0.001, 0.01) rounded to fp16.  Seeds: 1000*workload_id + 10*layer + tensor_id.
+U(0.001, 0.01) rounded to fp16; fp8 codes: N(0, 64^2) draws clamped to
++-448 and rounded to E4M3 by torch's float8_e4m3fn cast (the codes span the
+format, a few subnormals included), row scales U(0.5, 1.5) * 0.02 / 64 in
+fp32 (so the weights are about N(0, 0.02^2) like the bf16 ones).
+Seeds: 1000*workload_id + 10*layer + tensor_id.
 
 Layouts (all row-major, contiguous):
   x            [T, d]            bf16
@@ -30,9 +35,11 @@ Layouts (all row-major, contiguous):
   w_gate_up    [E, 2f, d]        bf16 (rows [0,f) gate, [f,2f) up)
                [E, 2f, d/2]      uint8 for int4 (element i in byte i/2, low
                                  nibble for even i, 4-bit two's complement)
-  w_down       [E, d, f]         bf16, or [E, d, f/2] uint8 for int4
-  scales_gu    [E, 2f, ceil(d/128)] fp16 (int4 only)
-  scales_d     [E, d, ceil(f/128)]  fp16 (int4 only)
+               [E, 2f, d]        uint8 for fp8 (E4M3 bytes)
+  w_down       [E, d, f]         bf16, or [E, d, f/2] uint8 for int4, or
+                                 [E, d, f] uint8 for fp8
+  scales_gu    [E, 2f, ceil(d/128)] fp16 (int4), [E, 2f] fp32 (fp8)
+  scales_d     [E, d, ceil(f/128)]  fp16 (int4), [E, d] fp32 (fp8)
 """
 from __future__ import annotations
 
@@ -46,6 +53,8 @@ GROUP = 128  # int4 quantisation group along the input dimension
 
 WDTYPE_BF16 = 0
 WDTYPE_INT4 = 1
+WDTYPE_FP8 = 2
+FP8_CODE_STD = 64.0   # spread of the E4M3 code draws
 
 
 @dataclasses.dataclass(frozen=True)
@@ -78,6 +87,8 @@ WORKLOADS = {
     "canvas": Workload("canvas", 1, T=256, d=2816, E=128, k=8, f=704),
     "canvas4": Workload("canvas4", 2, T=256, d=2816, E=128, k=8, f=704,
                         wdtype=WDTYPE_INT4, act_wid=1),
+    "canvas8": Workload("canvas8", 5, T=256, d=2816, E=128, k=8, f=704,
+                        wdtype=WDTYPE_FP8, act_wid=1),
     "encode": Workload("encode", 3, T=2048, d=2816, E=128, k=8, f=704),
     "stack30": Workload("stack30", 4, T=256, d=2816, E=128, k=8, f=704,
                         layers=30, zipf_s=1.1, residual=True, expert_norm=True),
@@ -139,6 +150,20 @@ def make_int4(shape, seed_codes, seed_scales, device):
     return pack_int4(codes), scales
 
 
+def make_fp8(shape, seed_codes, seed_scales, device):
+    """Random E4M3 codes (uint8 bytes) and fp32 scales, one per row: the
+    codes are N(0, 64^2) draws clamped to +-448 and rounded to E4M3 by
+    torch's float8_e4m3fn cast (no NaN code can come out); the scales are
+    U(0.5, 1.5) * 0.02 / 64."""
+    E, rows, cols = shape
+    v = _randn((E, rows, cols), FP8_CODE_STD, seed_codes, device, torch.float32)
+    codes = v.clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    gs = _gen(seed_scales, device)
+    scales = (torch.rand((E, rows), generator=gs, device=device, dtype=torch.float32) + 0.5) \
+        * (0.02 / FP8_CODE_STD)
+    return codes, scales
+
+
 def zipf_bias(E: int, s: float, seed: int, device) -> torch.Tensor:
     """Router bias whose exp() follows a Zipf(s) law over a seeded random
     ranking of the experts: b_e = -s * ln(rank_e), rank_e in 1..E."""
@@ -171,10 +196,11 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T: Optional[int] = Non
         out["scales_gate_up"] = None
         out["scales_down"] = None
     else:
-        out["w_gate_up"], out["scales_gate_up"] = make_int4(
+        mk = make_fp8 if w.wdtype == WDTYPE_FP8 else make_int4
+        out["w_gate_up"], out["scales_gate_up"] = mk(
             (w.E, 2 * w.f, w.d), seed_for(w.wid, layer, _TID_WGU),
             seed_for(w.wid, layer, _TID_SGU), device)
-        out["w_down"], out["scales_down"] = make_int4(
+        out["w_down"], out["scales_down"] = mk(
             (w.E, w.d, w.f), seed_for(w.wid, layer, _TID_WD),
             seed_for(w.wid, layer, _TID_SD), device)
     return out
@@ -199,7 +225,7 @@ def make_small(T, d, E, k, f, seed, wdtype=WDTYPE_BF16, bias=False, residual=Fal
         out["scales_gate_up"] = None
         out["scales_down"] = None
     else:
-        out["w_gate_up"], out["scales_gate_up"] = make_int4((E, 2 * f, d), base + 6, base + 8,
-                                                            device)
-        out["w_down"], out["scales_down"] = make_int4((E, d, f), base + 7, base + 9, device)
+        mk = make_fp8 if wdtype == WDTYPE_FP8 else make_int4
+        out["w_gate_up"], out["scales_gate_up"] = mk((E, 2 * f, d), base + 6, base + 8, device)
+        out["w_down"], out["scales_down"] = mk((E, d, f), base + 7, base + 9, device)
     return out

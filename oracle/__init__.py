@@ -17,6 +17,7 @@ from .oracle import (  # noqa: F401
     weight_row,
     decode_bf16,
     decode_fp16,
+    decode_e4m3,
     set_threads,
     get_threads,
 )

@@ -18,7 +18,11 @@
  *        down_proj 704->2816; quantization_config bits 4, group_size 128,
  *        sym True, data_type int).
  *  [RF]  Hugging Face card "kingjones777/DiffusionGemma-26B-A4B-it-ROCmFP4-GGUF":
- *        header (128 experts / top-8).
+ *        header (128 experts / top-8; FP4 / FP8 builds of the weights) and its
+ *        finding that at a 256-token canvas the 8-bit build steps faster.
+ *  [OCP] OCP 8-bit Floating Point Specification (OFP8), E4M3 encoding: the
+ *        8-bit float format of the fp8 weight storage (the pages name FP8
+ *        builds but do not define the encoding).
  *
  * Where the pages are silent this file follows the readings adopted by the
  * library (they are listed once, here):
@@ -34,10 +38,12 @@
  *  - router bias (optional) is added to the logits before the softmax;
  *  - int4: element i of a row sits in byte i/2, low nibble for even i, 4-bit
  *    two's complement; w = code * scale[i / 128] with fp16 scales, exact here;
+ *  - fp8: element i of a row is byte i, an E4M3 value [OCP]; w = value *
+ *    scale[row] with one fp32 scale per weight row (output channel), exact;
  *  - out = residual + sum_j w_j y_j, summed in j order (residual optional).
  *
  * Everything is computed in double precision from the exact bf16 / fp16 /
- * int4 values the GPU receives; nothing is rounded in between.
+ * int4 / fp8 values the GPU receives; nothing is rounded in between.
  */
 #include <math.h>
 #include <stdint.h>
@@ -49,6 +55,7 @@
 
 #define ORACLE_W_BF16 0
 #define ORACLE_W_INT4 1
+#define ORACLE_W_FP8 2
 #define ORACLE_GROUP 128
 
 /* ---- scalar decoders (IEEE definitions) -------------------------------- */
@@ -76,6 +83,24 @@ static double fp16_to_double(uint16_t h) {
   return sign ? -v : v;
 }
 
+/* OFP8 E4M3 [OCP]: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits;
+ * exponent 0 is subnormal (m/8 * 2^-6); exponent 15 with mantissa 7 is NaN
+ * (the format has no infinities, so 15 with mantissa 0..6 is an ordinary
+ * binade: the largest value is 1.75 * 2^8 = 448). */
+static double e4m3_to_double(uint8_t b) {
+  int sign = (b >> 7) & 1;
+  int ex = (b >> 3) & 0xf;
+  int man = b & 0x7;
+  double v;
+  if (ex == 0xf && man == 0x7)
+    v = NAN;
+  else if (ex == 0)
+    v = ldexp((double)man, -9); /* man/8 * 2^-6 */
+  else
+    v = ldexp(1.0 + man / 8.0, ex - 7);
+  return sign ? -v : v;
+}
+
 /* 4-bit two's complement code of element i of a packed row. */
 static int int4_code(const uint8_t* row, int i) {
   int byte = row[i / 2];
@@ -83,18 +108,23 @@ static int int4_code(const uint8_t* row, int i) {
   return nib >= 8 ? nib - 16 : nib;
 }
 
-/* One expert-weight element W[e][r][i] of a [E, R, C] weight in either
- * storage format.  int4: code * fp16 scale of group i/128 ([AR] w4g128). */
-static double weight_elem(int wdtype, const void* w, const uint16_t* scales, int R, int C, int e,
+/* One expert-weight element W[e][r][i] of a [E, R, C] weight in any of the
+ * storage formats.  int4: code * fp16 scale of group i/128 ([AR] w4g128);
+ * fp8: E4M3 value * fp32 scale of the row. */
+static double weight_elem(int wdtype, const void* w, const void* scales, int R, int C, int e,
                           int r, int i) {
   size_t row = (size_t)e * R + r;
   if (wdtype == ORACLE_W_BF16) {
     const uint16_t* wb = (const uint16_t*)w;
     return bf16_to_double(wb[row * C + i]);
   }
+  if (wdtype == ORACLE_W_FP8) {
+    const uint8_t* wp = (const uint8_t*)w + row * (size_t)C;
+    return e4m3_to_double(wp[i]) * (double)((const float*)scales)[row];
+  }
   const uint8_t* wp = (const uint8_t*)w + row * (size_t)(C / 2);
   int ng = (C + ORACLE_GROUP - 1) / ORACLE_GROUP;
-  double s = fp16_to_double(scales[row * ng + i / ORACLE_GROUP]);
+  double s = fp16_to_double(((const uint16_t*)scales)[row * ng + i / ORACLE_GROUP]);
   return (double)int4_code(wp, i) * s;
 }
 
@@ -169,7 +199,7 @@ void oracle_route_weights(int E, int k, const double* z, const int32_t* idx, dou
  *   h_r = gelu_tanh(g_r) * v_r
  *   y_m = sum_r Wd[e][m][r] h_r                                    (m < d) */
 void oracle_expert_ffn(int d, int f, int wdtype, const void* w_gu, const void* w_d,
-                       const uint16_t* s_gu, const uint16_t* s_d, int e, const double* x,
+                       const void* s_gu, const void* s_d, int e, const double* x,
                        double* y, double* h_out) {
   double* h = (double*)malloc(sizeof(double) * (size_t)f);
   for (int r = 0; r < f; r++) {
@@ -190,7 +220,7 @@ void oracle_expert_ffn(int d, int f, int wdtype, const void* w_gu, const void* w
 }
 
 /* Dequantised (or widened) row r of expert e of a [E, R, C] weight. */
-void oracle_weight_row(int wdtype, const void* w, const uint16_t* scales, int R, int C, int e,
+void oracle_weight_row(int wdtype, const void* w, const void* scales, int R, int C, int e,
                        int r, double* out) {
   for (int i = 0; i < C; i++) out[i] = weight_elem(wdtype, w, scales, R, C, e, r, i);
 }
@@ -252,7 +282,7 @@ void oracle_route(int T, int E, int k, int d, const uint16_t* x, const float* ro
 void oracle_moe_forward(int T, int E, int k, int d, int f, int wdtype, const uint16_t* x,
                         const float* router_w, const float* gamma, const float* bias,
                         const float* expert_gamma, double eps, const void* w_gu,
-                        const void* w_d, const uint16_t* s_gu, const uint16_t* s_d,
+                        const void* w_d, const void* s_gu, const void* s_d,
                         const uint16_t* residual, const int32_t* forced_idx, double* out,
                         int32_t* idx_out, double* w_out, double* gap_out) {
 #pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_get_threads())
@@ -307,4 +337,8 @@ void oracle_decode_bf16(int n, const uint16_t* in, double* out) {
 
 void oracle_decode_fp16(int n, const uint16_t* in, double* out) {
   for (int i = 0; i < n; i++) out[i] = fp16_to_double(in[i]);
+}
+
+void oracle_decode_e4m3(int n, const uint8_t* in, double* out) {
+  for (int i = 0; i < n; i++) out[i] = e4m3_to_double(in[i]);
 }

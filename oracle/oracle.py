@@ -22,6 +22,7 @@ _lib = None
 
 W_BF16 = 0
 W_INT4 = 1
+W_FP8 = 2
 
 
 def build(force: bool = False) -> str:
@@ -58,6 +59,7 @@ def lib():
             L.oracle_weight_row.argtypes = [I, P, P, I, I, I, I, P]
             L.oracle_decode_bf16.argtypes = [I, P, P]
             L.oracle_decode_fp16.argtypes = [I, P, P]
+            L.oracle_decode_e4m3.argtypes = [I, P, P]
             L.oracle_set_threads.argtypes = [I]
             L.oracle_get_threads.restype = I
             _lib = L
@@ -85,6 +87,15 @@ def _np(t, dtype=None):
     if dtype is not None and a.dtype != dtype:
         a = a.astype(dtype)
     return a
+
+
+def _wdtype(w, scales) -> int:
+    """Storage format of a weight array: bf16 (uint16 bits), int4 (packed
+    bytes with fp16 scales) or fp8 E4M3 (one byte per weight, fp32 row
+    scales)."""
+    if w.dtype != np.uint8:
+        return W_BF16
+    return W_FP8 if scales is not None and scales.dtype == np.float32 else W_INT4
 
 
 def _p(a):
@@ -168,10 +179,10 @@ def moe_forward(x, router_w, router_gamma, router_bias, w_gate_up, w_down, k: in
     eg = _np(expert_gamma, np.float32)
     T, d = x.shape
     E = rw.shape[0]
-    wdtype = W_INT4 if wgu.dtype == np.uint8 else W_BF16
+    wdtype = _wdtype(wgu, sgu)
     f = wgu.shape[1] // 2
     assert wgu.shape[0] == E and wd.shape[0] == E
-    if wdtype == W_INT4:
+    if wdtype != W_BF16:
         assert sgu is not None and sd is not None
     out = np.empty((T, d), np.float64)
     idx = np.empty((T, k), np.int32)
@@ -192,7 +203,7 @@ def expert_ffn(x_row, e: int, w_gate_up, w_down, scales_gate_up=None, scales_dow
     sd = _np(scales_down)
     d = x_row.size
     f = wgu.shape[1] // 2
-    wdtype = W_INT4 if wgu.dtype == np.uint8 else W_BF16
+    wdtype = _wdtype(wgu, sgu)
     y = np.empty(d, np.float64)
     h = np.empty(f, np.float64)
     lib().oracle_expert_ffn(d, f, wdtype, _p(wgu), _p(wd), _p(sgu), _p(sd), int(e), _p(x_row),
@@ -204,7 +215,7 @@ def weight_row(w, scales, e: int, r: int, cols: int) -> np.ndarray:
     """Row r of expert e of a [E,R,C] weight, widened / dequantised to fp64."""
     w = _np(w)
     s = _np(scales)
-    wdtype = W_INT4 if w.dtype == np.uint8 else W_BF16
+    wdtype = _wdtype(w, s)
     R = w.shape[1]
     out = np.empty(cols, np.float64)
     lib().oracle_weight_row(wdtype, _p(w), _p(s), R, cols, int(e), int(r), _p(out))
@@ -222,4 +233,12 @@ def decode_fp16(t) -> np.ndarray:
     a = _np(t)
     out = np.empty(a.shape, np.float64)
     lib().oracle_decode_fp16(a.size, _p(a), _p(out))
+    return out
+
+
+def decode_e4m3(t) -> np.ndarray:
+    """E4M3 bytes (uint8) -> float64 values (NaN for the NaN codes)."""
+    a = _np(t, np.uint8)
+    out = np.empty(a.shape, np.float64)
+    lib().oracle_decode_e4m3(a.size, _p(a), _p(out))
     return out

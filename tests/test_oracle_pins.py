@@ -23,10 +23,13 @@ EPS = 1e-6
 
 
 def dense_weights(w, scales, cols):
-    """[E,R,C] weight as float64 from its storage (bf16, or int4 codes x fp16
-    scales) -- written from the storage format, not from the oracle."""
+    """[E,R,C] weight as float64 from its storage (bf16, int4 codes x fp16
+    group scales, or E4M3 bytes x fp32 row scales) -- written from the
+    storage format with library casts, not from the oracle."""
     if scales is None:
         return w.double()
+    if scales.dtype == torch.float32:  # fp8: torch's own E4M3 decode
+        return w.view(torch.float8_e4m3fn).double() * scales.double()[..., None]
     codes = inputs.unpack_int4(w).double()
     s = scales.double().repeat_interleave(inputs.GROUP, dim=-1)[..., :cols]
     return codes * s
@@ -209,6 +212,8 @@ def test_tie_break_duplicated_router_rows():
     (3, 5, 5, False, True, inputs.WDTYPE_INT4, False),
     (4, 16, 2, True, True, inputs.WDTYPE_BF16, True),
     (5, 8, 3, False, False, inputs.WDTYPE_INT4, True),
+    (6, 16, 4, True, True, inputs.WDTYPE_FP8, False),
+    (7, 8, 2, False, False, inputs.WDTYPE_FP8, True),
 ])
 def test_layer_matches_brute_force(seed, E, k, bias, residual, wd, enorm):
     d, f = 256, 64
@@ -396,3 +401,76 @@ def test_decoders():
     np.testing.assert_array_equal(oracle.decode_bf16(b), b.double().numpy())
     sub = torch.tensor([2 ** -24, 3 * 2 ** -24, 2 ** -14], dtype=torch.float16)
     np.testing.assert_array_equal(oracle.decode_fp16(sub), sub.double().numpy())
+
+
+# ---------------------------------------------------------------- fp8 storage
+
+
+def test_e4m3_decode_matches_library_cast():
+    """All 256 byte values decode like torch's float8_e4m3fn -> float64 cast
+    (an independent library routine), NaN codes included."""
+    b = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    got = oracle.decode_e4m3(b)
+    ref = b.view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.isnan(got).sum() == 2  # 0x7F and 0xFF
+    np.testing.assert_array_equal(np.nan_to_num(got), np.nan_to_num(ref))
+
+
+def test_e4m3_closed_forms():
+    """OFP8 E4M3 (bias 7, 3 mantissa bits, no infinities): a few values by
+    hand, the subnormal step and sign symmetry."""
+    d = lambda v: float(oracle.decode_e4m3(np.array([v], np.uint8))[0])
+    assert d(0x38) == 1.0           # 0 0111 000
+    assert d(0x7E) == 448.0         # 0 1111 110: largest finite value
+    assert d(0x77) == 240.0         # 0 1110 111 = 1.875 * 2^7
+    assert d(0x08) == 2.0 ** -6     # smallest normal
+    assert d(0x01) == 2.0 ** -9     # smallest subnormal
+    assert d(0x07) == 7 * 2.0 ** -9
+    assert d(0x00) == 0.0 and d(0x80) == 0.0
+    for v in range(0x7F):
+        assert d(v | 0x80) == -d(v)
+
+
+def test_fp8_weight_row_closed_form():
+    """Rows decoded by the oracle equal value(code) * scale[row] for codes
+    and scales placed by hand (pins the byte order and the row scale)."""
+    E, R, C = 2, 3, 256
+    codes = torch.zeros(E, R, C, dtype=torch.uint8)
+    codes[1, 2, 0] = 0x38     # 1.0
+    codes[1, 2, 1] = 0xC4     # 1 1000 100 = -1.5 * 2
+    codes[1, 2, 130] = 0x01   # 2^-9
+    codes[1, 2, 255] = 0x7E   # 448
+    scales = torch.ones(E, R, dtype=torch.float32)
+    scales[1, 2] = 0.25
+    row = oracle.weight_row(codes, scales, 1, 2, C)
+    ref = np.zeros(C)
+    ref[0], ref[1], ref[130], ref[255] = 0.25, -0.75, 2.0 ** -11, 112.0
+    np.testing.assert_array_equal(row, ref)
+    assert np.all(oracle.weight_row(codes, scales, 0, 2, C) == 0)
+
+
+def test_fp8_single_code_closed_form():
+    """E = k = 1 with one nonzero code in each of gate, up and down:
+    out[m] = (v3 s3) * gelu_tanh(v1 s1 x_i) * (v2 s2 x_j), s the row scales."""
+    d, f = 256, 128
+    lay = inputs.make_small(T=3, d=d, E=1, k=1, f=f, seed=13, wdtype=inputs.WDTYPE_FP8)
+    cg = torch.zeros(1, 2 * f, d, dtype=torch.uint8)
+    cd = torch.zeros(1, d, f, dtype=torch.uint8)
+    r, i, j, m = 5, 130, 17, 200
+    cg[0, r, i] = 0x40        # 2.0, gate row r
+    cg[0, f + r, j] = 0xB4    # 1 0110 100 = -0.75, up row r
+    cd[0, m, r] = 0x44        # 0 1000 100 = 3.0, down column r
+    lay["w_gate_up"] = cg
+    lay["w_down"] = cd
+    s_gu = lay["scales_gate_up"]
+    s_d = lay["scales_down"]
+    out, _, _, _ = run_oracle(lay, 1)
+    x = lay["x"].double().numpy()
+    s1, s2, s3 = float(s_gu[0, r]), float(s_gu[0, f + r]), float(s_d[0, m])
+    a = 2.0 * s1 * x[:, i]
+    ref_m = 3.0 * s3 * (0.5 * a * (1 + np.tanh(math.sqrt(2 / math.pi) * (a + 0.044715 * a ** 3))))
+    ref_m = ref_m * (-0.75 * s2 * x[:, j])
+    ref = np.zeros((3, d))
+    ref[:, m] = ref_m
+    np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-300)
