@@ -167,12 +167,18 @@ def launches_per_layer(w, T: int, router: str) -> int:
     return 5
 
 
+# weight formats by moe_wdtype_t value (bf16, int4, fp8)
+WFMT = {0: "bf16", 1: "int4 w4g128", 2: "fp8 E4M3 (fp32 row scales)"}
+
+
 def layer_costs(w, touched: float, T: int):
     """Algorithmic bytes and FLOPs of one layer call: weights of the experts
     that receive a token (streamed once), x in, router tensors, out.  The
     expert kernel's share is those weights."""
-    if w.wdtype == 0:
+    if w.wdtype == 0:  # bf16
         wbytes = 3 * w.f * w.d * 2
+    elif w.wdtype == 2:  # fp8: E4M3 bytes + one fp32 scale per row
+        wbytes = 3 * w.f * w.d + 4 * (2 * w.f + w.d)
     else:
         wbytes = 3 * w.f * w.d // 2 + 2 * (2 * w.f * w.n_groups_d + w.d * w.n_groups_f)
     expert_bytes = touched * wbytes
@@ -420,6 +426,7 @@ def run_ours(args):
     desc = {
         "canvas": "one MoE layer over a T=256 token canvas",
         "canvas4": "one MoE layer over a T=256 token canvas, int4 w4g128 weights",
+        "canvas8": "one MoE layer over a T=256 token canvas, fp8 E4M3 weights",
         "encode": "one MoE layer over T=2048 tokens (1792 prompt + 256 canvas)",
         "stack30": "one denoising step: 30 stacked MoE layers (distinct weights, Zipf(1.1) "
                    "router bias, residual chained) over a T=256 canvas",
@@ -440,7 +447,7 @@ def run_ours(args):
         "data": "synthetic",
         "config": {
             "workload": f"{w.name}: {desc}, d={w.d}, E={w.E}, top-{w.k}, f={w.f}, "
-                        f"{'int4 w4g128' if w.wdtype else 'bf16'} weights",
+                        f"{WFMT[w.wdtype]} weights",
             "global_batch": world * T, "seq_len": T, "layers_per_step": L,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": f"weights {wbytes * w.E * L / 1e9:.2f} GB > L2; x/out rotated over "

@@ -330,7 +330,8 @@ struct GatherArgs {
   const float* gamma2;   // expert-side (1 + gamma2) RMSNorm, or NULL for raw x
   const int32_t* perm;
   const __nv_bfloat16* x;
-  __nv_bfloat16* x_perm;
+  __nv_bfloat16* x_perm;  // bf16, or fp16 bits when xf16 is set
+  int xf16;               // write x_perm as fp16 (the fp8-weight path's B operand)
 };
 
 struct CombineArgs {
@@ -351,7 +352,9 @@ struct ExpertArgs {
   int32_t* ready;
   const __half* scales_gu;  // int4: [E, 2f, ceil(d/128)]
   const __half* scales_d;   // int4: [E, d, ceil(f/128)]
-  __nv_bfloat16* h;   // [T*k, f]
+  const float* rows_gu;     // fp8: one fp32 scale per weight row [E, 2f]
+  const float* rows_d;      // fp8: [E, d]
+  __nv_bfloat16* h;   // [T*k, f] (fp16 bits on the fp8 path)
   void* y;            // [T*k, d], fp32 or (y_bf16) bf16
   int y_bf16;
   Ctl* ctl;
@@ -483,5 +486,8 @@ cudaError_t moe_launch_expert(const moe::ExpertArgs& a, const CUtensorMap& tm_wg
                               const CUtensorMap& tm_wd, const CUtensorMap& tm_xp,
                               const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_expert_w4(const moe::ExpertArgs& a, const CUtensorMap& tm_cgu,
+                                 const CUtensorMap& tm_cd, const CUtensorMap& tm_xp,
+                                 const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_expert_w8(const moe::ExpertArgs& a, const CUtensorMap& tm_cgu,
                                  const CUtensorMap& tm_cd, const CUtensorMap& tm_xp,
                                  const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);

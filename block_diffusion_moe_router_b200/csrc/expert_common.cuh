@@ -1,6 +1,6 @@
-// expert_common.cuh -- pieces shared by the bf16 and the int4 expert
+// expert_common.cuh -- pieces shared by the bf16, int4 and fp8 expert
 // kernels: the work-unit record, bounded waits, GELU-tanh and the epilogue
-// role (TMEM accumulators -> h = gelu(gate) * up in bf16, or y in fp32).
+// role (TMEM accumulators -> h = gelu(gate) * up in bf16 or fp16, or y).
 #pragma once
 
 #include "common.cuh"
@@ -36,7 +36,8 @@ enum {
   kWhereUnitFullEpi,
   kWhereTmemFull,
   kWhereDrain,
-  kWhereUnitFullB
+  kWhereUnitFullB,
+  kWhereScalesEpi
 };
 
 __device__ __forceinline__ float gelu_tanh(float g) {
@@ -78,6 +79,18 @@ __device__ inline bool mbar_wait_drain(uint64_t* bar, uint32_t parity, Ctl* ctl,
   return true;
 }
 
+// h in the epilogue's output type.
+template <typename HT>
+__device__ __forceinline__ HT to_h(float v);
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_h<__nv_bfloat16>(float v) {
+  return __float2bfloat16(v);
+}
+template <>
+__device__ __forceinline__ __half to_h<__half>(float v) {
+  return __float2half_rn(v);
+}
+
 // Epilogue role (warps 2..5, 128 threads): for each unit, read the fp32
 // accumulator from TMEM (lane = weight row, column = token), 32 tokens at a
 // time, and write
@@ -88,15 +101,22 @@ __device__ inline bool mbar_wait_drain(uint64_t* bar, uint32_t parity, Ctl* ctl,
 // store is a 16-byte piece of one token's row (coalesced rows instead of
 // 2-byte column scatters).  The leader does the waits and broadcasts the
 // outcome, so the 128 threads always pass the same named barriers.
+// kRowScale (fp8 weights): every accumulator row is first multiplied by its
+// weight row's fp32 scale, read from the unit's slot rscale + 128 * ur
+// (landed on sfull[ur]); HT is h's type (fp16 on that path).
+template <bool kRowScale = false, typename HT = __nv_bfloat16>
 __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInfo* units,
                                               uint64_t* ufull, uint64_t* uempty, uint64_t* tfull,
                                               uint64_t* tempty, float* xchg,
                                               volatile int* s_abort, volatile int* s_bcast,
                                               uint32_t tmem_base, int acc_cols, int warp,
-                                              int lane) {
+                                              int lane, uint64_t* sfull = nullptr,
+                                              const float* rscale = nullptr) {
   Ctl* ctl = a.ctl;
   __nv_bfloat16* tile =
       reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(xchg) + kXchgBytes);
+  HT* htile = reinterpret_cast<HT*>(tile);
+  HT* hout = reinterpret_cast<HT*>(a.h);
   const uint64_t pol_keep = l2_policy_evict_last();  // h and y are read back soon
   const int q4 = warp & 3;          // TMEM lane quarter this warp may access
   const int row = q4 * 32 + lane;   // accumulator row (TMEM lane)
@@ -112,6 +132,8 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
       bool ok = mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullEpi);
       if (ok && units[ur].type != kUnitStop)
         ok = mbar_wait(&tfull[acc], aphase, s_abort, ctl, a.timeout_ns, kWhereTmemFull);
+      if (kRowScale && ok && units[ur].type != kUnitStop)
+        ok = mbar_wait(&sfull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereScalesEpi);
       *s_bcast = ok ? 1 : 0;
     }
     named_barrier(1, 128);
@@ -120,6 +142,7 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
     named_barrier(1, 128);
     if (!ok || ui.type == kUnitStop) break;
     tc_fence_after();
+    const float rs = kRowScale ? rscale[ur * kBM + row] : 1.f;
     const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * acc_cols);
     const int nch = (ui.n + 31) / 32;
     if (ui.type == kUnitGateUp) {
@@ -130,16 +153,17 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
         if (row >= kGuHalf) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            xchg[(row - kGuHalf) * kXchgStride + i] = __uint_as_float(v[i]);
+            xchg[(row - kGuHalf) * kXchgStride + i] =
+                kRowScale ? __uint_as_float(v[i]) * rs : __uint_as_float(v[i]);
         }
         named_barrier(1, 128);
         const int cmax = min(32, ui.n - cc * 32);
         if (row < kGuHalf) {  // tile[token][r], 64 columns
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float g = __uint_as_float(v[i]);
+            const float g = kRowScale ? __uint_as_float(v[i]) * rs : __uint_as_float(v[i]);
             const float up = xchg[row * kXchgStride + i];
-            tile[i * kGuHalf + row] = __float2bfloat16(gelu_tanh(g) * up);
+            htile[i * kGuHalf + row] = to_h<HT>(gelu_tanh(g) * up);
           }
         }
         named_barrier(1, 128);
@@ -149,9 +173,9 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
           const int pc = et + 128 * k;
           const int tok = pc >> 3, piece = pc & 7;
           if (tok < cmax)
-            st_global_hint(a.h + (size_t)(ui.slot0 + cc * 32 + tok) * a.f + ui.m * kGuHalf +
+            st_global_hint(hout + (size_t)(ui.slot0 + cc * 32 + tok) * a.f + ui.m * kGuHalf +
                                piece * 8,
-                           *reinterpret_cast<const uint4*>(tile + tok * kGuHalf + piece * 8),
+                           *reinterpret_cast<const uint4*>(htile + tok * kGuHalf + piece * 8),
                            pol_keep);
         }
       }
@@ -164,7 +188,9 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
         const int cmax = min(32, ui.n - cc * 32);
         if (a.y_bf16) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) tile[i * kBM + row] = __float2bfloat16(__uint_as_float(v[i]));
+          for (int i = 0; i < 32; ++i)
+            tile[i * kBM + row] =
+                __float2bfloat16(kRowScale ? __uint_as_float(v[i]) * rs : __uint_as_float(v[i]));
           named_barrier(1, 128);
           // 32 tokens x 256 bytes: sixteen 16-byte pieces per token
           __nv_bfloat16* y = static_cast<__nv_bfloat16*>(a.y) + y0;
@@ -182,7 +208,9 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
           float* ycol = static_cast<float*>(a.y) + y0 + row;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (i < cmax) ycol[(size_t)(cc * 32 + i) * a.d] = __uint_as_float(v[i]);
+            if (i < cmax)
+              ycol[(size_t)(cc * 32 + i) * a.d] =
+                  kRowScale ? __uint_as_float(v[i]) * rs : __uint_as_float(v[i]);
         }
       }
     }

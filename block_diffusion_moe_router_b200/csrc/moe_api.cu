@@ -123,8 +123,8 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Tokens per scheduler chunk: 256 for bf16 weights, 128 for int4 (whose
-// kernel keeps dequantised A stages in TMEM next to the accumulators).
+// Tokens per scheduler chunk: 256 for bf16 weights, 128 for int4 and fp8
+// (whose kernels keep decoded A stages in TMEM next to the accumulators).
 int chunk_size(moe_plan_t p) { return p->wdtype == MOE_W_BF16 ? moe::kMaxN : 128; }
 
 int max_chunks(int E, int T, int k) { return E + (T * k) / 128 + 1; }
@@ -143,6 +143,22 @@ bool use_router_tc(moe_plan_t p, int T) {
 // x 64 bytes (one group of 128 codes), 64-byte swizzle.
 bool make_map_codes(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols_bytes,
                     uint32_t box_rows);
+
+// 2-D byte tensor map over fp8 codes [rows, cols]: box = box_rows x 128 bytes
+// (one 128-wide K stage), 128-byte swizzle.
+bool make_map_fp8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 moe_status_t check_device(moe_plan_t p) {
   int dev = -1;
@@ -248,8 +264,9 @@ moe_status_t validate_route(moe_plan_t p, int T, const void* x, const float* rw,
 
 // Bytes of the fused gate_up weight pulled into L2 during routing.
 uint64_t prefetch_bytes(moe_plan_t p) {
-  const uint64_t all = (uint64_t)p->E * 2 * p->f * p->d * (p->wdtype == MOE_W_BF16 ? 2 : 1) /
-                       (p->wdtype == MOE_W_BF16 ? 1 : 2);
+  const uint64_t n = (uint64_t)p->E * 2 * p->f * p->d;  // weights of the fused gate_up
+  const uint64_t all =
+      p->wdtype == MOE_W_BF16 ? 2 * n : (p->wdtype == MOE_W_FP8_E4M3 ? n : n / 2);
   const uint64_t want = (uint64_t)p->prefetch_mb << 20;
   return want < all ? want : all;
 }
@@ -311,7 +328,8 @@ moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, mo
   if (E < 1 || E > moe::kMaxE || k < 1 || k > E || k > moe::kMaxK) return MOE_ERR_UNSUPPORTED;
   if (d < 128 || d > 4096 || d % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (f < 64 || f > 4096 || f % 64 != 0) return MOE_ERR_UNSUPPORTED;
-  if (wdtype != MOE_W_BF16 && wdtype != MOE_W_INT4_G128) return MOE_ERR_UNSUPPORTED;
+  if (wdtype != MOE_W_BF16 && wdtype != MOE_W_INT4_G128 && wdtype != MOE_W_FP8_E4M3)
+    return MOE_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   int sms = 0;
@@ -422,14 +440,21 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int A = T * p->k;
   const bool w4 = p->wdtype == MOE_W_INT4_G128;
+  const bool w8 = p->wdtype == MOE_W_FP8_E4M3;
   CUtensorMap tm_wgu, tm_wd, tm_x, tm_h;
-  const bool maps_ok =
-      (w4 ? make_map_codes(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d / 2, moe::kGuHalf) &&
-                make_map_codes(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f / 2, moe::kBM)
-          : make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) &&
-                make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM)) &&
-      make_map_bf16(&tm_x, p->x_perm, (uint64_t)A, p->d, moe::kBRows) &&
-      make_map_bf16(&tm_h, p->h, (uint64_t)A, p->f, moe::kBRows);
+  bool maps_ok;
+  if (w4)
+    maps_ok = make_map_codes(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d / 2, moe::kGuHalf) &&
+              make_map_codes(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f / 2, moe::kBM);
+  else if (w8)
+    maps_ok = make_map_fp8(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) &&
+              make_map_fp8(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM);
+  else
+    maps_ok = make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) &&
+              make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM);
+  // x_perm and h (bf16, or fp16 on the fp8 path: 2-byte elements either way)
+  maps_ok = maps_ok && make_map_bf16(&tm_x, p->x_perm, (uint64_t)A, p->d, moe::kBRows) &&
+            make_map_bf16(&tm_h, p->h, (uint64_t)A, p->f, moe::kBRows);
   if (!maps_ok) return MOE_ERR_CUDA;
 
   st = launch_router(p, T, x, router_w, router_gamma, router_bias, p->idx, p->w, p->gap, s,
@@ -459,6 +484,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ga.perm = p->perm;
   ga.x = static_cast<const __nv_bfloat16*>(x);
   ga.x_perm = p->x_perm;
+  ga.xf16 = w8 ? 1 : 0;
   {
     ProfScope ps(p, MOE_K_PLAN, s);
     if (moe_launch_plan_gather(pa, ga, p->num_sms, s, p->pdl != 0) != cudaSuccess)
@@ -481,13 +507,16 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ea.ctl = p->ctl;
   ea.timeout_ns = (uint64_t)p->timeout_ms * 1000000ull;
   ea.test_stall = p->test_stall;
-  ea.scales_gu = static_cast<const __half*>(scales_gate_up);
-  ea.scales_d = static_cast<const __half*>(scales_down);
+  ea.scales_gu = w4 ? static_cast<const __half*>(scales_gate_up) : nullptr;
+  ea.scales_d = w4 ? static_cast<const __half*>(scales_down) : nullptr;
+  ea.rows_gu = w8 ? static_cast<const float*>(scales_gate_up) : nullptr;
+  ea.rows_d = w8 ? static_cast<const float*>(scales_down) : nullptr;
   {
     ProfScope ps(p, MOE_K_EXPERT, s);
     const cudaError_t le =
         w4 ? moe_launch_expert_w4(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0)
-           : moe_launch_expert(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0);
+        : w8 ? moe_launch_expert_w8(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0)
+             : moe_launch_expert(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0);
     if (le != cudaSuccess) return MOE_ERR_CUDA;
   }
 
@@ -751,6 +780,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ga.perm = perm;
   ga.x = static_cast<const __nv_bfloat16*>(x);
   ga.x_perm = x_perm;
+  ga.xf16 = 0;
   if (moe_launch_plan_gather(pa, ga, p->num_sms, s, p->pdl != 0) != cudaSuccess)
     return MOE_ERR_CUDA;
 
@@ -772,6 +802,8 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ea.test_stall = p->test_stall;
   ea.scales_gu = nullptr;
   ea.scales_d = nullptr;
+  ea.rows_gu = nullptr;
+  ea.rows_d = nullptr;
   if (moe_launch_expert(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0) !=
       cudaSuccess)
     return MOE_ERR_CUDA;

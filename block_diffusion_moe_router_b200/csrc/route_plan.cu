@@ -266,6 +266,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
 // expert-side norm bf16(x / sqrt(mean(x^2) + eps) * (1 + gamma2)) of that row
 // (the model's pre-FFN norm, whose only consumer is the fused gate_up).  One
 // warp per row, 16-byte moves, every load of the row issued before any use.
+// With xf16 the row is written as fp16 instead (exact for bf16 values of
+// magnitude 2^-14 .. 65504; the normed row is rounded once, to fp16).
 constexpr int kGatherVec = 16;  // uint4 per lane held in registers (d <= 4096)
 
 // One row (warp-wide, lane owns 16-byte pieces lane + 32j), in passes of
@@ -321,8 +323,24 @@ __device__ __forceinline__ void gather_row(const GatherArgs& a, int row, int t, 
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float2 f = __bfloat1622float2(h2[q]);
-            h2[q] = __floats2bfloat162_rn((f.x * inv) * (1.f + g[2 * q]),
-                                          (f.y * inv) * (1.f + g[2 * q + 1]));
+            const float y0 = (f.x * inv) * (1.f + g[2 * q]);
+            const float y1 = (f.y * inv) * (1.f + g[2 * q + 1]);
+            if (a.xf16)
+              *reinterpret_cast<__half2*>(&h2[q]) = __floats2half2_rn(y0, y1);
+            else
+              h2[q] = __floats2bfloat162_rn(y0, y1);
+          }
+        }
+      }
+    } else if (a.xf16) {
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) {
+        if (p0 + lane + 32 * j < n) {
+          __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[j]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(h2[q]);
+            *reinterpret_cast<__half2*>(&h2[q]) = __floats2half2_rn(f.x, f.y);
           }
         }
       }

@@ -12,7 +12,8 @@
  *   - per expert gate/up 2816->704, down 704->2816, act GELUTanh; optional
  *     symmetric int4 weights in groups of 128 (auto-round pull request "Add
  *     quantization support for DiffusionGemma", transformers backend test
- *     log);
+ *     log), or 8-bit floating-point weights (the ROCmFP4-GGUF card's FP8
+ *     builds; E4M3 with one fp32 scale per weight row here);
  *   - the canvas of 256 tokens is denoised in parallel, so each step is a set
  *     of large batched expert matmuls (the ROCmFP4-GGUF card, section "The
  *     4-bit is NOT the fastest here").
@@ -63,9 +64,19 @@ typedef enum {
 
 typedef enum {
   MOE_W_BF16 = 0,      /* w_gate_up bf16 [E,2f,d]; w_down bf16 [E,d,f]           */
-  MOE_W_INT4_G128 = 1  /* w_gate_up u8 [E,2f,d/2]; w_down u8 [E,d,f/2]; element i
+  MOE_W_INT4_G128 = 1, /* w_gate_up u8 [E,2f,d/2]; w_down u8 [E,d,f/2]; element i
                           of a row in byte i/2, low nibble for even i, 4-bit two's
                           complement; value = code * scale[row][i/128] (fp16)  */
+  MOE_W_FP8_E4M3 = 2   /* w_gate_up u8 [E,2f,d]; w_down u8 [E,d,f]; element i of a
+                          row is byte i, an OFP8 E4M3 value (OCP 8-bit Floating
+                          Point Specification; the NaN codes 0x7F / 0xFF must not
+                          occur); value = e4m3 * scale[row] with one fp32 scale
+                          per weight row.  The FP4 / FP8 weight builds are on the
+                          Hugging Face card "kingjones777/DiffusionGemma-26B-A4B-
+                          it-ROCmFP4-GGUF"; the pages do not fix the encoding.
+                          Activations (the experts' input rows and h) are carried
+                          as fp16 on this path: |x| (after the optional expert
+                          norm) and |h| must stay below 65504.                 */
 } moe_wdtype_t;
 
 /* Options for moe_plan_set_option. */
@@ -129,8 +140,8 @@ moe_status_t moe_plan_reserve(moe_plan_t plan, int max_T);
  *                  The router and the residual always see the raw x.
  *   w_gate_up      see moe_wdtype_t (rows [0,f) gate, [f,2f) up)
  *   w_down         see moe_wdtype_t
- *   scales_gate_up fp16 [E,2f,ceil(d/128)]  (int4 plans; must be NULL for bf16)
- *   scales_down    fp16 [E,d,ceil(f/128)]   (int4 plans; must be NULL for bf16)
+ *   scales_gate_up int4: fp16 [E,2f,ceil(d/128)]; fp8: fp32 [E,2f]; NULL for bf16
+ *   scales_down    int4: fp16 [E,d,ceil(f/128)];  fp8: fp32 [E,d];  NULL for bf16
  *   residual       bf16 [T,d] or NULL; may alias `out`
  *   out            bf16 [T,d]; must not overlap x
  * Asynchronous on `stream`; the plan's workspace holds the routing tables
@@ -179,8 +190,8 @@ moe_status_t moe_forward_host(moe_plan_t plan, int T, const void* x_host, const 
  *     call's contents (each call clears the words that must start at zero).
  *     Calls that overlap on the GPU (other streams, other threads, other
  *     plans) race on it and must be serialised by the caller.
- *   - bf16 plans only for now (int4 returns MOE_ERR_UNSUPPORTED, as in
- *     moe_forward); MOE_OPT_PROFILE is ignored. */
+ *   - bf16 plans only for now (int4 and fp8 plans return
+ *     MOE_ERR_UNSUPPORTED); MOE_OPT_PROFILE is ignored. */
 moe_status_t moe_forward_noalloc(moe_plan_t plan, int T, const void* x, const float* router_w,
                                  const float* router_gamma, const float* router_bias,
                                  const float* expert_gamma, const void* w_gate_up, const void* w_down,

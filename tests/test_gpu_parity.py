@@ -7,8 +7,8 @@ import torch
 import oracle
 from block_diffusion_moe_router_b200 import inputs
 import block_diffusion_moe_router_b200 as moe
-from parity_util import (TOL_BF16, TOL_INT4, check_routing, oracle_rows_for_sets, rel_l2,
-                         stable_tables)
+from parity_util import (TOL_BF16, TOL_FP8, TOL_INT4, check_routing, oracle_rows_for_sets,
+                         rel_l2, stable_tables)
 
 pytestmark = pytest.mark.gpu
 
@@ -40,10 +40,13 @@ def full_check(lay_cpu, lay_gpu, E, k, d, f, rows=None, residual=None, tol=TOL_B
     """Runs route + forward on the GPU and compares with the oracle (all rows
     or the sampled `rows`); `options` are plan options set before the calls."""
     T = lay_gpu["x"].shape[0]
-    int4 = lay_gpu["w_gate_up"].dtype == torch.uint8
+    coded = lay_gpu["w_gate_up"].dtype == torch.uint8
+    fp8 = coded and lay_gpu["scales_gate_up"].dtype == torch.float32
+    int4 = coded and not fp8
     if int4 and tol == TOL_BF16:
         tol = TOL_INT4
-    layer = moe.MoeLayer(E, k, d, f, moe.MOE_W_INT4_G128 if int4 else moe.MOE_W_BF16)
+    wdt = moe.MOE_W_FP8_E4M3 if fp8 else (moe.MOE_W_INT4_G128 if int4 else moe.MOE_W_BF16)
+    layer = moe.MoeLayer(E, k, d, f, wdt)
     try:
         for key, val in (options or {}).items():
             moe.moe_plan_set_option(layer.plan, key, val)
@@ -84,7 +87,7 @@ def full_check(lay_cpu, lay_gpu, E, k, d, f, rows=None, residual=None, tol=TOL_B
     assert np.all(np.isinf(gg[~fin]))
     np.testing.assert_allclose(gg[fin], ogap[fin], rtol=1e-3, atol=2e-5)
     # routing tables bit-exact (when the sets agree everywhere)
-    if check_tables and rows is None and len(mism) == 0 and not int4:
+    if check_tables and rows is None and len(mism) == 0 and not coded:
         off, perm, slot_of = stable_tables(oidx, E)
         assert np.array_equal(tables[0], off)
         assert np.array_equal(tables[1], perm)
@@ -123,7 +126,7 @@ def test_canvas_y_fp32(canvas):
     print("canvas y-fp32 rel-L2", err)
 
 
-@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4])
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4, inputs.WDTYPE_FP8])
 @pytest.mark.parametrize("ybf16", [0, 1])
 def test_y_dtype_ragged_residual(wd, ybf16):
     """Both y precisions with a residual, ragged T and both weight formats."""
@@ -241,6 +244,63 @@ def test_int4_hot_expert_chunks():
     print("int4 hot expert rel-L2", err)
 
 
+def test_canvas8_fp8_full_layer():
+    """T=256 canvas with E4M3 expert weights and fp32 row scales: every
+    token against the oracle's exact value * scale arithmetic."""
+    w = inputs.WORKLOADS["canvas8"]
+    lay_gpu = inputs.make_layer(w, device="cuda")
+    lay_cpu = _cpu(lay_gpu)
+    err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f, tol=TOL_FP8)
+    print("canvas8 fp8 rel-L2", err)
+
+
+@pytest.mark.parametrize("T,E,k,d,f,bias", [
+    (17, 16, 2, 256, 64, True),      # f=64: the only K stage of down is half out of bounds
+    (300, 33, 3, 384, 192, False),   # f=192: last stage of 64; E not a multiple of 32
+    (1, 4, 1, 128, 128, False),      # one token, one 128-wide stage each way
+])
+def test_fp8_edge_shapes(T, E, k, d, f, bias):
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=T + E + 2, bias=bias,
+                            wdtype=inputs.WDTYPE_FP8)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f, tol=TOL_FP8)
+    print("fp8", (T, E, k, d, f), "rel-L2", err)
+
+
+def test_fp8_hot_expert_chunks():
+    """fp8 units hold 128 tokens: one expert with 600 tokens spans 5 chunks."""
+    T, E, k, d, f = 600, 16, 2, 256, 128
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=79, bias=True,
+                            wdtype=inputs.WDTYPE_FP8)
+    lay["router_bias"] = torch.zeros(E)
+    lay["router_bias"][3] = 50.0
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f, tol=TOL_FP8)
+    print("fp8 hot expert rel-L2", err)
+
+
+@pytest.mark.parametrize("kind", ["subnormal", "extreme"])
+def test_fp8_code_ranges(kind):
+    """Every weight code subnormal (|v| < 2^-6), or every code at the
+    format's largest magnitudes (+-256 .. +-448): the decode must be exact
+    at both ends (a flushed subnormal or a saturated code would show)."""
+    T, E, k, d, f = 33, 8, 2, 256, 128
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=81, wdtype=inputs.WDTYPE_FP8)
+    g = torch.Generator().manual_seed(5)
+    for key in ("w_gate_up", "w_down"):
+        shape = lay[key].shape
+        sign = torch.randint(0, 2, shape, generator=g, dtype=torch.int32) << 7
+        if kind == "subnormal":   # exponent 0, mantissa 1..7
+            mag = torch.randint(1, 8, shape, generator=g, dtype=torch.int32)
+        else:                     # exponent 15 (256 .. 448), mantissa 0..6
+            mag = (15 << 3) | torch.randint(0, 7, shape, generator=g, dtype=torch.int32)
+        lay[key] = (sign | mag).to(torch.uint8)
+    # scales chosen so that the layer's values stay of order one
+    amp = 2.0 ** 9 / 4 if kind == "subnormal" else 1.0 / 350
+    lay["scales_gate_up"] = torch.full_like(lay["scales_gate_up"], amp * 0.02 * 3)
+    lay["scales_down"] = torch.full_like(lay["scales_down"], amp * 0.02 * 3)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f, tol=TOL_FP8)
+    print("fp8", kind, "rel-L2", err)
+
+
 # ------------------------------------------------------------------ edge cases
 
 
@@ -260,7 +320,7 @@ def test_edge_shapes(T, E, k, d, f, bias):
     print((T, E, k, d, f), "rel-L2", err)
 
 
-@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4])
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4, inputs.WDTYPE_FP8])
 def test_expert_side_norm(wd):
     """Experts read the (1+gamma2) RMSNorm of x (applied while gathering the
     rows); router and residual see the raw x."""
