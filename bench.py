@@ -33,10 +33,19 @@ METRIC = "canvas tokens/s per MoE layer (T=256, bf16) and % of HBM/tensor roofli
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "expert_kernel_canvas.txt")
-EXPERT_SOURCES = ["block_diffusion_moe_router_b200/csrc/expert.cu",
-                  "block_diffusion_moe_router_b200/csrc/expert_common.cuh",
-                  "block_diffusion_moe_router_b200/csrc/common.cuh"]
+_CSRC = "block_diffusion_moe_router_b200/csrc/"
+# Committed ncu summaries of the expert kernel per workload, and the sources
+# whose hash they record: the DRAM traffic is reported only while the kernel
+# still hashes to the profiled version.
+PROFILES = {
+    "canvas": ("expert_kernel_canvas.txt", "expert.cu"),
+    "canvas4": ("expert_w4_kernel_canvas4.txt", "expert_w4.cu"),
+    "canvas8": ("expert_w8_kernel_canvas8.txt", "expert_w8.cu"),
+}
+
+
+def expert_sources(workload: str):
+    return [_CSRC + PROFILES[workload][1], _CSRC + "expert_common.cuh", _CSRC + "common.cuh"]
 
 
 def parse():
@@ -71,26 +80,28 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def source_hash() -> str:
+def source_hash(workload: str = "canvas") -> str:
     h = hashlib.sha256()
-    for rel in EXPERT_SOURCES:
+    for rel in expert_sources(workload):
         with open(os.path.join(ROOT, rel), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
-    """DRAM bytes per launch of the expert kernel from the committed ncu
-    summary, or None if the summary is missing or the kernel changed since."""
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the expert kernel from the workload's committed
+    ncu summary, or None if there is none or the kernel changed since."""
+    if workload not in PROFILES:
+        return None
     try:
         kv = {}
-        for line in open(PROFILE_SUMMARY):
+        for line in open(os.path.join(ROOT, "profiles", PROFILES[workload][0])):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-        if kv.get("source_sha256_16") != source_hash():
+        if kv.get("source_sha256_16") != source_hash(workload):
             return None
-        return float(kv["dram_bytes_per_launch_full_canvas"])
+        return float(kv["dram_bytes_per_launch"])
     except Exception:
         return None
 
@@ -422,7 +433,7 @@ def run_ours(args):
     ms_step = ms / args.steps
     k_ms = kern["expert"]
     achieved = expert_bytes / (k_ms * 1e-3) / 1e9 if k_ms else None
-    traffic = recorded_traffic() if args.workload == "canvas" else None
+    traffic = recorded_traffic(args.workload)
     desc = {
         "canvas": "one MoE layer over a T=256 token canvas",
         "canvas4": "one MoE layer over a T=256 token canvas, int4 w4g128 weights",

@@ -5,24 +5,28 @@
 // builds of these weights and finds that, at a 256-token canvas, the 8-bit
 // build steps faster than the 4-bit one.
 //
-// Same work units, scheduler, unit ring and B operands as the int4 kernel
-// (expert_w4.cu); the A operand (weights) is decoded in TMEM:
-//   - TMA brings each 128-wide K stage of codes (128 rows x 128 bytes,
-//     128-byte swizzled) into shared memory;
-//   - 8 dequant warps widen them with the hardware E4M3 -> f16x2 conversion
-//     (exact: every E4M3 value is an fp16 value) and store the fp16 pairs
-//     straight into TMEM (tcgen05.st);
+// Same work units, scheduler, unit ring, B operands and epilogue as the bf16
+// and int4 kernels; the A operand (weights) is decoded in TMEM:
+//   - a code producer brings each 128-wide K stage of codes (128 rows x 128
+//     bytes, 128-byte swizzled) into a ring of its own by TMA; a B producer
+//     brings the matching activation tiles into a second ring.  A code stage
+//     is free again as soon as the dequant warps hold it in registers, so
+//     the code ring, which carries the HBM stream, is not held up by the
+//     UMMAs (a shared ring kept each stage ~3x longer and the stream at
+//     ~1,150 cycles per stage, latency-bound);
+//   - 8 dequant warps widen the codes with the hardware E4M3 -> f16x2
+//     conversion (exact: every E4M3 value is an fp16 value) and store the
+//     fp16 pairs straight into TMEM (tcgen05.st), two stages per hand-over;
 //   - the UMMA (kind::f16 with A and B both fp16) reads A from TMEM and the
 //     activations from shared memory: on this path x_perm and h are fp16;
 //   - the epilogue multiplies each accumulator row by its weight row's fp32
 //     scale before GELU-tanh(gate) * up (gate_up) or before writing y (down).
 // A unit's 128 row scales come in by bulk copy into the unit's slot when the
-// producer publishes the unit.  Per weight the SM moves one byte through
+// code producer publishes the unit.  Per weight the SM moves one byte through
 // shared memory and two bytes into TMEM, with one conversion per two weights.
 //
 // TMEM (512 columns): two 128-column fp32 accumulators (a unit holds at most
-// 128 tokens) and four 64-column A stages.
-#include <cuda_fp8.h>
+// 128 tokens) and two A slots of 128 columns (two K stages each).
 
 #include "expert_common.cuh"
 
@@ -30,28 +34,35 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 448;  // producer, UMMA, 4 epilogue, 8 dequant warps
+// warps: 0 code producer, 1 UMMA, 2-5 epilogue, 6-13 dequant, 14 B producer
+constexpr int kThreads = 480;
 constexpr int kDqWarp0 = 6;
-constexpr int kDqGroups = 2;              // dequant groups, each owning every other stage
+constexpr int kDqGroups = 2;              // dequant groups, each owning every other stage pair
 constexpr int kDqWarps = 4 * kDqGroups;   // a group is one warp per TMEM lane quarter
+constexpr int kBWarp = kDqWarp0 + kDqWarps;
 constexpr int kChunkN = 128;                 // tokens per unit
 constexpr int kBK8 = 128;                    // K per stage
 constexpr int kCodeBytes = kBM * kBK8;       // 16 KB of codes per stage
-constexpr int kAStages = 4;                  // TMEM A stages
-constexpr int kACols = kBK8 / 2;             // 64 columns of f16x2 per A stage
-constexpr int kAColBase = 2 * kChunkN;       // A stages after the accumulators
-constexpr int kMaxStages = 8;
-constexpr int kRingBytes = 192 * 1024;
+// TMEM A: two slots, each holding a pair of consecutive 128-wide K stages
+// (2 x 64 columns of f16x2).  The UMMA issuer and the dequant warps hand A
+// over once per pair: half the barrier round trips of one per stage.
+constexpr int kASlots = 2;
+constexpr int kACols = kBK8 / 2;             // 64 columns of f16x2 per K stage
+constexpr int kASlotCols = 2 * kACols;
+constexpr int kAColBase = 2 * kChunkN;       // A slots after the accumulators
+constexpr int kMaxCS = 10;                   // code stages
+constexpr int kMaxBS = 6;                    // B stages
+constexpr int kRingBytes = 192 * 1024;       // code ring + B ring
 // One row-scale slot per unit-ring entry: the unit's 128 fp32 row scales
 // (gate rows then up rows for gate_up, as the TMEM lanes hold them).
 constexpr int kScaleSlot = kBM * 4;
 constexpr int kScaleBytes = kUnitRing * kScaleSlot;
-constexpr int kBarBytes = 8 * (2 * kMaxStages + 2 * kAStages + 4 + 3 * kUnitRing + 1);
+constexpr int kBarBytes = 8 * (2 * kMaxCS + 2 * kMaxBS + 2 * kASlots + 4 + 3 * kUnitRing + 1);
 constexpr int kSmemBytes =
     1024 + kRingBytes + kScaleBytes + kEpiBytes + kBarBytes + 256;
-static_assert(kAColBase + kAStages * kACols <= kTmemCols, "TMEM budget");
+static_assert(kAColBase + kASlots * kASlotCols <= kTmemCols, "TMEM budget");
 
-enum { kWhereAFull = 20, kWhereAEmpty, kWhereDqFull };
+enum { kWhereAFull = 20, kWhereAEmpty, kWhereDqFull, kWhereBFull };
 
 // Instruction descriptor, kind::f16 with fp16 A and B (formats 0), fp32 D:
 // [4,6) D format = 1 (f32), [7,10) A = 0, [10,13) B = 0, K-major both,
@@ -127,12 +138,15 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 }
 
 // Four E4M3 codes (byte i = element i) -> two f16x2 words holding elements
-// (0,1) and (2,3), the lower element in the lower half.
+// (0,1) and (2,3), the lower element in the lower half (the hardware
+// conversion widens the two bytes of a 16-bit half in place).
 __device__ __forceinline__ void widen4(uint32_t w, uint32_t* out) {
-  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
-  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-  out[0] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
-  out[1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+      : "=r"(out[0]), "=r"(out[1])
+      : "r"(w));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -143,14 +157,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem;
+  uint8_t* ring = smem;  // [CS code stages][BS B stages]
   float* rsc = reinterpret_cast<float*>(smem + kRingBytes);  // [kUnitRing][128] row scales
   float* xchg = reinterpret_cast<float*>(smem + kRingBytes + kScaleBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRingBytes + kScaleBytes + kEpiBytes);
-  uint64_t* empty = full + kMaxStages;
-  uint64_t* afull = empty + kMaxStages;
-  uint64_t* aempty = afull + kAStages;
-  uint64_t* tfull = aempty + kAStages;
+  uint64_t* cfull = reinterpret_cast<uint64_t*>(smem + kRingBytes + kScaleBytes + kEpiBytes);
+  uint64_t* cempty = cfull + kMaxCS;
+  uint64_t* bfull = cempty + kMaxCS;
+  uint64_t* bempty = bfull + kMaxBS;
+  uint64_t* afull = bempty + kMaxBS;
+  uint64_t* aempty = afull + kASlots;
+  uint64_t* tfull = aempty + kASlots;
   uint64_t* tempty = tfull + 2;
   uint64_t* ufull = tempty + 2;
   uint64_t* uempty = ufull + kUnitRing;
@@ -169,11 +185,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   Ctl* ctl = a.ctl;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMaxStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 4 + 1);  // one dequant group reads codes, UMMA reads B
+    for (int i = 0; i < kMaxCS; ++i) {
+      mbar_init(&cfull[i], 1);
+      mbar_init(&cempty[i], 4);  // the dequant group's four warps hold the codes
     }
-    for (int i = 0; i < kAStages; ++i) {
+    for (int i = 0; i < kMaxBS; ++i) {
+      mbar_init(&bfull[i], 1);
+      mbar_init(&bempty[i], 1);  // UMMA commit
+    }
+    for (int i = 0; i < kASlots; ++i) {
       mbar_init(&afull[i], 4);
       mbar_init(&aempty[i], 1);
     }
@@ -183,7 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(&ufull[i], 1);
-      mbar_init(&uempty[i], 2 + kDqWarps);
+      // UMMA issuer, epilogue leader, B producer and every dequant warp
+      mbar_init(&uempty[i], 3 + kDqWarps);
       mbar_init(&sfull[i], 1);
     }
     mbar_init(drain, 1);
@@ -209,15 +230,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int maxn = max(1, min(kChunkN, ctl->max_chunk));
   const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
-  const int stage_bytes = kCodeBytes + 2 * NB * kBK * 2;  // codes + two 64-wide B sub-tiles
-  const int S = min(kMaxStages, kRingBytes / stage_bytes);
+  const int b_bytes = 4 * NB * kBK * 2;  // a stage pair: four 64-wide B sub-tiles of NB rows
+  const int BS = min(kMaxBS, max(2, (kRingBytes / 3) / b_bytes));
+  const int CS = min(kMaxCS, (kRingBytes - BS * b_bytes) / kCodeBytes);
+  uint8_t* ringB = ring + CS * kCodeBytes;
   const int n_chunks = ctl->n_chunks;
   const int U = n_chunks * (GU + DN);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ code producer
+    // Claims and publishes the units (with their row scales), then streams
+    // each unit's codes.
     const uint64_t pol_w = l2_policy_evict_first();
-    const uint64_t pol_act = l2_policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
     int ur = 0;
@@ -262,13 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             go = 0;
           }
         }
-        if (go && ui.type == kUnitDown) {
-          const int need = GU + (a.test_stall ? (1 << 30) : 0);
-          if (wait_count(a.ready + ui.q, need, s_abort, ctl, a.timeout_ns, kWhereReady))
-            fence_proxy_async_global();
-          else
-            go = 0;
-        }
         if (go && mbar_wait(&uempty[ur], uphase ^ 1, s_abort, ctl, a.timeout_ns,
                             kWhereUnitEmpty)) {
           if (ui.type != kUnitStop) {
@@ -297,8 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       go = __shfl_sync(0xffffffffu, go, 0);
       ui.type = __shfl_sync(0xffffffffu, ui.type, 0);
-      ui.n = __shfl_sync(0xffffffffu, ui.n, 0);
-      ui.slot0 = __shfl_sync(0xffffffffu, ui.slot0, 0);
+      ui.e = __shfl_sync(0xffffffffu, ui.e, 0);
+      ui.m = __shfl_sync(0xffffffffu, ui.m, 0);
       if (!go || ui.type == kUnitStop) break;
       if (++ur == kUnitRing) {
         ur = 0;
@@ -308,33 +325,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const int C = (ui.type == kUnitGateUp) ? a.d : a.f;
         const int nkb = (C + kBK8 - 1) / kBK8;
-        const int nbox = (ui.n + kBRows - 1) / kBRows;
-        const uint32_t tx = kCodeBytes + 2 * nbox * kBRows * kBK * 2;
-        const CUtensorMap* tb = (ui.type == kUnitGateUp) ? &tm_xp : &tm_h;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
+          if (!mbar_wait(&cempty[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
                          kWhereStageEmpty)) {
             ok = 0;
             break;
           }
-          uint8_t* sa = ring + stage * stage_bytes;
-          uint8_t* sb = sa + kCodeBytes;
-          mbar_arrive_expect_tx(&full[stage], tx);
+          uint8_t* sa = ring + stage * kCodeBytes;
+          mbar_arrive_expect_tx(&cfull[stage], kCodeBytes);
           const int cx = kb * kBK8;  // byte column of the codes
           if (ui.type == kUnitGateUp) {
             const int r0 = ui.e * 2 * a.f + ui.m * kGuHalf;
-            tma_load_2d(sa, &tm_cgu, cx, r0, &full[stage], pol_w);
-            tma_load_2d(sa + kCodeBytes / 2, &tm_cgu, cx, r0 + a.f, &full[stage], pol_w);
+            tma_load_2d(sa, &tm_cgu, cx, r0, &cfull[stage], pol_w);
+            tma_load_2d(sa + kCodeBytes / 2, &tm_cgu, cx, r0 + a.f, &cfull[stage], pol_w);
           } else {
-            tma_load_2d(sa, &tm_cd, cx, ui.e * a.d + ui.m * kBM, &full[stage], pol_w);
+            tma_load_2d(sa, &tm_cd, cx, ui.e * a.d + ui.m * kBM, &cfull[stage], pol_w);
           }
-          for (int h = 0; h < 2; ++h)
-            for (int bx = 0; bx < nbox; ++bx)
-              tma_load_2d(sb + h * NB * kBK * 2 + bx * kBRows * kBK * 2, tb, kb * kBK8 + h * kBK,
-                          ui.slot0 + bx * kBRows, &full[stage], pol_act);
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == S) {
+          if (++stage == CS) {
             stage = 0;
             phase ^= 1;
           }
@@ -344,20 +353,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
     }
     if (lane == 0) {
-      for (int s2 = 0; s2 < S; ++s2)
+      for (int s2 = 0; s2 < CS; ++s2)
         if ((issued >> s2) & 1u)
-          mbar_wait_drain(&full[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
+          mbar_wait_drain(&cfull[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
       for (int s2 = 0; s2 < kUnitRing; ++s2)
         if ((sissued >> s2) & 1u)
           mbar_wait_drain(&sfull[s2], (spar >> s2) & 1u, ctl, a.timeout_ns);
+    }
+  } else if (warp == kBWarp) {
+    // ------------------------------------------------------------ B producer
+    // Follows the unit ring; a down unit's h tiles wait for every gate_up
+    // unit of the chunk (the codes of the down unit stream meanwhile).
+    if (lane == 0) {
+      const uint64_t pol_act = l2_policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      int ur = 0;
+      uint32_t uphase = 0;
+      uint32_t issued = 0, issued_par = 0;
+      while (true) {
+        if (!mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullB)) break;
+        const UnitInfo ui = units[ur];
+        if (ui.type == kUnitStop) break;
+        if (ui.type == kUnitDown) {
+          const int need = GU + (a.test_stall ? (1 << 30) : 0);
+          if (!wait_count(a.ready + ui.q, need, s_abort, ctl, a.timeout_ns, kWhereReady)) break;
+          fence_proxy_async_global();
+        }
+        const int C = (ui.type == kUnitGateUp) ? a.d : a.f;
+        const int nkb = (C + kBK8 - 1) / kBK8;
+        const int nbox = (ui.n + kBRows - 1) / kBRows;
+        const CUtensorMap* tb = (ui.type == kUnitGateUp) ? &tm_xp : &tm_h;
+        bool ok = true;
+        for (int kb0 = 0; kb0 < nkb; kb0 += 2) {  // one B stage per K-stage pair
+          const int nst = min(2, nkb - kb0);
+          if (!mbar_wait(&bempty[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
+                         kWhereStageEmpty)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = ringB + stage * b_bytes;
+          mbar_arrive_expect_tx(&bfull[stage], nst * 2 * nbox * kBRows * kBK * 2);
+          for (int t = 0; t < 2 * nst; ++t)  // 64-wide sub-tiles
+            for (int bx = 0; bx < nbox; ++bx)
+              tma_load_2d(sb + t * NB * kBK * 2 + bx * kBRows * kBK * 2, tb, kb0 * kBK8 + t * kBK,
+                          ui.slot0 + bx * kBRows, &bfull[stage], pol_act);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == BS) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mbar_arrive(&uempty[ur]);
+        if (++ur == kUnitRing) {
+          ur = 0;
+          uphase ^= 1;
+        }
+      }
+      for (int s2 = 0; s2 < BS; ++s2)
+        if ((issued >> s2) & 1u)
+          mbar_wait_drain(&bfull[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     // The whole warp runs the loop (warp-uniform descriptors); the elected
     // lane issues the tcgen05 instructions.
-    int stage = 0;
-    uint32_t phase = 0;
-    int ast = 0;
+    int bst = 0;
+    uint32_t bph = 0;
+    int asl = 0;
     uint32_t aph = 0;
     int ur = 0;
     uint32_t uphase = 0;
@@ -376,29 +441,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t dt = tmem_base + (uint32_t)(acc * kChunkN);
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait_warp(&full[stage], phase, s_abort, ctl, a.timeout_ns, kWhereStageFull) ||
-            !mbar_wait_warp(&afull[ast], aph, s_abort, ctl, a.timeout_ns, kWhereAFull)) {
+      // one hand-over per K-stage pair: its A slot (dequant warps, which
+      // also waited for the pair's B stage) and its B stage
+      for (int kb0 = 0; kb0 < nkb; kb0 += 2) {
+        const int nst = min(2, nkb - kb0);
+        if (!mbar_wait_warp(&afull[asl], aph, s_abort, ctl, a.timeout_ns, kWhereAFull)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sb = smem_u32(ring + stage * stage_bytes + kCodeBytes);
-        const uint32_t ta = tmem_base + (uint32_t)(kAColBase + ast * kACols);
+        const uint32_t sb = smem_u32(ringB + bst * b_bytes);
+        const uint32_t ta = tmem_base + (uint32_t)(kAColBase + asl * kASlotCols);
+        for (int t = 0; t < nst; ++t) {
 #pragma unroll
-        for (int kk = 0; kk < kBK8 / kUmmaK; ++kk) {
-          const uint32_t b = sb + (kk >> 2) * NB * kBK * 2 + (kk & 3) * kUmmaK * 2;
-          if (elect_one())
-            umma_f16_ts(dt, ta + kk * (kUmmaK / 2), sdesc_k_sw128(b), idesc, (kb | kk) ? 1u : 0u);
+          for (int kk = 0; kk < kBK8 / kUmmaK; ++kk) {
+            const uint32_t b = sb + (2 * t + (kk >> 2)) * NB * kBK * 2 + (kk & 3) * kUmmaK * 2;
+            if (elect_one())
+              umma_f16_ts(dt, ta + t * kACols + kk * (kUmmaK / 2), sdesc_k_sw128(b), idesc,
+                          (kb0 | t | kk) ? 1u : 0u);
+          }
         }
-        umma_commit_elect(&empty[stage]);
-        umma_commit_elect(&aempty[ast]);
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
+        umma_commit_elect(&bempty[bst]);
+        umma_commit_elect(&aempty[asl]);
+        if (++bst == BS) {
+          bst = 0;
+          bph ^= 1;
         }
-        if (++ast == kAStages) {
-          ast = 0;
+        if (++asl == kASlots) {
+          asl = 0;
           aph ^= 1;
         }
       }
@@ -420,10 +490,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tmem_base, kChunkN, warp, lane, sfull, rsc);
   } else {
     // ------------------------------------------------------------ dequant warps
-    // Group g (one warp per TMEM lane quarter) takes the stages kb with
-    // kb % kDqGroups == g, a whole 128-code row per thread, so the groups
-    // work on different stages at once; a stage is signalled full as soon
-    // as its TMEM stores have landed.
+    // Group g (one warp per TMEM lane quarter) takes the stage pairs
+    // (kb / 2) % kDqGroups == g of each unit, a whole 128-code row per
+    // thread, so the groups work on different pairs at once; a pair is
+    // signalled full once the stores of its last stage have landed.
     const int dw = warp - kDqWarp0;        // 0..kDqWarps-1
     const int q4 = warp & 3;               // TMEM lane quarter
     const int row = q4 * 32 + lane;        // A row == TMEM lane
@@ -432,8 +502,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sw = row & 7;
     int stage = 0;
     uint32_t phase = 0;
-    int ast = 0;
+    int asl = 0;
     uint32_t aph = 0;
+    int bst = 0;  // the pair's B stage: waited for before the hand-over
+    uint32_t bph = 0;
     int ur = 0;
     uint32_t uphase = 0;
     while (true) {
@@ -450,21 +522,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int G = (C + kBK8 - 1) / kBK8;
       bool sok = true;
       for (int kb = 0; kb < G; ++kb) {
-        if (kb % kDqGroups == grp && sok) {
-          sok = mbar_wait(&full[stage], phase, s_abort, ctl, a.timeout_ns, kWhereDqFull) &&
-                mbar_wait(&aempty[ast], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty);
+        const bool pair_end = (kb & 1) || kb == G - 1;
+        if ((kb >> 1) % kDqGroups == grp && sok) {
+          if (!(kb & 1))
+            sok = mbar_wait(&aempty[asl], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty);
+          sok = sok && mbar_wait(&cfull[stage], phase, s_abort, ctl, a.timeout_ns, kWhereDqFull);
           if (sok) {
             // codes tile: 128-byte rows written by TMA with 128-byte
             // swizzling, i.e. 16-byte chunk c of row r sits at chunk c ^ (r & 7)
-            const uint8_t* crow = ring + stage * stage_bytes + row * kBK8;
+            const uint8_t* crow = ring + stage * kCodeBytes + row * kBK8;
             uint4 cw[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c)
               cw[c] = *reinterpret_cast<const uint4*>(crow + ((c ^ sw) << 4));
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[stage]);  // codes are in registers
+            if (lane == 0) mbar_arrive(&cempty[stage]);  // codes are in registers
             const uint32_t ta = tmem_base + ((uint32_t)(q4 * 32) << 16) +
-                                (uint32_t)(kAColBase + ast * kACols);
+                                (uint32_t)(kAColBase + asl * kASlotCols + (kb & 1) * kACols);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               uint32_t v[32];  // columns 32h .. 32h+31 = codes 64h .. 64h+63
@@ -477,20 +551,28 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               tmem_st32(ta + h * 32, v);
             }
-            // the stage is handed to the UMMA as soon as its stores land
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&afull[ast]);
+            if (pair_end) {  // the pair is handed to the UMMA once its stores land
+              tmem_wait_st();
+              tc_fence_before();
+              __syncwarp();
+              sok = mbar_wait(&bfull[bst], bph, s_abort, ctl, a.timeout_ns, kWhereBFull);
+              if (lane == 0 && sok) mbar_arrive(&afull[asl]);
+            }
           }
         }
-        if (++stage == S) {
+        if (++stage == CS) {
           stage = 0;
           phase ^= 1;
         }
-        if (++ast == kAStages) {
-          ast = 0;
-          aph ^= 1;
+        if (pair_end) {
+          if (++asl == kASlots) {
+            asl = 0;
+            aph ^= 1;
+          }
+          if (++bst == BS) {
+            bst = 0;
+            bph ^= 1;
+          }
         }
       }
       if (lane == 0) mbar_arrive(&uempty[ur]);  // this unit's slot is free
