@@ -342,3 +342,93 @@ void oracle_decode_fp16(int n, const uint16_t* in, double* out) {
 void oracle_decode_e4m3(int n, const uint8_t* in, double* out) {
   for (int i = 0; i < n; i++) out[i] = e4m3_to_double(in[i]);
 }
+
+/* ---- the step after the layer stack: lm_head over the canvas ------------
+ *
+ * Sources (page title, section):
+ *  [FU]  fucina docs "DiffusionGemma 26B-A4B -- block text-diffusion": the
+ *        runner denoises 256-token canvases with the entropy-bound sampler
+ *        (defaults from the model: <= 48 steps, temperature 0.8 -> 0.4,
+ *        bound 0.1); the mean canvas entropy is what the status line shows.
+ *  [AR]  auto-round pull request: EntropyBoundSamplerConfig, entropy_bound 0.1.
+ *  [QT]  Quant-Tuner pull request, Testing: the entropy-bound acceptance rule
+ *        is unit-tested there (its text is not on the pages).
+ * Readings (the pages fix none of these):
+ *  - logits z_v = h . W[v] over the whole vocabulary (W the lm_head / tied
+ *    embedding matrix, bf16), optionally soft-capped c * tanh(z / c);
+ *  - the sampler's distribution is p = softmax(z / temperature); a token's
+ *    entropy is H = -sum_v p_v log p_v = logZ - sum_v p_v u_v with
+ *    u = z / temperature and logZ = log sum_v exp(u_v);
+ *  - the proposed token is the argmax of z (lowest vocabulary index on ties);
+ *  - acceptance, over the still-masked positions: sort them by entropy
+ *    (ties by position) and accept the longest prefix whose entropies, all
+ *    but the largest, sum to at most the bound; the lowest-entropy position
+ *    is therefore always accepted (the entropy-bounded unmasking rule of
+ *    Ben-Hamu et al., "Accelerated Sampling from Masked Diffusion Models via
+ *    Entropy Bounded Unmasking", which the pages name only as the
+ *    entropy-bound sampler).  PARITY UNPINNED against the pages: they print
+ *    neither the rule nor an example; the pins check the definitions. */
+
+/* Statistics of token rows `rows[0..n)` of h [T, d] against W [V, d]:
+ * logZ, entropy H, argmax index and the gap between the two largest u. */
+void oracle_lmhead_stats(int V, int d, const uint16_t* h, const uint16_t* W, double inv_temp,
+                         double softcap, const int32_t* rows, int n, double* logz, double* H,
+                         int32_t* argmax, double* gap) {
+#pragma omp parallel for schedule(dynamic, 1) num_threads(oracle_get_threads())
+  for (int j = 0; j < n; j++) {
+    const uint16_t* hr = h + (size_t)rows[j] * d;
+    double* u = (double*)malloc(sizeof(double) * (size_t)V);
+    double* hx = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int i = 0; i < d; i++) hx[i] = bf16_to_double(hr[i]);
+    int best = 0;
+    for (int v = 0; v < V; v++) {
+      const uint16_t* wr = W + (size_t)v * d;
+      double z = 0.0;
+      for (int i = 0; i < d; i++) z += hx[i] * bf16_to_double(wr[i]);
+      if (softcap > 0.0) z = softcap * tanh(z / softcap);
+      u[v] = z * inv_temp;
+      if (u[v] > u[best]) best = v;
+    }
+    double second = -INFINITY;
+    for (int v = 0; v < V; v++)
+      if (v != best && u[v] > second) second = u[v];
+    double s = 0.0;
+    for (int v = 0; v < V; v++) s += exp(u[v] - u[best]);
+    const double lz = u[best] + log(s);
+    double eu = 0.0;
+    for (int v = 0; v < V; v++) eu += exp(u[v] - lz) * u[v];
+    logz[j] = lz;
+    H[j] = lz - eu;
+    argmax[j] = best;
+    gap[j] = u[best] - second;
+    free(u);
+    free(hx);
+  }
+}
+
+/* Entropy-bounded acceptance over the masked positions (reading above). */
+void oracle_eb_accept(int T, const double* H, const uint8_t* masked, double bound,
+                      uint8_t* accept) {
+  int* order = (int*)malloc(sizeof(int) * (size_t)(T > 0 ? T : 1));
+  int n = 0;
+  for (int t = 0; t < T; t++) {
+    accept[t] = 0;
+    if (!masked || masked[t]) order[n++] = t;
+  }
+  /* insertion sort by (H, position): plain and obviously stable */
+  for (int i = 1; i < n; i++) {
+    int t = order[i], j = i - 1;
+    while (j >= 0 && (H[order[j]] > H[t])) {
+      order[j + 1] = order[j];
+      j--;
+    }
+    order[j + 1] = t;
+  }
+  double below = 0.0; /* sum of the entropies before position i in the order */
+  for (int i = 0; i < n; i++) {
+    if (below > bound) break;
+    accept[order[i]] = 1;
+    below += H[order[i]];
+  }
+  free(order);
+}

@@ -60,6 +60,8 @@ def lib():
             L.oracle_decode_bf16.argtypes = [I, P, P]
             L.oracle_decode_fp16.argtypes = [I, P, P]
             L.oracle_decode_e4m3.argtypes = [I, P, P]
+            L.oracle_lmhead_stats.argtypes = [I, I, P, P, D, D, P, I, P, P, P, P]
+            L.oracle_eb_accept.argtypes = [I, P, P, D, P]
             L.oracle_set_threads.argtypes = [I]
             L.oracle_get_threads.restype = I
             _lib = L
@@ -242,3 +244,32 @@ def decode_e4m3(t) -> np.ndarray:
     out = np.empty(a.shape, np.float64)
     lib().oracle_decode_e4m3(a.size, _p(a), _p(out))
     return out
+
+
+def lmhead_stats(h, W, rows=None, temperature: float = 1.0, softcap: float = 0.0):
+    """Per token row of h [T,d] (bf16) against the lm_head W [V,d] (bf16):
+    (logZ, entropy H, argmax, gap between the two largest scaled logits),
+    all of softmax(z / temperature) with z = h . W (soft-capped if softcap > 0)."""
+    h = _np(h)
+    W = _np(W)
+    T, d = h.shape
+    V = W.shape[0]
+    rows = np.arange(T, dtype=np.int32) if rows is None else np.asarray(rows, np.int32)
+    n = rows.size
+    logz = np.empty(n, np.float64)
+    H = np.empty(n, np.float64)
+    am = np.empty(n, np.int32)
+    gap = np.empty(n, np.float64)
+    lib().oracle_lmhead_stats(V, d, _p(h), _p(W), 1.0 / temperature, float(softcap), _p(rows), n,
+                              _p(logz), _p(H), _p(am), _p(gap))
+    return logz, H, am, gap
+
+
+def eb_accept(H, masked, bound: float) -> np.ndarray:
+    """Entropy-bounded acceptance (uint8 per position) over the masked ones."""
+    H = _np(H, np.float64)
+    T = H.size
+    m = None if masked is None else _np(masked, np.uint8)
+    acc = np.empty(T, np.uint8)
+    lib().oracle_eb_accept(T, _p(H), _p(m), float(bound), _p(acc))
+    return acc
