@@ -510,10 +510,165 @@ def run_ours(args):
     rep.shutdown()
 
 
+LMHEAD_METRIC = ("canvas tokens/s through the lm_head step (T=256 logits over V=262144, "
+                 "entropy and argmax folded on chip, entropy-bound acceptance)")
+
+
+def run_lmhead(args):
+    """The step after the layer stack: one moe_lmhead_forward over a 256-token
+    canvas (V=262144, d=2816; W is 1.48 GB, far above L2, so no flush is
+    needed).  Same JSON contract as the layer bench."""
+    import torch
+    import block_diffusion_moe_router_b200 as moe
+    from block_diffusion_moe_router_b200 import inputs
+    from block_diffusion_moe_router_b200 import replicas as rep
+
+    rank, world, local = rep.dist_env()
+    torch.cuda.set_device(local)
+    rep.init("nccl", torch.device("cuda", local), timeout_s=120)
+    T, V, d = 256, inputs.LMHEAD_V, inputs.LMHEAD_D
+    temp, bound = 0.8, 0.1
+    nsets = 4
+    hs, W, _ = inputs.make_lmhead(T * nsets, V, d, seed=11 + rank, device="cuda")
+    hs = [hs[i * T:(i + 1) * T].contiguous() for i in range(nsets)]
+    g = torch.Generator().manual_seed(3)
+    masked = (torch.rand(T, generator=g) < 0.75).to(torch.uint8).cuda()
+    lh = moe.LmHead(V, d)
+    stream = torch.cuda.current_stream()
+    tok = torch.empty(T, dtype=torch.int32, device="cuda")
+    ent = torch.empty(T, dtype=torch.float32, device="cuda")
+    lz = torch.empty(T, dtype=torch.float32, device="cuda")
+    acc = torch.empty(T, dtype=torch.uint8, device="cuda")
+
+    def step(i):
+        moe.moe_lmhead_forward(lh.handle, T, hs[i % nsets], W, temp, 0.0, masked, bound, tok, ent,
+                               lz, acc, stream)
+
+    def timed(K, per_step=False):
+        rep.barrier()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1 if per_step else 2)]
+        ev[0].record(stream)
+        for i in range(K):
+            step(i)
+            if per_step:
+                ev[i + 1].record(stream)
+        ev[-1].record(stream)
+        torch.cuda.synchronize()
+        rep.barrier()
+        if per_step:
+            return [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+        return rep.max_over_ranks(ev[0].elapsed_time(ev[-1]), "cuda")
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = timed(args.steps)
+        moe.moe_lmhead_set_profile(lh.handle, True)
+        ms_prof = timed(args.steps)
+        moe.moe_lmhead_set_profile(lh.handle, False)
+    gemm_ms, n = moe.moe_lmhead_profile(lh.handle)
+    gemm_ms /= max(n, 1)
+    per_step = sorted(timed(args.steps, per_step=True))
+    pct = {f"p{q}": per_step[min(len(per_step) - 1, int(q / 100 * len(per_step)))]
+           for q in (10, 50, 90)}
+    if lh.sync_status() != moe.MOE_OK:
+        raise RuntimeError("lm_head step reported a device error")
+
+    # end to end: host h in, host token / entropy / accept out, every step
+    h_host = [x.cpu().pin_memory() for x in hs]
+    outs = [torch.empty(T, dtype=t.dtype).pin_memory() for t in (tok, ent, acc)]
+    rep.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        hs[0].copy_(h_host[i % nsets], non_blocking=True)
+        moe.moe_lmhead_forward(lh.handle, T, hs[0], W, temp, 0.0, masked, bound, tok, ent, lz,
+                               acc, stream)
+        for o, t in zip(outs, (tok, ent, acc)):
+            o.copy_(t, non_blocking=True)
+        stream.synchronize()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = rep.max_over_ranks(e0.elapsed_time(e1), "cuda")
+    lh.close()
+
+    hbm_gbs, bf16_tf, _, basis = peaks()
+    w_bytes = V * d * 2
+    alg_bytes = w_bytes + T * d * 2
+    flops = 2.0 * T * V * d
+    t_hbm = alg_bytes / (hbm_gbs * 1e9)
+    t_tc = flops / (bf16_tf * 1e12)
+    hbm_frac = (alg_bytes / (gemm_ms * 1e-3) / 1e9) / hbm_gbs
+    tc_frac = (flops / (gemm_ms * 1e-3) / 1e12) / bf16_tf
+    # the roofline is the slower of the two floors (they are within 1% here)
+    if t_tc >= t_hbm:
+        roof = {"bound": "tensor", "achieved": flops / (gemm_ms * 1e-3) / 1e12,
+                "peak": bf16_tf, "unit": "TFLOP/s", "frac": tc_frac,
+                "peak_basis": f"{basis} dense bf16 GEMM (burst)"}
+    else:
+        roof = {"bound": "hbm", "achieved": alg_bytes / (gemm_ms * 1e-3) / 1e9,
+                "peak": hbm_gbs, "unit": "GB/s", "frac": hbm_frac,
+                "peak_basis": f"{basis} HBM copy bandwidth"}
+    roof.update({"traffic": None, "kernel": "lm_head GEMM with the fused softmax statistics",
+                 "kernel_ms": gemm_ms, "hbm_fraction": hbm_frac, "tensor_fraction": tc_frac,
+                 "alg_bytes_per_launch": alg_bytes, "flops_per_launch": flops})
+    line = {
+        "metric": LMHEAD_METRIC,
+        "value": rep.job_rate(T, world, args.steps, ms),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"lmhead: T={T} canvas tokens, V={V}, d={d}, bf16 h and W, temperature "
+                        f"{temp}, entropy bound {bound}, 75% of positions masked",
+            "global_batch": world * T, "seq_len": T,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"W {w_bytes / 1e9:.2f} GB > L2; h rotated over {nsets} sets",
+            "timed_region": "CUDA events around the K steps; GEMM time from a second run "
+                            "with events around the GEMM launch",
+            "ms_per_step_with_kernel_events": ms_prof / args.steps,
+            "step_ms_percentiles_rank0": pct,
+            "t_hbm_ms": t_hbm * 1e3, "t_tensor_ms": t_tc * 1e3,
+        },
+        "roofline": roof,
+        "gpu_launches": 3 * args.steps,
+        "e2e": {"value": rep.job_rate(T, world, args.steps, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * d * 2, "d2h_bytes_per_step": T * (4 + 4 + 1)},
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        h_cpu, W_cpu = hs[0][:2].cpu(), W.cpu()
+        t0 = time.perf_counter()
+        oracle.lmhead_stats(h_cpu, W_cpu, temperature=temp)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": 2 / dt, "unit": "tokens/s",
+                                "cores": oracle.get_threads(), "kind": "oracle",
+                                "sample": "2 of the 256 canvas tokens over the full vocabulary, "
+                                          "fp64 oracle (one thread per token)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    rep.barrier()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "lmhead":
+        run_lmhead(args)
     else:
         run_ours(args)
 

@@ -19,7 +19,8 @@ from ._abi import (  # noqa: F401
     moe_plan_create, moe_plan_set_option, moe_plan_reserve, moe_forward, moe_forward_host,
     moe_forward_noalloc,
     moe_route, moe_plan_routing, moe_plan_sync_status, moe_plan_profile, moe_plan_destroy,
-    moe_status_str,
+    moe_status_str, moe_lmhead_create, moe_lmhead_forward, moe_lmhead_sync_status,
+    moe_lmhead_destroy, moe_lmhead_set_profile, moe_lmhead_profile,
 )
 
 
@@ -73,3 +74,33 @@ class MoeLayer:
 
     def sync_status(self, stream=None) -> int:
         return moe_plan_sync_status(self.plan, stream)
+
+
+class LmHead:
+    """lm_head over the canvas plus the entropy-bound acceptance step (a thin
+    owner of an moe_lmhead_t; every step runs in the library's kernels)."""
+
+    def __init__(self, V: int, d: int):
+        self.V, self.d = V, d
+        self.handle = moe_lmhead_create(V, d)
+
+    def step(self, h, w, temperature=1.0, softcap=0.0, masked=None, entropy_bound=0.1,
+             stream=None):
+        import torch
+        T = h.shape[0]
+        dev = h.device
+        token = torch.empty(T, dtype=torch.int32, device=dev)
+        ent = torch.empty(T, dtype=torch.float32, device=dev)
+        logz = torch.empty(T, dtype=torch.float32, device=dev)
+        acc = torch.empty(T, dtype=torch.uint8, device=dev)
+        moe_lmhead_forward(self.handle, T, h, w, temperature, softcap, masked, entropy_bound,
+                           token, ent, logz, acc, stream)
+        return token, ent, logz, acc
+
+    def sync_status(self, stream=None) -> int:
+        return moe_lmhead_sync_status(self.handle, stream)
+
+    def close(self):
+        if self.handle:
+            moe_lmhead_destroy(self.handle)
+            self.handle = None

@@ -43,6 +43,8 @@ EXPORTS = [
     "moe_plan_create", "moe_plan_set_option", "moe_plan_reserve", "moe_forward",
     "moe_forward_host", "moe_route", "moe_plan_routing", "moe_plan_sync_status",
     "moe_plan_profile", "moe_plan_destroy", "moe_status_str", "moe_forward_noalloc",
+    "moe_lmhead_create", "moe_lmhead_forward", "moe_lmhead_sync_status", "moe_lmhead_destroy",
+    "moe_lmhead_set_profile", "moe_lmhead_profile",
 ]
 
 _lock = threading.Lock()
@@ -89,6 +91,19 @@ def lib() -> ctypes.CDLL:
             L.moe_forward_noalloc.restype = I
             L.moe_status_str.argtypes = [I]
             L.moe_status_str.restype = ctypes.c_char_p
+            F = ctypes.c_float
+            L.moe_lmhead_create.argtypes = [I, I, ctypes.POINTER(P)]
+            L.moe_lmhead_create.restype = I
+            L.moe_lmhead_forward.argtypes = [P, I, P, P, F, F, P, F, P, P, P, P, P]
+            L.moe_lmhead_forward.restype = I
+            L.moe_lmhead_sync_status.argtypes = [P, P]
+            L.moe_lmhead_sync_status.restype = I
+            L.moe_lmhead_destroy.argtypes = [P]
+            L.moe_lmhead_destroy.restype = None
+            L.moe_lmhead_set_profile.argtypes = [P, I]
+            L.moe_lmhead_set_profile.restype = I
+            L.moe_lmhead_profile.argtypes = [P, ctypes.POINTER(D), ctypes.POINTER(I)]
+            L.moe_lmhead_profile.restype = I
             _lib = L
     return _lib
 
@@ -211,3 +226,39 @@ def moe_plan_destroy(plan) -> None:
 
 def moe_status_str(status: int) -> str:
     return status_str(status)
+
+
+def moe_lmhead_create(V: int, d: int) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().moe_lmhead_create(V, d, ctypes.byref(h)), "moe_lmhead_create", True)
+    return h.value
+
+
+def moe_lmhead_forward(lh, T, h, w, temperature, softcap, masked, entropy_bound, token_out,
+                       entropy_out, logz_out, accept_out, stream=None, check: bool = True):
+    st = lib().moe_lmhead_forward(lh, T, _ptr(h), _ptr(w), float(temperature), float(softcap),
+                                  _ptr(masked), float(entropy_bound), _ptr(token_out),
+                                  _ptr(entropy_out), _ptr(logz_out), _ptr(accept_out),
+                                  _stream(stream))
+    return _check(st, "moe_lmhead_forward", check)
+
+
+def moe_lmhead_sync_status(lh, stream=None) -> int:
+    return lib().moe_lmhead_sync_status(lh, _stream(stream))
+
+
+def moe_lmhead_destroy(lh) -> None:
+    lib().moe_lmhead_destroy(lh)
+
+
+def moe_lmhead_set_profile(lh, on: bool) -> None:
+    _check(lib().moe_lmhead_set_profile(lh, 1 if on else 0), "moe_lmhead_set_profile", True)
+
+
+def moe_lmhead_profile(lh):
+    """(total GEMM ms, launches) recorded since the last read."""
+    ms = ctypes.c_double()
+    n = ctypes.c_int()
+    _check(lib().moe_lmhead_profile(lh, ctypes.byref(ms), ctypes.byref(n)), "moe_lmhead_profile",
+           True)
+    return ms.value, n.value

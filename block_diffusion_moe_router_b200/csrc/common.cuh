@@ -363,6 +363,23 @@ struct ExpertArgs {
 };
 
 
+// lm_head over the canvas: statistics of softmax(z / temperature) per token
+// and entropy-bounded acceptance (lm_head.cu).
+struct LmHeadArgs {
+  int T, V, d;
+  float inv_temp;        // 1 / temperature
+  float softcap;         // z -> softcap * tanh(z / softcap) when > 0
+  float bound;           // entropy bound of the acceptance step
+  const uint8_t* masked; // [T] 1 = still masked (NULL: all)
+  float4* part;          // [T, ceil(V/128)] per-tile (max, sum exp, sum exp*u, argmax)
+  int32_t* token;        // [T] argmax
+  float* entropy;        // [T]
+  float* logz;           // [T]
+  uint8_t* accept;       // [T]
+  Ctl* ctl;
+  uint64_t timeout_ns;
+};
+
 // ---------------------------------------------------------------- top-k
 // Order-preserving map of a float to an unsigned key (-0 is folded into +0
 // first, so equal floats get equal keys).
@@ -488,6 +505,9 @@ cudaError_t moe_launch_expert(const moe::ExpertArgs& a, const CUtensorMap& tm_wg
 cudaError_t moe_launch_expert_w4(const moe::ExpertArgs& a, const CUtensorMap& tm_cgu,
                                  const CUtensorMap& tm_cd, const CUtensorMap& tm_xp,
                                  const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_lmhead_gemm(const moe::LmHeadArgs& a, const CUtensorMap& tm_w,
+                                   const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_lmhead_tail(const moe::LmHeadArgs& a, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_expert_w8(const moe::ExpertArgs& a, const CUtensorMap& tm_cgu,
                                  const CUtensorMap& tm_cd, const CUtensorMap& tm_xp,
                                  const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);

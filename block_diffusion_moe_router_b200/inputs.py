@@ -229,3 +229,26 @@ def make_small(T, d, E, k, f, seed, wdtype=WDTYPE_BF16, bias=False, residual=Fal
         out["w_gate_up"], out["scales_gate_up"] = mk((E, 2 * f, d), base + 6, base + 8, device)
         out["w_down"], out["scales_down"] = mk((E, d, f), base + 7, base + 9, device)
     return out
+
+
+# ---------------------------------------------------------------- lm_head step
+LMHEAD_V = 262144   # vocabulary of the lm_head (DiffusionGemma, vocab 262k)
+LMHEAD_D = 2816
+
+
+def make_lmhead(T: int, V: int, d: int, seed: int, device="cpu", logit_std: float = 2.0,
+                max_boost: float = 30.0):
+    """h [T, d] bf16 and W [V, d] bf16 for the lm_head step.  W ~ N(0,
+    logit_std^2 / d), so a random h ~ N(0, 1) gives logits of std logit_std
+    (a flat distribution); token t also gets c_t * W[v_t] / |W[v_t]|^2 added
+    with c_t spread over [0, max_boost] and v_t random, so its logit of v_t
+    is raised by about c_t and the entropies span flat to fully peaked, as
+    a denoising canvas does."""
+    g = _gen(seed, device)
+    W = torch.randn((V, d), generator=g, device=device) * (logit_std / math.sqrt(d))
+    h = torch.randn((T, d), generator=g, device=device)
+    tgt = torch.randint(0, V, (T,), generator=g, device=device)
+    c = torch.linspace(0.0, max_boost, T, device=device)[torch.randperm(T, generator=g, device=device)]
+    wt = W[tgt]
+    h += c[:, None] * wt / (wt * wt).sum(-1, keepdim=True)
+    return h.to(torch.bfloat16), W.to(torch.bfloat16), tgt

@@ -227,6 +227,63 @@ void moe_plan_destroy(moe_plan_t plan);
 /* Static description of a status code. */
 const char* moe_status_str(moe_status_t status);
 
+/* ---- lm_head over the canvas and the entropy-bound acceptance step -------
+ *
+ * The step after the layer stack (fucina docs "DiffusionGemma 26B-A4B --
+ * block text-diffusion": 256-token canvases denoised with the entropy-bound
+ * sampler, temperature 0.8 -> 0.4, bound 0.1; auto-round pull request:
+ * EntropyBoundSamplerConfig entropy_bound 0.1).  For each token t (h_t bf16
+ * [d], the lm_head / tied embedding W bf16 [V, d]):
+ *   z_v = h_t . W[v]  (fp32 accumulation), optionally softcap*tanh(z_v/softcap)
+ *   u_v = z_v / temperature;  logZ_t = log sum_v exp(u_v)
+ *   H_t = logZ_t - sum_v softmax(u)_v u_v            (entropy, nats)
+ *   token_t = argmax_v z_v (lowest v on ties)
+ * then, over the positions still masked: sorted by (H_t, t), accept the
+ * longest prefix whose entropies, all but the last, sum (in fp64) to at most
+ * entropy_bound; the lowest-entropy masked position is always accepted.
+ * The pages name the rule but do not state it; this is the entropy-bounded
+ * unmasking rule it is named after (the library's reading).
+ * The [T, V] logits are never written: the GEMM's epilogue folds them into
+ * per-(token, 128-row tile) softmax statistics on chip. */
+typedef struct moe_lmhead_s* moe_lmhead_t;
+
+/* Handle for a vocabulary of V rows of width d (1 <= V <= 2^24, d a multiple
+ * of 64 in [64, 8192]); no device memory until the first call. */
+moe_status_t moe_lmhead_create(int V, int d, moe_lmhead_t* out);
+
+/* Arguments (device pointers; h and w 16-byte aligned, outputs 4-byte
+ * aligned except accept_out):
+ *   T              tokens, 1..4096 (0: nothing launched)
+ *   h              bf16 [T, d]   final hidden states (after the final norm)
+ *   w              bf16 [V, d]   lm_head weight
+ *   temperature    > 0
+ *   softcap        >= 0 (0: no soft cap)
+ *   masked         uint8 [T], nonzero = still masked, or NULL (all masked)
+ *   entropy_bound  >= 0
+ *   token_out      int32 [T]     argmax token of every position
+ *   entropy_out    fp32 [T]      H_t
+ *   logz_out       fp32 [T]      logZ_t (NULL to skip)
+ *   accept_out     uint8 [T]     1 = masked and accepted this step
+ * Asynchronous on `stream`; bounded-wait expiry is reported by
+ * moe_lmhead_sync_status. */
+moe_status_t moe_lmhead_forward(moe_lmhead_t lh, int T, const void* h, const void* w,
+                                float temperature, float softcap, const uint8_t* masked,
+                                float entropy_bound, int32_t* token_out, float* entropy_out,
+                                float* logz_out, uint8_t* accept_out, void* stream);
+
+/* Synchronise `stream`, return the handle's device status word and clear it. */
+moe_status_t moe_lmhead_sync_status(moe_lmhead_t lh, void* stream);
+
+/* on != 0: moe_lmhead_forward records CUDA events around its GEMM launch
+ * (and launches without programmatic dependent launch, so the events bound
+ * the GEMM alone); moe_lmhead_profile returns the total GEMM time (ms) and
+ * the number of launches recorded since the last read, and clears them. */
+moe_status_t moe_lmhead_set_profile(moe_lmhead_t lh, int on);
+moe_status_t moe_lmhead_profile(moe_lmhead_t lh, double* gemm_ms, int* launches);
+
+/* Release the handle and its workspace (synchronous). NULL is ignored. */
+void moe_lmhead_destroy(moe_lmhead_t lh);
+
 #ifdef __cplusplus
 }
 #endif

@@ -77,3 +77,16 @@ def test_product_path_has_no_oracle_dependency():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dp, fn)).read()
                 assert "oracle" not in src.replace("CPU oracle", ""), fn
+
+
+def test_lmhead_create_rejects_bad_shapes_without_device(abi):
+    lib = abi.lib()
+    h = ctypes.c_void_p()
+    for V, d in [(0, 256), (1 << 25, 256), (1000, 32), (1000, 100), (1000, 16384)]:
+        assert lib.moe_lmhead_create(V, d, ctypes.byref(h)) == abi.MOE_ERR_UNSUPPORTED
+        assert h.value is None
+    assert lib.moe_lmhead_create(1000, 256, None) == abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_lmhead_forward(None, 4, None, None, 1.0, 0.0, None, 0.1, None, None, None,
+                                  None, None) == abi.MOE_ERR_INVALID_ARG
+    assert lib.moe_lmhead_sync_status(None, None) == abi.MOE_ERR_INVALID_ARG
+    lib.moe_lmhead_destroy(None)
