@@ -371,7 +371,7 @@ struct LmHeadArgs {
   float softcap;         // z -> softcap * tanh(z / softcap) when > 0
   float bound;           // entropy bound of the acceptance step
   const uint8_t* masked; // [T] 1 = still masked (NULL: all)
-  float4* part;          // [T, ceil(V/128)] per-tile (max, sum exp, sum exp*u, argmax)
+  float4* part;          // [T, ceil(V/256)] per-tile (max, sum exp, sum exp*u, argmax)
   int32_t* token;        // [T] argmax
   float* entropy;        // [T]
   float* logz;           // [T]

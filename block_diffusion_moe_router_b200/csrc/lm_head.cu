@@ -14,17 +14,19 @@
 // sum to at most the bound.
 //
 // Kernels:
-//   lmhead_gemm_kernel: persistent, one CTA per SM; a unit is (128-row tile
-//     of W, chunk of <= 256 tokens).  Swap-AB as in the expert kernels: W
-//     rows are the UMMA M, tokens N, so W streams from HBM once; h is
-//     re-read from L2 by every unit.  Warp 0 streams W (TMA, evict-first),
-//     warp 6 streams h (evict-last), warp 1 issues the tcgen05 UMMAs into
-//     two 256-column TMEM accumulators, warps 2..5 reduce each accumulator:
-//     the 128 x 32 tile of a 32-token slice goes through shared memory so
-//     that each thread folds 32 rows of one token into (max, sum exp, sum
-//     exp * u, argmax); four such partials per token are folded again and
-//     written as one float4 per (token, tile).  The logits never reach HBM.
-//   lmhead_finalize_kernel: one CTA per token folds its V/128 partials in a
+//   lmhead_gemm_pair_kernel: persistent, on pairs of CTAs (2-CTA clusters,
+//     one CTA per SM); a unit is (256 vocabulary rows, chunk of <= 256
+//     tokens).  One tcgen05 UMMA of M = 256 tokens (128 in each CTA) by
+//     N = 256 vocabulary rows (128 in each CTA's shared memory) per K = 16
+//     step, so W streams from HBM once and each SM reads half the operand
+//     bytes per multiply-add a 1-CTA M = 128 UMMA would.  Warp 0 streams W
+//     (TMA, evict-first), warp 6 streams h (evict-last), warp 1 of the even
+//     CTA issues the UMMAs into two 256-column TMEM accumulators per CTA,
+//     warps 2..5 reduce them: the TMEM lane is the token, so each thread
+//     folds its token's 256 logits in registers into (max, sum exp, sum
+//     exp * u, argmax) and writes one float4 per (token, 256-row tile).  The
+//     logits never reach HBM or shared memory.
+//   lmhead_finalize_kernel: one CTA per token folds its V/256 partials in a
 //     fixed order (deterministic) into logZ, H and the argmax.
 //   lmhead_accept_kernel: one CTA ranks the masked positions by (H, t) and
 //     walks them in that order summing the entropies in fp64.
@@ -36,20 +38,23 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 224;
-constexpr int kMaxA = 12;
-constexpr int kMaxB = 6;
-constexpr int kRingBytes = 200 * 1024;
-constexpr int kABytes = kBM * kBK * 2;    // 16 KB
-constexpr int kTileCols = 32;             // tokens per epilogue slice
-constexpr int kStatBytes = kBM * (kTileCols + 1) * 4 + 4 * kTileCols * 16;
-constexpr int kBarBytes = 8 * (2 * kMaxA + 2 * kMaxB + 4 + 1);
-constexpr int kSmemBytes = 1024 + kRingBytes + kStatBytes + kBarBytes + 256;
+constexpr int kRingBytes = 224 * 1024;
 enum { kWhereLmA = 40, kWhereLmB, kWhereLmMma, kWhereLmEpi };
 
 struct Stat {
   float m, s, q;
   int i;
 };
+
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kPastV = -1.0e30f;  // scaled logit of a row past V
+
+// 2^x by the hardware approximation (relative error ~2^-22; 2^-1e30 = 0)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Fold b into a: running max, sums rescaled to the new max, lowest index
 // among equal maxima.  An empty side has m = -inf.
@@ -72,152 +77,234 @@ __device__ __forceinline__ void fold(Stat& a, const Stat& b) {
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    lmhead_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
-                       const __grid_constant__ CUtensorMap tm_h, LmHeadArgs a) {
+// ---------------------------------------------------------------- CTA pairs
+// The GEMM runs on pairs of CTAs (a 2-CTA cluster): one UMMA of M = 256
+// covers both CTAs' 128 W rows against N tokens whose B rows are split
+// between the two CTAs' shared memory, so each SM reads half the B operand
+// per multiply-add that a 1-CTA M = 128 UMMA reads (at N = 256 the 1-CTA
+// kernel is bound by those shared-memory reads at ~50% of the tensor peak).
+// The even CTA of the pair issues the UMMAs and owns the full barriers; both
+// CTAs' TMA copies complete on them (the .cta_group::2 form allows the peer
+// CTA's barrier), and the UMMA commits arrive on both CTAs' barriers.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+
+// plain arrive on a barrier given by its shared::cluster address
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr)
+               : "memory");
+}
+
+// TMA tile into this CTA's shared memory, completing on the pair's barrier
+// at `bar_cl` (a shared::cluster address, possibly in the peer CTA)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, int x, int y,
+                                                 uint32_t bar_cl, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar_cl), "l"(policy)
+      : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T, M = 256
+__device__ __forceinline__ void umma_pair_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the barrier at the same offset in every CTA of `mask` when
+// the pair's UMMAs issued so far are done.
+__device__ __forceinline__ void umma_pair_commit(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)), "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+constexpr int kPairMaxA = 6;                 // h stages (L2)
+constexpr int kPairMaxB = 8;                 // W stages (HBM)
+constexpr int kPairTok = 128;                // token rows per CTA (UMMA M / 2)
+constexpr int kPairV = 256;                  // vocabulary rows per unit (UMMA N)
+constexpr int kPairStage = kPairTok * kBK * 2;  // 16 KB, also a CTA's half of a W stage
+constexpr int kPairBarBytes = 8 * (2 * kPairMaxA + 2 * kPairMaxB + 4 + 1);
+constexpr int kPairSmemBytes = 1024 + kRingBytes + kPairBarBytes + 256;
+
+// A unit of a pair is (256 vocabulary rows, chunk of <= 256 tokens).  The
+// UMMA is M = 256 tokens (128 per CTA: A = h, from each CTA's own smem) by
+// N = 256 vocabulary rows (B = W, 128 rows in each CTA's smem), so W is
+// streamed from HBM exactly once and each SM reads 4 KB of A and 4 KB of B
+// per K = 16 step.  The accumulator lane is the token: each epilogue thread
+// folds its own token's 256 logits in registers (online max / sums), with no
+// shared-memory transpose and no barriers, and writes one partial per
+// (token, 256-row tile).
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    lmhead_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
+                            const __grid_constant__ CUtensorMap tm_h, LmHeadArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  float* tile = reinterpret_cast<float*>(smem + kRingBytes);   // [128][33] u values
-  Stat* part = reinterpret_cast<Stat*>(tile + kBM * (kTileCols + 1));  // [4][32]
-  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + kRingBytes + kStatBytes);
-  uint64_t* emptyA = fullA + kMaxA;
-  uint64_t* fullB = emptyA + kMaxA;
-  uint64_t* emptyB = fullB + kMaxB;
-  uint64_t* tfull = emptyB + kMaxB;
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(smem + kRingBytes);
+  uint64_t* emptyA = fullA + kPairMaxA;
+  uint64_t* fullB = emptyA + kPairMaxA;
+  uint64_t* emptyB = fullB + kPairMaxB;
+  uint64_t* tfull = emptyB + kPairMaxB;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* s_bcast = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
   Ctl* ctl = a.ctl;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMaxA; ++i) {
+    // The full barriers of the leader collect both CTAs' copies: the leader
+    // arms them with both CTAs' bytes, and a peer's copy for a stage is only
+    // issued after that stage's previous use was consumed, so it always
+    // lands in the phase the leader arms (a peer arrival is not needed).
+    for (int i = 0; i < kPairMaxA; ++i) {
       mbar_init(&fullA[i], 1);
-      mbar_init(&emptyA[i], 1);
+      mbar_init(&emptyA[i], 1);  // the pair's UMMA commit
     }
-    for (int i = 0; i < kMaxB; ++i) {
+    for (int i = 0; i < kPairMaxB; ++i) {
       mbar_init(&fullB[i], 1);
       mbar_init(&emptyB[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], 8);  // four epilogue warps of each CTA (leader's copy used)
     }
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_h);
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_barrier();  // both CTAs' barriers initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // h may come from the previous kernel
+  pdl_wait();
   pdl_launch_dependents();
 
-  // Units: u = chunk * VT + tile, taken round-robin (they all cost the same).
-  const int VT = (a.V + kBM - 1) / kBM;
-  const int NC = (a.T + kMaxN - 1) / kMaxN;
-  const int U = VT * NC;
+  const int VT2 = (a.V + kPairV - 1) / kPairV;
+  const int NC = (a.T + 2 * kPairTok - 1) / (2 * kPairTok);
+  const int U = VT2 * NC;
+  const int nclus = gridDim.x / 2;
+  const int clus = blockIdx.x / 2;
   const int nkb = a.d / kBK;
-  const int NB = (min(a.T, kMaxN) + kBRows - 1) / kBRows * kBRows;
-  const int b_bytes = NB * kBK * 2;
-  const int SB = min(kMaxB, max(2, (kRingBytes / 3) / b_bytes));
-  const int SA = min(kMaxA, (kRingBytes - SB * b_bytes) / kABytes);
-  uint8_t* ringA = ring;
-  uint8_t* ringB = ring + SA * kABytes;
+  uint8_t* ringA = ring;                          // h
+  uint8_t* ringB = ring + kPairMaxA * kPairStage;  // W
 
   if (warp == 0) {
-    // ------------------------------------------------------------ W producer
+    // ------------------------------------------------------------ W producer (both CTAs)
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued = 0, issued_par = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const int vt = u % VT;
+      for (int u = clus; u < U && ok; u += nclus) {
+        const int vt2 = u % VT2;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&emptyA[stage], phase ^ 1, s_abort, ctl, a.timeout_ns, kWhereLmA)) {
+          if (!mbar_wait(&emptyB[stage], phase ^ 1, s_abort, ctl, a.timeout_ns, kWhereLmA)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&fullA[stage], kABytes);
-          tma_load_2d(ringA + stage * kABytes, &tm_w, kb * kBK, vt * kBM, &fullA[stage], pol_w);
-          issued |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == SA) {
+          if (leader) mbar_arrive_expect_tx(&fullB[stage], 2 * kPairStage);
+          tma_load_2d_pair(ringB + stage * kPairStage, &tm_w, kb * kBK,
+                           vt2 * kPairV + (int)rank * kPairTok,
+                           mapa_rank(smem_u32(&fullB[stage]), 0), pol_w);
+          if (++stage == kPairMaxB) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      for (int s2 = 0; s2 < SA; ++s2)
-        if ((issued >> s2) & 1u)
-          mbar_wait_drain(&fullA[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
     }
   } else if (warp == 6) {
-    // ------------------------------------------------------------ h producer
+    // ------------------------------------------------------------ h producer (both CTAs)
     if (lane == 0) {
       const uint64_t pol_act = l2_policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued = 0, issued_par = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const int ch = u / VT;
-        const int n = min(kMaxN, a.T - ch * kMaxN);
-        const int nbox = (n + kBRows - 1) / kBRows;
+      for (int u = clus; u < U && ok; u += nclus) {
+        const int ch = u / VT2;
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&emptyB[stage], phase ^ 1, s_abort, ctl, a.timeout_ns, kWhereLmB)) {
+          if (!mbar_wait(&emptyA[stage], phase ^ 1, s_abort, ctl, a.timeout_ns, kWhereLmB)) {
             ok = false;
             break;
           }
-          uint8_t* sb = ringB + stage * b_bytes;
-          mbar_arrive_expect_tx(&fullB[stage], nbox * kBRows * kBK * 2);
-          for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d(sb + bx * kBRows * kBK * 2, &tm_h, kb * kBK, ch * kMaxN + bx * kBRows,
-                        &fullB[stage], pol_act);
-          issued |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == SB) {
+          if (leader) mbar_arrive_expect_tx(&fullA[stage], 2 * kPairStage);
+          tma_load_2d_pair(ringA + stage * kPairStage, &tm_h, kb * kBK,
+                           ch * 2 * kPairTok + (int)rank * kPairTok,
+                           mapa_rank(smem_u32(&fullA[stage]), 0), pol_act);
+          if (++stage == kPairMaxA) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      for (int s2 = 0; s2 < SB; ++s2)
-        if ((issued >> s2) & 1u)
-          mbar_wait_drain(&fullB[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ UMMA issuer (leader)
+    if (leader && lane == 0) {
       int sa_i = 0, sb_i = 0;
       uint32_t pa = 0, pb = 0;
       int acc = 0;
       uint32_t aphase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const int ch = u / VT;
-        const int n = min(kMaxN, a.T - ch * kMaxN);
-        const uint32_t idesc = idesc_bf16_f32(kBM, (n + 15) & ~15);
+      const uint32_t idesc = idesc_bf16_f32(2 * kPairTok, kPairV);
+      for (int u = clus; u < U && ok; u += nclus) {
         if (!mbar_wait(&tempty[acc], aphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereLmMma)) break;
         tc_fence_after();
-        const uint32_t dt = tmem_base + (uint32_t)(acc * kMaxN);
+        const uint32_t dt = tmem_base + (uint32_t)(acc * kPairV);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&fullA[sa_i], pa, s_abort, ctl, a.timeout_ns, kWhereLmMma) ||
               !mbar_wait(&fullB[sb_i], pb, s_abort, ctl, a.timeout_ns, kWhereLmMma)) {
@@ -225,111 +312,102 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(ringA + sa_i * kABytes);
-          const uint32_t sb = smem_u32(ringB + sb_i * b_bytes);
+          const uint32_t sa = smem_u32(ringA + sa_i * kPairStage);
+          const uint32_t sb = smem_u32(ringB + sb_i * kPairStage);
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk)
-            umma_bf16(dt, sdesc_k_sw128(sa + kk * kUmmaK * 2), sdesc_k_sw128(sb + kk * kUmmaK * 2),
-                      idesc, (kb | kk) ? 1u : 0u);
-          umma_commit(&emptyA[sa_i]);
-          umma_commit(&emptyB[sb_i]);
-          if (++sa_i == SA) {
+            umma_pair_bf16(dt, sdesc_k_sw128(sa + kk * kUmmaK * 2),
+                           sdesc_k_sw128(sb + kk * kUmmaK * 2), idesc, (kb | kk) ? 1u : 0u);
+          umma_pair_commit(&emptyA[sa_i], 3);
+          umma_pair_commit(&emptyB[sb_i], 3);
+          if (++sa_i == kPairMaxA) {
             sa_i = 0;
             pa ^= 1;
           }
-          if (++sb_i == SB) {
+          if (++sb_i == kPairMaxB) {
             sb_i = 0;
             pb ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        umma_pair_commit(&tfull[acc], 3);
         acc ^= 1;
         if (acc == 0) aphase ^= 1;
       }
-      umma_commit(drain);
+      umma_pair_commit(drain, 1);
       mbar_wait_drain(drain, 0, ctl, a.timeout_ns);
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int q4 = warp & 3;           // TMEM lane quarter
-    const int row = q4 * 32 + lane;    // W row inside the tile (TMEM lane)
-    const int et = threadIdx.x - 64;   // 0..127
-    const int col = et & 31;           // token inside the slice (reduction phase)
-    const int rq = et >> 5;            // row quarter it folds
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q4 = warp & 3;
+    const int tl = q4 * 32 + lane;  // token inside this CTA's 128 (TMEM lane)
+    const float c2 = a.inv_temp * 1.4426950408889634f;  // log2(e) / temperature
+    const uint32_t tempty_l0 = mapa_rank(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_l1 = mapa_rank(smem_u32(&tempty[1]), 0);
     int acc = 0;
     uint32_t aphase = 0;
-    for (int u = blockIdx.x; u < U; u += gridDim.x) {
-      if (et == 0)
-        *s_bcast = mbar_wait(&tfull[acc], aphase, s_abort, ctl, a.timeout_ns, kWhereLmEpi) ? 1 : 0;
-      named_barrier(1, 128);
-      if (*s_bcast == 0) break;
+    for (int u = clus; u < U; u += nclus) {
+      if (!mbar_wait(&tfull[acc], aphase, s_abort, ctl, a.timeout_ns, kWhereLmEpi)) break;
       tc_fence_after();
-      const int vt = u % VT, ch = u / VT;
-      const int n = min(kMaxN, a.T - ch * kMaxN);
-      const int vrow = vt * kBM + row;
-      const bool valid = vrow < a.V;
-      const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kMaxN);
-      for (int c0 = 0; c0 < n; c0 += kTileCols) {
+      const int vt2 = u % VT2, ch = u / VT2;
+      const int tok = ch * 2 * kPairTok + (int)rank * kPairTok + tl;
+      const int v0 = vt2 * kPairV;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * kPairV);
+      Stat st;
+      st.m = -INFINITY;
+      st.s = 0.f;
+      st.q = 0.f;
+      st.i = 0;
+      for (int c0 = 0; c0 < kPairV; c0 += 32) {
         uint32_t v[32];
         tmem_ld32(tbase + c0, v);
         tmem_wait_ld();
+        // base-2 scaled logits w = u * log2(e); rows past V get a finite
+        // sentinel (so that 2^(w - max) * w is 0, not 0 * -inf)
+        float x[32];
+        float cm = kPastV;
+        int ci = 0;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           float z = __uint_as_float(v[i]);
           if (a.softcap > 0.f) z = a.softcap * tanhf(z / a.softcap);
-          tile[row * (kTileCols + 1) + i] = valid ? z * a.inv_temp : -INFINITY;
-        }
-        named_barrier(1, 128);
-        // thread (rq, col): rows [32 rq, 32 rq + 32) of token column col
-        Stat st;
-        st.m = -INFINITY;
-        st.i = 0;
-#pragma unroll 8
-        for (int r = 0; r < 32; ++r) {
-          const float x = tile[(rq * 32 + r) * (kTileCols + 1) + col];
-          if (x > st.m) {
-            st.m = x;
-            st.i = vt * kBM + rq * 32 + r;
+          x[i] = (v0 + c0 + i < a.V) ? z * c2 : kPastV;
+          if (x[i] > cm) {
+            cm = x[i];
+            ci = v0 + c0 + i;
           }
         }
-        st.s = 0.f;
-        st.q = 0.f;
-        if (st.m != -INFINITY) {
-#pragma unroll 8
-          for (int r = 0; r < 32; ++r) {
-            const float x = tile[(rq * 32 + r) * (kTileCols + 1) + col];
-            if (x != -INFINITY) {  // rows past V (0 * -inf would poison q)
-              const float e = expf(x - st.m);
-              st.s += e;
-              st.q = fmaf(e, x, st.q);
-            }
-          }
+        if (cm == kPastV) continue;  // the whole slice is past V
+        float s2 = 0.f, q2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float e = ex2_approx(x[i] - cm);
+          s2 += e;
+          q2 = fmaf(e, x[i], q2);
         }
-        part[rq * kTileCols + col] = st;
-        named_barrier(1, 128);
-        if (rq == 0) {
-          Stat t = part[col];
-          for (int k2 = 1; k2 < 4; ++k2) fold(t, part[k2 * kTileCols + col]);
-          const int tok = ch * kMaxN + c0 + col;
-          if (c0 + col < n)
-            a.part[(size_t)tok * VT + vt] = make_float4(t.m, t.s, t.q, __int_as_float(t.i));
-        }
-        named_barrier(1, 128);
+        Stat b;  // back to natural units: max u, sum e^(u - max), sum e^(u - max) u
+        b.m = cm * kLn2;
+        b.s = s2;
+        b.q = q2 * kLn2;
+        b.i = ci;
+        fold(st, b);
       }
+      if (tok < a.T) a.part[(size_t)tok * VT2 + vt2] = make_float4(st.m, st.s, st.q, __int_as_float(st.i));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) mbar_arrive_remote(acc ? tempty_l1 : tempty_l0);
       acc ^= 1;
       if (acc == 0) aphase ^= 1;
     }
   }
 
+  // Neither CTA leaves (or frees TMEM) while the pair's UMMAs may still read
+  // its shared memory or write its TMEM: the leader drained them above.
   tc_fence_before();
-  __syncthreads();
+  cluster_barrier();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -339,7 +417,7 @@ __global__ void __launch_bounds__(256) lmhead_finalize_kernel(LmHeadArgs a) {
   __shared__ Stat sh[256];
   pdl_wait();
   const int t = blockIdx.x;
-  const int VT = (a.V + kBM - 1) / kBM;
+  const int VT = (a.V + kPairV - 1) / kPairV;  // partials per token (256-row tiles)
   Stat st;
   st.m = -INFINITY;
   st.s = st.q = 0.f;
@@ -411,15 +489,33 @@ __global__ void __launch_bounds__(1024) lmhead_accept_kernel(LmHeadArgs a) {
 
 cudaError_t moe_launch_lmhead_gemm(const moe::LmHeadArgs& a, const CUtensorMap& tm_w,
                                    const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl) {
-  static_assert(moe::kSmemBytes <= 232448, "lm_head kernel smem above the sm_100 limit");
-  cudaError_t err = cudaFuncSetAttribute(moe::lmhead_gemm_kernel,
+  static_assert(moe::kPairSmemBytes <= 232448, "lm_head kernel smem above the sm_100 limit");
+  cudaError_t err = cudaFuncSetAttribute(moe::lmhead_gemm_pair_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         moe::kSmemBytes);
+                                         moe::kPairSmemBytes);
   if (err != cudaSuccess) return err;
-  const int VT = (a.V + moe::kBM - 1) / moe::kBM;
-  const int U = VT * ((a.T + moe::kMaxN - 1) / moe::kMaxN);
-  return moe::launch_pdl(moe::lmhead_gemm_kernel, dim3(min(num_sms, U)), dim3(moe::kThreads),
-                         (size_t)moe::kSmemBytes, s, pdl, tm_w, tm_h, a);
+  // as many CTA pairs as can be resident at once (one CTA per SM), but no
+  // more than there are units
+  static int max_pairs[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && max_pairs[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(moe::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = moe::kPairSmemBytes;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, moe::lmhead_gemm_pair_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = num_sms / 2;
+    }
+    max_pairs[dev] = n > 0 ? n : 1;
+  }
+  const int VT2 = (a.V + moe::kPairV - 1) / moe::kPairV;
+  const int U = VT2 * ((a.T + 2 * moe::kPairTok - 1) / (2 * moe::kPairTok));
+  const int pairs = min(min(dev < 64 ? max_pairs[dev] : num_sms / 2, num_sms / 2), U);
+  return moe::launch_pdl(moe::lmhead_gemm_pair_kernel, dim3(2 * pairs), dim3(moe::kThreads),
+                         (size_t)moe::kPairSmemBytes, s, pdl, tm_w, tm_h, a);
 }
 
 cudaError_t moe_launch_lmhead_tail(const moe::LmHeadArgs& a, cudaStream_t s, bool pdl) {

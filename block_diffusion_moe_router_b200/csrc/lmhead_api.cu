@@ -107,7 +107,7 @@ moe_status_t moe_lmhead_forward(moe_lmhead_t p, int T, const void* h, const void
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev != p->device) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int VT = (p->V + moe::kBM - 1) / moe::kBM;
+  const int VT = (p->V + 255) / 256;  // partials per token: one per 256-row tile
   if (!p->ws || T > p->cap_T) {
     int cap = p->cap_T > 0 ? p->cap_T : 64;
     while (cap < T) cap *= 2;
@@ -132,7 +132,7 @@ moe_status_t moe_lmhead_forward(moe_lmhead_t p, int T, const void* h, const void
                          : reinterpret_cast<float*>(p->part + (size_t)p->cap_T * VT);
   CUtensorMap tm_w, tm_h;
   if (!map_bf16(&tm_w, w, (uint64_t)p->V, (uint64_t)p->d, moe::kBM) ||
-      !map_bf16(&tm_h, h, (uint64_t)T, (uint64_t)p->d, moe::kBRows))
+      !map_bf16(&tm_h, h, (uint64_t)T, (uint64_t)p->d, 128))
     return MOE_ERR_CUDA;
   moe::LmHeadArgs a;
   a.T = T;
