@@ -452,22 +452,28 @@ __global__ void __launch_bounds__(256) lmhead_finalize_kernel(LmHeadArgs a) {
 }
 
 // Entropy-bounded acceptance over the masked positions: rank by (H, t),
-// then one thread walks the ranks summing entropies in fp64.
+// then one thread walks the ranks summing entropies in fp64.  Entropies and
+// the mask are staged in shared memory first (each rank reads all of them).
 __global__ void __launch_bounds__(1024) lmhead_accept_kernel(LmHeadArgs a) {
-  extern __shared__ int s_order[];  // [T] position at each rank (-1: none)
+  extern __shared__ int s_order[];  // [T] position at each rank (-1: none), then H [T], mask [T]
+  float* s_h = reinterpret_cast<float*>(s_order + a.T);
+  uint8_t* s_m = reinterpret_cast<uint8_t*>(s_h + a.T);
   pdl_wait();
   const int T = a.T;
-  for (int t = threadIdx.x; t < T; t += blockDim.x) s_order[t] = -1;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    s_order[t] = -1;
+    s_h[t] = a.entropy[t];
+    s_m[t] = a.masked ? (a.masked[t] != 0) : 1;
+  }
   __syncthreads();
   for (int t = threadIdx.x; t < T; t += blockDim.x) {
     a.accept[t] = 0;
-    if (a.masked && !a.masked[t]) continue;
-    const float ht = a.entropy[t];
+    if (!s_m[t]) continue;
+    const float ht = s_h[t];
     int rank = 0;
-    for (int s = 0; s < T; ++s) {
-      if (a.masked && !a.masked[s]) continue;
-      const float hs = a.entropy[s];
-      rank += (hs < ht || (hs == ht && s < t)) ? 1 : 0;
+    for (int q = 0; q < T; ++q) {
+      const float hs = s_h[q];
+      rank += (s_m[q] && (hs < ht || (hs == ht && q < t))) ? 1 : 0;
     }
     s_order[rank] = t;
   }
@@ -478,7 +484,7 @@ __global__ void __launch_bounds__(1024) lmhead_accept_kernel(LmHeadArgs a) {
       const int t = s_order[r];
       if (t < 0 || below > (double)a.bound) break;
       a.accept[t] = 1;
-      below += (double)a.entropy[t];
+      below += (double)s_h[t];
     }
   }
 }
@@ -522,5 +528,5 @@ cudaError_t moe_launch_lmhead_tail(const moe::LmHeadArgs& a, cudaStream_t s, boo
   cudaError_t err = moe::launch_pdl(moe::lmhead_finalize_kernel, dim3(a.T), dim3(256), 0, s, pdl, a);
   if (err != cudaSuccess) return err;
   return moe::launch_pdl(moe::lmhead_accept_kernel, dim3(1), dim3(1024),
-                         (size_t)a.T * sizeof(int), s, pdl, a);
+                         (size_t)a.T * (sizeof(int) + sizeof(float) + 1), s, pdl, a);
 }
