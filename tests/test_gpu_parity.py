@@ -188,6 +188,22 @@ def test_encode_sampled_rows():
     print("encode sampled rel-L2", err)
 
 
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_INT4, inputs.WDTYPE_FP8])
+def test_encode_shape_coded_weights_sampled_rows(wd):
+    """T=2048 with int4 or fp8 expert weights: ~128 tokens per expert, so the
+    coded kernels run their largest chunks (and the fp8 kernel its shallowest
+    code ring); the oracle checks 48 sampled rows including both ends."""
+    T, d, E, k, f = 2048, 2816, 128, 8, 704
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=120 + wd, wdtype=wd, device="cuda")
+    lay_cpu = _cpu(lay)
+    g = np.random.default_rng(4)
+    rows = np.unique(np.concatenate([np.arange(8), np.arange(T - 8, T),
+                                     g.choice(T, 32, replace=False)]))
+    err, _ = full_check(lay_cpu, lay, E, k, d, f, rows=rows,
+                        tol=TOL_INT4 if wd == inputs.WDTYPE_INT4 else TOL_FP8)
+    print("encode-shape", "int4" if wd == inputs.WDTYPE_INT4 else "fp8", "sampled rel-L2", err)
+
+
 def test_stack30_layer_zipf_bias_and_residual():
     """One layer of the 30-layer stack: Zipf-skewed router bias, residual added
     in place (out aliases residual).  The delta is checked with the residual
