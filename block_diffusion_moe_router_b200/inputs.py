@@ -12,6 +12,8 @@ per-expert intermediate 704, symmetric int4 weights in groups of 128):
   canvas   T=256,  d=2816, E=128, k=8, f=704, bf16 weights
   canvas4  T=256,  d=2816, E=128, k=8, f=704, int4 w4g128 weights + fp16 scales
   canvas8  T=256,  d=2816, E=128, k=8, f=704, fp8 E4M3 weights + fp32 row scales
+  canvas4f T=256,  d=2816, E=128, k=8, f=704, fp4 E2M1 weights + E4M3 block
+           scales (16 elements) + fp32 row scales
   encode   T=2048, d=2816, E=128, k=8, f=704, bf16 weights (prompt + canvas)
   stack30  30 layers of `canvas`, distinct weights, Zipf(1.1)-skewed router bias,
            residual carried between layers, experts reading the (1+gamma2)
@@ -54,6 +56,8 @@ GROUP = 128  # int4 quantisation group along the input dimension
 WDTYPE_BF16 = 0
 WDTYPE_INT4 = 1
 WDTYPE_FP8 = 2
+WDTYPE_FP4 = 3
+FP4_BLOCK = 16        # elements per E4M3 block scale of the fp4 weights
 FP8_CODE_STD = 64.0   # spread of the E4M3 code draws
 
 
@@ -89,6 +93,8 @@ WORKLOADS = {
                         wdtype=WDTYPE_INT4, act_wid=1),
     "canvas8": Workload("canvas8", 5, T=256, d=2816, E=128, k=8, f=704,
                         wdtype=WDTYPE_FP8, act_wid=1),
+    "canvas4f": Workload("canvas4f", 6, T=256, d=2816, E=128, k=8, f=704,
+                         wdtype=WDTYPE_FP4, act_wid=1),
     "encode": Workload("encode", 3, T=2048, d=2816, E=128, k=8, f=704),
     "stack30": Workload("stack30", 4, T=256, d=2816, E=128, k=8, f=704,
                         layers=30, zipf_s=1.1, residual=True, expert_norm=True),
@@ -164,6 +170,36 @@ def make_fp8(shape, seed_codes, seed_scales, device):
     return codes, scales
 
 
+def make_fp4(shape, seed_codes, seed_scales, device):
+    """Random E2M1 codes (uniform over the 16 nibbles, packed two per byte
+    like the int4 codes) and their scale records: per expert e, the fp32 row
+    scales [R] (U(0.5, 1.5) * 0.01) then the E4M3 block scales [NB][R] (N(1,
+    0.25^2) draws clamped to [0.25, 4] and rounded to E4M3 by torch's cast),
+    NB = ceil(C/16), all as one uint8 tensor [E, 4R + NB R]."""
+    E, rows, cols = shape
+    g = _gen(seed_codes, device)
+    nib = torch.randint(0, 16, (E, rows, cols), generator=g, device=device, dtype=torch.int16)
+    codes = (nib[..., 0::2] | (nib[..., 1::2] << 4)).to(torch.uint8)
+    nb = (cols + FP4_BLOCK - 1) // FP4_BLOCK
+    gs = _gen(seed_scales, device)
+    srow = (torch.rand((E, rows), generator=gs, device=device) + 0.5) * 0.01
+    blk = (torch.randn((E, nb, rows), generator=gs, device=device) * 0.25 + 1.0).clamp_(0.25, 4.0)
+    blk = blk.to(torch.float8_e4m3fn).view(torch.uint8)
+    rec = torch.cat([srow.contiguous().view(torch.uint8).reshape(E, rows * 4),
+                     blk.reshape(E, nb * rows)], dim=1)
+    return codes, rec.contiguous()
+
+
+def fp4_scale_record(rec: torch.Tensor, rows: int, cols: int):
+    """Split scale records (see make_fp4) into fp32 row scales [E, R] and
+    E4M3 block-scale bytes [E, NB, R] (byte reinterpretation only)."""
+    E = rec.shape[0]
+    nb = (cols + FP4_BLOCK - 1) // FP4_BLOCK
+    srow = rec[:, :rows * 4].contiguous().view(torch.float32).reshape(E, rows)
+    blk = rec[:, rows * 4:].reshape(E, nb, rows)
+    return srow, blk
+
+
 def zipf_bias(E: int, s: float, seed: int, device) -> torch.Tensor:
     """Router bias whose exp() follows a Zipf(s) law over a seeded random
     ranking of the experts: b_e = -s * ln(rank_e), rank_e in 1..E."""
@@ -196,7 +232,7 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T: Optional[int] = Non
         out["scales_gate_up"] = None
         out["scales_down"] = None
     else:
-        mk = make_fp8 if w.wdtype == WDTYPE_FP8 else make_int4
+        mk = {WDTYPE_FP8: make_fp8, WDTYPE_FP4: make_fp4}.get(w.wdtype, make_int4)
         out["w_gate_up"], out["scales_gate_up"] = mk(
             (w.E, 2 * w.f, w.d), seed_for(w.wid, layer, _TID_WGU),
             seed_for(w.wid, layer, _TID_SGU), device)
@@ -225,7 +261,7 @@ def make_small(T, d, E, k, f, seed, wdtype=WDTYPE_BF16, bias=False, residual=Fal
         out["scales_gate_up"] = None
         out["scales_down"] = None
     else:
-        mk = make_fp8 if wdtype == WDTYPE_FP8 else make_int4
+        mk = {WDTYPE_FP8: make_fp8, WDTYPE_FP4: make_fp4}.get(wdtype, make_int4)
         out["w_gate_up"], out["scales_gate_up"] = mk((E, 2 * f, d), base + 6, base + 8, device)
         out["w_down"], out["scales_down"] = mk((E, d, f), base + 7, base + 9, device)
     return out

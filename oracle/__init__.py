@@ -18,6 +18,7 @@ from .oracle import (  # noqa: F401
     decode_bf16,
     decode_fp16,
     decode_e4m3,
+    decode_e2m1,
     lmhead_stats,
     eb_accept,
     set_threads,

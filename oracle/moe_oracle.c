@@ -23,6 +23,9 @@
  *  [OCP] OCP 8-bit Floating Point Specification (OFP8), E4M3 encoding: the
  *        8-bit float format of the fp8 weight storage (the pages name FP8
  *        builds but do not define the encoding).
+ *  [MX]  OCP Microscaling Formats (MX) Specification, FP4 E2M1 element
+ *        encoding: the 4-bit float of the fp4 weight storage (the pages name
+ *        FP4 builds but do not define them).
  *
  * Where the pages are silent this file follows the readings adopted by the
  * library (they are listed once, here):
@@ -40,6 +43,11 @@
  *    two's complement; w = code * scale[i / 128] with fp16 scales, exact here;
  *  - fp8: element i of a row is byte i, an E4M3 value [OCP]; w = value *
  *    scale[row] with one fp32 scale per weight row (output channel), exact;
+ *  - fp4: element i of a row is the nibble of byte i/2 (low nibble for even
+ *    i), an E2M1 value [MX]; w = value * e4m3(block[i/16][row]) * s[row]:
+ *    an E4M3 scale per 16 consecutive elements and an fp32 scale per row.
+ *    The scales of expert e form one record {fp32 s[R]; uint8 block[NB][R]}
+ *    (NB = ceil(C/16); each block's rows contiguous), records back to back;
  *  - out = residual + sum_j w_j y_j, summed in j order (residual optional).
  *
  * Everything is computed in double precision from the exact bf16 / fp16 /
@@ -56,6 +64,7 @@
 #define ORACLE_W_BF16 0
 #define ORACLE_W_INT4 1
 #define ORACLE_W_FP8 2
+#define ORACLE_W_FP4 3
 #define ORACLE_GROUP 128
 
 /* ---- scalar decoders (IEEE definitions) -------------------------------- */
@@ -101,6 +110,17 @@ static double e4m3_to_double(uint8_t b) {
   return sign ? -v : v;
 }
 
+/* MX FP4 E2M1 [MX]: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit;
+ * exponent 0 is subnormal (m * 0.5); no infinities or NaN.  The magnitudes
+ * are 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+static double e2m1_to_double(int nib) {
+  int sign = (nib >> 3) & 1;
+  int ex = (nib >> 1) & 0x3;
+  int man = nib & 0x1;
+  double v = (ex == 0) ? 0.5 * man : ldexp(1.0 + 0.5 * man, ex - 1);
+  return sign ? -v : v;
+}
+
 /* 4-bit two's complement code of element i of a packed row. */
 static int int4_code(const uint8_t* row, int i) {
   int byte = row[i / 2];
@@ -121,6 +141,17 @@ static double weight_elem(int wdtype, const void* w, const void* scales, int R, 
   if (wdtype == ORACLE_W_FP8) {
     const uint8_t* wp = (const uint8_t*)w + row * (size_t)C;
     return e4m3_to_double(wp[i]) * (double)((const float*)scales)[row];
+  }
+  if (wdtype == ORACLE_W_FP4) {
+    const uint8_t* wp = (const uint8_t*)w + row * (size_t)(C / 2);
+    int byte = wp[i / 2];
+    int nib = (i % 2 == 0) ? (byte & 0xf) : ((byte >> 4) & 0xf);
+    const size_t NB = (size_t)(C + 15) / 16;
+    const uint8_t* rec = (const uint8_t*)scales + (size_t)e * ((size_t)R * 4 + NB * R);
+    float srow;
+    memcpy(&srow, rec + (size_t)r * 4, sizeof srow);
+    const uint8_t blk = rec[(size_t)R * 4 + (size_t)(i / 16) * R + r];
+    return e2m1_to_double(nib) * e4m3_to_double(blk) * (double)srow;
   }
   const uint8_t* wp = (const uint8_t*)w + row * (size_t)(C / 2);
   int ng = (C + ORACLE_GROUP - 1) / ORACLE_GROUP;
@@ -337,6 +368,10 @@ void oracle_decode_bf16(int n, const uint16_t* in, double* out) {
 
 void oracle_decode_fp16(int n, const uint16_t* in, double* out) {
   for (int i = 0; i < n; i++) out[i] = fp16_to_double(in[i]);
+}
+
+void oracle_decode_e2m1(int n, const uint8_t* in, double* out) {
+  for (int i = 0; i < n; i++) out[i] = e2m1_to_double(in[i] & 0xf);
 }
 
 void oracle_decode_e4m3(int n, const uint8_t* in, double* out) {

@@ -23,6 +23,7 @@ _lib = None
 W_BF16 = 0
 W_INT4 = 1
 W_FP8 = 2
+W_FP4 = 3
 
 
 def build(force: bool = False) -> str:
@@ -60,6 +61,7 @@ def lib():
             L.oracle_decode_bf16.argtypes = [I, P, P]
             L.oracle_decode_fp16.argtypes = [I, P, P]
             L.oracle_decode_e4m3.argtypes = [I, P, P]
+            L.oracle_decode_e2m1.argtypes = [I, P, P]
             L.oracle_lmhead_stats.argtypes = [I, I, P, P, D, D, P, I, P, P, P, P]
             L.oracle_eb_accept.argtypes = [I, P, P, D, P]
             L.oracle_set_threads.argtypes = [I]
@@ -93,11 +95,15 @@ def _np(t, dtype=None):
 
 def _wdtype(w, scales) -> int:
     """Storage format of a weight array: bf16 (uint16 bits), int4 (packed
-    bytes with fp16 scales) or fp8 E4M3 (one byte per weight, fp32 row
-    scales)."""
+    bytes with fp16 scales), fp8 E4M3 (one byte per weight, fp32 row
+    scales) or fp4 E2M1 (packed bytes, scale records as uint8 bytes)."""
     if w.dtype != np.uint8:
         return W_BF16
-    return W_FP8 if scales is not None and scales.dtype == np.float32 else W_INT4
+    if scales is not None and scales.dtype == np.float32:
+        return W_FP8
+    if scales is not None and scales.dtype == np.uint8:
+        return W_FP4
+    return W_INT4
 
 
 def _p(a):
@@ -235,6 +241,14 @@ def decode_fp16(t) -> np.ndarray:
     a = _np(t)
     out = np.empty(a.shape, np.float64)
     lib().oracle_decode_fp16(a.size, _p(a), _p(out))
+    return out
+
+
+def decode_e2m1(t) -> np.ndarray:
+    """E2M1 codes (the low nibble of each uint8) -> float64 values."""
+    a = _np(t, np.uint8)
+    out = np.empty(a.shape, np.float64)
+    lib().oracle_decode_e2m1(a.size, _p(a), _p(out))
     return out
 
 

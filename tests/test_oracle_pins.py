@@ -17,6 +17,9 @@ import oracle
 from block_diffusion_moe_router_b200 import inputs
 
 EPS = 1e-6
+# MX FP4 E2M1 values of the 16 nibbles (OCP Microscaling Formats specification)
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0,
+              -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
 
 
 # ---------------------------------------------------------------- helpers
@@ -30,6 +33,14 @@ def dense_weights(w, scales, cols):
         return w.double()
     if scales.dtype == torch.float32:  # fp8: torch's own E4M3 decode
         return w.view(torch.float8_e4m3fn).double() * scales.double()[..., None]
+    if scales.dtype == torch.uint8:  # fp4: the MX E2M1 table, torch's E4M3 decode
+        E, R = w.shape[0], w.shape[1]
+        nib = torch.stack([w & 0xF, w >> 4], dim=-1).reshape(E, R, -1).long()
+        vals = torch.tensor(E2M1_TABLE, dtype=torch.float64)[nib]
+        srow, blk = inputs.fp4_scale_record(scales, R, cols)
+        bs = blk.view(torch.float8_e4m3fn).double().permute(0, 2, 1)  # [E, R, NB]
+        bs = bs.repeat_interleave(inputs.FP4_BLOCK, dim=-1)[..., :cols]
+        return vals * bs * srow.double()[..., None]
     codes = inputs.unpack_int4(w).double()
     s = scales.double().repeat_interleave(inputs.GROUP, dim=-1)[..., :cols]
     return codes * s
@@ -214,6 +225,8 @@ def test_tie_break_duplicated_router_rows():
     (5, 8, 3, False, False, inputs.WDTYPE_INT4, True),
     (6, 16, 4, True, True, inputs.WDTYPE_FP8, False),
     (7, 8, 2, False, False, inputs.WDTYPE_FP8, True),
+    (8, 16, 4, True, True, inputs.WDTYPE_FP4, False),
+    (9, 8, 3, False, False, inputs.WDTYPE_FP4, True),
 ])
 def test_layer_matches_brute_force(seed, E, k, bias, residual, wd, enorm):
     d, f = 256, 64
@@ -474,3 +487,37 @@ def test_fp8_single_code_closed_form():
     ref = np.zeros((3, d))
     ref[:, m] = ref_m
     np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-300)
+
+
+# ---------------------------------------------------------------- fp4 storage
+
+
+def test_e2m1_decode_table():
+    """The 16 E2M1 nibbles decode to the MX table (1 sign, 2 exponent bits
+    with bias 1, 1 mantissa bit; exponent 0 is subnormal)."""
+    got = oracle.decode_e2m1(np.arange(16, dtype=np.uint8))
+    np.testing.assert_array_equal(got, np.array(E2M1_TABLE))
+    assert np.array_equal(np.signbit(got[8:]), np.ones(8, bool))
+
+
+def test_fp4_weight_row_closed_form():
+    """Hand-placed nibbles, block scales and row scales (pins the nibble
+    order, the block index i // 16 and the record layout)."""
+    E, R, C = 2, 3, 64
+    nib = torch.zeros(E, R, C, dtype=torch.int16)
+    nib[1, 2, 0] = 0x2      # 1.0
+    nib[1, 2, 1] = 0xF      # -6.0
+    nib[1, 2, 17] = 0x7     # 6.0 in block 1
+    nib[1, 2, 63] = 0x9     # -0.5 in block 3
+    codes = (nib[..., 0::2] | (nib[..., 1::2] << 4)).to(torch.uint8)
+    srow = torch.ones(E, R)
+    srow[1, 2] = 0.5
+    blk = torch.full((E, 4, R), 1.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    blk[1, 1, 2] = torch.tensor(2.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    blk[1, 3, 2] = torch.tensor(0.25).to(torch.float8_e4m3fn).view(torch.uint8)
+    rec = torch.cat([srow.view(torch.uint8).reshape(E, R * 4), blk.reshape(E, 4 * R)], 1)
+    row = oracle.weight_row(codes, rec.contiguous(), 1, 2, C)
+    ref = np.zeros(C)
+    ref[0], ref[1], ref[17], ref[63] = 0.5, -3.0, 6.0, -0.0625
+    np.testing.assert_array_equal(row, ref)
+    assert np.all(oracle.weight_row(codes, rec.contiguous(), 0, 2, C) == 0)
