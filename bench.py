@@ -178,8 +178,9 @@ def launches_per_layer(w, T: int, router: str) -> int:
     return 5
 
 
-# weight formats by moe_wdtype_t value (bf16, int4, fp8)
-WFMT = {0: "bf16", 1: "int4 w4g128", 2: "fp8 E4M3 (fp32 row scales)"}
+# weight formats by moe_wdtype_t value (bf16, int4, fp8, fp4)
+WFMT = {0: "bf16", 1: "int4 w4g128", 2: "fp8 E4M3 (fp32 row scales)",
+        3: "fp4 E2M1 (E4M3 scales per 16 weights, fp32 row scales)"}
 
 
 def layer_costs(w, touched: float, T: int):
@@ -190,6 +191,8 @@ def layer_costs(w, touched: float, T: int):
         wbytes = 3 * w.f * w.d * 2
     elif w.wdtype == 2:  # fp8: E4M3 bytes + one fp32 scale per row
         wbytes = 3 * w.f * w.d + 4 * (2 * w.f + w.d)
+    elif w.wdtype == 3:  # fp4: packed E2M1 + scale records (fp32 per row, E4M3 per 16)
+        wbytes = 3 * w.f * w.d // 2 + 2 * w.f * (4 + w.d // 16) + w.d * (4 + w.f // 16)
     else:
         wbytes = 3 * w.f * w.d // 2 + 2 * (2 * w.f * w.n_groups_d + w.d * w.n_groups_f)
     expert_bytes = touched * wbytes
@@ -438,6 +441,7 @@ def run_ours(args):
         "canvas": "one MoE layer over a T=256 token canvas",
         "canvas4": "one MoE layer over a T=256 token canvas, int4 w4g128 weights",
         "canvas8": "one MoE layer over a T=256 token canvas, fp8 E4M3 weights",
+        "canvas4f": "one MoE layer over a T=256 token canvas, fp4 E2M1 weights",
         "encode": "one MoE layer over T=2048 tokens (1792 prompt + 256 canvas)",
         "stack30": "one denoising step: 30 stacked MoE layers (distinct weights, Zipf(1.1) "
                    "router bias, residual chained) over a T=256 canvas",
@@ -454,7 +458,7 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "fp16" if w.wdtype in (2, 3) else "bf16",
         "data": "synthetic",
         "config": {
             "workload": f"{w.name}: {desc}, d={w.d}, E={w.E}, top-{w.k}, f={w.f}, "

@@ -25,6 +25,7 @@ MOE_ERR_DEVICE_CHECK = 6
 MOE_W_BF16 = 0
 MOE_W_INT4_G128 = 1
 MOE_W_FP8_E4M3 = 2
+MOE_W_FP4_E2M1 = 3
 
 MOE_OPT_EPS = 0
 MOE_OPT_TIMEOUT_MS = 1

@@ -12,6 +12,14 @@
 #include "common.cuh"
 #include "moe.h"
 
+// fp4 expert kernel (expert_w4f.cu): the fp8 launcher's arguments plus the
+// block-scale tensor maps of both weights.
+cudaError_t moe_launch_expert_w4f(const moe::ExpertArgs& a, const CUtensorMap& tm_cgu,
+                                  const CUtensorMap& tm_cd, const CUtensorMap& tm_xp,
+                                  const CUtensorMap& tm_h, const CUtensorMap& tm_bgu,
+                                  const CUtensorMap& tm_bd, int num_sms, cudaStream_t s,
+                                  bool pdl);
+
 namespace {
 
 using moe::Ctl;
@@ -160,6 +168,25 @@ bool make_map_fp8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
   return r == CUDA_SUCCESS;
 }
 
+// 3-D byte tensor map over the E4M3 block scales of fp4 scale records: the
+// records are {fp32 s[R]; uint8 block[NB][R]} back to back, so the block
+// scales form an [E][NB][R] array with row stride R and expert stride equal to
+// the record size.  Box = box_rows x 8 blocks (one 128-wide K stage).
+bool make_map_blk(CUtensorMap* m, const void* records, uint64_t E, uint64_t R, uint64_t NB,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {R, NB, E};
+  cuuint64_t strides[2] = {R, R * (4 + NB)};
+  cuuint32_t box[3] = {box_rows, 8, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  void* base = const_cast<uint8_t*>(static_cast<const uint8_t*>(records) + 4 * R);
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 moe_status_t check_device(moe_plan_t p) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -266,7 +293,7 @@ moe_status_t validate_route(moe_plan_t p, int T, const void* x, const float* rw,
 uint64_t prefetch_bytes(moe_plan_t p) {
   const uint64_t n = (uint64_t)p->E * 2 * p->f * p->d;  // weights of the fused gate_up
   const uint64_t all =
-      p->wdtype == MOE_W_BF16 ? 2 * n : (p->wdtype == MOE_W_FP8_E4M3 ? n : n / 2);
+      p->wdtype == MOE_W_BF16 ? 2 * n : (p->wdtype == MOE_W_FP8_E4M3 ? n : n / 2);  // int4, fp4: n/2
   const uint64_t want = (uint64_t)p->prefetch_mb << 20;
   return want < all ? want : all;
 }
@@ -328,7 +355,8 @@ moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, mo
   if (E < 1 || E > moe::kMaxE || k < 1 || k > E || k > moe::kMaxK) return MOE_ERR_UNSUPPORTED;
   if (d < 128 || d > 4096 || d % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (f < 64 || f > 4096 || f % 64 != 0) return MOE_ERR_UNSUPPORTED;
-  if (wdtype != MOE_W_BF16 && wdtype != MOE_W_INT4_G128 && wdtype != MOE_W_FP8_E4M3)
+  if (wdtype != MOE_W_BF16 && wdtype != MOE_W_INT4_G128 && wdtype != MOE_W_FP8_E4M3 &&
+      wdtype != MOE_W_FP4_E2M1)
     return MOE_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -441,9 +469,15 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   const int A = T * p->k;
   const bool w4 = p->wdtype == MOE_W_INT4_G128;
   const bool w8 = p->wdtype == MOE_W_FP8_E4M3;
-  CUtensorMap tm_wgu, tm_wd, tm_x, tm_h;
+  const bool w4f = p->wdtype == MOE_W_FP4_E2M1;
+  CUtensorMap tm_wgu, tm_wd, tm_x, tm_h, tm_bgu, tm_bd;
   bool maps_ok;
-  if (w4)
+  if (w4f)
+    maps_ok = make_map_codes(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d / 2, moe::kGuHalf) &&
+              make_map_codes(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f / 2, moe::kBM) &&
+              make_map_blk(&tm_bgu, scales_gate_up, p->E, 2 * p->f, p->d / 16, moe::kGuHalf) &&
+              make_map_blk(&tm_bd, scales_down, p->E, p->d, p->f / 16, moe::kBM);
+  else if (w4)
     maps_ok = make_map_codes(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d / 2, moe::kGuHalf) &&
               make_map_codes(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f / 2, moe::kBM);
   else if (w8)
@@ -452,7 +486,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   else
     maps_ok = make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) &&
               make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM);
-  // x_perm and h (bf16, or fp16 on the fp8 path: 2-byte elements either way)
+  // x_perm and h (bf16, or fp16 on the fp8 and fp4 paths: 2-byte elements either way)
   maps_ok = maps_ok && make_map_bf16(&tm_x, p->x_perm, (uint64_t)A, p->d, moe::kBRows) &&
             make_map_bf16(&tm_h, p->h, (uint64_t)A, p->f, moe::kBRows);
   if (!maps_ok) return MOE_ERR_CUDA;
@@ -484,7 +518,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ga.perm = p->perm;
   ga.x = static_cast<const __nv_bfloat16*>(x);
   ga.x_perm = p->x_perm;
-  ga.xf16 = w8 ? 1 : 0;
+  ga.xf16 = (w8 || w4f) ? 1 : 0;
   {
     ProfScope ps(p, MOE_K_PLAN, s);
     if (moe_launch_plan_gather(pa, ga, p->num_sms, s, p->pdl != 0) != cudaSuccess)
@@ -509,13 +543,16 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ea.test_stall = p->test_stall;
   ea.scales_gu = w4 ? static_cast<const __half*>(scales_gate_up) : nullptr;
   ea.scales_d = w4 ? static_cast<const __half*>(scales_down) : nullptr;
-  ea.rows_gu = w8 ? static_cast<const float*>(scales_gate_up) : nullptr;
-  ea.rows_d = w8 ? static_cast<const float*>(scales_down) : nullptr;
+  // fp8: the fp32 row scales; fp4: the scale records, which open with them
+  ea.rows_gu = (w8 || w4f) ? static_cast<const float*>(scales_gate_up) : nullptr;
+  ea.rows_d = (w8 || w4f) ? static_cast<const float*>(scales_down) : nullptr;
   {
     ProfScope ps(p, MOE_K_EXPERT, s);
     const cudaError_t le =
         w4 ? moe_launch_expert_w4(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0)
         : w8 ? moe_launch_expert_w8(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0)
+        : w4f ? moe_launch_expert_w4f(ea, tm_wgu, tm_wd, tm_x, tm_h, tm_bgu, tm_bd, p->num_sms, s,
+                                      p->pdl != 0)
              : moe_launch_expert(ea, tm_wgu, tm_wd, tm_x, tm_h, p->num_sms, s, p->pdl != 0);
     if (le != cudaSuccess) return MOE_ERR_CUDA;
   }

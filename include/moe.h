@@ -13,7 +13,9 @@
  *     symmetric int4 weights in groups of 128 (auto-round pull request "Add
  *     quantization support for DiffusionGemma", transformers backend test
  *     log), or 8-bit floating-point weights (the ROCmFP4-GGUF card's FP8
- *     builds; E4M3 with one fp32 scale per weight row here);
+ *     builds; E4M3 with one fp32 scale per weight row here), or 4-bit
+ *     floating-point weights (the card's FP4 builds; MX E2M1 with an E4M3
+ *     scale per 16 weights and an fp32 scale per row here);
  *   - the canvas of 256 tokens is denoised in parallel, so each step is a set
  *     of large batched expert matmuls (the ROCmFP4-GGUF card, section "The
  *     4-bit is NOT the fastest here").
@@ -67,7 +69,7 @@ typedef enum {
   MOE_W_INT4_G128 = 1, /* w_gate_up u8 [E,2f,d/2]; w_down u8 [E,d,f/2]; element i
                           of a row in byte i/2, low nibble for even i, 4-bit two's
                           complement; value = code * scale[row][i/128] (fp16)  */
-  MOE_W_FP8_E4M3 = 2   /* w_gate_up u8 [E,2f,d]; w_down u8 [E,d,f]; element i of a
+  MOE_W_FP8_E4M3 = 2,  /* w_gate_up u8 [E,2f,d]; w_down u8 [E,d,f]; element i of a
                           row is byte i, an OFP8 E4M3 value (OCP 8-bit Floating
                           Point Specification; the NaN codes 0x7F / 0xFF must not
                           occur); value = e4m3 * scale[row] with one fp32 scale
@@ -77,6 +79,16 @@ typedef enum {
                           Activations (the experts' input rows and h) are carried
                           as fp16 on this path: |x| (after the optional expert
                           norm) and |h| must stay below 65504.                 */
+  MOE_W_FP4_E2M1 = 3   /* w_gate_up u8 [E,2f,d/2]; w_down u8 [E,d,f/2]; element i
+                          of a row in byte i/2, low nibble for even i, an MX E2M1
+                          value (OCP Microscaling Formats specification: 0, 0.5,
+                          1, 1.5, 2, 3, 4, 6 and their negatives); value =
+                          e2m1 * block[i/16][row] * s[row].  The scales of each
+                          expert form one record {fp32 s[R]; u8 block[R*C/16]},
+                          R the tensor's rows, C its columns, block[j][r] the
+                          OFP8 E4M3 scale (no NaN) of elements 16j..16j+15 of
+                          row r; records back to back, R*(4 + C/16) bytes each.
+                          Activations are fp16 as for MOE_W_FP8_E4M3.          */
 } moe_wdtype_t;
 
 /* Options for moe_plan_set_option. */
@@ -142,6 +154,8 @@ moe_status_t moe_plan_reserve(moe_plan_t plan, int max_T);
  *   w_down         see moe_wdtype_t
  *   scales_gate_up int4: fp16 [E,2f,ceil(d/128)]; fp8: fp32 [E,2f]; NULL for bf16
  *   scales_down    int4: fp16 [E,d,ceil(f/128)];  fp8: fp32 [E,d];  NULL for bf16
+ *                  fp4: E scale records each (see MOE_W_FP4_E2M1), R = 2f, C = d for
+ *                  gate_up and R = d, C = f for down
  *   residual       bf16 [T,d] or NULL; may alias `out`
  *   out            bf16 [T,d]; must not overlap x
  * Asynchronous on `stream`; the plan's workspace holds the routing tables

@@ -22,6 +22,7 @@ GAP_FLAG = 1e-5
 TOL_BF16 = 5e-3
 TOL_INT4 = 1e-2
 TOL_FP8 = TOL_BF16
+TOL_FP4 = TOL_BF16  # exact block-scaled decode; fp16 activations as on the fp8 path
 
 
 def rel_l2(a, b) -> float:

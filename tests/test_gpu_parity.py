@@ -7,7 +7,7 @@ import torch
 import oracle
 from block_diffusion_moe_router_b200 import inputs
 import block_diffusion_moe_router_b200 as moe
-from parity_util import (TOL_BF16, TOL_FP8, TOL_INT4, check_routing, oracle_rows_for_sets,
+from parity_util import (TOL_BF16, TOL_FP4, TOL_FP8, TOL_INT4, check_routing, oracle_rows_for_sets,
                          rel_l2, stable_tables)
 
 pytestmark = pytest.mark.gpu
@@ -42,10 +42,12 @@ def full_check(lay_cpu, lay_gpu, E, k, d, f, rows=None, residual=None, tol=TOL_B
     T = lay_gpu["x"].shape[0]
     coded = lay_gpu["w_gate_up"].dtype == torch.uint8
     fp8 = coded and lay_gpu["scales_gate_up"].dtype == torch.float32
-    int4 = coded and not fp8
+    fp4 = coded and lay_gpu["scales_gate_up"].dtype == torch.uint8  # scale records
+    int4 = coded and not fp8 and not fp4
     if int4 and tol == TOL_BF16:
         tol = TOL_INT4
-    wdt = moe.MOE_W_FP8_E4M3 if fp8 else (moe.MOE_W_INT4_G128 if int4 else moe.MOE_W_BF16)
+    wdt = (moe.MOE_W_FP8_E4M3 if fp8 else moe.MOE_W_FP4_E2M1 if fp4
+           else moe.MOE_W_INT4_G128 if int4 else moe.MOE_W_BF16)
     layer = moe.MoeLayer(E, k, d, f, wdt)
     try:
         for key, val in (options or {}).items():
@@ -126,7 +128,8 @@ def test_canvas_y_fp32(canvas):
     print("canvas y-fp32 rel-L2", err)
 
 
-@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4, inputs.WDTYPE_FP8])
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4, inputs.WDTYPE_FP8,
+                                inputs.WDTYPE_FP4])
 @pytest.mark.parametrize("ybf16", [0, 1])
 def test_y_dtype_ragged_residual(wd, ybf16):
     """Both y precisions with a residual, ragged T and both weight formats."""
@@ -188,9 +191,9 @@ def test_encode_sampled_rows():
     print("encode sampled rel-L2", err)
 
 
-@pytest.mark.parametrize("wd", [inputs.WDTYPE_INT4, inputs.WDTYPE_FP8])
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_INT4, inputs.WDTYPE_FP8, inputs.WDTYPE_FP4])
 def test_encode_shape_coded_weights_sampled_rows(wd):
-    """T=2048 with int4 or fp8 expert weights: ~128 tokens per expert, so the
+    """T=2048 with int4, fp8 or fp4 expert weights: ~128 tokens per expert, so the
     coded kernels run their largest chunks (and the fp8 kernel its shallowest
     code ring); the oracle checks 48 sampled rows including both ends."""
     T, d, E, k, f = 2048, 2816, 128, 8, 704
@@ -201,7 +204,8 @@ def test_encode_shape_coded_weights_sampled_rows(wd):
                                      g.choice(T, 32, replace=False)]))
     err, _ = full_check(lay_cpu, lay, E, k, d, f, rows=rows,
                         tol=TOL_INT4 if wd == inputs.WDTYPE_INT4 else TOL_FP8)
-    print("encode-shape", "int4" if wd == inputs.WDTYPE_INT4 else "fp8", "sampled rel-L2", err)
+    print("encode-shape", {inputs.WDTYPE_INT4: "int4", inputs.WDTYPE_FP8: "fp8"}.get(wd, "fp4"),
+          "sampled rel-L2", err)
 
 
 def test_stack30_layer_zipf_bias_and_residual():
@@ -317,6 +321,65 @@ def test_fp8_code_ranges(kind):
     print("fp8", kind, "rel-L2", err)
 
 
+def test_canvas4f_fp4_full_layer():
+    """T=256 canvas with E2M1 expert weights, E4M3 scales per 16 weights and
+    fp32 row scales: every token against the oracle's exact decode."""
+    w = inputs.WORKLOADS["canvas4f"]
+    lay_gpu = inputs.make_layer(w, device="cuda")
+    lay_cpu = _cpu(lay_gpu)
+    err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f, tol=TOL_FP4)
+    print("canvas4f fp4 rel-L2", err)
+
+
+@pytest.mark.parametrize("T,E,k,d,f,bias", [
+    (17, 16, 2, 256, 64, True),      # f=64: down's only K stage is half out of bounds (codes and blocks)
+    (300, 33, 3, 384, 192, False),   # f=192: last stage of 64; E not a multiple of 32
+    (1, 4, 1, 128, 128, False),      # one token, one 128-wide stage each way
+])
+def test_fp4_edge_shapes(T, E, k, d, f, bias):
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=T + E + 3, bias=bias,
+                            wdtype=inputs.WDTYPE_FP4)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f, tol=TOL_FP4)
+    print("fp4", (T, E, k, d, f), "rel-L2", err)
+
+
+def test_fp4_hot_expert_chunks():
+    """fp4 units hold 128 tokens: one expert with 600 tokens spans 5 chunks."""
+    T, E, k, d, f = 600, 16, 2, 256, 128
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=83, bias=True,
+                            wdtype=inputs.WDTYPE_FP4)
+    lay["router_bias"] = torch.zeros(E)
+    lay["router_bias"][3] = 50.0
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f, tol=TOL_FP4)
+    print("fp4 hot expert rel-L2", err)
+
+
+@pytest.mark.parametrize("kind", ["subnormal", "extreme"])
+def test_fp4_block_scale_ranges(kind):
+    """Every E4M3 block scale subnormal (2^-9 .. 7 * 2^-9), or every one at
+    the format's largest magnitudes (256 .. 448), over all 16 E2M1 codes: the
+    scaled decode must stay exact at both ends (a flushed subnormal scale or an
+    fp16 product out of range would show)."""
+    T, E, k, d, f = 33, 8, 2, 256, 128
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=85, wdtype=inputs.WDTYPE_FP4)
+    g = torch.Generator().manual_seed(6)
+    for key, (R, C) in (("scales_gate_up", (2 * f, d)), ("scales_down", (d, f))):
+        rec = lay[key].clone()
+        nb = C // inputs.FP4_BLOCK
+        if kind == "subnormal":   # exponent 0, mantissa 1..7
+            blk = torch.randint(1, 8, (E, nb * R), generator=g, dtype=torch.int32)
+            srow = 2.0 ** 9 / 4 * 0.01
+        else:                     # exponent 15, mantissa 0..6 (256 .. 448)
+            blk = (15 << 3) | torch.randint(0, 7, (E, nb * R), generator=g, dtype=torch.int32)
+            srow = 0.01 / 350
+        rec[:, 4 * R:] = blk.to(torch.uint8)
+        rows = torch.full((E, R), srow, dtype=torch.float32)
+        rec[:, :4 * R] = rows.view(torch.uint8).reshape(E, 4 * R)
+        lay[key] = rec
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f, tol=TOL_FP4)
+    print("fp4", kind, "rel-L2", err)
+
+
 # ------------------------------------------------------------------ edge cases
 
 
@@ -336,7 +399,8 @@ def test_edge_shapes(T, E, k, d, f, bias):
     print((T, E, k, d, f), "rel-L2", err)
 
 
-@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4, inputs.WDTYPE_FP8])
+@pytest.mark.parametrize("wd", [inputs.WDTYPE_BF16, inputs.WDTYPE_INT4, inputs.WDTYPE_FP8,
+                                inputs.WDTYPE_FP4])
 def test_expert_side_norm(wd):
     """Experts read the (1+gamma2) RMSNorm of x (applied while gathering the
     rows); router and residual see the raw x."""
