@@ -41,6 +41,7 @@ PROFILES = {
     "canvas": ("expert_kernel_canvas.txt", "expert.cu"),
     "canvas4": ("expert_w4_kernel_canvas4.txt", "expert_w4.cu"),
     "canvas8": ("expert_w8_kernel_canvas8.txt", "expert_w8.cu"),
+    "canvas4f": ("expert_w4f_kernel_canvas4f.txt", "expert_w4f.cu"),
 }
 
 
