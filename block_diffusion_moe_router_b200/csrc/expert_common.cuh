@@ -99,6 +99,15 @@ __device__ __forceinline__ __half to_h<__half>(float v) {
   return __float2half_rn(v);
 }
 
+// v += the fp32 accumulator columns at taddr (a second split-K partial).
+__device__ __forceinline__ void add_partial(uint32_t taddr, uint32_t (&v)[32]) {
+  uint32_t w[32];
+  tmem_ld32(taddr, w);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
+}
+
 // Epilogue role (warps 2..5, 128 threads): for each unit, read the fp32
 // accumulator from TMEM (lane = weight row, column = token), 32 tokens at a
 // time, and write
@@ -119,7 +128,8 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
                                               volatile int* s_abort, volatile int* s_bcast,
                                               uint32_t tmem_base, int acc_cols, int warp,
                                               int lane, uint64_t* sfull = nullptr,
-                                              const float* rscale = nullptr) {
+                                              const float* rscale = nullptr,
+                                              int split_kpair = 0) {
   Ctl* ctl = a.ctl;
   __nv_bfloat16* tile =
       reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(xchg) + kXchgBytes);
@@ -153,11 +163,19 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
     const float rs = kRowScale ? rscale[ur * kBM + row] : 1.f;
     const uint32_t tbase = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * acc_cols);
     const int nch = (ui.n + 31) / 32;
+    // Split K (kernels with two UMMA issuers, split_kpair = the K width of a
+    // stage pair): a unit of at most acc_cols / 2 tokens spanning two or more
+    // pairs is accumulated in two partials, acc_cols / 2 columns apart, which
+    // are summed here.
+    const int Ck = ui.type == kUnitGateUp ? a.d : a.f;
+    const bool split = split_kpair > 0 && ui.n <= acc_cols / 2 && Ck > split_kpair;
+    const uint32_t poff = (uint32_t)(acc_cols / 2);
     if (ui.type == kUnitGateUp) {
       for (int cc = 0; cc < nch; ++cc) {
         uint32_t v[32];
         tmem_ld32(tbase + cc * 32, v);
         tmem_wait_ld();
+        if (split) add_partial(tbase + poff + cc * 32, v);
         if (row >= kGuHalf) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -193,6 +211,7 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
         uint32_t v[32];
         tmem_ld32(tbase + cc * 32, v);
         tmem_wait_ld();
+        if (split) add_partial(tbase + poff + cc * 32, v);
         const int cmax = min(32, ui.n - cc * 32);
         if (a.y_bf16) {
 #pragma unroll

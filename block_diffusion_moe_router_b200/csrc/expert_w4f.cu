@@ -30,12 +30,14 @@ namespace moe {
 
 namespace {
 
-// warps: 0 code producer, 1 UMMA, 2-5 epilogue, 6-13 dequant, 14 B producer
-constexpr int kThreads = 480;
+// warps: 0 code producer, 1 UMMA (partial 0), 2-5 epilogue, 6-13 dequant,
+// 14 B producer, 15 UMMA (partial 1)
+constexpr int kThreads = 512;
 constexpr int kDqWarp0 = 6;
 constexpr int kDqGroups = 2;              // dequant groups, each owning every other stage pair
 constexpr int kDqWarps = 4 * kDqGroups;   // a group is one warp per TMEM lane quarter
 constexpr int kBWarp = kDqWarp0 + kDqWarps;
+constexpr int kMmaWarp2 = kBWarp + 1;
 constexpr int kChunkN = 128;                 // tokens per unit
 constexpr int kBK8 = 128;                    // K per stage
 constexpr int kCodeBytes = kBM * kBK8 / 2;   // 8 KB of packed codes per stage
@@ -57,7 +59,7 @@ constexpr int kRingBytes = 192 * 1024;       // code ring + B ring
 // (gate rows then up rows for gate_up, as the TMEM lanes hold them).
 constexpr int kScaleSlot = kBM * 4;
 constexpr int kScaleBytes = kUnitRing * kScaleSlot;
-constexpr int kBarBytes = 8 * (2 * kMaxCS + 2 * kMaxBS + 2 * kASlots + 4 + 3 * kUnitRing + 1);
+constexpr int kBarBytes = 8 * (2 * kMaxCS + 2 * kMaxBS + 2 * kASlots + 4 + 3 * kUnitRing + 3);
 constexpr int kSmemBytes =
     1024 + kRingBytes + kScaleBytes + kEpiBytes + kBarBytes + 256;
 static_assert(kAColBase + kASlots * kASlotCols <= kTmemCols, "TMEM budget");
@@ -200,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* uempty = ufull + kUnitRing;
   uint64_t* sfull = uempty + kUnitRing;  // the unit's row scales have landed
   uint64_t* drain = sfull + kUnitRing;
-  UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 1);
+  uint64_t* uend = drain + 2;  // both UMMA warps are done with a unit's A slots
+  UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 3);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(units + kUnitRing);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* s_bcast = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -222,20 +225,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bempty[i], 1);  // UMMA commit
     }
     for (int i = 0; i < kASlots; ++i) {
-      mbar_init(&afull[i], 4);
+      mbar_init(&afull[i], 8);  // both dequant groups' warps (one stage each)
       mbar_init(&aempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&tfull[i], 1);
+      mbar_init(&tfull[i], 2);  // one commit from each UMMA warp
       mbar_init(&tempty[i], 4);
     }
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(&ufull[i], 1);
-      // UMMA issuer, epilogue leader, B producer and every dequant warp
-      mbar_init(&uempty[i], 3 + kDqWarps);
+      // both UMMA warps, epilogue leader, B producer and every dequant warp
+      mbar_init(&uempty[i], 4 + kDqWarps);
       mbar_init(&sfull[i], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
+    mbar_init(uend, 2);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -459,10 +464,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((issued >> s2) & 1u)
           mbar_wait_drain(&bfull[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
-    // The whole warp runs the loop (warp-uniform descriptors); the elected
-    // lane issues the tcgen05 instructions.
+  } else if (warp == 1 || warp == kMmaWarp2) {
+    // ------------------------------------------------------------ UMMA issuers
+    // Each warp runs the loop whole (warp-uniform descriptors); the elected
+    // lane issues the tcgen05 instructions.  An UMMA costs its issuing warp
+    // ~70-110 cycles whatever N is (small N here), and issuers in different
+    // warps overlap, so two warps split K: for a unit of at most 64 tokens
+    // with two or more stage pairs, warp 1 takes the even pairs into columns
+    // [0, 64) of the accumulator and warp 15 the odd ones into [64, 128); the
+    // epilogue adds the two partials.  Larger units stay with warp 1.
+    // A slot s serves the pairs of global index = s (mod 2) and its full
+    // barrier is waited for by parity, so a warp that takes a slot over from
+    // the other must not run two phases ahead of it: at the end of every
+    // unit both warps meet on `uend` (a bounded wait), after the old owner has
+    // passed its last wait on each slot.
+    const int mw = warp == 1 ? 0 : 1;
+    uint32_t eph = 0;
     int bst = 0;
     uint32_t bph = 0;
     int asl = 0;
@@ -482,12 +499,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_warp(&tempty[acc], aphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereTmemEmpty))
         break;
       tc_fence_after();
-      const uint32_t dt = tmem_base + (uint32_t)(acc * kChunkN);
+      const bool split = ui.n <= kChunkN / 2 && nkb > 2;
+      const uint32_t dt = tmem_base + (uint32_t)(acc * kChunkN) + (split && mw ? kChunkN / 2 : 0);
       bool ok = true;
+      uint32_t first = 1;  // the next UMMA of this warp is its first of the unit
       // one hand-over per K-stage pair: its A slot (dequant warps, which
       // also waited for the pair's B stage) and its B stage
       for (int kb0 = 0; kb0 < nkb; kb0 += 2) {
         const int nst = min(2, nkb - kb0);
+        const bool mine = split ? ((kb0 >> 1) & 1) == mw : mw == 0;
+        if (!mine) {  // the other warp's pair: keep the ring positions in step
+          if (++bst == BS) {
+            bst = 0;
+            bph ^= 1;
+          }
+          if (++asl == kASlots) {
+            asl = 0;
+            aph ^= 1;
+          }
+          continue;
+        }
         if (!mbar_wait_warp(&afull[asl], aph, s_abort, ctl, a.timeout_ns, kWhereAFull)) {
           ok = false;
           break;
@@ -501,9 +532,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t b = sb + (2 * t + (kk >> 2)) * NB * kBK * 2 + (kk & 3) * kUmmaK * 2;
             if (elect_one())
               umma_f16_ts(dt, ta + t * kACols + kk * (kUmmaK / 2), sdesc_k_sw128(b), idesc,
-                          (kb0 | t | kk) ? 1u : 0u);
+                          (first && t == 0 && kk == 0) ? 0u : 1u);
           }
         }
+        first = 0;
         umma_commit_elect(&bempty[bst]);
         umma_commit_elect(&aempty[asl]);
         if (++bst == BS) {
@@ -516,6 +548,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) break;
+      if (lane == 0) mbar_arrive(uend);
+      if (!mbar_wait_warp(uend, eph, s_abort, ctl, a.timeout_ns, kWhereAFull)) break;
+      eph ^= 1;
       umma_commit_elect(&tfull[acc]);
       if (lane == 0) mbar_arrive(&uempty[ur]);
       if (++ur == kUnitRing) {
@@ -525,12 +560,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc ^= 1;
       if (acc == 0) aphase ^= 1;
     }
-    umma_commit_elect(drain);
-    if (lane == 0) mbar_wait_drain(drain, 0, ctl, a.timeout_ns);
+    umma_commit_elect(&drain[mw]);
+    if (lane == 0) mbar_wait_drain(&drain[mw], 0, ctl, a.timeout_ns);
     __syncwarp();
   } else if (warp < kDqWarp0) {
     epilogue_role<true, __half>(a, units, ufull, uempty, tfull, tempty, xchg, s_abort, s_bcast,
-                                tmem_base, kChunkN, warp, lane, sfull, rsc);
+                                tmem_base, kChunkN, warp, lane, sfull, rsc, 2 * kBK8);
   } else {
     // ------------------------------------------------------------ dequant warps
     // Group g (one warp per TMEM lane quarter) takes the stage pairs
@@ -566,9 +601,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool sok = true;
       for (int kb = 0; kb < G; ++kb) {
         const bool pair_end = (kb & 1) || kb == G - 1;
-        if ((kb >> 1) % kDqGroups == grp && sok) {
-          if (!(kb & 1))
-            sok = mbar_wait(&aempty[asl], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty);
+        if ((kb & 1) != grp && sok && grp == 1 && kb == G - 1) {
+          // a last pair of one stage: group 1 has nothing to decode but its
+          // four arrivals still complete the pair's hand-over, in its phase
+          sok = mbar_wait(&aempty[asl], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty) &&
+                mbar_wait(&bfull[bst], bph, s_abort, ctl, a.timeout_ns, kWhereBFull);
+          __syncwarp();
+          if (lane == 0 && sok) mbar_arrive(&afull[asl]);
+        }
+        if ((kb & 1) == grp && sok) {
+          sok = mbar_wait(&aempty[asl], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty);
           sok = sok && mbar_wait(&cfull[stage], phase, s_abort, ctl, a.timeout_ns, kWhereDqFull);
           if (sok) {
             // codes tile: 64-byte rows written by TMA with 64-byte swizzling,
@@ -608,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               tmem_st32(ta + h * 32, v);
             }
-            if (pair_end) {  // the pair is handed to the UMMA once its stores land
+            {  // the pair is handed to the UMMA once both groups' stores land
               tmem_wait_st();
               tc_fence_before();
               __syncwarp();
