@@ -40,10 +40,14 @@ constexpr int kBWarp = kDqWarp0 + kDqWarps;
 constexpr int kMmaWarp2 = kBWarp + 1;
 constexpr int kChunkN = 128;                 // tokens per unit
 constexpr int kBK8 = 128;                    // K per stage
-constexpr int kCodeBytes = kBM * kBK8 / 2;   // 8 KB of packed codes per stage
+// The code ring holds stage PAIRS: 128 rows x 128 bytes of packed codes (two
+// 128-wide K stages; 128-byte rows halve the TMA row requests of 64-byte
+// ones) and the pair's 16 x 128 block scales.
+constexpr int kCodeBytes = kBM * kBK8;       // 16 KB of packed codes per pair
 constexpr int kBlk = 16;                     // weights per block scale
 constexpr int kBlkPerStage = kBK8 / kBlk;    // 8
-constexpr int kBlkBytes = kBlkPerStage * kBM;  // 1 KB of block scales per stage
+constexpr int kBlkPerPair = 2 * kBlkPerStage;
+constexpr int kBlkBytes = kBlkPerPair * kBM;   // 2 KB of block scales per pair
 constexpr int kStageBytes = kCodeBytes + kBlkBytes;
 // TMEM A: two slots, each holding a pair of consecutive 128-wide K stages
 // (2 x 64 columns of f16x2).  The UMMA issuer and the dequant warps hand A
@@ -52,7 +56,7 @@ constexpr int kASlots = 2;
 constexpr int kACols = kBK8 / 2;             // 64 columns of f16x2 per K stage
 constexpr int kASlotCols = 2 * kACols;
 constexpr int kAColBase = 2 * kChunkN;       // A slots after the accumulators
-constexpr int kMaxCS = 16;                   // code stages
+constexpr int kMaxCS = 8;                    // code ring entries (stage pairs)
 constexpr int kMaxBS = 6;                    // B stages
 constexpr int kRingBytes = 192 * 1024;       // code ring + B ring
 // One row-scale slot per unit-ring entry: the unit's 128 fp32 row scales
@@ -218,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMaxCS; ++i) {
       mbar_init(&cfull[i], 1);
-      mbar_init(&cempty[i], 4);  // the dequant group's four warps hold the codes
+      mbar_init(&cempty[i], 8);  // both dequant groups' warps hold their stage's codes
     }
     for (int i = 0; i < kMaxBS; ++i) {
       mbar_init(&bfull[i], 1);
@@ -367,21 +371,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const int C = (ui.type == kUnitGateUp) ? a.d : a.f;
         const int nkb = (C + kBK8 - 1) / kBK8;
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = 0; kb < nkb; kb += 2) {  // one ring entry per stage pair
           if (!mbar_wait(&cempty[stage], phase ^ 1, s_abort, ctl, a.timeout_ns,
                          kWhereStageEmpty)) {
             ok = 0;
             break;
           }
           uint8_t* sa = ring + stage * kStageBytes;
-          uint8_t* sbk = sa + kCodeBytes;  // [8 blocks][128 rows] of e4m3 scales
+          uint8_t* sbk = sa + kCodeBytes;  // [16 blocks][128 rows] of e4m3 scales
           mbar_arrive_expect_tx(&cfull[stage], kStageBytes);
-          const int cx = kb * (kBK8 / 2);  // byte column of the packed codes
+          const int cx = kb * (kBK8 / 2);  // byte column of the packed codes (a multiple of 128)
           if (ui.type == kUnitGateUp) {
             const int r0 = ui.e * 2 * a.f + ui.m * kGuHalf;
             tma_load_2d(sa, &tm_cgu, cx, r0, &cfull[stage], pol_w);
             tma_load_2d(sa + kCodeBytes / 2, &tm_cgu, cx, r0 + a.f, &cfull[stage], pol_w);
-            // block scales: gate rows into [8][64] at 0, up rows at 512
+            // block scales: gate rows into [16][64] at 0, up rows at 1024
             tma_load_3d(sbk, &tm_bgu, ui.m * kGuHalf, kb * kBlkPerStage, ui.e, &cfull[stage], pol_w);
             tma_load_3d(sbk + kBlkBytes / 2, &tm_bgu, a.f + ui.m * kGuHalf, kb * kBlkPerStage, ui.e,
                         &cfull[stage], pol_w);
@@ -577,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q4 * 32 + lane;        // A row == TMEM lane
     const int grp = dw >> 2;
     const int dt = threadIdx.x - kDqWarp0 * 32;
-    const int sw = (row >> 1) & 3;
+    const int sw = row & 7;
     int stage = 0;
     uint32_t phase = 0;
     int asl = 0;
@@ -603,8 +607,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool pair_end = (kb & 1) || kb == G - 1;
         if ((kb & 1) != grp && sok && grp == 1 && kb == G - 1) {
           // a last pair of one stage: group 1 has nothing to decode but its
-          // four arrivals still complete the pair's hand-over, in its phase
-          sok = mbar_wait(&aempty[asl], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty) &&
+          // four arrivals still complete the pair's ring entry and hand-over,
+          // each in its phase
+          sok = mbar_wait(&cfull[stage], phase, s_abort, ctl, a.timeout_ns, kWhereDqFull);
+          __syncwarp();
+          if (lane == 0 && sok) mbar_arrive(&cempty[stage]);
+          sok = sok && mbar_wait(&aempty[asl], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty) &&
                 mbar_wait(&bfull[bst], bph, s_abort, ctl, a.timeout_ns, kWhereBFull);
           __syncwarp();
           if (lane == 0 && sok) mbar_arrive(&afull[asl]);
@@ -613,20 +621,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           sok = mbar_wait(&aempty[asl], aph ^ 1, s_abort, ctl, a.timeout_ns, kWhereAEmpty);
           sok = sok && mbar_wait(&cfull[stage], phase, s_abort, ctl, a.timeout_ns, kWhereDqFull);
           if (sok) {
-            // codes tile: 64-byte rows written by TMA with 64-byte swizzling,
-            // i.e. 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3);
-            // block scales: [8][128] (down) or gate [8][64] + up [8][64]
+            // codes tile: 128-byte rows (the pair's two stages, 64 bytes
+            // each) written by TMA with 128-byte swizzling, i.e. 16-byte
+            // chunk c of row r sits at chunk c ^ (r & 7); this group's stage
+            // is chunks 4 (kb & 1) .. +3.  Block scales: [16][128] (down) or
+            // gate [16][64] + up [16][64]; this stage's are blocks 8 (kb & 1) ..
             const uint8_t* st_base = ring + stage * kStageBytes;
-            const uint8_t* crow = st_base + row * (kBK8 / 2);
+            const uint8_t* crow = st_base + row * kBK8;
+            const int c0 = (kb & 1) * 4;
             uint4 cw[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-              cw[c] = *reinterpret_cast<const uint4*>(crow + ((c ^ sw) << 4));
+              cw[c] = *reinterpret_cast<const uint4*>(crow + (((c0 + c) ^ sw) << 4));
             const uint8_t* bk = st_base + kCodeBytes;
-            const uint8_t* bkr = ui.type == kUnitGateUp
-                                     ? bk + (row < kGuHalf ? row : kBlkBytes / 2 + row - kGuHalf)
-                                     : bk + row;
             const int bstride = ui.type == kUnitGateUp ? kGuHalf : kBM;
+            const uint8_t* bkr = (ui.type == kUnitGateUp
+                                      ? bk + (row < kGuHalf ? row : kBlkBytes / 2 + row - kGuHalf)
+                                      : bk + row) +
+                                 (kb & 1) * kBlkPerStage * bstride;
             uint16_t sb[kBlkPerStage / 2];
 #pragma unroll
             for (int q = 0; q < kBlkPerStage / 2; ++q)
@@ -659,11 +671,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (++stage == CS) {
-          stage = 0;
-          phase ^= 1;
-        }
         if (pair_end) {
+          if (++stage == CS) {
+            stage = 0;
+            phase ^= 1;
+          }
           if (++asl == kASlots) {
             asl = 0;
             aph ^= 1;

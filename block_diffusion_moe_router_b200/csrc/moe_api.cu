@@ -168,17 +168,33 @@ bool make_map_fp8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols
   return r == CUDA_SUCCESS;
 }
 
+// 2-D byte tensor map over packed fp4 codes [rows, cols_bytes]: box =
+// box_rows x 128 bytes (two 128-wide K stages), 128-byte swizzle.
+bool make_map_codes_pair(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols_bytes,
+                         uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols_bytes, rows};
+  cuuint64_t strides[1] = {cols_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 3-D byte tensor map over the E4M3 block scales of fp4 scale records: the
 // records are {fp32 s[R]; uint8 block[NB][R]} back to back, so the block
 // scales form an [E][NB][R] array with row stride R and expert stride equal to
-// the record size.  Box = box_rows x 8 blocks (one 128-wide K stage).
+// the record size.  Box = box_rows x 16 blocks (a pair of 128-wide K stages).
 bool make_map_blk(CUtensorMap* m, const void* records, uint64_t E, uint64_t R, uint64_t NB,
                   uint32_t box_rows) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {R, NB, E};
   cuuint64_t strides[2] = {R, R * (4 + NB)};
-  cuuint32_t box[3] = {box_rows, 8, 1};
+  cuuint32_t box[3] = {box_rows, 16, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   void* base = const_cast<uint8_t*>(static_cast<const uint8_t*>(records) + 4 * R);
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, estr,
@@ -473,8 +489,9 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   CUtensorMap tm_wgu, tm_wd, tm_x, tm_h, tm_bgu, tm_bd;
   bool maps_ok;
   if (w4f)
-    maps_ok = make_map_codes(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d / 2, moe::kGuHalf) &&
-              make_map_codes(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f / 2, moe::kBM) &&
+    maps_ok = make_map_codes_pair(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d / 2,
+                                  moe::kGuHalf) &&
+              make_map_codes_pair(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f / 2, moe::kBM) &&
               make_map_blk(&tm_bgu, scales_gate_up, p->E, 2 * p->f, p->d / 16, moe::kGuHalf) &&
               make_map_blk(&tm_bd, scales_down, p->E, p->d, p->f / 16, moe::kBM);
   else if (w4)
