@@ -6,15 +6,15 @@
 // it finds the 8-bit build faster at a 256-token canvas).
 //
 // The fp8 kernel's pipeline (expert_w8.cu) with another decode:
-//   - the code producer brings each 128-wide K stage of packed codes (128
-//     rows x 64 bytes, 64-byte swizzled) and the stage's block scales (8
-//     blocks x 128 rows of E4M3 bytes, by a 3-D TMA over the scale records)
-//     into the code ring; a B producer brings the activation tiles of each
-//     pair of K stages into a second ring;
+//   - the code producer brings each pair of 128-wide K stages of packed
+//     codes (128 rows x 128 bytes, 128-byte swizzled) and the pair's block
+//     scales (16 blocks x 128 rows of E4M3 bytes, by a 3-D TMA over the
+//     scale records) into the code ring; a B producer brings the activation
+//     tiles of each pair of K stages into a second ring;
 //   - 8 dequant warps widen the codes with the hardware E2M1 -> f16x2
 //     conversion (exact), multiply each pair by its block's scale (E4M3 ->
-//     fp16, exact) and store the fp16 pairs straight into TMEM, two stages per
-//     hand-over.  The product is exact too: an E2M1 value has 2 significant
+//     fp16, exact) and store the fp16 pairs straight into TMEM, one stage
+//     per group, both stages of a pair per hand-over.  The product is exact too: an E2M1 value has 2 significant
 //     bits and an E4M3 scale 4, so it fits fp16's 11, and its smallest
 //     magnitude 2^-10 is above fp16's subnormal range;
 //   - the UMMA (kind::f16, A and B both fp16) reads A from TMEM and the fp16
@@ -34,7 +34,7 @@ namespace {
 // 14 B producer, 15 UMMA (partial 1)
 constexpr int kThreads = 512;
 constexpr int kDqWarp0 = 6;
-constexpr int kDqGroups = 2;              // dequant groups, each owning every other stage pair
+constexpr int kDqGroups = 2;              // dequant groups, each owning one stage of every pair
 constexpr int kDqWarps = 4 * kDqGroups;   // a group is one warp per TMEM lane quarter
 constexpr int kBWarp = kDqWarp0 + kDqWarps;
 constexpr int kMmaWarp2 = kBWarp + 1;
@@ -572,10 +572,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tmem_base, kChunkN, warp, lane, sfull, rsc, 2 * kBK8);
   } else {
     // ------------------------------------------------------------ dequant warps
-    // Group g (one warp per TMEM lane quarter) takes the stage pairs
-    // (kb / 2) % kDqGroups == g of each unit, a whole 128-code row per
-    // thread, so the groups work on different pairs at once; a pair is
-    // signalled full once the stores of its last stage have landed.
+    // Group g (one warp per TMEM lane quarter) takes the stages kb % 2 == g
+    // of each unit, a whole 128-code row per thread, so the two stages of a
+    // pair are widened at once; the pair's A slot is signalled full once both
+    // groups' stores have landed (eight arrivals; for a last pair of one
+    // stage group 1 arrives without data).
     const int dw = warp - kDqWarp0;        // 0..kDqWarps-1
     const int q4 = warp & 3;               // TMEM lane quarter
     const int row = q4 * 32 + lane;        // A row == TMEM lane

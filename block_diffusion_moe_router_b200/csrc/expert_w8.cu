@@ -16,7 +16,8 @@
 //     ~1,150 cycles per stage, latency-bound);
 //   - 8 dequant warps widen the codes with the hardware E4M3 -> f16x2
 //     conversion (exact: every E4M3 value is an fp16 value) and store the
-//     fp16 pairs straight into TMEM (tcgen05.st), two stages per hand-over;
+//     fp16 pairs straight into TMEM (tcgen05.st), one stage per group, both
+//     stages of a pair per hand-over;
 //   - the UMMA (kind::f16 with A and B both fp16) reads A from TMEM and the
 //     activations from shared memory: on this path x_perm and h are fp16;
 //   - the epilogue multiplies each accumulator row by its weight row's fp32
@@ -38,7 +39,7 @@ namespace {
 // 14 B producer, 15 UMMA (partial 1)
 constexpr int kThreads = 512;
 constexpr int kDqWarp0 = 6;
-constexpr int kDqGroups = 2;              // dequant groups, each owning every other stage pair
+constexpr int kDqGroups = 2;              // dequant groups, each owning one stage of every pair
 constexpr int kDqWarps = 4 * kDqGroups;   // a group is one warp per TMEM lane quarter
 constexpr int kBWarp = kDqWarp0 + kDqWarps;
 constexpr int kMmaWarp2 = kBWarp + 1;
@@ -525,10 +526,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tmem_base, kChunkN, warp, lane, sfull, rsc, 2 * kBK8);
   } else {
     // ------------------------------------------------------------ dequant warps
-    // Group g (one warp per TMEM lane quarter) takes the stage pairs
-    // (kb / 2) % kDqGroups == g of each unit, a whole 128-code row per
-    // thread, so the groups work on different pairs at once; a pair is
-    // signalled full once the stores of its last stage have landed.
+    // Group g (one warp per TMEM lane quarter) takes the stages kb % 2 == g
+    // of each unit, a whole 128-code row per thread, so the two stages of a
+    // pair are widened at once; the pair's A slot is signalled full once both
+    // groups' stores have landed (eight arrivals; for a last pair of one
+    // stage group 1 arrives without data).
     const int dw = warp - kDqWarp0;        // 0..kDqWarps-1
     const int q4 = warp & 3;               // TMEM lane quarter
     const int row = q4 * 32 + lane;        // A row == TMEM lane
