@@ -7,9 +7,13 @@ f=704, bf16 weights (synthetic, seeded; inputs resident in HBM).  The metric
 is canvas tokens/s per MoE layer; the JSON line also carries the expert
 kernel's HBM roofline fraction, an end-to-end figure through
 moe_forward_host (host buffers, copies inside the timed region) and the CPU
-oracle timed on a bounded sample.
+oracle timed on a bounded sample.  The same line also carries, under the keys
+"encode" and "stack30", the T=2048 prompt+canvas layer (graded on its
+tensor-core fraction) and the 30-layer denoising step, each measured in the
+same run with its own step time, per-kernel times and roofline fractions.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--extra encode,stack30 | --no-extra]
 
 N > 1 runs N independent replicas (one canvas per GPU, no collective on the
 data path), launched one process per GPU by torch.distributed.run.
@@ -65,6 +69,10 @@ def parse():
                    help="router path (auto: tensor cores when E <= 128)")
     p.add_argument("--prefetch-mb", type=int, default=None,
                    help="MiB of gate_up weights pulled into L2 during routing")
+    p.add_argument("--extra", default="encode,stack30",
+                   help="other workloads measured in the same run, reported under their "
+                        "own keys of the JSON line")
+    p.add_argument("--no-extra", action="store_true", help="measure the main workload only")
     return p.parse_args()
 
 
@@ -219,6 +227,17 @@ def oracle_sample_rate(lay_cpu, k, n_tokens, eps=1e-6):
     return n_tokens / (time.perf_counter() - t0)
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(lay_cpu, w, budget_s=12.0):
     import oracle
     cores = oracle.get_threads()
@@ -227,6 +246,7 @@ def cpu_baseline(lay_cpu, w, budget_s=12.0):
     n = int(max(probe, min(w.T, round(r * budget_s / cores) * cores)))
     r = oracle_sample_rate(lay_cpu, w.k, n)
     return {"value": r, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "omp_threads": cores, "host_cpus": os.cpu_count(),
             "sample": f"first {n} of the {w.T} canvas tokens, fp64 oracle, one layer"}
 
 
@@ -279,11 +299,198 @@ def run_reference(args):
         "config": {"workload": f"{w.name}: T={w.T} d={w.d} E={w.E} k={w.k} f={w.f} bf16 weights",
                    "sample_tokens_per_step": per},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "cpu_model": cpu_model(), "omp_threads": cores,
+                         "host_cpus": os.cpu_count(), "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+class LayerRun:
+    """One workload resident on this rank's GPU: its layers' weights, input
+    sets rotated so that every step's working set (with the weights) exceeds
+    L2, and a plan.  A step is one pass of the whole hot path: one moe_forward
+    per layer (router -> plan -> gather -> expert GEMMs -> combine), layers
+    chained through the residual."""
+
+    def __init__(self, w, args, rank):
+        import torch
+        import block_diffusion_moe_router_b200 as moe
+        from block_diffusion_moe_router_b200 import inputs
+        from block_diffusion_moe_router_b200 import replicas as rep
+        self.torch, self.moe, self.rep = torch, moe, rep
+        self.w = w
+        T, L = w.T, w.layers
+        self.T, self.L = T, L
+        self.lays = [inputs.make_layer(w, layer=l, device="cuda", with_x=False)
+                     for l in range(L)]
+        lay = self.lays[0]
+        self.small = T * w.d * 2 * 2 + (w.E * w.d * 4 + w.d * 4 if L == 1 else 0)
+        self.nsets = nsets = args.sets or max(2, math.ceil(1.1 * L2_BYTES / self.small))
+        self.xs = [inputs._randn((T, w.d), 1.0, rep.replica_seed(rank, i), "cuda",
+                                 torch.bfloat16) for i in range(nsets)]
+        if L == 1:
+            self.rws = [lay["router_w"]] + [
+                lay["router_w"][torch.randperm(w.E, device="cuda")].contiguous()
+                for _ in range(nsets - 1)]
+            self.gms = [lay["router_gamma"]] + [lay["router_gamma"].roll(i).contiguous()
+                                                for i in range(1, nsets)]
+        self.outs = [torch.empty((T, w.d), dtype=torch.bfloat16, device="cuda")
+                     for _ in range(nsets)]
+        self.bufs = [torch.empty((T, w.d), dtype=torch.bfloat16, device="cuda")
+                     for _ in range(2)]
+        self.plan = moe.moe_plan_create(w.E, w.k, w.d, w.f, w.wdtype)
+        moe.moe_plan_reserve(self.plan, T)
+        moe.moe_plan_set_option(self.plan, moe.MOE_OPT_PDL, 0 if args.no_pdl else 1)
+        moe.moe_plan_set_option(self.plan, moe.MOE_OPT_ROUTER,
+                                {"auto": 0, "ffma": 1, "tc": 2}[args.router])
+        if args.prefetch_mb is not None:
+            moe.moe_plan_set_option(self.plan, moe.MOE_OPT_L2_PREFETCH_MB, args.prefetch_mb)
+        moe.moe_plan_set_option(self.plan, moe.MOE_OPT_Y_BF16, 0 if args.y_fp32 else 1)
+        self.stream = torch.cuda.current_stream()
+        # experts that receive a token (their weights are the bytes the layer
+        # must stream), per layer, averaged over the input sets
+        self.touched = [0.0] * L
+        off = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+
+        def count(l):
+            moe.moe_plan_routing(self.plan, off, None, None, self.stream)
+            self.touched[l] += float(((off[1:] - off[:-1]) > 0).sum().item()) / nsets
+
+        for i in range(nsets):
+            self.step(i, count)
+        self.check()
+
+    def layer_call(self, l, x, out, residual, rw=None, gm=None):
+        ly = self.lays[l]
+        self.moe.moe_forward(self.plan, self.T, x, ly["router_w"] if rw is None else rw,
+                             ly["router_gamma"] if gm is None else gm, ly["router_bias"],
+                             ly["w_gate_up"], ly["w_down"], ly["scales_gate_up"],
+                             ly["scales_down"], residual, out, self.stream,
+                             expert_gamma=ly["expert_gamma"])
+
+    def step(self, i, per_layer=None):
+        j = i % self.nsets
+        if self.L == 1:
+            self.layer_call(0, self.xs[j], self.outs[j], None, self.rws[j], self.gms[j])
+            if per_layer is not None:
+                per_layer(0)
+            return self.outs[j]
+        cur = self.xs[j]
+        for l in range(self.L):  # x_{l+1} = x_l + MoE_l(x_l)
+            nxt = self.bufs[l % 2]
+            self.layer_call(l, cur, nxt, cur)
+            if per_layer is not None:
+                per_layer(l)
+            cur = nxt
+        return cur
+
+    def check(self):
+        st = self.moe.moe_plan_sync_status(self.plan, self.stream)
+        if st != self.moe.MOE_OK:
+            raise RuntimeError(self.moe.moe_status_str(st))
+
+    def timed(self, K, profile, per_step=False):
+        """Device time of K steps (CUDA events on the launching stream, barrier
+        and synchronize on both sides, max over ranks), or the per-step list."""
+        torch, moe, rep = self.torch, self.moe, self.rep
+        moe.moe_plan_set_option(self.plan, moe.MOE_OPT_PROFILE, 1 if profile else 0)
+        rep.barrier()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1 if per_step else 2)]
+        ev[0].record(self.stream)
+        for i in range(K):
+            self.step(i)
+            if per_step:
+                ev[i + 1].record(self.stream)
+        ev[-1].record(self.stream)
+        torch.cuda.synchronize()
+        rep.barrier()
+        moe.moe_plan_set_option(self.plan, moe.MOE_OPT_PROFILE, 0)
+        if per_step:
+            return [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+        return rep.max_over_ranks(ev[0].elapsed_time(ev[-1]), "cuda")
+
+    def warm(self, W):
+        for i in range(W):
+            self.step(i)
+        self.torch.cuda.synchronize()
+        for kk in range(len(self.moe.KERNEL_NAMES)):  # discard warm-up records
+            self.moe.moe_plan_profile(self.plan, kk)
+
+    def kernel_ms(self):
+        kern = {}
+        for kk, name in enumerate(self.moe.KERNEL_NAMES):
+            tot, n = self.moe.moe_plan_profile(self.plan, kk)
+            kern[name] = (tot / n) if n else None
+        return kern
+
+    def costs(self):
+        """Per step: algorithmic bytes of the expert kernels (per launch), of
+        the whole step, FLOPs, and the expert weight bytes per touched expert."""
+        expert_bytes, layer_bytes, flops = 0.0, 0.0, 0.0
+        for l in range(self.L):
+            eb, lb, fl, wbytes = layer_costs(self.w, self.touched[l], self.T)
+            expert_bytes += eb
+            layer_bytes += lb
+            flops += fl
+        return expert_bytes / self.L, layer_bytes, flops, wbytes
+
+    def close(self):
+        self.moe.moe_plan_destroy(self.plan)
+        self.lays = self.xs = self.outs = self.bufs = None
+        self.torch.cuda.empty_cache()
+
+
+def sub_record(name, args, rank, steps, warmup):
+    """A second workload measured in the same run, for the same JSON line:
+    its step time (events around the K steps), per-kernel times (a second run
+    with events between the launches) and its roofline fractions against the
+    measured HBM copy bandwidth and both measured bf16 GEMM peaks."""
+    import torch
+    from block_diffusion_moe_router_b200 import inputs
+    w = inputs.WORKLOADS[name]
+    run = LayerRun(w, args, rank)
+    run.warm(warmup)
+    _, local = rank, int(os.environ.get("LOCAL_RANK", "0"))
+    with ClockSampler(local) as clk:
+        ms = run.timed(steps, profile=False)
+        run.timed(steps, profile=True)
+    kern = run.kernel_ms()
+    per_step = sorted(run.timed(steps, profile=False, per_step=True))
+    run.check()
+    expert_bytes, step_bytes, flops, wbytes = run.costs()
+    hbm, bf16, bf16_sus, basis = peaks()
+    ms_step = ms / steps
+    t = ms_step * 1e-3
+    rec = {
+        "workload": f"{w.name}: T={w.T}, d={w.d}, E={w.E}, top-{w.k}, f={w.f}, "
+                    f"{WFMT[w.wdtype]} weights, {w.layers} layer(s) per step",
+        "steps": steps, "warmup": warmup,
+        "ms_per_step": ms_step,
+        "ms_per_layer": ms_step / w.layers,
+        "tokens_per_s_per_layer": w.T * w.layers / t,
+        "step_ms_p10_p50_p90": [per_step[int(q * (len(per_step) - 1))] for q in (0.1, 0.5, 0.9)],
+        "touched_experts_per_layer": sum(run.touched) / w.layers,
+        "alg_bytes_per_step": step_bytes,
+        "flops_per_step": flops,
+        "hbm_frac": step_bytes / t / (hbm * 1e9),
+        "tensor_frac_of_burst_peak": flops / t / (bf16 * 1e12),
+        "tensor_frac_of_sustained_peak": flops / t / (bf16_sus * 1e12),
+        "frac_of_roofline": max(step_bytes / (hbm * 1e9), flops / (bf16_sus * 1e12)) / t,
+        "peak_basis": f"{basis}: HBM {hbm} GB/s, bf16 {bf16} TFLOP/s burst, "
+                      f"{bf16_sus} TFLOP/s sustained",
+        "kernel_ms_per_layer": kern,
+        "expert_kernel_hbm_frac": (expert_bytes / (kern["expert"] * 1e-3) / 1e9 / hbm)
+        if kern.get("expert") else None,
+        "clocks": clk.summary(),
+        "gpu_launches": launches_per_layer(w, w.T, args.router) * w.layers * steps,
+    }
+    run.close()
+    del run
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_ours(args):
@@ -297,111 +504,24 @@ def run_ours(args):
     rep.init("nccl", torch.device("cuda", local), timeout_s=120)
     w = inputs.WORKLOADS[args.workload]
     T, L = w.T, w.layers
-    lays = [inputs.make_layer(w, layer=l, device="cuda", with_x=False) for l in range(L)]
-    lay = lays[0]
-    # rotate the small per-call inputs so that, with the weights, the working
-    # set exceeds L2 on every step
-    small = T * w.d * 2 * 2 + (w.E * w.d * 4 + w.d * 4 if L == 1 else 0)
-    nsets = args.sets or max(2, math.ceil(1.1 * L2_BYTES / small))
-    xs = [inputs._randn((T, w.d), 1.0, rep.replica_seed(rank, i), "cuda", torch.bfloat16)
-          for i in range(nsets)]
-    if L == 1:
-        rws = [lay["router_w"]] + [lay["router_w"][torch.randperm(w.E, device="cuda")]
-                                   .contiguous() for _ in range(nsets - 1)]
-        gms = [lay["router_gamma"]] + [lay["router_gamma"].roll(i).contiguous()
-                                       for i in range(1, nsets)]
-    outs = [torch.empty((T, w.d), dtype=torch.bfloat16, device="cuda") for _ in range(nsets)]
-    bufs = [torch.empty((T, w.d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    plan = moe.moe_plan_create(w.E, w.k, w.d, w.f, w.wdtype)
-    moe.moe_plan_reserve(plan, T)
-    moe.moe_plan_set_option(plan, moe.MOE_OPT_PDL, 0 if args.no_pdl else 1)
-    moe.moe_plan_set_option(plan, moe.MOE_OPT_ROUTER,
-                            {"auto": 0, "ffma": 1, "tc": 2}[args.router])
-    if args.prefetch_mb is not None:
-        moe.moe_plan_set_option(plan, moe.MOE_OPT_L2_PREFETCH_MB, args.prefetch_mb)
-    moe.moe_plan_set_option(plan, moe.MOE_OPT_Y_BF16, 0 if args.y_fp32 else 1)
-    stream = torch.cuda.current_stream()
-
-    def layer_call(l, x, out, residual, rw=None, gm=None):
-        ly = lays[l]
-        moe.moe_forward(plan, T, x, ly["router_w"] if rw is None else rw,
-                        ly["router_gamma"] if gm is None else gm, ly["router_bias"],
-                        ly["w_gate_up"], ly["w_down"], ly["scales_gate_up"], ly["scales_down"],
-                        residual, out, stream, expert_gamma=ly["expert_gamma"])
-
-    def step(i, per_layer=None):
-        j = i % nsets
-        if L == 1:
-            layer_call(0, xs[j], outs[j], None, rws[j], gms[j])
-            if per_layer is not None:
-                per_layer(0)
-            return outs[j]
-        cur = xs[j]
-        for l in range(L):  # x_{l+1} = x_l + MoE_l(x_l)
-            nxt = bufs[l % 2]
-            layer_call(l, cur, nxt, cur)
-            if per_layer is not None:
-                per_layer(l)
-            cur = nxt
-        return cur
-
-    # experts that receive a token (their weights are the bytes the layer
-    # must stream), per layer, averaged over the input sets
-    touched = [0.0] * L
-    off = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
-
-    def count(l):
-        moe.moe_plan_routing(plan, off, None, None, stream)
-        touched[l] += float(((off[1:] - off[:-1]) > 0).sum().item()) / nsets
-
-    for i in range(nsets):
-        step(i, count)
-    st = moe.moe_plan_sync_status(plan, stream)
-    if st != moe.MOE_OK:
-        raise RuntimeError(moe.moe_status_str(st))
-
-    def timed(K, profile, per_step=False):
-        moe.moe_plan_set_option(plan, moe.MOE_OPT_PROFILE, 1 if profile else 0)
-        rep.barrier()
-        torch.cuda.synchronize()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1 if per_step else 2)]
-        ev[0].record(stream)
-        for i in range(K):
-            step(i)
-            if per_step:
-                ev[i + 1].record(stream)
-        ev[-1].record(stream)
-        torch.cuda.synchronize()
-        rep.barrier()
-        moe.moe_plan_set_option(plan, moe.MOE_OPT_PROFILE, 0)
-        if per_step:
-            return [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
-        return rep.max_over_ranks(ev[0].elapsed_time(ev[-1]), "cuda")
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    for kk in range(len(moe.KERNEL_NAMES)):  # discard warm-up records
-        moe.moe_plan_profile(plan, kk)
+    run = LayerRun(w, args, rank)
+    lay, plan, stream = run.lays[0], run.plan, run.stream
+    nsets = run.nsets
+    run.warm(args.warmup)
     with ClockSampler(local) as clk:
         # the reported time: K steps, CUDA events around the region only
-        ms = timed(args.steps, profile=False)
+        ms = run.timed(args.steps, profile=False)
         # diagnostics: the same K steps with per-kernel events between the
         # launches (they break the launch overlap, so this run is slower)
-        ms_prof = timed(args.steps, profile=True)
-    kern = {}
-    for kk, name in enumerate(moe.KERNEL_NAMES):
-        tot, n = moe.moe_plan_profile(plan, kk)
-        kern[name] = (tot / n) if n else None
-    per_step = sorted(timed(args.steps, profile=False, per_step=True))
+        ms_prof = run.timed(args.steps, profile=True)
+    kern = run.kernel_ms()
+    per_step = sorted(run.timed(args.steps, profile=False, per_step=True))
     pct = {f"p{q}": per_step[min(len(per_step) - 1, int(q / 100 * len(per_step)))]
            for q in (10, 50, 90)}
-    st = moe.moe_plan_sync_status(plan, stream)
-    if st != moe.MOE_OK:
-        raise RuntimeError(moe.moe_status_str(st))
+    run.check()
 
     # end to end: host x in, host result out, every step, through the C ABI
-    x_host = [xs[i].cpu().pin_memory() for i in range(min(nsets, 4))]
+    x_host = [run.xs[i].cpu().pin_memory() for i in range(min(nsets, 4))]
     out_host = torch.empty((T, w.d), dtype=torch.bfloat16).pin_memory()
     K2 = args.steps
     rep.barrier()
@@ -411,33 +531,32 @@ def run_ours(args):
     h0.record(stream)
     for i in range(K2):
         if L == 1:
-            moe.moe_forward_host(plan, T, x_host[i % len(x_host)], rws[0], gms[0],
+            moe.moe_forward_host(plan, T, x_host[i % len(x_host)], run.rws[0], run.gms[0],
                                  lay["router_bias"], lay["w_gate_up"], lay["w_down"],
                                  lay["scales_gate_up"], lay["scales_down"], None, out_host,
                                  stream, expert_gamma=lay["expert_gamma"])
         else:
-            xs[0].copy_(x_host[i % len(x_host)], non_blocking=True)
-            out_host.copy_(step(0), non_blocking=True)
+            run.xs[0].copy_(x_host[i % len(x_host)], non_blocking=True)
+            out_host.copy_(run.step(0), non_blocking=True)
             stream.synchronize()
     h1.record(stream)
     torch.cuda.synchronize()
     e2e_s = rep.max_over_ranks(h0.elapsed_time(h1), "cuda") * 1e-3
-    st = moe.moe_plan_sync_status(plan, stream)
-    if st != moe.MOE_OK:
-        raise RuntimeError(moe.moe_status_str(st))
+    run.check()
 
     hbm, bf16, bf16_sus, basis = peaks()
-    expert_bytes, layer_bytes, flops = 0.0, 0.0, 0.0
-    for l in range(L):
-        eb, lb, fl, wbytes = layer_costs(w, touched[l], T)
-        expert_bytes += eb
-        layer_bytes += lb
-        flops += fl
-    expert_bytes /= L  # per expert-kernel launch
+    expert_bytes, layer_bytes, flops, wbytes = run.costs()
     ms_step = ms / args.steps
     k_ms = kern["expert"]
     achieved = expert_bytes / (k_ms * 1e-3) / 1e9 if k_ms else None
     traffic = recorded_traffic(args.workload)
+    touched = run.touched
+    lay_cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        lay_cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in lay.items()}
+        lay_cpu["x"] = run.xs[0].cpu()
+    run.close()
+    del run
     desc = {
         "canvas": "one MoE layer over a T=256 token canvas",
         "canvas4": "one MoE layer over a T=256 token canvas, int4 w4g128 weights",
@@ -467,7 +586,7 @@ def run_ours(args):
             "global_batch": world * T, "seq_len": T, "layers_per_step": L,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": f"weights {wbytes * w.E * L / 1e9:.2f} GB > L2; x/out rotated over "
-                  f"{nsets} sets ({nsets * small / 2**20:.0f} MiB)",
+                  f"{nsets} sets ({nsets * run_small(w, nsets) / 2**20:.0f} MiB)",
             "timed_region": "CUDA events around the K steps; per-kernel times from a second "
                             "timed run with events between the launches",
             "ms_per_step_with_kernel_events": ms_prof / args.steps,
@@ -500,10 +619,13 @@ def run_ours(args):
                 "h2d_bytes_per_step": T * w.d * 2, "d2h_bytes_per_step": T * w.d * 2},
         "clocks": clk.summary(),
     }
-    moe.moe_plan_destroy(plan)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        lay_cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in lay.items()}
-        lay_cpu["x"] = xs[0].cpu()
+    # the other workloads the layer is graded on, measured in the same run:
+    # the T=2048 encode layer (tensor-core target) and the 30-layer step
+    extras = [] if args.no_extra else [x for x in args.extra.split(",") if x and x != w.name]
+    for name in extras:
+        steps, warm = {"encode": (100, 20), "stack30": (20, 5)}.get(name, (50, 10))
+        line[name] = sub_record(name, args, rank, steps, warm)
+    if lay_cpu is not None:
         cb = cpu_baseline(lay_cpu, w)
         if L > 1:
             cb["value"] /= L
@@ -513,6 +635,10 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     rep.barrier()
     rep.shutdown()
+
+
+def run_small(w, nsets):
+    return w.T * w.d * 2 * 2 + (w.E * w.d * 4 + w.d * 4 if w.layers == 1 else 0)
 
 
 LMHEAD_METRIC = ("canvas tokens/s through the lm_head step (T=256 logits over V=262144, "

@@ -35,6 +35,10 @@ MOE_OPT_PDL = 4
 MOE_OPT_L2_PREFETCH_MB = 5
 MOE_OPT_ROUTER = 6
 MOE_OPT_Y_BF16 = 7
+MOE_OPT_DEBUG = 8
+
+MOE_MAX_T = 65536
+MOE_MAX_ASSIGNMENTS = 1 << 19
 
 MOE_K_ROUTER, MOE_K_PLAN, MOE_K_EXPERT, MOE_K_COMBINE = range(4)
 KERNEL_NAMES = ["router", "plan_gather", "expert", "combine"]

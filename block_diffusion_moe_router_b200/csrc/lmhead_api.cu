@@ -109,15 +109,21 @@ moe_status_t moe_lmhead_forward(moe_lmhead_t p, int T, const void* h, const void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int VT = (p->V + 255) / 256;  // partials per token: one per 256-row tile
   if (!p->ws || T > p->cap_T) {
+    // stream-ordered growth: the host does not wait for earlier calls
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return MOE_ERR_UNSUPPORTED;
     int cap = p->cap_T > 0 ? p->cap_T : 64;
     while (cap < T) cap *= 2;
+    if (cap > kMaxT) cap = kMaxT;
     const size_t bytes = 256 + (size_t)cap * VT * sizeof(float4) + (size_t)cap * 4;
     if (p->ws) {
-      if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
-      cudaFree(p->ws);
+      if (cudaFreeAsync(p->ws, s) != cudaSuccess) return MOE_ERR_CUDA;
       p->ws = nullptr;
+      p->cap_T = 0;
     }
-    if (cudaMalloc(&p->ws, bytes) != cudaSuccess) {
+    if (cudaMallocAsync(&p->ws, bytes, s) != cudaSuccess) {
+      cudaGetLastError();
       p->ws = nullptr;
       p->cap_T = 0;
       return MOE_ERR_ALLOC;
@@ -125,7 +131,7 @@ moe_status_t moe_lmhead_forward(moe_lmhead_t p, int T, const void* h, const void
     p->ctl = static_cast<moe::Ctl*>(p->ws);
     p->part = reinterpret_cast<float4*>(static_cast<uint8_t*>(p->ws) + 256);
     p->cap_T = cap;
-    if (cudaMemset(p->ctl, 0, sizeof(moe::Ctl)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(p->ctl, 0, sizeof(moe::Ctl), s) != cudaSuccess) return MOE_ERR_CUDA;
   }
   // logZ goes to the caller's array, else to scratch after the partials
   float* logz = logz_out ? logz_out

@@ -44,9 +44,12 @@ struct moe_plan_s {
   int prefetch_mb;
   int y_bf16;
   int router_sel;
+  int debug;       // MOE_OPT_DEBUG: lay the next workspace out with guard blocks
   int cap_T;
   int last_T;
   void* ws;  // one device allocation holding everything below
+  std::vector<size_t> guards;  // offsets of the workspace's guard blocks (debug layout)
+  Ctl* noalloc_ctl;            // status word of this plan's last moe_forward_noalloc call
   Ctl* ctl;
   int32_t *idx, *perm, *slot_of, *offsets, *ready;
   int4* chunk_info;
@@ -135,7 +138,7 @@ size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 // (whose kernels keep decoded A stages in TMEM next to the accumulators).
 int chunk_size(moe_plan_t p) { return p->wdtype == MOE_W_BF16 ? moe::kMaxN : 128; }
 
-int max_chunks(int E, int T, int k) { return E + (T * k) / 128 + 1; }
+size_t max_chunks(int E, size_t T, int k) { return (size_t)E + (T * (size_t)k) / 128 + 1; }
 
 // Experts rounded up to the UMMA N granularity for the tensor-core router.
 int router_ep(int E) { return (E + 15) / 16 * 16; }
@@ -209,40 +212,77 @@ moe_status_t check_device(moe_plan_t p) {
   return dev == p->device ? MOE_OK : MOE_ERR_INVALID_ARG;
 }
 
-moe_status_t ensure_workspace(moe_plan_t p, int T) {
+constexpr size_t kGuardBytes = 256;
+constexpr int kGuardByte = 0xA5;
+
+// T within the token limits of include/moe.h.
+bool tokens_ok(const moe_plan_s* p, int T) {
+  return T <= MOE_MAX_T && (int64_t)T * p->k <= (int64_t)MOE_MAX_ASSIGNMENTS;
+}
+
+// Grows the workspace to hold T tokens (T within tokens_ok), stream-ordered
+// on `s`: the old allocation is released with cudaFreeAsync and the new one
+// taken with cudaMallocAsync and cleared with cudaMemsetAsync, so the host
+// never waits.  With the debug layout a guard block of kGuardBytes follows
+// every region.
+moe_status_t ensure_workspace(moe_plan_t p, int T, cudaStream_t s) {
   if (p->ws && T <= p->cap_T) return MOE_OK;
-  int cap = p->cap_T > 0 ? p->cap_T : 16;
-  while (cap < T) cap *= 2;
-  const size_t A = (size_t)cap * p->k;
-  const size_t MC = (size_t)max_chunks(p->E, cap, p->k);
+  {
+    // growth inside a stream capture would put allocation nodes into the
+    // caller's graph: the workspace must be reserved before capturing
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return MOE_ERR_UNSUPPORTED;
+  }
+  size_t cap = p->cap_T > 0 ? (size_t)p->cap_T : 16;
+  while (cap < (size_t)T) cap *= 2;
+  if (cap > (size_t)MOE_MAX_T) cap = MOE_MAX_T;
+  if (cap * (size_t)p->k > (size_t)MOE_MAX_ASSIGNMENTS) cap = (size_t)T;
+  const size_t A = cap * p->k;
+  const size_t MC = max_chunks(p->E, cap, p->k);
+  const bool dbg = p->debug != 0;
+  std::vector<size_t> guards;
   size_t sz = 0;
   auto take = [&](size_t bytes) {
     size_t o = sz;
     sz += align256(bytes);
+    if (dbg) {
+      guards.push_back(sz);
+      sz += kGuardBytes;
+    }
     return o;
   };
   const size_t o_ctl = take(sizeof(Ctl));
-  const size_t o_idx = take(A * 4), o_w = take(A * 4), o_gap = take((size_t)cap * 4);
+  const size_t o_idx = take(A * 4), o_w = take(A * 4), o_gap = take(cap * 4);
   const size_t o_perm = take(A * 4), o_slot = take(A * 4), o_off = take((size_t)(p->E + 1) * 4);
   const size_t o_ci = take(MC * 16), o_rd = take(MC * 4);
   const size_t o_xp = take(A * p->d * 2);
   const size_t o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
-  const size_t o_xd = take((size_t)cap * p->d * 2), o_rs = take((size_t)cap * p->d * 2);
-  const size_t o_od = take((size_t)cap * p->d * 2);
+  const size_t o_xd = take(cap * p->d * 2), o_rs = take(cap * p->d * 2);
+  const size_t o_od = take(cap * p->d * 2);
   if (p->ws) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
-    cudaFree(p->ws);
+    if (cudaFreeAsync(p->ws, s) != cudaSuccess) return MOE_ERR_CUDA;
     p->ws = nullptr;
+    p->cap_T = 0;
   }
   void* ws = nullptr;
-  if (cudaMalloc(&ws, sz) != cudaSuccess) {
+  if (cudaMallocAsync(&ws, sz, s) != cudaSuccess) {
     cudaGetLastError();
     p->cap_T = 0;
     return MOE_ERR_ALLOC;
   }
-  if (cudaMemset(ws, 0, sz) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sz, s) != cudaSuccess) {
+    cudaFreeAsync(ws, s);
+    return MOE_ERR_CUDA;
+  }
   char* b = static_cast<char*>(ws);
+  for (size_t g : guards)
+    if (cudaMemsetAsync(b + g, kGuardByte, kGuardBytes, s) != cudaSuccess) {
+      cudaFreeAsync(ws, s);
+      return MOE_ERR_CUDA;
+    }
   p->ws = ws;
+  p->guards.swap(guards);
   p->ctl = reinterpret_cast<Ctl*>(b + o_ctl);
   p->idx = reinterpret_cast<int32_t*>(b + o_idx);
   p->w = reinterpret_cast<float*>(b + o_w);
@@ -258,7 +298,7 @@ moe_status_t ensure_workspace(moe_plan_t p, int T) {
   p->x_dev = reinterpret_cast<__nv_bfloat16*>(b + o_xd);
   p->res_dev = reinterpret_cast<__nv_bfloat16*>(b + o_rs);
   p->out_dev = reinterpret_cast<__nv_bfloat16*>(b + o_od);
-  p->cap_T = cap;
+  p->cap_T = (int)cap;
   return MOE_OK;
 }
 
@@ -299,6 +339,7 @@ moe_status_t validate_route(moe_plan_t p, int T, const void* x, const float* rw,
   if (!p) return MOE_ERR_INVALID_ARG;
   if (T < 0) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
+  if (!tokens_ok(p, T)) return MOE_ERR_UNSUPPORTED;
   if (!x || !rw || !gamma) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(rw) || !aligned16(gamma)) return MOE_ERR_INVALID_ARG;
   if (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)) return MOE_ERR_INVALID_ARG;
@@ -395,9 +436,11 @@ moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, mo
   p->prefetch_mb = 0;
   p->y_bf16 = 1;
   p->router_sel = 0;
+  p->debug = 0;
   p->cap_T = 0;
   p->last_T = 0;
   p->ws = nullptr;
+  p->noalloc_ctl = nullptr;
   *out = p;
   return MOE_OK;
 }
@@ -433,15 +476,21 @@ moe_status_t moe_plan_set_option(moe_plan_t p, int key, double value) {
     case MOE_OPT_Y_BF16:
       p->y_bf16 = value != 0.0;
       return MOE_OK;
+    case MOE_OPT_DEBUG:
+      p->debug = value != 0.0;
+      return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
 }
 
 moe_status_t moe_plan_reserve(moe_plan_t p, int max_T) {
   if (!p || max_T < 0) return MOE_ERR_INVALID_ARG;
+  if (!tokens_ok(p, max_T)) return MOE_ERR_UNSUPPORTED;
   moe_status_t st = check_device(p);
   if (st != MOE_OK) return st;
-  return ensure_workspace(p, max_T > 0 ? max_T : 1);
+  st = ensure_workspace(p, max_T > 0 ? max_T : 1, nullptr);
+  if (st != MOE_OK) return st;
+  return cudaStreamSynchronize(nullptr) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_route(moe_plan_t p, int T, const void* x, const float* router_w,
@@ -453,7 +502,7 @@ moe_status_t moe_route(moe_plan_t p, int T, const void* x, const float* router_w
   if ((reinterpret_cast<uintptr_t>(idx_out) & 3u) || (reinterpret_cast<uintptr_t>(w_out) & 3u) ||
       (gap_out && (reinterpret_cast<uintptr_t>(gap_out) & 3u)))
     return MOE_ERR_INVALID_ARG;
-  st = ensure_workspace(p, 1);
+  st = ensure_workspace(p, 1, static_cast<cudaStream_t>(stream));
   if (st != MOE_OK) return st;
   return launch_router(p, T, x, router_w, router_gamma, router_bias, idx_out, w_out, gap_out,
                        static_cast<cudaStream_t>(stream));
@@ -478,11 +527,11 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   const size_t act = (size_t)T * p->d * 2;
   if (overlap(out, act, x, act)) return MOE_ERR_INVALID_ARG;
   if (residual && residual != out && overlap(out, act, residual, act)) return MOE_ERR_INVALID_ARG;
-  st = ensure_workspace(p, T);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = ensure_workspace(p, T, s);
   if (st != MOE_OK) return st;
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int A = T * p->k;
+  const int A = T * p->k;  // <= MOE_MAX_ASSIGNMENTS
   const bool w4 = p->wdtype == MOE_W_INT4_G128;
   const bool w8 = p->wdtype == MOE_W_FP8_E4M3;
   const bool w4f = p->wdtype == MOE_W_FP4_E2M1;
@@ -600,12 +649,13 @@ moe_status_t moe_forward_host(moe_plan_t p, int T, const void* x_host, const flo
                               const void* residual_host, void* out_host, void* stream) {
   if (!p || T < 0) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
+  if (!tokens_ok(p, T)) return MOE_ERR_UNSUPPORTED;
   if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
   moe_status_t st = check_device(p);
   if (st != MOE_OK) return st;
-  st = ensure_workspace(p, T);
-  if (st != MOE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = ensure_workspace(p, T, s);
+  if (st != MOE_OK) return st;
   const size_t act = (size_t)T * p->d * 2;
   if (cudaMemcpyAsync(p->x_dev, x_host, act, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -643,16 +693,35 @@ moe_status_t moe_plan_sync_status(moe_plan_t p, void* stream) {
   if (!p) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
-  if (!p->ws) return MOE_OK;
-  Ctl c;
-  if (cudaMemcpy(&c, p->ctl, sizeof(Ctl), cudaMemcpyDeviceToHost) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (c.status != 0) {
-    const int zero[2] = {0, 0};
-    if (cudaMemcpy(p->ctl, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
-      return MOE_ERR_CUDA;
+  int status = 0;
+  // The plan's own word first, then the word its last noalloc call left in
+  // the library's array; each is cleared once read.
+  Ctl* words[2] = {p->ws ? p->ctl : nullptr, p->noalloc_ctl};
+  for (Ctl* w : words) {
+    if (!w) continue;
+    int c[2] = {0, 0};
+    if (cudaMemcpy(c, w, sizeof(c), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (c[0] != 0) {
+      if (status == 0) status = c[0];
+      const int zero[2] = {0, 0};
+      if (cudaMemcpy(w, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
   }
-  return static_cast<moe_status_t>(c.status);
+  if (p->ws && !p->guards.empty()) {
+    unsigned char g[kGuardBytes];
+    for (size_t off : p->guards) {
+      if (cudaMemcpy(g, static_cast<char*>(p->ws) + off, kGuardBytes, cudaMemcpyDeviceToHost) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
+      for (size_t i = 0; i < kGuardBytes; ++i)
+        if (g[i] != (unsigned char)kGuardByte) {
+          if (status == 0) status = MOE_ERR_DEVICE_CHECK;
+          break;
+        }
+    }
+  }
+  return static_cast<moe_status_t>(status);
 }
 
 moe_status_t moe_plan_profile(moe_plan_t p, int kernel, double* total_ms, int* launches) {
@@ -714,13 +783,21 @@ namespace {
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[128] = {};
 
-// Device address of the array on device `dev` (must be current).  Looked up
-// once per device; in host code the array's name is only a stand-in, so it
-// is never passed to a kernel directly.
-void* noalloc_scratch(int dev) {
+// Device address of the array on device `dev` (must be current).  In host
+// code the array's name is only a stand-in, so it is never passed to a kernel
+// directly.  The address is looked up again on every call whose stream is
+// not capturing (a device reset reloads the module and moves the array);
+// during a capture, which must not trigger a module load, the last address
+// looked up on the device is used.
+void* noalloc_scratch(int dev, cudaStream_t s) {
   if (dev < 0 || dev >= 128) return nullptr;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, moe_noalloc_scratch) != cudaSuccess || !ptr) {
       cudaGetLastError();
@@ -747,7 +824,6 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   if (expert_gamma && !aligned16(expert_gamma)) return MOE_ERR_INVALID_ARG;
   if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
   if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 3u)) return MOE_ERR_INVALID_ARG;
-  if (expert_gamma && !aligned16(expert_gamma)) return MOE_ERR_INVALID_ARG;
   if (p->wdtype == MOE_W_BF16) {
     if (scales_gate_up || scales_down) return MOE_ERR_INVALID_ARG;
   } else {
@@ -759,7 +835,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
 
   // Carve the intermediates for T tokens; refuse what does not fit.
   const size_t A = (size_t)T * p->k;
-  const size_t MC = (size_t)max_chunks(p->E, T, p->k);
+  const size_t MC = max_chunks(p->E, T, p->k);
   size_t sz = 0;
   auto take = [&](size_t bytes) {
     size_t o = sz;
@@ -774,7 +850,8 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   const size_t o_h = take(A * p->f * 2), o_y = take(A * p->d * 4);
   if (sz > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
 
-  char* b = static_cast<char*>(noalloc_scratch(p->device));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* b = static_cast<char*>(noalloc_scratch(p->device, s));
   if (!b) return MOE_ERR_CUDA;
   Ctl* ctl = reinterpret_cast<Ctl*>(b + o_ctl);
   int32_t* idx = reinterpret_cast<int32_t*>(b + o_idx);
@@ -789,7 +866,6 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(b + o_h);
   float* y = reinterpret_cast<float*>(b + o_y);
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tm_wgu, tm_wd, tm_x, tm_h;
   if (!make_map_bf16(&tm_wgu, w_gate_up, (uint64_t)p->E * 2 * p->f, p->d, moe::kGuHalf) ||
       !make_map_bf16(&tm_wd, w_down, (uint64_t)p->E * p->d, p->f, moe::kBM) ||
@@ -800,6 +876,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   // The status word must start at zero; the plan kernel resets the scheduler
   // counters and chunk tables itself on every call.
   if (cudaMemsetAsync(ctl, 0, sizeof(Ctl), s) != cudaSuccess) return MOE_ERR_CUDA;
+  p->noalloc_ctl = ctl;  // moe_plan_sync_status reads this call's status here
 
   {
     const bool prof = p->profile != 0;

@@ -27,7 +27,7 @@
  *   S   = the k largest z_e, ties to the lower index; j order = (z desc, e asc)
  *   w_j = softmax(z)[S_j] / sum_j' softmax(z)[S_j']
  *   h   = gelu_tanh(Wgu[S_j][0:f] xe) * (Wgu[S_j][f:2f] xe)     (bf16 h)
- *   y_j = Wd[S_j] h                                              (fp32 y)
+ *   y_j = Wd[S_j] h          (bf16 y by default; fp32 with MOE_OPT_Y_BF16 = 0)
  *   out_t = residual_t + sum_j w_j y_j  (j order, fp32, one rounding to bf16)
  *
  * Conventions for every entry point:
@@ -39,7 +39,9 @@
  *     stream).  Calls are asynchronous on that stream except where stated.
  *     A plan is used by one stream at a time.
  *   - On any invalid argument nothing is launched and an error is returned.
- *     Launch failures return MOE_ERR_CUDA.  Faults the kernels detect
+ *     Launch failures return MOE_ERR_CUDA.
+ *   - Token counts: 0 <= T <= MOE_MAX_T and T * k <= MOE_MAX_ASSIGNMENTS;
+ *     a larger T returns MOE_ERR_UNSUPPORTED before anything is launched.  Faults the kernels detect
  *     themselves (a bounded wait that ran out, an index out of range) are
  *     recorded in a device status word read by moe_plan_sync_status.
  */
@@ -53,6 +55,11 @@ extern "C" {
 #endif
 
 typedef struct moe_plan_s* moe_plan_t;
+
+/* Largest token count of one call, and largest T * k (token-expert
+ * assignments) of one call. */
+#define MOE_MAX_T 65536
+#define MOE_MAX_ASSIGNMENTS (1 << 19)
 
 typedef enum {
   MOE_OK = 0,
@@ -109,9 +116,17 @@ enum {
                              router pulls into L2 while routing runs, so the
                              expert kernel's first wave finds it there
                              (default 0 = off)                                   */
-  MOE_OPT_Y_BF16 = 7      /* 1 (default): the per-slot expert outputs y are kept
+  MOE_OPT_Y_BF16 = 7,     /* 1 (default): the per-slot expert outputs y are kept
                              in bf16 (one more rounding before the fp32
                              combine, half the bytes); 0: fp32                   */
+  MOE_OPT_DEBUG = 8       /* 1: the workspace is laid out with a 256-byte guard
+                             block after every region, filled with a fixed
+                             pattern when the workspace is (re)allocated;
+                             moe_plan_sync_status then also checks every guard
+                             and returns MOE_ERR_DEVICE_CHECK if a kernel wrote
+                             past its region.  Takes effect at the next
+                             workspace (re)allocation (set it before the first
+                             call or moe_plan_reserve).  Default 0.             */
 };
 
 /* Kernels of one moe_forward, for moe_plan_profile. */
@@ -126,7 +141,8 @@ enum {
 
 /* Create a plan for E experts, top-k, hidden d, per-expert intermediate f.
  * Limits: 1 <= E <= 256; 1 <= k <= min(E, 32); d % 128 == 0, 128 <= d <= 4096;
- * f % 64 == 0, 64 <= f <= 4096.  Binds the plan to the current CUDA device.
+ * f % 64 == 0, 64 <= f <= 4096 (every DiffusionGemma shape and the test
+ * shapes fit; d % 128 keeps an int4 scale group inside one row of x).  Binds the plan to the current CUDA device.
  * Returns MOE_ERR_UNSUPPORTED outside the limits, MOE_ERR_INVALID_ARG on a
  * NULL `out`.  Allocates nothing on the device until the first call. */
 moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, moe_plan_t* out);
@@ -134,9 +150,13 @@ moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, mo
 /* Set an option (see MOE_OPT_*).  Synchronous, host only. */
 moe_status_t moe_plan_set_option(moe_plan_t plan, int key, double value);
 
-/* Grow the plan-owned workspace to hold max_T tokens (synchronous device
- * allocation).  moe_forward grows it on demand; call this first when the
- * calls are to be captured in a CUDA graph. */
+/* Grow the plan-owned workspace to hold max_T tokens (allocated on the
+ * legacy default stream, then synchronised).  moe_forward grows it on demand,
+ * stream-ordered: the old workspace is released with cudaFreeAsync and the
+ * new one taken with cudaMallocAsync on the call's stream, so the call does
+ * not synchronise the host.  Call this first when the calls are to be
+ * captured in a CUDA graph: a call that would grow the workspace while its
+ * stream is capturing returns MOE_ERR_UNSUPPORTED and launches nothing. */
 moe_status_t moe_plan_reserve(moe_plan_t plan, int max_T);
 
 /* The whole layer for T tokens (T = 0 is a no-op).
@@ -187,7 +207,10 @@ moe_status_t moe_forward_host(moe_plan_t plan, int T, const void* x_host, const 
  * Same arguments, layouts, results and errors as moe_forward, plus
  * status_out: a DEVICE int32 (or NULL) that receives this call's device
  * status word (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK) in stream
- * order.  The caller still passes every input and output.  All intermediates
+ * order.  The same status also stays in the array: moe_plan_sync_status on
+ * the plan reports it (with the plan's own status word, first error first)
+ * as long as no later moe_forward_noalloc call on the device has replaced
+ * it, so a caller that passes NULL still learns of a device-side error.  The caller still passes every input and output.  All intermediates
  * (routing tables, gathered rows, h, y, counters) live in one file-scope
  * __device__ array of MOE_NOALLOC_SCRATCH_BYTES; the call never calls
  * cudaMalloc, cudaFree or any allocating routine.
@@ -195,17 +218,20 @@ moe_status_t moe_forward_host(moe_plan_t plan, int T, const void* x_host, const 
  *     T*k*(6d + 2f) + T*(16k + 4) bytes plus small tables; one
  *     256-token canvas of the 2816/704/128/top-8 layer needs 37.5 MB).  A larger call
  *     returns MOE_ERR_UNSUPPORTED and launches nothing.
- *   - Set-up: the first call on each device (with that device current) looks
- *     up the array's device address once; make that first call before any
- *     stream capture.
+ *   - Set-up: a call looks up the array's device address on its device
+ *     (cudaGetSymbolAddress, the device current) whenever its stream is not
+ *     capturing, so the address stays right after a device reset reloads the
+ *     library's module; while a capture is in progress the address of the
+ *     last lookup on that device is used.  Make the first call on each device
+ *     before any stream capture.
  *   - The array is part of the library's device image: every GPU that loads
  *     it holds the 40 MiB until the process exits.
  *   - Every call on a device shares the one array and it keeps the last
  *     call's contents (each call clears the words that must start at zero).
  *     Calls that overlap on the GPU (other streams, other threads, other
  *     plans) race on it and must be serialised by the caller.
- *   - bf16 plans only for now (int4 and fp8 plans return
- *     MOE_ERR_UNSUPPORTED); MOE_OPT_PROFILE is ignored. */
+ *   - bf16 plans only (int4, fp8 and fp4 plans return MOE_ERR_UNSUPPORTED);
+ *     MOE_OPT_PROFILE and MOE_OPT_DEBUG are ignored. */
 moe_status_t moe_forward_noalloc(moe_plan_t plan, int T, const void* x, const float* router_w,
                                  const float* router_gamma, const float* router_bias,
                                  const float* expert_gamma, const void* w_gate_up, const void* w_down,
@@ -227,7 +253,10 @@ moe_status_t moe_plan_routing(moe_plan_t plan, int32_t* offsets, int32_t* perm, 
                               void* stream);
 
 /* Synchronise `stream`, return the device status word (MOE_OK, MOE_ERR_TIMEOUT
- * or MOE_ERR_DEVICE_CHECK) and clear it. */
+ * or MOE_ERR_DEVICE_CHECK) and clear it.  The plan's own word comes first;
+ * if it is clear, the word of the plan's last moe_forward_noalloc call (see
+ * there) is reported and cleared.  With MOE_OPT_DEBUG on, a damaged
+ * workspace guard block is reported as MOE_ERR_DEVICE_CHECK. */
 moe_status_t moe_plan_sync_status(moe_plan_t plan, void* stream);
 
 /* With MOE_OPT_PROFILE on: total device time (ms) and number of launches of
@@ -258,7 +287,7 @@ const char* moe_status_str(moe_status_t status);
  * The pages name the rule but do not state it; this is the entropy-bounded
  * unmasking rule it is named after (the library's reading).
  * The [T, V] logits are never written: the GEMM's epilogue folds them into
- * per-(token, 128-row tile) softmax statistics on chip. */
+ * per-(token, 256-row tile) softmax statistics on chip. */
 typedef struct moe_lmhead_s* moe_lmhead_t;
 
 /* Handle for a vocabulary of V rows of width d (1 <= V <= 2^24, d a multiple
@@ -279,7 +308,9 @@ moe_status_t moe_lmhead_create(int V, int d, moe_lmhead_t* out);
  *   logz_out       fp32 [T]      logZ_t (NULL to skip)
  *   accept_out     uint8 [T]     1 = masked and accepted this step
  * Asynchronous on `stream`; bounded-wait expiry is reported by
- * moe_lmhead_sync_status. */
+ * moe_lmhead_sync_status.  The handle's workspace grows stream-ordered on
+ * `stream` when T exceeds every earlier call's (a growth while the stream is
+ * capturing returns MOE_ERR_UNSUPPORTED: make a call of the largest T first). */
 moe_status_t moe_lmhead_forward(moe_lmhead_t lh, int T, const void* h, const void* w,
                                 float temperature, float softcap, const uint8_t* masked,
                                 float entropy_bound, int32_t* token_out, float* entropy_out,

@@ -90,3 +90,20 @@ def test_lmhead_create_rejects_bad_shapes_without_device(abi):
                                   None, None) == abi.MOE_ERR_INVALID_ARG
     assert lib.moe_lmhead_sync_status(None, None) == abi.MOE_ERR_INVALID_ARG
     lib.moe_lmhead_destroy(None)
+
+
+def test_binding_constants_match_the_header(abi):
+    """Every status, weight format, option and limit the header defines has the
+    same value in the Python binding."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    enums = dict((n, int(v)) for n, v in re.findall(r"\b(MOE_(?:ERR_\w+|OK|W_\w+|OPT_\w+|K_\w+))"
+                                                    r"\s*=\s*(\d+)", src))
+    assert len(enums) >= 25
+    for name, val in enums.items():
+        if name == "MOE_K_COUNT":
+            continue
+        assert getattr(abi, name) == val, name
+    defines = dict(re.findall(r"#define\s+(MOE_MAX_\w+)\s+\(?([^)\n]+)\)?", src))
+    assert eval(defines["MOE_MAX_T"]) == abi.MOE_MAX_T
+    assert eval(defines["MOE_MAX_ASSIGNMENTS"].replace("(", "").replace(")", "")) == \
+        abi.MOE_MAX_ASSIGNMENTS
