@@ -349,44 +349,6 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
                : "memory");
 }
 
-// Bounded wait with cluster-scope acquire: for barriers that the peer CTA
-// arrives on (its writes before a release.cluster arrive become visible).
-__device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                             Ctl* ctl, uint64_t timeout_ns, int where) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait_cl(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait_cl(a, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > timeout_ns) {
-      record_error(ctl, MOE_ERR_TIMEOUT, where);
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
-// 32-bit store into the shared memory of a CTA of the cluster
-// (shared::cluster address from mapa_rank).
-__device__ __forceinline__ void st_cluster_u32(uint32_t cl_addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cl_addr), "r"(v) : "memory");
-}
-
 // Programmatic dependent launch: wait until the preceding grid in the stream
 // has completed and its memory is visible (a no-op when the kernel was not
 // launched with the attribute), and let the next grid begin launching.

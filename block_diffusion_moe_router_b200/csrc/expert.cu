@@ -18,18 +18,29 @@
 // the expert are N (16..256), so every weight byte is streamed from HBM once
 // per chunk, and at 256 tokens per canvas one chunk covers every expert.
 //
-// Roles (224 threads): warp 0 = scheduler (claims units: its CTA index
-// first, then from a global counter) and weight (A) producer, warp 1 = UMMA issuer (owns the TMEM
-// allocation), warps 2..5 = epilogue (TMEM -> registers -> global), warp 6 =
-// activation (B) producer.  Weights and activations have rings of their own,
+// Roles (256 threads): warp 0 = scheduler (claims units: its CTA index
+// first, then from a global counter) and weight (A) producer, warps 1 and 7
+// = UMMA issuers (warp 1 owns the TMEM allocation), warps 2..5 = epilogue
+// (TMEM -> registers -> global), warp 6 = activation (B) producer.  One
+// issuing thread sustains one M=128 K=16 UMMA per ~90-110 cycles whatever N
+// is (below N ~ 180), which at 4 UMMAs per 64-wide K stage is slower than a
+// stage's share of the weight stream once the chunks grow past ~100 tokens;
+// UMMAs from two threads overlap, so, while every chunk has at most 128
+// tokens (a canvas), the two issuers split K: warp 1 takes the even K stages
+// of every unit and warp 7 the odd ones, each into its own partial
+// accumulator, and the epilogue adds the two partials (fixed order, so the
+// result does not depend on timing).  With larger chunks the two partials of
+// a unit would fill half of TMEM and the epilogue would stall the tensor
+// cores at every unit, so warp 1 issues alone.  Weights and activations have rings of their own,
 // sized at run time from the largest chunk: the weight ring is deep, since
 // its tiles come from HBM and are the bytes the kernel exists to stream,
 // while the activation tiles come from L2.  So the weights of a unit keep
 // streaming while its activations are still being produced: a down unit's
 // W_d tiles are fetched before every gate_up unit of its chunk has published
 // h, and only its h tiles wait (per-chunk counter, acquire/release).  TMEM
-// holds two 256-column fp32 accumulators so the epilogue of one unit overlaps
-// the MMAs of the next.
+// (512 columns) holds two units' accumulators (two 128-column partials each
+// when K is split, else one of 256 columns), so the epilogue of one unit
+// overlaps the MMAs of the next.
 //
 // Every wait is bounded by %globaltimer; on expiry the kernel records
 // MOE_ERR_TIMEOUT, the roles leave their loops, in-flight TMA copies and
@@ -40,13 +51,13 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 224;
+constexpr int kThreads = 256;
 constexpr int kMaxA = 12;  // weight stages
 constexpr int kMaxB = 8;   // activation stages
-constexpr int kMinB = 3;
+constexpr int kMinB = 3;  // 2 when rounded down to even
 constexpr int kRingBytes = 200 * 1024;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
-constexpr int kBarBytes = 8 * (2 * kMaxA + 2 * kMaxB + 4 + 2 * kUnitRing + 1);
+constexpr int kBarBytes = 8 * (2 * kMaxA + 2 * kMaxB + 4 + 2 * kUnitRing + 2);
 constexpr int kSmemBytes = 1024 + kRingBytes + kEpiBytes + kBarBytes + 256;
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -68,7 +79,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* ufull = tempty + 2;
   uint64_t* uempty = ufull + kUnitRing;
   uint64_t* drain = uempty + kUnitRing;
-  UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 1);
+  UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(units + kUnitRing);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* s_bcast = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -89,14 +100,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&emptyB[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&tfull[i], 1);
+      mbar_init(&tfull[i], 2);   // one commit per UMMA issuer
       mbar_init(&tempty[i], 4);  // one arrival per epilogue warp
     }
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(&ufull[i], 1);
-      mbar_init(&uempty[i], 3);  // UMMA issuer, epilogue leader, B producer
+      mbar_init(&uempty[i], 4);  // two UMMA issuers, epilogue leader, B producer
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -120,14 +132,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   // B-operand rows per stage: the largest chunk, rounded up to the TMA box.
   // The activation ring takes kMinB..kMaxB stages (as many as fit half of
   // the ring: at 2048 tokens a chunk's B stage is larger than its A stage
-  // and its L2 latency must be hidden too), the weights the rest.
+  // and its L2 latency must be hidden too), the weights the rest.  When two
+  // issuers split K (splitk, below) both depths are even: a ring slot then
+  // always holds stages of the same issuer (global stage parity), so an
+  // issuer waiting on its stage q has itself consumed stage q - depth in
+  // that slot and the parity wait cannot be satisfied by a phase two behind
+  // (with an odd depth the slot's previous stage belongs to the other issuer
+  // and may still be in flight).
   const int maxn = max(1, min(kMaxN, ctl->max_chunk));
+  const bool splitk = maxn <= 128;
+  const int even = splitk ? ~1 : ~0;
   const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
   const int b_bytes = NB * kBK * 2;
-  const int SB = min(kMaxB, max(kMinB, (kRingBytes / 2) / b_bytes));
-  const int SA = min(kMaxA, (kRingBytes - SB * b_bytes) / kABytes);
+  const int SB = min(kMaxB, max(kMinB, (kRingBytes / 2) / b_bytes)) & even;
+  const int SA = min(kMaxA, (kRingBytes - SB * b_bytes) / kABytes) & even;
   uint8_t* ringA = ring;
   uint8_t* ringB = ring + SA * kABytes;
+  // Accumulators, two units in flight.  Chunks of at most 128 tokens: the
+  // two issuers split K, each unit holding two partials of 128 columns.
+  // Larger chunks: their partials would leave room for one unit only, and
+  // the epilogue would then stall the tensor cores at every unit, so warp 1
+  // issues every stage into one 256-column accumulator (warp 7 only keeps
+  // the barrier protocol).
+  const int W = splitk ? 128 : kMaxN;      // columns of one partial
+  const int ACC = splitk ? 2 * W : kMaxN;  // columns of one unit's accumulator
+  const int NBUF = kTmemCols / ACC;        // 2
   const int n_chunks = ctl->n_chunks;
   const int U = n_chunks * (GU + DN);
 
@@ -230,15 +259,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s2 = 0; s2 < SA; ++s2)
         if ((issued >> s2) & 1u)
           mbar_wait_drain(&fullA[s2], (issued_par >> s2) & 1u, ctl, a.timeout_ns);
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ UMMA issuer
+  } else if (warp == 1 || warp == 7) {
+    // ------------------------------------------------------------ UMMA issuers
+    // Issuer par (0: warp 1, 1: warp 7) takes the K stages kb % 2 == par of
+    // every unit into partial par of the unit's accumulator.  Both always
+    // wait for the accumulator to be free and commit its full barrier (count
+    // 2), so neither can run a phase ahead of the epilogue.
     if (lane == 0) {
-      int sa_i = 0, sb_i = 0;
-      uint32_t pa = 0, pb = 0;
+      const int par = warp == 1 ? 0 : 1;
+      const int first = splitk ? par : (par == 0 ? 0 : 1 << 30);  // this issuer's first stage
+      const int step = splitk ? 2 : 1;
+      int g = 0;  // ring stages used by all earlier units
       int ur = 0;
       uint32_t uphase = 0;
-      int acc = 0;
-      uint32_t aphase = 0;
+      int buf = 0;
+      uint32_t bphase = 0;
       while (true) {
         if (!mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullMma)) break;
         const UnitInfo ui = units[ur];
@@ -246,12 +281,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nkb = (ui.type == kUnitGateUp) ? a.d / kBK : a.f / kBK;
         const int N = (ui.n + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kBM, N);
-        if (!mbar_wait(&tempty[acc], aphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereTmemEmpty))
+        if (!mbar_wait(&tempty[buf], bphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereTmemEmpty))
           break;
         tc_fence_after();
-        const uint32_t dt = tmem_base + (uint32_t)(acc * kMaxN);
+        const uint32_t dt = tmem_base + (uint32_t)(buf * ACC + (splitk ? par * W : 0));
+        const int g0 = g + (first < nkb ? first : 0);
+        int sa_i = g0 % SA, sb_i = g0 % SB;
+        uint32_t pa = (uint32_t)(g0 / SA) & 1u, pb = (uint32_t)(g0 / SB) & 1u;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = first; kb < nkb; kb += step) {
           if (!mbar_wait(&fullA[sa_i], pa, s_abort, ctl, a.timeout_ns, kWhereStageFull) ||
               !mbar_wait(&fullB[sb_i], pb, s_abort, ctl, a.timeout_ns, kWhereStageFull)) {
             ok = false;
@@ -263,31 +301,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk)
             umma_bf16(dt, sdesc_k_sw128(sa + kk * kUmmaK * 2), sdesc_k_sw128(sb + kk * kUmmaK * 2),
-                      idesc, (kb | kk) ? 1u : 0u);
+                      idesc, (kb > first || kk > 0) ? 1u : 0u);
           umma_commit(&emptyA[sa_i]);
           umma_commit(&emptyB[sb_i]);
-          if (++sa_i == SA) {
-            sa_i = 0;
+          sa_i += step;
+          if (sa_i >= SA) {
+            sa_i -= SA;
             pa ^= 1;
           }
-          if (++sb_i == SB) {
-            sb_i = 0;
+          sb_i += step;
+          if (sb_i >= SB) {
+            sb_i -= SB;
             pb ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        umma_commit(&tfull[buf]);
         mbar_arrive(&uempty[ur]);
+        g += nkb;
         if (++ur == kUnitRing) {
           ur = 0;
           uphase ^= 1;
         }
-        acc ^= 1;
-        if (acc == 0) aphase ^= 1;
+        if (++buf == NBUF) {
+          buf = 0;
+          bphase ^= 1;
+        }
       }
       // Drain: all issued UMMAs complete before TMEM is released.
-      umma_commit(drain);
-      mbar_wait_drain(drain, 0, ctl, a.timeout_ns);
+      umma_commit(&drain[par]);
+      mbar_wait_drain(&drain[par], 0, ctl, a.timeout_ns);
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------ B producer
@@ -345,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     epilogue_role(a, units, ufull, uempty, tfull, tempty, xchg, s_abort, s_bcast, tmem_base,
-                  kMaxN, warp, lane);
+                  ACC, warp, lane, nullptr, nullptr, splitk ? kBK : 0, NBUF);
   }
 
   tc_fence_before();

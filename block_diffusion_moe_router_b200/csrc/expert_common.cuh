@@ -120,7 +120,9 @@ __device__ __forceinline__ void add_partial(uint32_t taddr, uint32_t (&v)[32]) {
 // outcome, so the 128 threads always pass the same named barriers.
 // kRowScale (fp8 weights): every accumulator row is first multiplied by its
 // weight row's fp32 scale, read from the unit's slot rscale + 128 * ur
-// (landed on sfull[ur]); HT is h's type (fp16 on that path).
+// (landed on sfull[ur]); HT is h's type (fp16 on that path).  The units
+// rotate over `nbuf` accumulators of acc_cols columns each (tfull / tempty
+// per accumulator).
 template <bool kRowScale = false, typename HT = __nv_bfloat16>
 __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInfo* units,
                                               uint64_t* ufull, uint64_t* uempty, uint64_t* tfull,
@@ -129,7 +131,7 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
                                               uint32_t tmem_base, int acc_cols, int warp,
                                               int lane, uint64_t* sfull = nullptr,
                                               const float* rscale = nullptr,
-                                              int split_kpair = 0) {
+                                              int split_kpair = 0, int nbuf = 2) {
   Ctl* ctl = a.ctl;
   __nv_bfloat16* tile =
       reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(xchg) + kXchgBytes);
@@ -258,8 +260,10 @@ __device__ __forceinline__ void epilogue_role(const ExpertArgs& a, const UnitInf
       ur = 0;
       uphase ^= 1;
     }
-    acc ^= 1;
-    if (acc == 0) aphase ^= 1;
+    if (++acc == nbuf) {
+      acc = 0;
+      aphase ^= 1;
+    }
   }
 }
 
