@@ -21,7 +21,8 @@ from ._abi import (  # noqa: F401
     moe_forward_noalloc,
     moe_route, moe_plan_routing, moe_plan_sync_status, moe_plan_profile, moe_plan_destroy,
     moe_status_str, moe_lmhead_create, moe_lmhead_forward, moe_lmhead_sync_status,
-    moe_lmhead_destroy, moe_lmhead_set_profile, moe_lmhead_profile,
+    moe_lmhead_destroy, moe_lmhead_set_profile, moe_lmhead_profile, moe_ep_dispatch,
+    moe_expert_rows, moe_combine_rows,
 )
 
 

@@ -49,7 +49,8 @@ EXPORTS = [
     "moe_forward_host", "moe_route", "moe_plan_routing", "moe_plan_sync_status",
     "moe_plan_profile", "moe_plan_destroy", "moe_status_str", "moe_forward_noalloc",
     "moe_lmhead_create", "moe_lmhead_forward", "moe_lmhead_sync_status", "moe_lmhead_destroy",
-    "moe_lmhead_set_profile", "moe_lmhead_profile",
+    "moe_lmhead_set_profile", "moe_lmhead_profile", "moe_ep_dispatch", "moe_expert_rows",
+    "moe_combine_rows",
 ]
 
 _lock = threading.Lock()
@@ -94,6 +95,12 @@ def lib() -> ctypes.CDLL:
             L.moe_plan_destroy.restype = None
             L.moe_forward_noalloc.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P, P, P, P]
             L.moe_forward_noalloc.restype = I
+            L.moe_ep_dispatch.argtypes = [P, I, P, P, I, P, P, P, P, P, P]
+            L.moe_ep_dispatch.restype = I
+            L.moe_expert_rows.argtypes = [P, I, P, P, P, P, P, P, P, P, P]
+            L.moe_expert_rows.restype = I
+            L.moe_combine_rows.argtypes = [P, I, P, P, P, P, P, P]
+            L.moe_combine_rows.restype = I
             L.moe_status_str.argtypes = [I]
             L.moe_status_str.restype = ctypes.c_char_p
             F = ctypes.c_float
@@ -197,6 +204,28 @@ def moe_forward_noalloc(plan, T, x, router_w, router_gamma, router_bias, w_gate_
                                    _ptr(scales_gate_up), _ptr(scales_down), _ptr(residual),
                                    _ptr(out), _ptr(status_out), _stream(stream))
     return _check(st, "moe_forward_noalloc", check)
+
+
+def moe_ep_dispatch(plan, T, x, idx, n_ranks, expert_gamma, send_rows, send_expert, pos,
+                    send_counts, stream=None, check: bool = True):
+    st = lib().moe_ep_dispatch(plan, T, _ptr(x), _ptr(idx), n_ranks, _ptr(expert_gamma),
+                               _ptr(send_rows), _ptr(send_expert), _ptr(pos), _ptr(send_counts),
+                               _stream(stream))
+    return _check(st, "moe_ep_dispatch", check)
+
+
+def moe_expert_rows(plan, R, x_rows, row_expert, expert_gamma, w_gate_up, w_down, scales_gate_up,
+                    scales_down, y_rows, stream=None, check: bool = True):
+    st = lib().moe_expert_rows(plan, R, _ptr(x_rows), _ptr(row_expert), _ptr(expert_gamma),
+                               _ptr(w_gate_up), _ptr(w_down), _ptr(scales_gate_up),
+                               _ptr(scales_down), _ptr(y_rows), _stream(stream))
+    return _check(st, "moe_expert_rows", check)
+
+
+def moe_combine_rows(plan, T, y_rows, pos, w, residual, out, stream=None, check: bool = True):
+    st = lib().moe_combine_rows(plan, T, _ptr(y_rows), _ptr(pos), _ptr(w), _ptr(residual),
+                                _ptr(out), _stream(stream))
+    return _check(st, "moe_combine_rows", check)
 
 
 def moe_route(plan, T, x, router_w, router_gamma, router_bias, idx_out, w_out, gap_out,

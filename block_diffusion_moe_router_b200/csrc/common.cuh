@@ -404,11 +404,13 @@ struct GatherArgs {
 struct CombineArgs {
   int T, k, d;
   const int32_t* slot_of;
-  const float* w;
-  const void* y;       // fp32 or bf16 [T*k, d]
+  const float* w;      // [T, k], or NULL: every weight 1
+  const void* y;       // fp32 or bf16 [rows, d]
   int y_bf16;
   const __nv_bfloat16* residual;
   __nv_bfloat16* out;
+  int rows = 0;        // rows of y: a slot outside [0, rows) is clamped and reported
+  Ctl* ctl = nullptr;
 };
 
 struct ExpertArgs {
@@ -566,6 +568,11 @@ cudaError_t moe_launch_gather(const moe::GatherArgs& a, int num_sms, cudaStream_
 cudaError_t moe_launch_plan_gather(const moe::PlanArgs& a, const moe::GatherArgs& g, int num_sms,
                                    cudaStream_t s, bool pdl);
 cudaError_t moe_launch_combine(const moe::CombineArgs& a, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_ep_keys(const int32_t* idx, int A, int E, int per, int32_t* keys,
+                               moe::Ctl* ctl, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t moe_launch_ep_meta(const int32_t* idx, const int32_t* pos, const int32_t* offsets,
+                               int A, int E, int per, int ranks, int32_t* send_expert,
+                               int32_t* send_counts, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t moe_launch_expert(const moe::ExpertArgs& a, const CUtensorMap& tm_wgu,
                               const CUtensorMap& tm_wd, const CUtensorMap& tm_xp,
                               const CUtensorMap& tm_h, int num_sms, cudaStream_t s, bool pdl);

@@ -508,12 +508,20 @@ moe_status_t moe_route(moe_plan_t p, int T, const void* x, const float* router_w
                        static_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router_w,
-                         const float* router_gamma, const float* router_bias,
-                         const float* expert_gamma, const void* w_gate_up, const void* w_down, const void* scales_gate_up,
-                         const void* scales_down, const void* residual, void* out, void* stream) {
-  moe_status_t st = validate_route(p, T, x, router_w, router_gamma, router_bias);
-  if (st != MOE_OK || T == 0) return st;
+}  // extern "C"
+
+namespace {
+
+// The layer, or (row_expert != NULL) its expert part alone: rows x[t] routed
+// to expert row_expert[t] with weight 1 (a plan with k == 1), no router.
+// The router arguments are validated by the caller.
+moe_status_t forward_impl(moe_plan_t p, int T, const void* x, const float* router_w,
+                          const float* router_gamma, const float* router_bias,
+                          const int32_t* row_expert, const float* expert_gamma,
+                          const void* w_gate_up, const void* w_down, const void* scales_gate_up,
+                          const void* scales_down, const void* residual, void* out,
+                          cudaStream_t s) {
+  moe_status_t st = MOE_OK;
   if (!w_gate_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   if (expert_gamma && !aligned16(expert_gamma)) return MOE_ERR_INVALID_ARG;
@@ -527,7 +535,6 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   const size_t act = (size_t)T * p->d * 2;
   if (overlap(out, act, x, act)) return MOE_ERR_INVALID_ARG;
   if (residual && residual != out && overlap(out, act, residual, act)) return MOE_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = ensure_workspace(p, T, s);
   if (st != MOE_OK) return st;
 
@@ -557,9 +564,11 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
             make_map_bf16(&tm_h, p->h, (uint64_t)A, p->f, moe::kBRows);
   if (!maps_ok) return MOE_ERR_CUDA;
 
-  st = launch_router(p, T, x, router_w, router_gamma, router_bias, p->idx, p->w, p->gap, s,
-                     w_gate_up, prefetch_bytes(p));
-  if (st != MOE_OK) return st;
+  if (!row_expert) {
+    st = launch_router(p, T, x, router_w, router_gamma, router_bias, p->idx, p->w, p->gap, s,
+                       w_gate_up, prefetch_bytes(p));
+    if (st != MOE_OK) return st;
+  }
 
   moe::PlanArgs pa;
   pa.T = T;
@@ -568,7 +577,7 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   pa.d = p->d;
   pa.f = p->f;
   pa.chunk = chunk_size(p);
-  pa.idx = p->idx;
+  pa.idx = row_expert ? row_expert : p->idx;
   pa.offsets = p->offsets;
   pa.perm = p->perm;
   pa.slot_of = p->slot_of;
@@ -628,11 +637,13 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
   ca.k = p->k;
   ca.d = p->d;
   ca.slot_of = p->slot_of;
-  ca.w = p->w;
+  ca.w = row_expert ? nullptr : p->w;
   ca.y = p->y;
   ca.y_bf16 = p->y_bf16;
   ca.residual = static_cast<const __nv_bfloat16*>(residual);
   ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.rows = A;
+  ca.ctl = p->ctl;
   {
     ProfScope ps(p, MOE_K_COMBINE, s);
     if (moe_launch_combine(ca, p->num_sms, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
@@ -640,6 +651,138 @@ moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router
 
   p->last_T = T;
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_forward(moe_plan_t p, int T, const void* x, const float* router_w,
+                         const float* router_gamma, const float* router_bias,
+                         const float* expert_gamma, const void* w_gate_up, const void* w_down,
+                         const void* scales_gate_up, const void* scales_down, const void* residual,
+                         void* out, void* stream) {
+  moe_status_t st = validate_route(p, T, x, router_w, router_gamma, router_bias);
+  if (st != MOE_OK || T == 0) return st;
+  return forward_impl(p, T, x, router_w, router_gamma, router_bias, nullptr, expert_gamma,
+                      w_gate_up, w_down, scales_gate_up, scales_down, residual, out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_rows(moe_plan_t p, int R, const void* x_rows, const int32_t* row_expert,
+                             const float* expert_gamma, const void* w_gate_up, const void* w_down,
+                             const void* scales_gate_up, const void* scales_down, void* y_rows,
+                             void* stream) {
+  if (!p || R < 0) return MOE_ERR_INVALID_ARG;
+  if (p->k != 1) return MOE_ERR_INVALID_ARG;
+  if (R == 0) return MOE_OK;
+  if (!tokens_ok(p, R)) return MOE_ERR_UNSUPPORTED;
+  if (!x_rows || !row_expert || !aligned16(x_rows) ||
+      (reinterpret_cast<uintptr_t>(row_expert) & 3u))
+    return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device(p);
+  if (st != MOE_OK) return st;
+  return forward_impl(p, R, x_rows, nullptr, nullptr, nullptr, row_expert, expert_gamma,
+                      w_gate_up, w_down, scales_gate_up, scales_down, nullptr, y_rows,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_ep_dispatch(moe_plan_t p, int T, const void* x, const int32_t* idx, int n_ranks,
+                             const float* expert_gamma, void* send_rows, int32_t* send_expert,
+                             int32_t* pos, int32_t* send_counts, void* stream) {
+  if (!p || T < 0) return MOE_ERR_INVALID_ARG;
+  if (n_ranks < 1 || n_ranks > p->E || n_ranks > moe::kMaxE || p->E % n_ranks != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!send_counts || (reinterpret_cast<uintptr_t>(send_counts) & 3u)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    moe_status_t st = check_device(p);
+    if (st != MOE_OK) return st;
+    return cudaMemsetAsync(send_counts, 0, (size_t)n_ranks * 4, s) == cudaSuccess ? MOE_OK
+                                                                                    : MOE_ERR_CUDA;
+  }
+  if (!tokens_ok(p, T)) return MOE_ERR_UNSUPPORTED;
+  if (!x || !idx || !send_rows || !send_expert || !pos) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(send_rows) || (expert_gamma && !aligned16(expert_gamma)) ||
+      ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(send_expert) |
+        reinterpret_cast<uintptr_t>(pos)) & 3u))
+    return MOE_ERR_INVALID_ARG;
+  const size_t A = (size_t)T * p->k;
+  if (overlap(send_rows, A * p->d * 2, x, (size_t)T * p->d * 2)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device(p);
+  if (st != MOE_OK) return st;
+  st = ensure_workspace(p, T, s);
+  if (st != MOE_OK) return st;
+  const bool pdl = p->pdl != 0;
+  const int per = p->E / n_ranks;
+  // owner keys into the plan workspace, then the plan keyed by owner: pos is
+  // the plan's slot of every assignment, perm the token of every send row
+  if (moe_launch_ep_keys(idx, (int)A, p->E, per, p->idx, p->ctl, p->num_sms, s, pdl) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  moe::PlanArgs pa;
+  pa.T = T;
+  pa.E = n_ranks;
+  pa.k = p->k;
+  pa.d = p->d;
+  pa.f = p->f;
+  pa.chunk = chunk_size(p);
+  pa.idx = p->idx;
+  pa.offsets = p->offsets;
+  pa.perm = p->perm;
+  pa.slot_of = pos;
+  pa.chunk_info = p->chunk_info;
+  pa.ready = p->ready;
+  pa.ctl = p->ctl;
+  if (moe_launch_plan(pa, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
+  moe::GatherArgs ga;
+  ga.rows = (int)A;
+  ga.d = p->d;
+  ga.eps = p->eps;
+  ga.gamma2 = expert_gamma;
+  ga.perm = p->perm;
+  ga.x = static_cast<const __nv_bfloat16*>(x);
+  ga.x_perm = static_cast<__nv_bfloat16*>(send_rows);
+  ga.xf16 = 0;
+  if (moe_launch_gather(ga, p->num_sms, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe_launch_ep_meta(idx, pos, p->offsets, (int)A, p->E, per, n_ranks, send_expert,
+                         send_counts, p->num_sms, s, pdl) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_combine_rows(moe_plan_t p, int T, const void* y_rows, const int32_t* pos,
+                              const float* w, const void* residual, void* out, void* stream) {
+  if (!p || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!tokens_ok(p, T)) return MOE_ERR_UNSUPPORTED;
+  if (!y_rows || !pos || !w || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_rows) || !aligned16(out) || (residual && !aligned16(residual)) ||
+      ((reinterpret_cast<uintptr_t>(pos) | reinterpret_cast<uintptr_t>(w)) & 3u))
+    return MOE_ERR_INVALID_ARG;
+  const size_t act = (size_t)T * p->d * 2;
+  const size_t A = (size_t)T * p->k;
+  if (overlap(out, act, y_rows, A * p->d * 2)) return MOE_ERR_INVALID_ARG;
+  if (residual && residual != out && overlap(out, act, residual, act)) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device(p);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = ensure_workspace(p, 1, s);  // the status word
+  if (st != MOE_OK) return st;
+  moe::CombineArgs ca;
+  ca.T = T;
+  ca.k = p->k;
+  ca.d = p->d;
+  ca.slot_of = pos;
+  ca.w = w;
+  ca.y = y_rows;
+  ca.y_bf16 = 1;
+  ca.residual = static_cast<const __nv_bfloat16*>(residual);
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.rows = (int)A;
+  ca.ctl = p->ctl;
+  return moe_launch_combine(ca, p->num_sms, s, p->pdl != 0) == cudaSuccess ? MOE_OK
+                                                                           : MOE_ERR_CUDA;
 }
 
 moe_status_t moe_forward_host(moe_plan_t p, int T, const void* x_host, const float* router_w,
@@ -949,6 +1092,8 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   ca.y_bf16 = p->y_bf16;
   ca.residual = static_cast<const __nv_bfloat16*>(residual);
   ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.rows = (int)A;
+  ca.ctl = ctl;
   if (moe_launch_combine(ca, p->num_sms, s, p->pdl != 0) != cudaSuccess) return MOE_ERR_CUDA;
 
   if (status_out && cudaMemcpyAsync(status_out, &ctl->status, sizeof(int32_t),

@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(kSmallT) plan_gather_small_kernel(PlanArgs a, 
 }
 
 // out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32, one
-// rounding).  One token per CTA step (grid-stride over tokens, a few CTAs per
+// rounding; w NULL: every weight 1, so with k = 1 a row is copied exactly).  One token per CTA step (grid-stride over tokens, a few CTAs per
 // SM, so the whole grid is resident at once); a thread owns up to kCombCols
 // 16-byte column groups of the row and issues the loads of up to kCombK
 // contributions per column group before accumulating them.  slot_of and w of
@@ -543,6 +543,15 @@ __device__ __forceinline__ void widen(const uint4& r, const __nv_bfloat16*, floa
   }
 }
 
+// A slot outside the y rows is clamped (and reported) instead of read.
+__device__ __forceinline__ int checked_slot(const CombineArgs& a, int sl) {
+  if (a.rows > 0 && (sl < 0 || sl >= a.rows)) {
+    if (a.ctl) record_error(a.ctl, MOE_ERR_DEVICE_CHECK, 120);
+    return sl < 0 ? 0 : a.rows - 1;
+  }
+  return sl;
+}
+
 template <typename YT>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
   constexpr int V = YVec<YT>::n;
@@ -558,8 +567,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
 #pragma unroll
     for (int j = 0; j < kCombK; ++j) {
       const bool in = t < a.T && j < a.k;
-      sl0[j] = in ? __ldg(a.slot_of + (size_t)t * a.k + j) : 0;
-      wt0[j] = in ? __ldg(a.w + (size_t)t * a.k + j) : 0.f;
+      sl0[j] = in ? checked_slot(a, __ldg(a.slot_of + (size_t)t * a.k + j)) : 0;
+      wt0[j] = in ? (a.w ? __ldg(a.w + (size_t)t * a.k + j) : 1.f) : 0.f;
     }
   }
   pdl_wait();  // y comes from the expert kernel
@@ -578,8 +587,11 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
       const bool pre = t == (int)blockIdx.x && j0 == 0;
 #pragma unroll
       for (int j = 0; j < kCombK; ++j) {
-        sl[j] = pre ? sl0[j] : (j0 + j < a.k) ? __ldg(a.slot_of + (size_t)t * a.k + j0 + j) : 0;
-        wt[j] = pre ? wt0[j] : (j0 + j < a.k) ? __ldg(a.w + (size_t)t * a.k + j0 + j) : 0.f;
+        sl[j] = pre ? sl0[j]
+                    : (j0 + j < a.k) ? checked_slot(a, __ldg(a.slot_of + (size_t)t * a.k + j0 + j))
+                                     : 0;
+        wt[j] = pre ? wt0[j]
+                    : (j0 + j < a.k) ? (a.w ? __ldg(a.w + (size_t)t * a.k + j0 + j) : 1.f) : 0.f;
       }
 #pragma unroll
       for (int q = 0; q < kCombCols; ++q) {
@@ -629,6 +641,45 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(CombineArgs a) {
         *reinterpret_cast<uint2*>(a.out + o + i) = ov;
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------- expert parallel
+// Dispatch of the token-expert assignments to the ranks that own the experts
+// (rank r owns experts [r * per, (r + 1) * per)): the assignments are sorted
+// by owner with the plan kernel, keyed by owner instead of expert, so each
+// owner's rows are contiguous and in (token, j) order.
+
+// keys[a] = idx[a] / per (the owner of the assignment's expert).
+__global__ void __launch_bounds__(256) ep_keys_kernel(const int32_t* idx, int A, int E, int per,
+                                                      int32_t* keys, Ctl* ctl) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A; i += gridDim.x * blockDim.x) {
+    int e = idx[i];
+    if (e < 0 || e >= E) {
+      record_error(ctl, MOE_ERR_DEVICE_CHECK, 110);
+      e = 0;
+    }
+    keys[i] = e / per;
+  }
+}
+
+// send_expert[pos[a]] = idx[a] % per (the expert's index on its owner), and
+// send_counts[r] = rows for owner r.
+__global__ void __launch_bounds__(256) ep_meta_kernel(const int32_t* idx, const int32_t* pos,
+                                                      const int32_t* offsets, int A, int E, int per,
+                                                      int ranks, int32_t* send_expert,
+                                                      int32_t* send_counts) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int i0 = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i0 < ranks) send_counts[i0] = offsets[i0 + 1] - offsets[i0];
+  for (int i = i0; i < A; i += gridDim.x * blockDim.x) {
+    int e = idx[i];
+    if (e < 0 || e >= E) e = 0;
+    const int p = pos[i];
+    if (p >= 0 && p < A) send_expert[p] = e % per;
   }
 }
 
@@ -698,4 +749,21 @@ cudaError_t moe_launch_combine(const moe::CombineArgs& a, int num_sms, cudaStrea
                            s, pdl, a);
   return moe::launch_pdl(moe::combine_kernel<float>, grid, dim3(moe::kCombThreads), 0, s, pdl,
                          a);
+}
+
+cudaError_t moe_launch_ep_keys(const int32_t* idx, int A, int E, int per, int32_t* keys,
+                               moe::Ctl* ctl, int num_sms, cudaStream_t s, bool pdl) {
+  if (A == 0) return cudaSuccess;
+  const int blocks = std::max(1, std::min((A + 255) / 256, 4 * std::max(num_sms, 1)));
+  return moe::launch_pdl(moe::ep_keys_kernel, dim3(blocks), dim3(256), 0, s, pdl, idx, A, E, per,
+                         keys, ctl);
+}
+
+cudaError_t moe_launch_ep_meta(const int32_t* idx, const int32_t* pos, const int32_t* offsets,
+                               int A, int E, int per, int ranks, int32_t* send_expert,
+                               int32_t* send_counts, int num_sms, cudaStream_t s, bool pdl) {
+  const int n = std::max(A, ranks);
+  const int blocks = std::max(1, std::min((n + 255) / 256, 4 * std::max(num_sms, 1)));
+  return moe::launch_pdl(moe::ep_meta_kernel, dim3(blocks), dim3(256), 0, s, pdl, idx, pos,
+                         offsets, A, E, per, ranks, send_expert, send_counts);
 }

@@ -245,6 +245,76 @@ moe_status_t moe_route(moe_plan_t plan, int T, const void* x, const float* route
                        const float* router_gamma, const float* router_bias, int32_t* idx_out,
                        float* w_out, float* gap_out, void* stream);
 
+/* ---- expert parallelism over the GPUs of one node -----------------------
+ *
+ * The pages run the whole model on one device (Hugging Face card
+ * "Infatoshi/diffusiongemma-26B-A4B-iq2xxs-4070": every layer offloaded to one
+ * card; auto-round pull request, transformers backend test log: one GPU).
+ * These three calls are the library's own extension that spreads each
+ * layer's experts
+ * over N ranks of one node, rank r owning experts [r*E/N, (r+1)*E/N).
+ * The pages' model has 128 experts with 8 active per token (Quant-Tuner pull
+ * request, Summary; the ROCmFP4-GGUF card's header).  A layer call is:
+ *   1. moe_route (every rank, its own tokens) -> idx, w;
+ *   2. moe_ep_dispatch: the token-expert assignments sorted by owner, each
+ *      owner's rows contiguous in (token, j) order, x rows packed to match;
+ *   3. the caller exchanges counts, rows and expert ids with an all-to-all
+ *      (e.g. NCCL through torch.distributed; no library kernel reads another
+ *      GPU's memory);
+ *   4. moe_expert_rows on every owner (a plan of its E/N experts, k = 1):
+ *      y rows in the order received;
+ *   5. the caller returns the y rows with the reverse all-to-all;
+ *   6. moe_combine_rows: out_t = residual_t + sum_j w_tj y_(t,j) in j order.
+ * With bf16 y rows (MOE_OPT_Y_BF16 on, the default) every rank's out equals
+ * moe_forward's bytes for bf16 and int4 weights (and for fp8 / fp4 weights
+ * without expert_gamma: those paths carry fp16 rows, and a row normalised
+ * on the sender travels as bf16), provided the bf16 expert kernel takes the
+ * same accumulation in both: it splits K between two issuing threads when
+ * every expert chunk of the call has at most 128 tokens and not otherwise,
+ * so an owner whose chunks are all small can round differently from a
+ * moe_forward call that also holds a larger chunk (within the layer's
+ * tolerance either way). */
+
+/* Step 2, on the routing plan (E experts, top-k) of the sending rank.
+ *   x             bf16 [T, d]  the rank's tokens
+ *   idx           int32 [T, k] the experts moe_route chose
+ *   n_ranks       owners; E % n_ranks == 0, 1 <= n_ranks <= min(E, 256)
+ *   expert_gamma  fp32 [d] or NULL: rows are sent as the expert-side RMSNorm
+ *                 of x (as in moe_forward), else as x
+ *   send_rows     bf16 [T*k, d] out: rows for owner 0, then owner 1, ...
+ *   send_expert   int32 [T*k] out: each send row's expert index on its owner
+ *   pos           int32 [T*k] out: send row of assignment t*k + j
+ *   send_counts   int32 [n_ranks] out (device): rows for each owner
+ * Asynchronous on `stream`; an expert id outside [0, E) is reported as
+ * MOE_ERR_DEVICE_CHECK by moe_plan_sync_status. */
+moe_status_t moe_ep_dispatch(moe_plan_t plan, int T, const void* x, const int32_t* idx,
+                             int n_ranks, const float* expert_gamma, void* send_rows,
+                             int32_t* send_expert, int32_t* pos, int32_t* send_counts,
+                             void* stream);
+
+/* Step 4, on a plan created with the owner's expert count and k = 1: y_rows[r]
+ * = expert row_expert[r] applied to x_rows[r] (gate_up, GELU-tanh * up,
+ * down), rounded to bf16.  Weights and scales are the owner's slice of the
+ * layer's tensors, laid out as for moe_forward.
+ *   x_rows        bf16 [R, d]   rows as received (already normalised)
+ *   row_expert    int32 [R]     expert of each row on this owner, [0, E)
+ *   expert_gamma  fp32 [d] or NULL (normally NULL: the sender normalised)
+ *   y_rows        bf16 [R, d]   out, same row order
+ * R = 0 is a no-op.  A plan with k != 1 returns MOE_ERR_INVALID_ARG. */
+moe_status_t moe_expert_rows(moe_plan_t plan, int R, const void* x_rows, const int32_t* row_expert,
+                             const float* expert_gamma, const void* w_gate_up, const void* w_down,
+                             const void* scales_gate_up, const void* scales_down, void* y_rows,
+                             void* stream);
+
+/* Step 6, on the sending rank's routing plan: out_t = residual_t + sum_j
+ * w[t,j] * y_rows[pos[t*k+j]], j in order, fp32, one rounding to bf16.
+ *   y_rows    bf16 [T*k, d] the returned rows, in send order
+ *   pos, w    from moe_ep_dispatch / moe_route
+ *   residual  bf16 [T, d] or NULL; may alias out
+ * A pos outside [0, T*k) is clamped and reported as MOE_ERR_DEVICE_CHECK. */
+moe_status_t moe_combine_rows(moe_plan_t plan, int T, const void* y_rows, const int32_t* pos,
+                              const float* w, const void* residual, void* out, void* stream);
+
 /* Device-to-device copies of the last moe_forward's routing tables (NULL to
  * skip one): offsets int32 [E+1] (expert segment starts in slot order),
  * perm int32 [T*k] (token of each slot), slot_of int32 [T*k] (slot of
