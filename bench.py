@@ -238,16 +238,39 @@ def cpu_model() -> str:
     return platform.processor() or "unknown"
 
 
+def oracle_f32_sample_rate(lay_cpu, k, n_tokens, eps=1e-6):
+    """Tokens/s of the oracle's single-precision timing build on the first
+    n_tokens rows (all host threads)."""
+    import oracle
+    x = lay_cpu["x"][:n_tokens]
+    t0 = time.perf_counter()
+    oracle.moe_forward_f32(x, lay_cpu["router_w"], lay_cpu["router_gamma"],
+                           lay_cpu.get("router_bias"), lay_cpu["w_gate_up"], lay_cpu["w_down"], k,
+                           scales_gate_up=lay_cpu.get("scales_gate_up"),
+                           scales_down=lay_cpu.get("scales_down"), eps=eps,
+                           expert_gamma=lay_cpu.get("expert_gamma"))
+    return n_tokens / (time.perf_counter() - t0)
+
+
 def cpu_baseline(lay_cpu, w, budget_s=12.0):
+    """The fp64 oracle as it stands (the value), and beside it the same
+    definition compiled in single precision, each on a bounded sample."""
     import oracle
     cores = oracle.get_threads()
     probe = max(1, min(w.T, cores))
     r = oracle_sample_rate(lay_cpu, w.k, probe)
     n = int(max(probe, min(w.T, round(r * budget_s / cores) * cores)))
     r = oracle_sample_rate(lay_cpu, w.k, n)
+    oracle.build_f32()
+    r32 = oracle_f32_sample_rate(lay_cpu, w.k, probe)
+    n32 = int(max(probe, min(w.T, round(r32 * budget_s / 2 / cores) * cores)))
+    r32 = oracle_f32_sample_rate(lay_cpu, w.k, n32)
     return {"value": r, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "cpu_model": cpu_model(), "omp_threads": cores, "host_cpus": os.cpu_count(),
-            "sample": f"first {n} of the {w.T} canvas tokens, fp64 oracle, one layer"}
+            "sample": f"first {n} of the {w.T} canvas tokens, fp64 oracle, one layer",
+            "fp32_timing_build": {"value": r32, "unit": "tokens/s",
+                                  "sample": f"first {n32} of the {w.T} canvas tokens, the "
+                                            f"oracle compiled in single precision, one layer"}}
 
 
 # ---------------------------------------------------------------- arms

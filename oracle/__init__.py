@@ -13,6 +13,8 @@ from .oracle import (  # noqa: F401
     route_weights,
     route,
     moe_forward,
+    moe_forward_f32,
+    build_f32,
     expert_ffn,
     weight_row,
     decode_bf16,

@@ -38,6 +38,67 @@ def build(force: bool = False) -> str:
     return _SO
 
 
+_SRC32 = os.path.join(_HERE, "moe_oracle_f32.c")
+_SO32 = os.path.join(_BUILD, "liboracle_f32.so")
+_lib32 = None
+
+
+def build_f32(force: bool = False) -> str:
+    """Compile the single-precision timing build (moe_oracle_f32.c, which
+    includes moe_oracle.c with every double made a float)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC32))
+    if force or not os.path.exists(_SO32) or os.path.getmtime(_SO32) < newest:
+        tmp = _SO32 + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-D_DEFAULT_SOURCE", "-fPIC", "-shared", "-fopenmp",
+               "-fno-fast-math", "-Wall", "-o", tmp, _SRC32, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _SO32)
+    return _SO32
+
+
+def lib_f32():
+    """The timing build: the same entry points with float arguments."""
+    global _lib32
+    with _lock:
+        if _lib32 is None:
+            build_f32()
+            L = ctypes.CDLL(_SO32)
+            P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+            L.oracle_moe_forward.argtypes = [I, I, I, I, I, I, P, P, P, P, P, F, P, P, P, P, P,
+                                             P, P, P, P, P]
+            L.oracle_set_threads.argtypes = [I]
+            L.oracle_get_threads.restype = I
+            _lib32 = L
+    return _lib32
+
+
+def moe_forward_f32(x, router_w, router_gamma, router_bias, w_gate_up, w_down, k: int,
+                    scales_gate_up=None, scales_down=None, residual=None, eps: float = 1e-6,
+                    expert_gamma=None):
+    """The whole layer in single precision (timing build): out [T,d] float32."""
+    x = _np(x)
+    rw = _np(router_w, np.float32)
+    g = _np(router_gamma, np.float32)
+    b = _np(router_bias, np.float32)
+    wgu = _np(w_gate_up)
+    wd = _np(w_down)
+    sgu = _np(scales_gate_up)
+    sd = _np(scales_down)
+    res = _np(residual)
+    eg = _np(expert_gamma, np.float32)
+    T, d = x.shape
+    E = rw.shape[0]
+    out = np.empty((T, d), np.float32)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    gap = np.empty(T, np.float32)
+    lib_f32().oracle_moe_forward(T, E, k, d, wgu.shape[1] // 2, _wdtype(wgu, sgu), _p(x), _p(rw),
+                                 _p(g), _p(b), _p(eg), float(eps), _p(wgu), _p(wd), _p(sgu),
+                                 _p(sd), _p(res), None, _p(out), _p(idx), _p(w), _p(gap))
+    return out
+
+
 def lib():
     global _lib
     with _lock:

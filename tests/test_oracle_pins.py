@@ -521,3 +521,18 @@ def test_fp4_weight_row_closed_form():
     ref[0], ref[1], ref[17], ref[63] = 0.5, -3.0, 6.0, -0.0625
     np.testing.assert_array_equal(row, ref)
     assert np.all(oracle.weight_row(codes, rec.contiguous(), 0, 2, C) == 0)
+
+
+def test_single_precision_timing_build_computes_the_same_layer():
+    """The fp32 build the bench times beside the fp64 oracle is the same
+    definition in single precision: on a tiny layer its output agrees with
+    the fp64 oracle to single-precision accuracy (it is never a reference)."""
+    lay = inputs.make_small(T=12, d=256, E=16, k=4, f=64, seed=404, bias=True, residual=True)
+    ref, _, _, _ = oracle.moe_forward(lay["x"], lay["router_w"], lay["router_gamma"],
+                                      lay["router_bias"], lay["w_gate_up"], lay["w_down"], 4,
+                                      residual=lay["residual"])
+    got = oracle.moe_forward_f32(lay["x"], lay["router_w"], lay["router_gamma"],
+                                 lay["router_bias"], lay["w_gate_up"], lay["w_down"], 4,
+                                 residual=lay["residual"])
+    err = np.linalg.norm(got.astype(np.float64) - ref) / np.linalg.norm(ref)
+    assert err < 1e-5, err
