@@ -26,10 +26,10 @@
 // is (below N ~ 180), which at 4 UMMAs per 64-wide K stage is slower than a
 // stage's share of the weight stream once the chunks grow past ~100 tokens;
 // UMMAs from two threads overlap, so, while every chunk has at most 128
-// tokens (a canvas), the two issuers split K: warp 1 takes the even K stages
-// of every unit and warp 7 the odd ones, each into its own partial
-// accumulator, and the epilogue adds the two partials (fixed order, so the
-// result does not depend on timing).  With larger chunks the two partials of
+// tokens (a canvas), the two issuers split K: warp 1 takes the stages of
+// even global index and warp 7 those of odd index, each into its own
+// partial accumulator, and the epilogue adds the two partials (fixed order,
+// so the result does not depend on timing).  With larger chunks the two partials of
 // a unit would fill half of TMEM and the epilogue would stall the tensor
 // cores at every unit, so warp 1 issues alone.  Weights and activations have rings of their own,
 // sized at run time from the largest chunk: the weight ring is deep, since
@@ -57,7 +57,7 @@ constexpr int kMaxB = 8;   // activation stages
 constexpr int kMinB = 3;  // 2 when rounded down to even
 constexpr int kRingBytes = 200 * 1024;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
-constexpr int kBarBytes = 8 * (2 * kMaxA + 2 * kMaxB + 4 + 2 * kUnitRing + 2);
+constexpr int kBarBytes = 8 * (2 * kMaxA + 2 * kMaxB + 4 + 2 * kUnitRing + 3);
 constexpr int kSmemBytes = 1024 + kRingBytes + kEpiBytes + kBarBytes + 256;
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* ufull = tempty + 2;
   uint64_t* uempty = ufull + kUnitRing;
   uint64_t* drain = uempty + kUnitRing;
-  UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 2);
+  uint64_t* meet = drain + 2;  // the two UMMA issuers' end-of-unit rendezvous
+  UnitInfo* units = reinterpret_cast<UnitInfo*>(drain + 3);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(units + kUnitRing);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* s_bcast = reinterpret_cast<volatile int*>(tmem_slot + 2);
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(meet, 2);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -133,12 +135,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The activation ring takes kMinB..kMaxB stages (as many as fit half of
   // the ring: at 2048 tokens a chunk's B stage is larger than its A stage
   // and its L2 latency must be hidden too), the weights the rest.  When two
-  // issuers split K (splitk, below) both depths are even: a ring slot then
-  // always holds stages of the same issuer (global stage parity), so an
-  // issuer waiting on its stage q has itself consumed stage q - depth in
-  // that slot and the parity wait cannot be satisfied by a phase two behind
-  // (with an odd depth the slot's previous stage belongs to the other issuer
-  // and may still be in flight).
+  // issuers split K (splitk, below) both depths are even, so within a unit
+  // a ring slot comes back to the same issuer; across units the issuers'
+  // end-of-unit rendezvous covers it (see there).  Without both, an issuer
+  // could wait on a slot whose previous stage belongs to the other issuer
+  // and is still in flight, and its parity wait would pass a phase early.
   const int maxn = max(1, min(kMaxN, ctl->max_chunk));
   const bool splitk = maxn <= 128;
   const int even = splitk ? ~1 : ~0;
@@ -267,13 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 2), so neither can run a phase ahead of the epilogue.
     if (lane == 0) {
       const int par = warp == 1 ? 0 : 1;
-      const int first = splitk ? par : (par == 0 ? 0 : 1 << 30);  // this issuer's first stage
       const int step = splitk ? 2 : 1;
       int g = 0;  // ring stages used by all earlier units
       int ur = 0;
       uint32_t uphase = 0;
       int buf = 0;
       uint32_t bphase = 0;
+      uint32_t mphase = 0;
       while (true) {
         if (!mbar_wait(&ufull[ur], uphase, s_abort, ctl, a.timeout_ns, kWhereUnitFullMma)) break;
         const UnitInfo ui = units[ur];
@@ -284,7 +285,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&tempty[buf], bphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereTmemEmpty))
           break;
         tc_fence_after();
-        const uint32_t dt = tmem_base + (uint32_t)(buf * ACC + (splitk ? par * W : 0));
+        // This issuer's first stage of the unit (split K by the stage's
+        // parity inside the unit, so a unit's result does not depend on the
+        // order the units were claimed in); a unit of one stage has no
+        // second partial, and its one stage lands in columns [0, W).
+        const int first = splitk ? par : (par == 0 ? 0 : 1 << 30);
+        const uint32_t dt =
+            tmem_base + (uint32_t)(buf * ACC + (splitk && nkb > 1 ? par * W : 0));
         const int g0 = g + (first < nkb ? first : 0);
         int sa_i = g0 % SA, sb_i = g0 % SB;
         uint32_t pa = (uint32_t)(g0 / SA) & 1u, pb = (uint32_t)(g0 / SB) & 1u;
@@ -316,6 +323,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
+        // The two issuers meet at the end of every unit: a ring slot then
+        // holds, before it comes back to an issuer, either its own stage of
+        // the same unit (the depths are even) or a stage of an earlier unit
+        // that both issuers have waited on, so no parity wait can be
+        // satisfied by a phase two behind.
+        mbar_arrive(meet);
+        if (!mbar_wait(meet, mphase, s_abort, ctl, a.timeout_ns, kWhereStageFull)) break;
+        mphase ^= 1;
         umma_commit(&tfull[buf]);
         mbar_arrive(&uempty[ur]);
         g += nkb;
