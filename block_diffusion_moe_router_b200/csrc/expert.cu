@@ -25,13 +25,12 @@
 // issuing thread sustains one M=128 K=16 UMMA per ~90-110 cycles whatever N
 // is (below N ~ 180), which at 4 UMMAs per 64-wide K stage is slower than a
 // stage's share of the weight stream once the chunks grow past ~100 tokens;
-// UMMAs from two threads overlap, so, while every chunk has at most 128
-// tokens (a canvas), the two issuers split K: warp 1 takes the stages of
-// even global index and warp 7 those of odd index, each into its own
-// partial accumulator, and the epilogue adds the two partials (fixed order,
-// so the result does not depend on timing).  With larger chunks the two partials of
-// a unit would fill half of TMEM and the epilogue would stall the tensor
-// cores at every unit, so warp 1 issues alone.  Weights and activations have rings of their own,
+// UMMAs from two threads overlap, so for every unit of at most 128 tokens
+// the two issuers split K: warp 1 takes the unit's even K stages and warp 7
+// the odd ones, each into its own 128-column partial, and the epilogue adds
+// the two partials (fixed order, so the result does not depend on timing).
+// A larger unit's partials would not leave TMEM room for a second unit in
+// flight, so warp 1 issues it alone into 256 columns.  Weights and activations have rings of their own,
 // sized at run time from the largest chunk: the weight ring is deep, since
 // its tiles come from HBM and are the bytes the kernel exists to stream,
 // while the activation tiles come from L2.  So the weights of a unit keep
@@ -134,29 +133,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   // B-operand rows per stage: the largest chunk, rounded up to the TMA box.
   // The activation ring takes kMinB..kMaxB stages (as many as fit half of
   // the ring: at 2048 tokens a chunk's B stage is larger than its A stage
-  // and its L2 latency must be hidden too), the weights the rest.  When two
-  // issuers split K (splitk, below) both depths are even, so within a unit
-  // a ring slot comes back to the same issuer; across units the issuers'
-  // end-of-unit rendezvous covers it (see there).  Without both, an issuer
-  // could wait on a slot whose previous stage belongs to the other issuer
-  // and is still in flight, and its parity wait would pass a phase early.
+  // and its L2 latency must be hidden too), the weights the rest.  Both
+  // depths are even, so within a unit whose K is split a ring slot comes
+  // back to the same issuer; across units the issuers' end-of-unit
+  // rendezvous covers it (see there).  Without both, an issuer could wait on
+  // a slot whose previous stage belongs to the other issuer and is still in
+  // flight, and its parity wait would pass a phase early.
   const int maxn = max(1, min(kMaxN, ctl->max_chunk));
-  const bool splitk = maxn <= 128;
-  const int even = splitk ? ~1 : ~0;
   const int NB = (maxn + kBRows - 1) / kBRows * kBRows;
   const int b_bytes = NB * kBK * 2;
-  const int SB = min(kMaxB, max(kMinB, (kRingBytes / 2) / b_bytes)) & even;
-  const int SA = min(kMaxA, (kRingBytes - SB * b_bytes) / kABytes) & even;
+  const int SB = min(kMaxB, max(kMinB, (kRingBytes / 2) / b_bytes)) & ~1;
+  const int SA = min(kMaxA, (kRingBytes - SB * b_bytes) / kABytes) & ~1;
   uint8_t* ringA = ring;
   uint8_t* ringB = ring + SA * kABytes;
-  // Accumulators, two units in flight.  Chunks of at most 128 tokens: the
-  // two issuers split K, each unit holding two partials of 128 columns.
-  // Larger chunks: their partials would leave room for one unit only, and
-  // the epilogue would then stall the tensor cores at every unit, so warp 1
-  // issues every stage into one 256-column accumulator (warp 7 only keeps
-  // the barrier protocol).
-  const int W = splitk ? 128 : kMaxN;      // columns of one partial
-  const int ACC = splitk ? 2 * W : kMaxN;  // columns of one unit's accumulator
+  // Accumulators: two units in flight, 256 columns each.  A unit of at most
+  // 128 tokens (and two or more K stages) has its K split between the two
+  // issuers, each into a 128-column partial; a larger unit is issued by warp
+  // 1 alone into all 256 columns (warp 7 then only keeps the barrier
+  // protocol).  The choice depends on the unit alone, so a unit's result
+  // does not depend on the other units of the call.
+  constexpr int W = 128;                   // columns of one partial
+  constexpr int ACC = kMaxN;               // columns of one unit's accumulator
   const int NBUF = kTmemCols / ACC;        // 2
   const int n_chunks = ctl->n_chunks;
   const int U = n_chunks * (GU + DN);
@@ -268,7 +265,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 2), so neither can run a phase ahead of the epilogue.
     if (lane == 0) {
       const int par = warp == 1 ? 0 : 1;
-      const int step = splitk ? 2 : 1;
       int g = 0;  // ring stages used by all earlier units
       int ur = 0;
       uint32_t uphase = 0;
@@ -285,13 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&tempty[buf], bphase ^ 1, s_abort, ctl, a.timeout_ns, kWhereTmemEmpty))
           break;
         tc_fence_after();
-        // This issuer's first stage of the unit (split K by the stage's
-        // parity inside the unit, so a unit's result does not depend on the
-        // order the units were claimed in); a unit of one stage has no
-        // second partial, and its one stage lands in columns [0, W).
+        // Split K by the stage's parity inside the unit (a unit's result then
+        // does not depend on the order the units were claimed in): this
+        // issuer's first stage and step.  A unit of one stage, or of more
+        // than W tokens, is warp 1's alone, in columns [0, ACC).
+        const bool splitk = nkb > 1 && N <= W;
         const int first = splitk ? par : (par == 0 ? 0 : 1 << 30);
-        const uint32_t dt =
-            tmem_base + (uint32_t)(buf * ACC + (splitk && nkb > 1 ? par * W : 0));
+        const int step = splitk ? 2 : 1;
+        const uint32_t dt = tmem_base + (uint32_t)(buf * ACC + (splitk ? par * W : 0));
         const int g0 = g + (first < nkb ? first : 0);
         int sa_i = g0 % SA, sb_i = g0 % SB;
         uint32_t pa = (uint32_t)(g0 / SA) & 1u, pb = (uint32_t)(g0 / SB) & 1u;
@@ -403,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     epilogue_role(a, units, ufull, uempty, tfull, tempty, xchg, s_abort, s_bcast, tmem_base,
-                  ACC, warp, lane, nullptr, nullptr, splitk ? kBK : 0, NBUF);
+                  ACC, warp, lane, nullptr, nullptr, kBK, NBUF);
   }
 
   tc_fence_before();

@@ -268,12 +268,9 @@ moe_status_t moe_route(moe_plan_t plan, int T, const void* x, const float* route
  * With bf16 y rows (MOE_OPT_Y_BF16 on, the default) every rank's out equals
  * moe_forward's bytes for bf16 and int4 weights (and for fp8 / fp4 weights
  * without expert_gamma: those paths carry fp16 rows, and a row normalised
- * on the sender travels as bf16), provided the bf16 expert kernel takes the
- * same accumulation in both: it splits K between two issuing threads when
- * every expert chunk of the call has at most 128 tokens and not otherwise,
- * so an owner whose chunks are all small can round differently from a
- * moe_forward call that also holds a larger chunk (within the layer's
- * tolerance either way). */
+ * on the sender travels as bf16): an expert's tokens form the same chunks
+ * on the owner as in moe_forward, and the expert kernels' arithmetic for a
+ * chunk depends on that chunk alone. */
 
 /* Step 2, on the routing plan (E experts, top-k) of the sending rank.
  *   x             bf16 [T, d]  the rank's tokens

@@ -1,8 +1,8 @@
 """Expert parallelism on the GPU, through the C ABI (moe_route,
 moe_ep_dispatch, moe_expert_rows, moe_combine_rows) and the orchestration in
-block_diffusion_moe_router_b200.expert_parallel.  Every shape here keeps all
-expert chunks at 128 tokens or fewer, so the expert kernel accumulates the
-same way on an owner as in moe_forward and the bytes must agree:
+block_diffusion_moe_router_b200.expert_parallel.  An expert's tokens form the
+same chunks on an owner as in moe_forward and the kernels' arithmetic for a
+chunk depends on that chunk alone, so the bytes must agree:
 
   - one rank: bit-identical to moe_forward on the same inputs;
   - four ranks emulated in one process on one GPU (the all-to-alls done by
@@ -97,9 +97,13 @@ def test_one_rank_bit_identical_to_moe_forward(wd):
 
 def test_four_emulated_ranks_on_the_canvas():
     """The canvas layer (T=256, d=2816, 128 experts, top-8, f=704) over four
-    emulated ranks of 64 tokens and 32 experts each, with a residual."""
+    emulated ranks of 64 tokens and 32 experts each, with a residual and a
+    router bias that sends every token to expert 5 (a 256-token chunk next
+    to small ones)."""
     w = inputs.WORKLOADS["canvas"]
     lay = inputs.make_layer(w, device="cuda")
+    lay["router_bias"] = torch.zeros(w.E, device="cuda")
+    lay["router_bias"][5] = 50.0
     res = inputs._randn((w.T, w.d), 1.0, 78, "cuda", torch.bfloat16)
     want = _reference(lay, w.E, w.k, w.d, w.f, inputs.WDTYPE_BF16, res)
     got = _emulated(lay, w.E, w.k, w.d, w.f, inputs.WDTYPE_BF16, 4, res)
