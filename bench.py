@@ -460,6 +460,62 @@ class LayerRun:
             flops += fl
         return expert_bytes / self.L, layer_bytes, flops, wbytes
 
+    def forward_into(self, x, out):
+        """One step on input x, the last layer writing into out (layers chained
+        through the residual, as in step())."""
+        if self.L == 1:
+            self.layer_call(0, x, out, None, self.rws[0], self.gms[0])
+            return out
+        cur = x
+        for l in range(self.L):
+            nxt = out if l == self.L - 1 else self.bufs[l % 2]
+            self.layer_call(l, cur, nxt, cur)
+            cur = nxt
+        return out
+
+    def e2e_pipelined(self, K, x_host):
+        """Device time of K end-to-end steps: each step copies its input from
+        pinned host memory, runs the layer(s) and copies its result back to
+        pinned host memory.  Two input and two output buffers; the copies run
+        on two side streams, so step i+1's input and step i-1's result move
+        while step i computes (the layer calls stay in order on the plan's
+        stream)."""
+        torch = self.torch
+        T, d = self.T, self.w.d
+        comp = self.stream
+        cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+        xin = [torch.empty((T, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        outd = [torch.empty((T, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        hout = [torch.empty((T, d), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        for b in range(2):
+            ev_done[b].record(comp)
+            ev_out[b].record(cout)
+        self.rep.barrier()
+        torch.cuda.synchronize()
+        h0 = torch.cuda.Event(enable_timing=True)
+        h1 = torch.cuda.Event(enable_timing=True)
+        h0.record(cin)
+        for i in range(K):
+            b = i % 2
+            cin.wait_event(ev_done[b])  # step i-2 no longer reads xin[b]
+            with torch.cuda.stream(cin):
+                xin[b].copy_(x_host[i % len(x_host)], non_blocking=True)
+            ev_in[b].record(cin)
+            comp.wait_event(ev_in[b])
+            comp.wait_event(ev_out[b])  # step i-2's result has left outd[b]
+            self.forward_into(xin[b], outd[b])
+            ev_done[b].record(comp)
+            cout.wait_event(ev_done[b])
+            with torch.cuda.stream(cout):
+                hout[b].copy_(outd[b], non_blocking=True)
+            ev_out[b].record(cout)
+        h1.record(cout)
+        torch.cuda.synchronize()
+        return h0.elapsed_time(h1)
+
     def close(self):
         self.moe.moe_plan_destroy(self.plan)
         self.lays = self.xs = self.outs = self.bufs = None
@@ -543,10 +599,15 @@ def run_ours(args):
            for q in (10, 50, 90)}
     run.check()
 
-    # end to end: host x in, host result out, every step, through the C ABI
+    # end to end: host x in, host result out, every step, through the C ABI.
+    # Reported: the pipelined form (copies on side streams overlap the layer,
+    # two buffers each way); beside it the blocking form, one
+    # moe_forward_host call per step (copy in, layer, copy out, synchronise).
     x_host = [run.xs[i].cpu().pin_memory() for i in range(min(nsets, 4))]
     out_host = torch.empty((T, w.d), dtype=torch.bfloat16).pin_memory()
     K2 = args.steps
+    run.e2e_pipelined(min(K2, 5), x_host)  # warm the side streams
+    e2e_s = rep.max_over_ranks(run.e2e_pipelined(K2, x_host), "cuda") * 1e-3
     rep.barrier()
     torch.cuda.synchronize()
     h0 = torch.cuda.Event(enable_timing=True)
@@ -564,7 +625,7 @@ def run_ours(args):
             stream.synchronize()
     h1.record(stream)
     torch.cuda.synchronize()
-    e2e_s = rep.max_over_ranks(h0.elapsed_time(h1), "cuda") * 1e-3
+    e2e_block_s = rep.max_over_ranks(h0.elapsed_time(h1), "cuda") * 1e-3
     run.check()
 
     hbm, bf16, bf16_sus, basis = peaks()
@@ -639,7 +700,14 @@ def run_ours(args):
         "kernel_ms": kern,
         "gpu_launches": launches_per_layer(w, T, args.router) * L * args.steps,
         "e2e": {"value": rep.job_rate(T, world, K2, e2e_s * 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * w.d * 2, "d2h_bytes_per_step": T * w.d * 2},
+                "h2d_bytes_per_step": T * w.d * 2, "d2h_bytes_per_step": T * w.d * 2,
+                "form": "every step: x from pinned host memory, the layer call(s), the "
+                        "result to pinned host memory; copies on two side streams overlap "
+                        "the layer (two buffers each way), device time by CUDA events",
+                "blocking": {"value": rep.job_rate(T, world, K2, e2e_block_s * 1e3),
+                             "unit": "tokens/s",
+                             "form": "one synchronous moe_forward_host call per step"
+                                     if L == 1 else "copy in, step, copy out, synchronise"}},
         "clocks": clk.summary(),
     }
     # the other workloads the layer is graded on, measured in the same run:
