@@ -7,13 +7,16 @@ f=704, bf16 weights (synthetic, seeded; inputs resident in HBM).  The metric
 is canvas tokens/s per MoE layer; the JSON line also carries the expert
 kernel's HBM roofline fraction, an end-to-end figure through
 moe_forward_host (host buffers, copies inside the timed region) and the CPU
-oracle timed on a bounded sample.  The same line also carries, under the keys
-"encode" and "stack30", the T=2048 prompt+canvas layer (graded on its
-tensor-core fraction) and the 30-layer denoising step, each measured in the
-same run with its own step time, per-kernel times and roofline fractions.
+oracle timed on a bounded sample.  The same line also carries, under their
+own keys, the other workloads measured in the same run: "encode" (the T=2048
+prompt+canvas layer, graded on its tensor-core fraction), "stack30" (the
+30-layer denoising step), "canvas4" / "canvas8" / "canvas4f" (the canvas
+layer with int4, fp8 and fp4 expert weights) and "lmhead" (the lm_head step
+with entropy-bounded acceptance), each with its own step time, per-kernel
+times, roofline fractions and clock record.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--extra encode,stack30 | --no-extra]
+                  [--workload NAME] [--extra NAME,... | --no-extra]
 
 N > 1 runs N independent replicas (one canvas per GPU, no collective on the
 data path), launched one process per GPU by torch.distributed.run.
@@ -69,7 +72,7 @@ def parse():
                    help="router path (auto: tensor cores when E <= 128)")
     p.add_argument("--prefetch-mb", type=int, default=None,
                    help="MiB of gate_up weights pulled into L2 during routing")
-    p.add_argument("--extra", default="encode,stack30",
+    p.add_argument("--extra", default="encode,stack30,canvas4,canvas8,canvas4f,lmhead",
                    help="other workloads measured in the same run, reported under their "
                         "own keys of the JSON line")
     p.add_argument("--no-extra", action="store_true", help="measure the main workload only")
@@ -572,6 +575,68 @@ def sub_record(name, args, rank, steps, warmup):
     return rec
 
 
+def lmhead_record(args, rank, steps, warmup):
+    """The lm_head step over a 256-token canvas (V=262144, d=2816) measured in
+    the same run: step time, GEMM time and its fractions of the measured HBM
+    bandwidth and of the sustained bf16 peak."""
+    import torch
+    import block_diffusion_moe_router_b200 as moe
+    from block_diffusion_moe_router_b200 import inputs
+    T, V, d = 256, inputs.LMHEAD_V, inputs.LMHEAD_D
+    temp, bound = 0.8, 0.1
+    nsets = 4
+    hs, W, _ = inputs.make_lmhead(T * nsets, V, d, seed=11 + rank, device="cuda")
+    hs = [hs[i * T:(i + 1) * T].contiguous() for i in range(nsets)]
+    g = torch.Generator().manual_seed(3)
+    masked = (torch.rand(T, generator=g) < 0.75).to(torch.uint8).cuda()
+    lh = moe.LmHead(V, d)
+    stream = torch.cuda.current_stream()
+    outs = [torch.empty(T, dtype=dt, device="cuda")
+            for dt in (torch.int32, torch.float32, torch.float32, torch.uint8)]
+
+    def run(K):
+        for i in range(K):
+            moe.moe_lmhead_forward(lh.handle, T, hs[i % nsets], W, temp, 0.0, masked, bound,
+                                   *outs, stream)
+
+    run(warmup)
+    torch.cuda.synchronize()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    with ClockSampler(local) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run(steps)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        moe.moe_lmhead_set_profile(lh.handle, True)
+        run(steps)
+        moe.moe_lmhead_set_profile(lh.handle, False)
+    ms = e0.elapsed_time(e1) / steps
+    gemm_ms, n = moe.moe_lmhead_profile(lh.handle)
+    gemm_ms /= max(n, 1)
+    if lh.sync_status() != moe.MOE_OK:
+        raise RuntimeError("lm_head step reported a device error")
+    lh.close()
+    del hs, W
+    torch.cuda.empty_cache()
+    hbm, bf16, bf16_sus, basis = peaks()
+    alg_bytes = V * d * 2 + T * d * 2
+    flops = 2.0 * T * V * d
+    return {
+        "workload": f"lmhead: T={T} canvas tokens, V={V}, d={d}, bf16 h and W, temperature "
+                    f"{temp}, entropy bound {bound}, 75% of positions masked",
+        "steps": steps, "warmup": warmup,
+        "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3),
+        "gemm_ms": gemm_ms,
+        "gemm_hbm_frac": alg_bytes / (gemm_ms * 1e-3) / 1e9 / hbm,
+        "gemm_tensor_frac_of_sustained_peak": flops / (gemm_ms * 1e-3) / 1e12 / bf16_sus,
+        "gemm_tensor_frac_of_burst_peak": flops / (gemm_ms * 1e-3) / 1e12 / bf16,
+        "peak_basis": f"{basis}: HBM {hbm} GB/s, bf16 {bf16} / {bf16_sus} TFLOP/s",
+        "clocks": clk.summary(),
+        "gpu_launches": 3 * steps,
+    }
+
+
 def run_ours(args):
     import torch
     import block_diffusion_moe_router_b200 as moe
@@ -714,8 +779,11 @@ def run_ours(args):
     # the T=2048 encode layer (tensor-core target) and the 30-layer step
     extras = [] if args.no_extra else [x for x in args.extra.split(",") if x and x != w.name]
     for name in extras:
-        steps, warm = {"encode": (100, 20), "stack30": (20, 5)}.get(name, (50, 10))
-        line[name] = sub_record(name, args, rank, steps, warm)
+        steps, warm = {"encode": (100, 20), "stack30": (20, 5)}.get(name, (100, 20))
+        if name == "lmhead":
+            line[name] = lmhead_record(args, rank, steps, warm)
+        else:
+            line[name] = sub_record(name, args, rank, steps, warm)
     if lay_cpu is not None:
         cb = cpu_baseline(lay_cpu, w)
         if L > 1:
