@@ -186,8 +186,9 @@ def router_on_tensor_cores(w, T: int, router: str) -> bool:
 
 def launches_per_layer(w, T: int, router: str) -> int:
     """Kernels one moe_forward launches: router, route plan, gather, expert
-    GEMMs, combine."""
-    return 5
+    GEMMs, combine; the plan and the gather are one launch for one canvas
+    (T <= 256, k <= 8)."""
+    return 4 if (T <= 256 and w.k <= 8) else 5
 
 
 # weight formats by moe_wdtype_t value (bf16, int4, fp8, fp4)

@@ -465,6 +465,24 @@ def test_coded_split_k_boundary(wd, T):
     print("split-K boundary", wd, T, "rel-L2", err)
 
 
+@pytest.mark.parametrize("f", [64, 320])
+@pytest.mark.parametrize("T", [1, 128, 129, 144, 145, 200, 256, 300])
+def test_bf16_issuer_split_boundary(T, f):
+    """k = E: every expert gets all T tokens.  The bf16 kernel's two UMMA
+    issuers split K for a unit of at most 128 tokens with two or more K
+    stages; a larger unit, or one of a single K stage, is one issuer's.
+    d=640 gives gate_up ten K stages; f=320 gives down five, f=64 one (a
+    single-issuer down unit at every T).  T=128/129 and 144/145 sit on either
+    side of the split boundary and of a 16-column UMMA step; T=300 makes a
+    256-token chunk next to a 44-token one, so the widest activation stage
+    and a split unit share the ring."""
+    E = k = 2
+    d = 640
+    lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=400 + T + f)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f)
+    print("issuer split boundary", T, f, "rel-L2", err)
+
+
 # ------------------------------------------------------------------ edge cases
 
 
