@@ -451,13 +451,14 @@ def test_fp4_block_scale_ranges(kind):
 
 
 @pytest.mark.parametrize("wd", [inputs.WDTYPE_FP8, inputs.WDTYPE_FP4])
-@pytest.mark.parametrize("T", [64, 65, 128, 129])
+@pytest.mark.parametrize("T", [1, 16, 32, 33, 64, 65, 128, 129])
 def test_coded_split_k_boundary(wd, T):
     """k = E: every expert gets all T tokens.  The fp8 and fp4 kernels split
     K between their two UMMA warps only for units of at most 64 tokens with
-    two or more stage pairs: T=64 splits, 65 and 128 do not, 129 makes a
-    128-token chunk and a 1-token chunk that splits.  d=640 gives gate_up
-    five K stages (a last pair of one stage), f=320 gives down three."""
+    two or more stage pairs: T=1 … 64 split (T=1 and 16 with UMMA N=16, 33
+    across a 32-column step), 65 and 128 do not, 129 makes a 128-token chunk
+    and a 1-token chunk that splits.  d=640 gives gate_up five K stages (a
+    last pair of one stage), f=320 gives down three."""
     E = k = 2
     d, f = 640, 320
     lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=200 + T + wd, wdtype=wd)
