@@ -14,7 +14,7 @@ from ._abi import (  # noqa: F401
     MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_ALLOC, MOE_ERR_CUDA,
     MOE_ERR_TIMEOUT, MOE_ERR_DEVICE_CHECK, MOE_W_BF16, MOE_W_INT4_G128, MOE_W_FP8_E4M3, MOE_W_FP4_E2M1, MOE_OPT_EPS,
     MOE_OPT_TIMEOUT_MS, MOE_OPT_PROFILE, MOE_OPT_TEST_STALL, MOE_OPT_PDL,
-    MOE_OPT_L2_PREFETCH_MB, MOE_OPT_ROUTER, MOE_OPT_Y_BF16, MOE_OPT_DEBUG, MOE_MAX_T,
+    MOE_OPT_L2_PREFETCH_MB, MOE_OPT_ROUTER, MOE_OPT_Y_BF16, MOE_OPT_DEBUG, MOE_OPT_CHUNK_TOKENS, MOE_MAX_T,
     MOE_MAX_ASSIGNMENTS, MOE_K_ROUTER, MOE_K_PLAN,
     MOE_K_EXPERT, MOE_K_COMBINE, KERNEL_NAMES, MoeError,
     moe_plan_create, moe_plan_set_option, moe_plan_reserve, moe_forward, moe_forward_host,

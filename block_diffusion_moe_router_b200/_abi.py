@@ -36,6 +36,7 @@ MOE_OPT_L2_PREFETCH_MB = 5
 MOE_OPT_ROUTER = 6
 MOE_OPT_Y_BF16 = 7
 MOE_OPT_DEBUG = 8
+MOE_OPT_CHUNK_TOKENS = 9
 
 MOE_MAX_T = 65536
 MOE_MAX_ASSIGNMENTS = 1 << 19

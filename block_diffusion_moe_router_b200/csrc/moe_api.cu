@@ -45,6 +45,7 @@ struct moe_plan_s {
   int y_bf16;
   int router_sel;
   int debug;       // MOE_OPT_DEBUG: lay the next workspace out with guard blocks
+  int chunk_tokens;  // MOE_OPT_CHUNK_TOKENS: 0 (by call size), 128 or 256
   int cap_T;
   int last_T;
   void* ws;  // one device allocation holding everything below
@@ -134,9 +135,19 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Tokens per scheduler chunk: 256 for bf16 weights, 128 for int4 and fp8
-// (whose kernels keep decoded A stages in TMEM next to the accumulators).
-int chunk_size(moe_plan_t p) { return p->wdtype == MOE_W_BF16 ? moe::kMaxN : 128; }
+// Tokens per scheduler chunk.  128 for the int4, fp8 and fp4 kernels (which
+// keep decoded A stages in TMEM next to the accumulators).  bf16:
+// MOE_OPT_CHUNK_TOKENS, by default 128 for a call of at most 256 tokens and
+// 256 above.  At one canvas a hot expert then becomes chunks of at most 128
+// tokens, each with two UMMA issuers and activation stages of at most 16 KB
+// (a 256-token chunk sizes every stage at 32 KB and leaves two); for long
+// calls, where most experts get 100-200 tokens, one 256-token chunk streams
+// each expert's weights once.
+int chunk_size(moe_plan_t p, int T) {
+  if (p->wdtype != MOE_W_BF16) return 128;
+  if (p->chunk_tokens == 128 || p->chunk_tokens == moe::kMaxN) return p->chunk_tokens;
+  return T <= 256 ? 128 : moe::kMaxN;
+}
 
 size_t max_chunks(int E, size_t T, int k) { return (size_t)E + (T * (size_t)k) / 128 + 1; }
 
@@ -437,6 +448,7 @@ moe_status_t moe_plan_create(int E, int k, int d, int f, moe_wdtype_t wdtype, mo
   p->y_bf16 = 1;
   p->router_sel = 0;
   p->debug = 0;
+  p->chunk_tokens = 0;
   p->cap_T = 0;
   p->last_T = 0;
   p->ws = nullptr;
@@ -478,6 +490,10 @@ moe_status_t moe_plan_set_option(moe_plan_t p, int key, double value) {
       return MOE_OK;
     case MOE_OPT_DEBUG:
       p->debug = value != 0.0;
+      return MOE_OK;
+    case MOE_OPT_CHUNK_TOKENS:
+      if (value != 0.0 && value != 128.0 && value != (double)moe::kMaxN) return MOE_ERR_INVALID_ARG;
+      p->chunk_tokens = (int)value;
       return MOE_OK;
   }
   return MOE_ERR_INVALID_ARG;
@@ -576,7 +592,7 @@ moe_status_t forward_impl(moe_plan_t p, int T, const void* x, const float* route
   pa.k = p->k;
   pa.d = p->d;
   pa.f = p->f;
-  pa.chunk = chunk_size(p);
+  pa.chunk = chunk_size(p, T);
   pa.idx = row_expert ? row_expert : p->idx;
   pa.offsets = p->offsets;
   pa.perm = p->perm;
@@ -726,7 +742,7 @@ moe_status_t moe_ep_dispatch(moe_plan_t p, int T, const void* x, const int32_t* 
   pa.k = p->k;
   pa.d = p->d;
   pa.f = p->f;
-  pa.chunk = chunk_size(p);
+  pa.chunk = chunk_size(p, T);
   pa.idx = p->idx;
   pa.offsets = p->offsets;
   pa.perm = p->perm;
@@ -1037,7 +1053,7 @@ extern "C" moe_status_t moe_forward_noalloc(moe_plan_t p, int T, const void* x,
   pa.k = p->k;
   pa.d = p->d;
   pa.f = p->f;
-  pa.chunk = chunk_size(p);
+  pa.chunk = chunk_size(p, T);
   pa.idx = idx;
   pa.offsets = offsets;
   pa.perm = perm;

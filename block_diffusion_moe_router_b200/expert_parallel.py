@@ -50,12 +50,17 @@ def local_slice(t: Optional[torch.Tensor], E: int, world: int, rank: int):
 
 class LibraryOps:
     """The layer's steps on the GPU, through the C ABI: a routing plan (E
-    experts, top-k) and an owner plan (the rank's E / world experts, k = 1)."""
+    experts, top-k) and an owner plan (the rank's E / world experts, k = 1).
+    `chunk_tokens` is the owner plan's MOE_OPT_CHUNK_TOKENS (0: by the size
+    of each call); give moe_forward's plan the same explicit value where the
+    two must agree byte for byte."""
 
-    def __init__(self, E: int, k: int, d: int, f: int, wdtype: int, world: int):
+    def __init__(self, E: int, k: int, d: int, f: int, wdtype: int, world: int,
+                 chunk_tokens: int = 0):
         self.E, self.k, self.d, self.f = E, k, d, f
         self.route_plan = _abi.moe_plan_create(E, k, d, f, wdtype)
         self.owner_plan = _abi.moe_plan_create(E // world, 1, d, f, wdtype)
+        _abi.moe_plan_set_option(self.owner_plan, _abi.MOE_OPT_CHUNK_TOKENS, chunk_tokens)
 
     def route(self, x, router_w, router_gamma, router_bias, stream=None):
         T = x.shape[0]
@@ -148,11 +153,12 @@ class ExpertParallelLayer:
     rank's slices of w_gate_up / w_down (and scales), see `local_slice`."""
 
     def __init__(self, E: int, k: int, d: int, f: int, wdtype: int = _abi.MOE_W_BF16,
-                 rank: int = 0, world: int = 1, exchange=None, ops=None):
+                 rank: int = 0, world: int = 1, exchange=None, ops=None, chunk_tokens: int = 0):
         owned_experts(E, world, rank)  # validates the split
         self.E, self.k, self.d, self.f = E, k, d, f
         self.rank, self.world = rank, world
-        self.ops = ops if ops is not None else LibraryOps(E, k, d, f, wdtype, world)
+        self.ops = ops if ops is not None else LibraryOps(E, k, d, f, wdtype, world,
+                                                          chunk_tokens)
         if exchange is None:
             exchange = LocalExchange() if world == 1 else TorchExchange()
         self.exchange = exchange

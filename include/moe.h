@@ -119,7 +119,7 @@ enum {
   MOE_OPT_Y_BF16 = 7,     /* 1 (default): the per-slot expert outputs y are kept
                              in bf16 (one more rounding before the fp32
                              combine, half the bytes); 0: fp32                   */
-  MOE_OPT_DEBUG = 8       /* 1: the workspace is laid out with a 256-byte guard
+  MOE_OPT_DEBUG = 8,      /* 1: the workspace is laid out with a 256-byte guard
                              block after every region, filled with a fixed
                              pattern when the workspace is (re)allocated;
                              moe_plan_sync_status then also checks every guard
@@ -127,6 +127,18 @@ enum {
                              past its region.  Takes effect at the next
                              workspace (re)allocation (set it before the first
                              call or moe_plan_reserve).  Default 0.             */
+  MOE_OPT_CHUNK_TOKENS = 9 /* bf16 weights: tokens per work chunk of an expert,
+                             128 or 256; 0 (default) picks 128 for a call of
+                             at most 256 tokens and 256 above.  An expert
+                             with more tokens than a chunk is split into
+                             chunks, each streaming the expert's weights;
+                             chunks of at most 128 tokens are multiplied by
+                             two UMMA issuers that split K, so the fp32
+                             summation order, and the result's last bits,
+                             depend on the chunking: give two plans whose
+                             results must agree byte for byte (expert-parallel
+                             owners and moe_forward) the same explicit value.
+                             The int4, fp8 and fp4 kernels always use 128.   */
 };
 
 /* Kernels of one moe_forward, for moe_plan_profile. */
@@ -268,9 +280,11 @@ moe_status_t moe_route(moe_plan_t plan, int T, const void* x, const float* route
  * With bf16 y rows (MOE_OPT_Y_BF16 on, the default) every rank's out equals
  * moe_forward's bytes for bf16 and int4 weights (and for fp8 / fp4 weights
  * without expert_gamma: those paths carry fp16 rows, and a row normalised
- * on the sender travels as bf16): an expert's tokens form the same chunks
- * on the owner as in moe_forward, and the expert kernels' arithmetic for a
- * chunk depends on that chunk alone. */
+ * on the sender travels as bf16), provided the owner plan and moe_forward's
+ * plan have the same explicit MOE_OPT_CHUNK_TOKENS (its default depends on
+ * the call's size, which differs between them): an expert's tokens then
+ * form the same chunks on the owner as in moe_forward, and the expert
+ * kernels' arithmetic for a chunk depends on that chunk alone. */
 
 /* Step 2, on the routing plan (E experts, top-k) of the sending rank.
  *   x             bf16 [T, d]  the rank's tokens

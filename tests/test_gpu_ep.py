@@ -26,9 +26,10 @@ def _cuda(lay):
     return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in lay.items()}
 
 
-def _reference(lay, E, k, d, f, wd, residual):
+def _reference(lay, E, k, d, f, wd, residual, chunk_tokens=0):
     layer = moe.MoeLayer(E, k, d, f, wd)
     try:
+        moe.moe_plan_set_option(layer.plan, moe.MOE_OPT_CHUNK_TOKENS, chunk_tokens)
         out = layer.forward(lay["x"], lay["router_w"], lay["router_gamma"], lay["w_gate_up"],
                             lay["w_down"], router_bias=lay.get("router_bias"),
                             scales_gate_up=lay.get("scales_gate_up"),
@@ -45,12 +46,13 @@ def _weights(lay, E, world, rank):
             for key in ("w_gate_up", "w_down", "scales_gate_up", "scales_down")}
 
 
-def _emulated(lay, E, k, d, f, wd, world, residual):
+def _emulated(lay, E, k, d, f, wd, world, residual, chunk_tokens=0):
     """All ranks in this process: phases in turn, exchanges by concatenation."""
     T = lay["x"].shape[0]
     sl = [slice(r * T // world, (r + 1) * T // world) for r in range(world)]
     layers = [ep.ExpertParallelLayer(E, k, d, f, wd, rank=r, world=world,
-                                     exchange=ep.LocalExchange()) for r in range(world)]
+                                     exchange=ep.LocalExchange(), chunk_tokens=chunk_tokens)
+              for r in range(world)]
     try:
         st = [layers[r].begin(lay["x"][sl[r]].contiguous(), lay["router_w"], lay["router_gamma"],
                               lay.get("router_bias"), lay.get("expert_gamma"))
@@ -95,18 +97,22 @@ def test_one_rank_bit_identical_to_moe_forward(wd):
     assert torch.equal(got, want)
 
 
-def test_four_emulated_ranks_on_the_canvas():
+@pytest.mark.parametrize("chunk_tokens", [128, 256])
+def test_four_emulated_ranks_on_the_canvas(chunk_tokens):
     """The canvas layer (T=256, d=2816, 128 experts, top-8, f=704) over four
     emulated ranks of 64 tokens and 32 experts each, with a residual and a
-    router bias that sends every token to expert 5 (a 256-token chunk next
-    to small ones)."""
+    router bias that sends every token to expert 5 (two 128-token chunks, or
+    one 256-token chunk, next to small ones).  The owners' plans and the
+    reference plan take the same explicit chunk size: by default it follows
+    each call's size, and an owner's call (all rows it receives) is not the
+    size of the whole layer's."""
     w = inputs.WORKLOADS["canvas"]
     lay = inputs.make_layer(w, device="cuda")
     lay["router_bias"] = torch.zeros(w.E, device="cuda")
     lay["router_bias"][5] = 50.0
     res = inputs._randn((w.T, w.d), 1.0, 78, "cuda", torch.bfloat16)
-    want = _reference(lay, w.E, w.k, w.d, w.f, inputs.WDTYPE_BF16, res)
-    got = _emulated(lay, w.E, w.k, w.d, w.f, inputs.WDTYPE_BF16, 4, res)
+    want = _reference(lay, w.E, w.k, w.d, w.f, inputs.WDTYPE_BF16, res, chunk_tokens)
+    got = _emulated(lay, w.E, w.k, w.d, w.f, inputs.WDTYPE_BF16, 4, res, chunk_tokens)
     assert torch.equal(got, want)
 
 

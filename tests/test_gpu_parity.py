@@ -466,9 +466,10 @@ def test_coded_split_k_boundary(wd, T):
     print("split-K boundary", wd, T, "rel-L2", err)
 
 
+@pytest.mark.parametrize("chunk", [0, 256])
 @pytest.mark.parametrize("f", [64, 320])
 @pytest.mark.parametrize("T", [1, 128, 129, 144, 145, 200, 256, 300])
-def test_bf16_issuer_split_boundary(T, f):
+def test_bf16_issuer_split_boundary(T, f, chunk):
     """k = E: every expert gets all T tokens.  The bf16 kernel's two UMMA
     issuers split K for a unit of at most 128 tokens with two or more K
     stages; a larger unit, or one of a single K stage, is one issuer's.
@@ -476,12 +477,15 @@ def test_bf16_issuer_split_boundary(T, f):
     single-issuer down unit at every T).  T=128/129 and 144/145 sit on either
     side of the split boundary and of a 16-column UMMA step; T=300 makes a
     256-token chunk next to a 44-token one, so the widest activation stage
-    and a split unit share the ring."""
+    and a split unit share the ring.  With the default chunk size (chunk=0)
+    a call of at most 256 tokens is cut into chunks of at most 128, so the
+    single-issuer units above 128 tokens appear there only with chunk=256."""
     E = k = 2
     d = 640
     lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=400 + T + f)
-    err, _ = full_check(lay, _cuda(lay), E, k, d, f)
-    print("issuer split boundary", T, f, "rel-L2", err)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f,
+                        options={moe.MOE_OPT_CHUNK_TOKENS: chunk})
+    print("issuer split boundary", T, f, chunk, "rel-L2", err)
 
 
 # ------------------------------------------------------------------ edge cases
@@ -537,15 +541,17 @@ def test_awq_fold_invariance_on_gpu():
     assert torch.equal(outs[0], outs[1])
 
 
-def test_hot_expert_multi_chunk():
+@pytest.mark.parametrize("chunk", [0, 128])
+def test_hot_expert_multi_chunk(chunk):
     """One expert receives every token (T=600 > 256): its work splits into
-    three 256-token chunks; the widest B stage is exercised."""
+    three chunks of at most 256 tokens (the default above 256 tokens; the
+    widest B stage is exercised), or five of at most 128."""
     T, E, k, d, f = 600, 16, 2, 256, 128
     lay = inputs.make_small(T=T, d=d, E=E, k=k, f=f, seed=77, bias=True)
     lay["router_bias"] = torch.zeros(E)
     lay["router_bias"][5] = 50.0
-    err, _ = full_check(lay, _cuda(lay), E, k, d, f)
-    print("hot expert rel-L2", err)
+    err, _ = full_check(lay, _cuda(lay), E, k, d, f, options={moe.MOE_OPT_CHUNK_TOKENS: chunk})
+    print("hot expert rel-L2", chunk, err)
 
 
 def test_zero_tokens_is_noop():
@@ -575,6 +581,20 @@ def test_forward_host_matches_device(canvas):
 
 
 # ------------------------------------------------------------------ error paths
+
+
+def test_chunk_option_values():
+    """MOE_OPT_CHUNK_TOKENS takes 0, 128 or 256 and nothing else."""
+    layer = moe.MoeLayer(16, 2, 256, 64)
+    try:
+        for v in (0, 128, 256):
+            assert moe.moe_plan_set_option(layer.plan, moe.MOE_OPT_CHUNK_TOKENS, v,
+                                           check=False) == moe.MOE_OK
+        for v in (64, 100, 512, -1):
+            assert moe.moe_plan_set_option(layer.plan, moe.MOE_OPT_CHUNK_TOKENS, v,
+                                           check=False) == moe.MOE_ERR_INVALID_ARG
+    finally:
+        layer.close()
 
 
 def test_invalid_arguments_launch_nothing():
