@@ -1,6 +1,6 @@
 // expert.cu -- grouped expert GEMMs of the MoE FFN on tcgen05 tensor cores.
 //
-// One persistent kernel runs every (expert, 256-token chunk) work unit of both
+// One persistent kernel runs every (expert, chunk of <= 256 tokens) work unit of both
 // projections (auto-round pull request "Add quantization support for
 // DiffusionGemma", transformers backend test log: gate_proj / up_proj
 // 2816->704, down_proj 704->2816, act GELUTanh; Quant-Tuner pull request,
@@ -12,11 +12,12 @@
 //     the epilogue pairs TMEM lane r (gate) with lane 64+r (up) and writes
 //     h = gelu_tanh(gate) * up in bf16.
 //   down unit (e, chunk, m): rows [m*128, m*128+128) of W_d[e] against the
-//     chunk's h rows; the epilogue writes y (fp32) per slot.
+//     chunk's h rows; the epilogue writes y (bf16, or fp32) per slot.
 //
 // "Swap-AB": weight rows are the UMMA M dimension and the tokens routed to
 // the expert are N (16..256), so every weight byte is streamed from HBM once
-// per chunk, and at 256 tokens per canvas one chunk covers every expert.
+// per chunk; the plan cuts an expert's tokens into chunks of 128 or 256
+// (the host's choice), so at one canvas only a hot expert has two.
 //
 // Roles (256 threads): warp 0 = scheduler (claims units: its CTA index
 // first, then from a global counter) and weight (A) producer, warps 1 and 7
