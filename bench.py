@@ -554,6 +554,7 @@ def sub_record(name, args, rank, steps, warmup):
         "ms_per_step": ms_step,
         "ms_per_layer": ms_step / w.layers,
         "tokens_per_s_per_layer": w.T * w.layers / t,
+        "canvas_tokens_per_s_per_step": w.T / t,  # T tokens through all the step's layers
         "step_ms_p10_p50_p90": [per_step[int(q * (len(per_step) - 1))] for q in (0.1, 0.5, 0.9)],
         "touched_experts_per_layer": sum(run.touched) / w.layers,
         "alg_bytes_per_step": step_bytes,
