@@ -269,13 +269,16 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(PlanArgs a) {
 // With xf16 the row is written as fp16 instead (exact for bf16 values of
 // magnitude 2^-14 .. 65504; the normed row is rounded once, to fp16).
 constexpr int kGatherVec = 16;  // uint4 per lane held in registers (d <= 4096)
+constexpr int kGatherMaxD = 4096;
 
 // One row (warp-wide, lane owns 16-byte pieces lane + 32j), in passes of
 // VEC pieces per lane with every load of a pass issued before any use.  With
 // the expert norm, the row's sum of squares is taken first (an extra read
-// when the row needs more than one pass).
+// when the row needs more than one pass); g1, when given, holds 1 + gamma2
+// (in shared memory), else gamma2 is read from global memory.
 template <int VEC>
-__device__ __forceinline__ void gather_row(const GatherArgs& a, int row, int t, int lane) {
+__device__ __forceinline__ void gather_row(const GatherArgs& a, int row, int t, int lane,
+                                           const float* g1 = nullptr) {
   const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d);
   uint4* dst = reinterpret_cast<uint4*>(a.x_perm + (size_t)row * a.d);
   const int n = a.d / 8;
@@ -317,14 +320,23 @@ __device__ __forceinline__ void gather_row(const GatherArgs& a, int row, int t, 
       for (int j = 0; j < VEC; ++j) {
         const int i = p0 + lane + 32 * j;
         if (i < n) {
-          const float4 ga = __ldg(g4 + 2 * i), gb = __ldg(g4 + 2 * i + 1);
-          const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          float g[8];  // 1 + gamma2 of the piece's eight columns
+          if (g1) {
+            const float4 ga = reinterpret_cast<const float4*>(g1)[2 * i];
+            const float4 gb = reinterpret_cast<const float4*>(g1)[2 * i + 1];
+            g[0] = ga.x; g[1] = ga.y; g[2] = ga.z; g[3] = ga.w;
+            g[4] = gb.x; g[5] = gb.y; g[6] = gb.z; g[7] = gb.w;
+          } else {
+            const float4 ga = __ldg(g4 + 2 * i), gb = __ldg(g4 + 2 * i + 1);
+            g[0] = 1.f + ga.x; g[1] = 1.f + ga.y; g[2] = 1.f + ga.z; g[3] = 1.f + ga.w;
+            g[4] = 1.f + gb.x; g[5] = 1.f + gb.y; g[6] = 1.f + gb.z; g[7] = 1.f + gb.w;
+          }
           __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&v[j]);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float2 f = __bfloat1622float2(h2[q]);
-            const float y0 = (f.x * inv) * (1.f + g[2 * q]);
-            const float y1 = (f.y * inv) * (1.f + g[2 * q + 1]);
+            const float y0 = (f.x * inv) * g[2 * q];
+            const float y1 = (f.y * inv) * g[2 * q + 1];
             if (a.xf16)
               *reinterpret_cast<__half2*>(&h2[q]) = __floats2half2_rn(y0, y1);
             else
@@ -390,6 +402,7 @@ __global__ void __launch_bounds__(kSmallT) plan_gather_small_kernel(PlanArgs a, 
   __shared__ int s_maxc;
   __shared__ int s_bad;
   __shared__ int s_perm[kSmallA];
+  __shared__ __align__(16) float s_g1[kGatherMaxD];  // 1 + gamma2 (expert norm)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -407,6 +420,10 @@ __global__ void __launch_bounds__(kSmallT) plan_gather_small_kernel(PlanArgs a, 
   // The expert kernel may launch at once: it waits for this grid to complete.
   pdl_launch_dependents();
   pdl_wait();  // idx comes from the router
+  // the expert norm's 1 + gamma2 into shared memory; its loads overlap the
+  // plan below (the gather, after the plan's barriers, reads it)
+  if (g.gamma2)
+    for (int i = tid; i < g.d; i += kSmallT) s_g1[i] = 1.f + __ldg(g.gamma2 + i);
   __syncthreads();
 
   int ev[kSmallK];
@@ -507,7 +524,7 @@ __global__ void __launch_bounds__(kSmallT) plan_gather_small_kernel(PlanArgs a, 
     for (int i = tid; i < A; i += kSmallT) a.perm[i] = s_perm[i];
   // this CTA's rows of x_perm (a warp per row)
   for (int row = blockIdx.x * (kSmallT / 32) + warp; row < A; row += gridDim.x * (kSmallT / 32))
-    gather_row<kGatherVec>(g, row, s_perm[row], lane);
+    gather_row<kGatherVec>(g, row, s_perm[row], lane, g.gamma2 ? s_g1 : nullptr);
 }
 
 // out[t] = residual[t] + sum_j w[t,j] * y[slot_of[t,j]]   (j order, fp32, one
