@@ -278,17 +278,22 @@ def test_encode_shape_coded_weights_sampled_rows(wd):
           "sampled rel-L2", err)
 
 
-def test_stack30_layer_zipf_bias_and_residual():
+@pytest.mark.parametrize("chunk", [0, 256])
+def test_stack30_layer_zipf_bias_and_residual(chunk):
     """One layer of the 30-layer stack: Zipf-skewed router bias, residual added
     in place (out aliases residual).  The delta is checked with the residual
-    off, the residual path on the full output."""
+    off, the residual path on the full output.  chunk=0 cuts the hot experts'
+    tokens into 128-token chunks (the default at one canvas), chunk=256 keeps
+    each in one chunk of up to 256 tokens."""
     w = inputs.WORKLOADS["stack30"]
     lay_gpu = inputs.make_layer(w, layer=7, device="cuda")
     lay_cpu = _cpu(lay_gpu)
-    err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f)
+    opts = {moe.MOE_OPT_CHUNK_TOKENS: chunk}
+    err, _ = full_check(lay_cpu, lay_gpu, w.E, w.k, w.d, w.f, options=opts)
     res = inputs._randn((w.T, w.d), 1.0, 4242, "cuda", torch.bfloat16)
     layer = moe.MoeLayer(w.E, w.k, w.d, w.f)
     try:
+        moe.moe_plan_set_option(layer.plan, moe.MOE_OPT_CHUNK_TOKENS, chunk)
         delta = run_gpu(layer, lay_gpu, w.T).float()
         buf = res.clone()
         out = run_gpu(layer, lay_gpu, w.T, residual=buf, out=buf).float()
